@@ -1,0 +1,147 @@
+"""fp64 CPU oracle for Kimi Delta Attention (KDA) -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference leg may import this package. The CUDA library never does, and the
+two share no code: this side is plain C (``kda_oracle.c``, compiled with gcc)
+plus the numpy marshalling below.
+
+Functions and the passages they follow (pages cited by title and section):
+
+* :func:`recurrent` -- the KDA recurrence token by token, "[Kimi-2] Kimi
+  Linear：用 KDA 重写长上下文注意力" §3 (boxed update, three-step form) with the
+  §1 readout ``o_t = S_t^T q_t`` and §6.2 L2 normalisation of q, k.
+* :func:`chunkwise` -- the same outputs through the chunkwise form of §5 (UT
+  transform inside a chunk, state passed between chunks), derived in the C
+  source's comment.
+* :func:`decode_step` -- one token of the recurrence on a resident state,
+  §5 ("S_(t-1) + current token -> S_t + output").
+
+Arrays are ``numpy`` (any real dtype; converted to fp64). Layouts::
+
+    q, k, log_alpha [T, H, dk]   v [T, H, dv]   beta [T, H]
+    S0, S_T         [N, H, dk, dv]              cu_seqlens [N+1]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+
+
+def build(force: bool = False) -> str:
+    """Compile ``kda_oracle.c`` into ``libkda_oracle.so`` with gcc (plain -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
+             "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def load_library(path: str | None = None):
+    """Load the oracle library (building it first if needed)."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _bind(lib):
+    i, d = ctypes.c_int, ctypes.c_double
+    lib.kda_oracle_recurrent.argtypes = [_D, _D, _D, _D, _D, _D, _I64, i, i, i, i, i, d, _D, _D, i]
+    lib.kda_oracle_chunkwise.argtypes = [_D, _D, _D, _D, _D, _D, _I64, i, i, i, i, i, d, i, _D, _D, i]
+    lib.kda_oracle_decode_step.argtypes = [_D, _D, _D, _D, _D, _D, i, i, i, i, i, d, _D]
+    for f in (lib.kda_oracle_recurrent, lib.kda_oracle_chunkwise, lib.kda_oracle_decode_step):
+        f.restype = ctypes.c_int
+    return lib
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(x):
+    return None if x is None else x.ctypes.data_as(_D)
+
+
+def _prep(q, k, v, log_alpha, beta, S0, cu_seqlens):
+    q, k, v, la, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if k.shape != (T, H, dk) or la.shape != (T, H, dk) or v.shape[:2] != (T, H) or b.shape != (T, H):
+        raise ValueError("inconsistent shapes")
+    cu = np.array([0, T] if cu_seqlens is None else np.asarray(cu_seqlens), dtype=np.int64)
+    N = len(cu) - 1
+    if cu[-1] != T:
+        raise ValueError("cu_seqlens[-1] must equal T")
+    if S0 is not None:
+        S0 = _f64(S0)
+        if S0.shape != (N, H, dk, dv):
+            raise ValueError("S0 shape")
+    return q, k, v, la, b, S0, cu, T, H, dk, dv, N
+
+
+def _threads(threads):
+    return threads if threads else (os.cpu_count() or 1)
+
+
+def recurrent(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, l2norm=True, eps=1e-6,
+              threads=None):
+    """Token-by-token KDA recurrence in fp64. Returns ``(o [T,H,dv], S_T [N,H,dk,dv])``."""
+    q, k, v, la, b, S0, cu, T, H, dk, dv, N = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
+    o = np.zeros((T, H, dv))
+    ST = np.zeros((N, H, dk, dv))
+    rc = load_library().kda_oracle_recurrent(
+        _p(q), _p(k), _p(v), _p(la), _p(b), _p(S0), cu.ctypes.data_as(_I64), N, H, dk, dv,
+        int(bool(l2norm)), float(eps), _p(o), _p(ST), _threads(threads))
+    if rc:
+        raise RuntimeError("kda_oracle_recurrent failed (%d)" % rc)
+    return o, ST
+
+
+def chunkwise(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, chunk=64, l2norm=True,
+              eps=1e-6, threads=None):
+    """Chunkwise (UT-transform) KDA in fp64. Returns ``(o, S_T)`` like :func:`recurrent`."""
+    q, k, v, la, b, S0, cu, T, H, dk, dv, N = _prep(q, k, v, log_alpha, beta, S0, cu_seqlens)
+    o = np.zeros((T, H, dv))
+    ST = np.zeros((N, H, dk, dv))
+    rc = load_library().kda_oracle_chunkwise(
+        _p(q), _p(k), _p(v), _p(la), _p(b), _p(S0), cu.ctypes.data_as(_I64), N, H, dk, dv,
+        int(bool(l2norm)), float(eps), int(chunk), _p(o), _p(ST), _threads(threads))
+    if rc:
+        raise RuntimeError("kda_oracle_chunkwise failed (%d)" % rc)
+    return o, ST
+
+
+def decode_step(q, k, v, log_alpha, beta, S, l2norm=True, eps=1e-6):
+    """One decode step for N sequences: inputs ``[N,H,d]``, state ``[N,H,dk,dv]``.
+
+    Returns ``(o [N,H,dv], S_new [N,H,dk,dv])``; the input ``S`` is not modified.
+    """
+    q, k, v, la = (_f64(x) for x in (q, k, v, log_alpha))
+    b = _f64(beta)
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    Snew = np.array(S, dtype=np.float64, copy=True, order="C")
+    if Snew.shape != (N, H, dk, dv) or b.shape != (N, H):
+        raise ValueError("inconsistent shapes")
+    o = np.zeros((N, H, dv))
+    rc = load_library().kda_oracle_decode_step(
+        _p(q), _p(k), _p(v), _p(la), _p(b), _p(Snew), N, H, dk, dv, int(bool(l2norm)),
+        float(eps), _p(o))
+    if rc:
+        raise RuntimeError("kda_oracle_decode_step failed (%d)" % rc)
+    return o, Snew

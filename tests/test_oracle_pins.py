@@ -1,0 +1,362 @@
+"""Pins for the fp64 oracle against what the pages and the mathematics fix.
+
+Each check here computes its expected value by a route other than the
+oracle's own three-step update: the worked decay example printed on a page,
+closed forms, the gradient-step definition of the delta rule (via autograd),
+explicit transition matrices (product / DPLR / GDN / DeltaNet forms), the
+read-back property of the delta rule, and the chunkwise form against the
+token recurrence. ``test_pins_catch_planted_mistakes`` plants plausible
+mistakes in a copy of the oracle's C source and checks that the pins fail.
+"""
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def rnd(seed, T, H, dk, dv, unit=True, mu=-1.0, N=1):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((T, H, dk))
+    k = rng.standard_normal((T, H, dk))
+    if unit:
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, H, dv))
+    la = -np.log1p(np.exp(rng.standard_normal((T, H, dk)) + mu))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, H))))
+    S0 = 0.3 * rng.standard_normal((N, H, dk, dv))
+    return q, k, v, la, beta, S0
+
+
+# ---------------------------------------------------------------- pins ----
+
+def pin_worked_decay_example(orc):
+    """Page "Kimi Linear — 逐通道的遺忘", section "KDA：把衰減拆到每個通道": (8,6) -> (4,3) / (8,0.6)."""
+    rows = []
+    with open(os.path.join(HERE, "golden", "channel_decay_example.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append([np.array(p.split(), dtype=float) for p in line.split("|")])
+    assert len(rows) == 2
+    for s_before, alpha, s_after in rows:
+        S0 = s_before.reshape(1, 1, 2, 1)
+        for ch in range(2):
+            q = np.zeros((1, 1, 2)); q[0, 0, ch] = 1.0
+            k = np.array([[[1.0, 0.0]]])
+            v = np.array([[[5.0]]])
+            la = np.log(alpha).reshape(1, 1, 2)
+            beta = np.zeros((1, 1))  # decay step only: no correction/write
+            o, ST = orc.recurrent(q, k, v, la, beta, S0)
+            np.testing.assert_allclose(ST.reshape(2), s_after, rtol=0, atol=1e-14)
+            np.testing.assert_allclose(o[0, 0, 0], s_after[ch], rtol=0, atol=1e-14)
+
+
+def pin_pure_decay_closed_form(orc):
+    """beta = 0 leaves only per-channel decay: S_T = Diag(exp(sum log alpha)) S0."""
+    q, k, v, la, beta, S0 = rnd(1, 9, 2, 5, 3)
+    beta[:] = 0.0
+    o, ST = orc.recurrent(q, k, v, la, beta, S0)
+    G = np.cumsum(la, axis=0)  # [T,H,dk]
+    for h in range(2):
+        np.testing.assert_allclose(ST[0, h], np.exp(G[-1, h])[:, None] * S0[0, h], rtol=1e-13, atol=1e-15)
+        for t in range(9):
+            St = np.exp(G[t, h])[:, None] * S0[0, h]
+            np.testing.assert_allclose(o[t, h], St.T @ q[t, h], rtol=1e-12, atol=1e-14)
+
+
+def pin_delta_readback(orc):
+    """beta = 1 and a unit key: the updated state reads back exactly v_t at k_t,
+    whatever the decay (page "[Kimi-2] Kimi Linear" §2: error ~ 0 once written)."""
+    q, k, v, la, beta, S0 = rnd(2, 12, 2, 6, 4)
+    beta[:] = 1.0
+    q = k.copy()
+    o, _ = orc.recurrent(q, k, v, la, beta, S0)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-12)
+
+
+def pin_overwrite(orc):
+    """Two writes to the same key with beta = 1, alpha = 1: only the last value is read."""
+    rng = np.random.default_rng(3)
+    kk = rng.standard_normal(5); kk /= np.linalg.norm(kk)
+    k = np.stack([kk, kk, kk])[:, None, :]
+    v = rng.standard_normal((3, 1, 4))
+    la = np.zeros((3, 1, 5))
+    beta = np.array([[1.0], [1.0], [0.0]])
+    o, _ = orc.recurrent(k.copy(), k, v, la, beta, 0.5 * rng.standard_normal((1, 1, 5, 4)))
+    np.testing.assert_allclose(o[2, 0], v[1, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o[1, 0], v[1, 0], rtol=0, atol=1e-12)
+
+
+def pin_gradient_step(orc):
+    """Page "[Kimi-2] Kimi Linear" §2-§3: the update is one gradient step of size beta_t on
+    1/2 ||S~^T k_t - v_t||^2 taken at the decayed state S~ = Diag(alpha_t) S_{t-1}.
+    The gradient comes from torch autograd, not from a closed form."""
+    T, dk, dv = 10, 5, 4
+    q, k, v, la, beta, S0 = rnd(4, T, 1, dk, dv)
+    o, ST = orc.recurrent(q, k, v, la, beta, S0)
+    S = torch.tensor(S0[0, 0])
+    for t in range(T):
+        St = (torch.exp(torch.tensor(la[t, 0]))[:, None] * S).detach().requires_grad_(True)
+        kt, vt = torch.tensor(k[t, 0]), torch.tensor(v[t, 0])
+        loss = 0.5 * ((St.T @ kt - vt) ** 2).sum()
+        (g,) = torch.autograd.grad(loss, St)
+        S = (St - float(beta[t, 0]) * g).detach()
+        np.testing.assert_allclose(o[t, 0], (S.T @ torch.tensor(q[t, 0])).numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ST[0, 0], S.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def _A(la_t, k_t, b_t):
+    return (np.eye(len(k_t)) - b_t * np.outer(k_t, k_t)) @ np.diag(np.exp(la_t))
+
+
+def pin_unrolled_product_form(orc):
+    """Page "[Kimi-2] Kimi Linear" §8: o_t = sum_i [q_t^T (prod_{j=i+1..t} A_j) k_i] v_i,
+    read with the write strength beta_i restored and the S0 term added."""
+    T, dk, dv = 7, 4, 3
+    q, k, v, la, beta, S0 = rnd(5, T, 1, dk, dv)
+    o, ST = orc.recurrent(q, k, v, la, beta, S0)
+    A = [_A(la[j, 0], k[j, 0], beta[j, 0]) for j in range(T)]
+
+    def prod(i, t):  # A_t A_{t-1} ... A_{i}  (i > t -> identity)
+        M = np.eye(dk)
+        for j in range(i, t + 1):
+            M = A[j] @ M
+        return M
+
+    for t in range(T):
+        St = prod(0, t) @ S0[0, 0]
+        for i in range(t + 1):
+            St = St + beta[i, 0] * np.outer(prod(i + 1, t) @ k[i, 0], v[i, 0])
+        np.testing.assert_allclose(o[t, 0], St.T @ q[t, 0], rtol=1e-12, atol=1e-13)
+        if t == T - 1:
+            np.testing.assert_allclose(ST[0, 0], St, rtol=1e-12, atol=1e-13)
+
+
+def pin_dplr_form(orc):
+    """Page "[Kimi-2] Kimi Linear" §4: A_t = D_t - a_t b_t^T with D = Diag(alpha), a = beta k,
+    b = alpha * k (both sides tied to the same key)."""
+    T, dk, dv = 8, 5, 3
+    q, k, v, la, beta, S0 = rnd(6, T, 1, dk, dv)
+    o, ST = orc.recurrent(q, k, v, la, beta, S0)
+    S = S0[0, 0].copy()
+    for t in range(T):
+        al = np.exp(la[t, 0])
+        A = np.diag(al) - np.outer(beta[t, 0] * k[t, 0], al * k[t, 0])
+        S = A @ S + beta[t, 0] * np.outer(k[t, 0], v[t, 0])
+        np.testing.assert_allclose(o[t, 0], S.T @ q[t, 0], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ST[0, 0], S, rtol=1e-12, atol=1e-13)
+
+
+def pin_gdn_special_case(orc):
+    """Channel-constant alpha reduces KDA to Gated DeltaNet, page "[Kimi-2] Kimi Linear" §3:
+    S_t = alpha_t (I - beta_t k k^T) S_{t-1} + beta_t k v^T."""
+    T, dk, dv = 9, 4, 6
+    q, k, v, la, beta, S0 = rnd(7, T, 1, dk, dv)
+    la[:] = la[:, :, :1]
+    o, ST = orc.recurrent(q, k, v, la, beta, S0)
+    S = S0[0, 0].copy()
+    for t in range(T):
+        a = np.exp(la[t, 0, 0])
+        S = a * (np.eye(dk) - beta[t, 0] * np.outer(k[t, 0], k[t, 0])) @ S + beta[t, 0] * np.outer(k[t, 0], v[t, 0])
+        np.testing.assert_allclose(o[t, 0], S.T @ q[t, 0], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(ST[0, 0], S, rtol=1e-12, atol=1e-13)
+
+
+def pin_deltanet_special_case(orc):
+    """alpha = 1 reduces KDA to DeltaNet, page "[Kimi-2] Kimi Linear" §2:
+    S_t = S_{t-1} + beta_t k_t (v_t - S_{t-1}^T k_t)^T."""
+    T, dk, dv = 9, 6, 5
+    q, k, v, la, beta, S0 = rnd(8, T, 1, dk, dv)
+    la[:] = 0.0
+    o, ST = orc.recurrent(q, k, v, la, beta, S0)
+    S = S0[0, 0].copy()
+    for t in range(T):
+        S = S + beta[t, 0] * np.outer(k[t, 0], v[t, 0] - S.T @ k[t, 0])
+        np.testing.assert_allclose(o[t, 0], S.T @ q[t, 0], rtol=1e-12, atol=1e-13)
+
+
+def pin_l2norm(orc):
+    """Page "[Kimi-2] Kimi Linear" §6.2: q, k are L2-normalised, so scaling them changes nothing."""
+    q, k, v, la, beta, S0 = rnd(9, 11, 2, 5, 3)
+    o1, S1 = orc.recurrent(q, k, v, la, beta, S0)
+    sc = np.random.default_rng(10).uniform(0.1, 7.0, size=(11, 2, 1))
+    o2, S2 = orc.recurrent(q * sc, k * sc[::-1], v, la, beta, S0)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S2, S1, rtol=1e-12, atol=1e-13)
+    o3, S3 = orc.recurrent(q, k, v, la, beta, S0, l2norm=False)
+    np.testing.assert_allclose(o3, o1, rtol=1e-12, atol=1e-13)
+
+
+def pin_decode_step(orc):
+    """Page "[Kimi-2] Kimi Linear" §5: a decode step is one token of the same recurrence."""
+    N, H, dk, dv = 3, 2, 5, 4
+    q, k, v, la, beta, S0 = rnd(11, N, H, dk, dv, N=N)
+    o, S1 = orc.decode_step(q, k, v, la, beta, S0)
+    for s in range(N):
+        o_r, S_r = orc.recurrent(q[s:s + 1], k[s:s + 1], v[s:s + 1], la[s:s + 1], beta[s:s + 1], S0[s:s + 1])
+        np.testing.assert_allclose(o[s], o_r[0], rtol=1e-14, atol=1e-15)
+        np.testing.assert_allclose(S1[s], S_r[0], rtol=1e-14, atol=1e-15)
+
+
+def pin_chunkwise_equals_recurrent(orc):
+    """Page "[Kimi-2] Kimi Linear" §5: the chunkwise form reaches the recurrence's result."""
+    lengths = [1, 63, 64, 65, 150]
+    cu = np.cumsum([0] + lengths)
+    q, k, v, la, beta, S0 = rnd(12, int(cu[-1]), 2, 8, 6, N=len(lengths))
+    o_r, S_r = orc.recurrent(q, k, v, la, beta, S0, cu)
+    for C in (1, 3, 16, 64):
+        o_c, S_c = orc.chunkwise(q, k, v, la, beta, S0, cu, chunk=C)
+        np.testing.assert_allclose(o_c, o_r, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(S_c, S_r, rtol=1e-11, atol=1e-12)
+
+
+ALL_PINS = [pin_worked_decay_example, pin_pure_decay_closed_form, pin_delta_readback,
+            pin_overwrite, pin_gradient_step, pin_unrolled_product_form, pin_dplr_form,
+            pin_gdn_special_case, pin_deltanet_special_case, pin_l2norm, pin_decode_step,
+            pin_chunkwise_equals_recurrent]
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(pin):
+    pin(oracle)
+
+
+# ------------------------------------------------------ structural tests ----
+
+def test_varlen_packing_equals_separate_calls():
+    lengths = [5, 1, 17, 64, 70]
+    cu = np.cumsum([0] + lengths)
+    q, k, v, la, beta, S0 = rnd(13, int(cu[-1]), 3, 6, 7, N=len(lengths))
+    for fn in (oracle.recurrent, lambda *a, **kw: oracle.chunkwise(*a, chunk=16, **kw)):
+        o, ST = fn(q, k, v, la, beta, S0, cu)
+        for s in range(len(lengths)):
+            a, b = cu[s], cu[s + 1]
+            o1, S1 = oracle.recurrent(q[a:b], k[a:b], v[a:b], la[a:b], beta[a:b], S0[s:s + 1])
+            np.testing.assert_allclose(o[a:b], o1, rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(ST[s], S1[0], rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("t0", [1, 37, 64, 100])
+def test_split_continuity(t0):
+    """prefill(x[0:T]) == prefill(x[t0:T], S0 = prefill(x[0:t0]).S_T) (chunk-boundary state)."""
+    T = 160
+    q, k, v, la, beta, S0 = rnd(14, T, 2, 8, 8)
+    o, ST = oracle.chunkwise(q, k, v, la, beta, S0, chunk=64)
+    oa, Sa = oracle.chunkwise(q[:t0], k[:t0], v[:t0], la[:t0], beta[:t0], S0, chunk=64)
+    ob, Sb = oracle.chunkwise(q[t0:], k[t0:], v[t0:], la[t0:], beta[t0:], Sa, chunk=64)
+    np.testing.assert_allclose(np.concatenate([oa, ob]), o, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(Sb, ST, rtol=1e-11, atol=1e-12)
+
+
+def test_strong_decay_chunkwise_finite():
+    """log alpha far below what exp(+-G) factorisations survive: chunkwise stays exact."""
+    q, k, v, la, beta, S0 = rnd(15, 130, 1, 8, 4)
+    la[:] = -np.abs(la) * 40.0
+    o_r, S_r = oracle.recurrent(q, k, v, la, beta, S0)
+    o_c, S_c = oracle.chunkwise(q, k, v, la, beta, S0, chunk=64)
+    assert np.isfinite(o_c).all()
+    np.testing.assert_allclose(o_c, o_r, rtol=1e-11, atol=1e-12)
+
+
+def test_state_norm_bounded():
+    """Invariant: with unit k, beta in [0,1] and alpha in (0,1] the transition is a
+    contraction (||A_t||_2 <= 1), so ||S_t||_F <= ||S0||_F + sum_t beta_t ||v_t||."""
+    q, k, v, la, beta, S0 = rnd(16, 200, 1, 6, 5, mu=-4.0)
+    o, ST = oracle.recurrent(q, k, v, la, beta, S0)
+    bound = np.linalg.norm(S0) + np.sum(beta[:, 0] * np.linalg.norm(v[:, 0], axis=-1))
+    assert np.linalg.norm(ST) <= bound
+    for t in range(20):
+        A = _A(la[t, 0], k[t, 0], beta[t, 0])
+        assert np.linalg.norm(A, 2) <= 1.0 + 1e-12
+
+
+def test_threads_do_not_change_results():
+    lengths = [40, 90]
+    cu = np.cumsum([0] + lengths)
+    q, k, v, la, beta, S0 = rnd(17, int(cu[-1]), 4, 8, 8, N=2)
+    o1, S1 = oracle.recurrent(q, k, v, la, beta, S0, cu, threads=1)
+    o2, S2 = oracle.recurrent(q, k, v, la, beta, S0, cu, threads=5)
+    assert np.array_equal(o1, o2) and np.array_equal(S1, S2)
+
+
+# ---------------------------------------------- planted-mistake check ----
+
+class _Orc:
+    """The oracle's Python wrapper bound to another build of its C source."""
+
+    def __init__(self, lib):
+        self.lib = lib
+
+    def _call(self, fn, *a, **kw):
+        saved = oracle._lib
+        oracle._lib = self.lib
+        try:
+            return fn(*a, **kw)
+        finally:
+            oracle._lib = saved
+
+    def recurrent(self, *a, **kw):
+        return self._call(oracle.recurrent, *a, **kw)
+
+    def chunkwise(self, *a, **kw):
+        return self._call(oracle.chunkwise, *a, **kw)
+
+    def decode_step(self, *a, **kw):
+        return self._call(oracle.decode_step, *a, **kw)
+
+
+_O_BLOCK = """    /* o_t = S_t^T q_t. */
+    for (int j = 0; j < dv; ++j) o[j] = 0.0;
+    for (int i = 0; i < dk; ++i) {
+        const double *row = S + (size_t)i * dv;
+        for (int j = 0; j < dv; ++j) o[j] += row[j] * qn[i];
+    }
+"""
+_DECAY_MARK = "    /* S~ = Diag(alpha_t) S_{t-1}"
+
+MUTANTS = {
+    "sign_of_correction": [("y[j] = beta * (v[j] - y[j]);", "y[j] = beta * (v[j] + y[j]);")],
+    "dropped_beta": [("y[j] = beta * (v[j] - y[j]);", "y[j] = (v[j] - y[j]);")],
+    "gate_not_exponentiated": [("double a = exp(la[i]);", "double a = 1.0 + la[i];")],
+    "gate_index_dropped": [("double a = exp(la[i]);", "double a = exp(la[0]);")],
+    "write_along_query": [("row[j] += kn[i] * y[j];", "row[j] += qn[i] * y[j];")],
+    "read_before_update": [(_O_BLOCK, ""), (_DECAY_MARK, _O_BLOCK + _DECAY_MARK)],
+    "no_l2norm": [("    if (!on) {\n        memcpy", "    if (1) {\n        memcpy")],
+    "chunk_solve_without_beta": [("for (int c = 0; c < wx; ++c) xr[c] *= b;", "")],
+    "chunk_exponent_sign": [("double e = exp(G[(size_t)r * dk + c] - G[(size_t)i * dk + c]);",
+                             "double e = exp(G[(size_t)i * dk + c] - G[(size_t)r * dk + c]);")],
+    "chunk_P_without_diagonal": [("P[(size_t)r * C + i] = (i <= r) ? p : 0.0;",
+                                  "P[(size_t)r * C + i] = (i < r) ? p : 0.0;")],
+    "chunk_state_not_decayed": [("double acc = exp(gl[c]) * S[(size_t)c * dv + j];",
+                                 "double acc = S[(size_t)c * dv + j];")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(name, tmp_path):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "kda_oracle.c")).read()
+    for old, new in MUTANTS[name]:
+        assert src.count(old) == 1, (name, old)
+        src = src.replace(old, new)
+    c = tmp_path / "mutant.c"
+    c.write_text(src)
+    so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-pthread", "-o",
+                           str(so), str(c), "-lm"])
+    orc = _Orc(oracle.load_library(str(so)))
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, "planted mistake %r passed every pin" % name
