@@ -1,0 +1,335 @@
+"""Benchmark of the KDA hot path on B200: prefill tokens/s and decode-step HBM GB/s.
+
+One timed "step" is one chunkwise prefill of the single-sequence workload
+(B=1, H=32, T=8192, d_k=d_v=128, bf16 q/k/v, fp32 gates and state; inputs
+~404 MB > L2, so no flush is needed). The decode step of the batched workload
+(256 sequences x 32 heads, 512 MiB fp32 state in place, > L2) is timed as a
+second region and reported in ``decode``. Everything runs in libkda's CUDA
+kernels; inputs are seeded synthetic tensors (``kda_inputs``).
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+Multi-GPU: launched with torchrun, one rank per GPU; every rank runs its own
+independent batch (weak scaling, no data-path collective).
+
+``--impl reference`` times the fp64 CPU oracle (the only other implementation
+of this path; it is test infrastructure) on the host cores, on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_inputs as KI  # noqa: E402
+
+METRIC = "KDA prefill tokens/s at H=32,d=128; decode-step HBM GB/s vs B200 peak"
+PREFILL = "prefill_8k"
+T8K, H, D = 8192, 32, 128
+DEC_N, DEC_STEPS_POOL = 256, 64
+# Algorithmic HBM bytes (inputs read once, outputs written once):
+#   prefill per token (all 32 heads): q,k,v bf16 3*32*128*2 + log_alpha 32*128*4 + beta 32*4
+#   + o 32*128*2 = 49,280 B; plus S0 read and S_T written (2 MiB each at H=32).
+PREFILL_BYTES_PER_TOKEN = 3 * H * D * 2 + H * D * 4 + H * 4 + H * D * 2
+PREFILL_STATE_BYTES = 2 * H * D * D * 4
+# decode per step: state read + write, q,k,v bf16, log_alpha fp32, beta fp32, o bf16
+DECODE_BYTES = DEC_N * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class Clocks:
+    """Sample SM clocks and throttle reasons while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, x in enumerate(r) if x == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() and args.impl == "kda" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------- oracle ----
+
+def oracle_sample(seconds_target=10.0, device="cpu"):
+    """Time the fp64 oracle on a bounded sample of the prefill workload (some heads,
+    all 8192 tokens). Returns (tokens/s at H=32, cores, description)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    heads = max(1, min(H, cores))
+    inp = KI.prefill_workload(PREFILL, "cpu", heads=heads)
+    f = lambda x: x.to(torch.float64).numpy()
+    args = [f(inp[n]) for n in ("q", "k", "v", "log_alpha", "beta")]
+    S0 = f(inp["S0"])
+    reps, elapsed = 0, 0.0
+    while reps == 0 or (elapsed < seconds_target and reps < 50):
+        t0 = time.perf_counter()
+        oracle.recurrent(*args, S0, threads=cores)
+        elapsed += time.perf_counter() - t0
+        reps += 1
+    tok = reps * T8K * heads / H  # tokens-equivalent of a 32-head token
+    desc = "%d of %d heads x %d tokens, %d repetitions, fp64 recurrence, %d threads" % (
+        heads, H, T8K, reps, cores)
+    return tok / elapsed, cores, desc
+
+
+def run_reference(args, world, rank):
+    """Each step is one bounded oracle sample (``cores`` heads x 8192 tokens)."""
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(seconds_target=0.0)
+    rates = []
+    for _ in range(args.steps):
+        r, cores, desc = oracle_sample(seconds_target=0.0)
+        rates.append(r)
+    v = len(rates) / sum(1.0 / r for r in rates)  # total tokens / total time
+    desc = "%d steps, each: %s" % (args.steps, desc)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * T8K / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "prefill_8k: B=1 H=32 T=8192 d_k=d_v=128 (oracle sample)"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- kda ----
+
+def run_kda(args, world, rank, local):
+    import gated_delta_rule_125_b200 as kda
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    hbm, peak_src = peaks()
+
+    # ---- prefill workload, resident in HBM
+    inp = KI.prefill_workload(PREFILL, dev, seed=rank)
+    q, k, v, la, beta, S0, cu = (inp[n] for n in ("q", "k", "v", "log_alpha", "beta", "S0", "cu_seqlens"))
+    o = torch.empty_like(v)
+    S_T = torch.empty_like(S0)
+    wsb = kda.kda_prefill_workspace_size(1, T8K, T8K, H, D, D, torch.bfloat16)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    launches_prefill = kda.kda_prefill_launches(1, T8K, T8K, H, D, D, torch.bfloat16, wsb)
+
+    def prefill():
+        kda.kda_prefill(q, k, v, la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
+
+    for _ in range(args.warmup):
+        prefill()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            prefill()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = max_over_ranks(ms, world, dev)
+    tokens_per_s = world * T8K / (ms_max * 1e-3)
+    bytes_pass = T8K * PREFILL_BYTES_PER_TOKEN + PREFILL_STATE_BYTES
+    achieved = bytes_pass / (ms * 1e-3) / 1e9
+
+    # ---- end to end through the C ABI: pinned host inputs -> device -> host
+    h_in = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v", "log_alpha", "beta", "S0")}
+    h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h_S = torch.empty(S_T.shape, dtype=S_T.dtype).pin_memory()
+    d_in = {n: torch.empty_like(inp[n]) for n in h_in}
+    h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+    d2h = h_o.numel() * h_o.element_size() + h_S.numel() * h_S.element_size()
+
+    def e2e_step():
+        for n in h_in:
+            d_in[n].copy_(h_in[n], non_blocking=True)
+        kda.kda_prefill(d_in["q"], d_in["k"], d_in["v"], d_in["log_alpha"], d_in["beta"],
+                        d_in["S0"], cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
+        h_o.copy_(o, non_blocking=True)
+        h_S.copy_(S_T, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    del d_in, h_in
+
+    # ---- decode: 256 x 32 heads, state 512 MiB in place
+    dec = KI.decode_workload(DEC_N, H, D, DEC_STEPS_POOL, torch.bfloat16, dev, seed=rank)
+    S = dec["S0"].clone()
+    od = torch.empty((DEC_N, H, D), dtype=torch.bfloat16, device=dev)
+
+    def decode(t):
+        i = t % DEC_STEPS_POOL
+        kda.kda_decode_step(dec["q"][i], dec["k"][i], dec["v"][i], dec["log_alpha"][i],
+                            dec["beta"][i], S, o=od)
+
+    dsteps = args.decode_steps
+    for t in range(max(3, args.warmup)):
+        decode(t)
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for t in range(dsteps):
+        decode(t)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    dec_us = ev0.elapsed_time(ev1) * 1e3 / dsteps
+    dec_us_max = max_over_ranks(dec_us, world, dev)
+    dec_gbs = DECODE_BYTES / (dec_us * 1e-6) / 1e9
+
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill_8k: B=1 H=32 T=8192 d_k=d_v=128 bf16 q/k/v, fp32 "
+                               "gates/state, chunk 64, S0~N(0,0.01^2), per rank",
+                   "global_batch": world, "seq_len": T8K,
+                   "l2": "inputs 404 MB > 126 MB L2 (no flush)",
+                   "parallelism": "independent batch per GPU" if world > 1 else "1 GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "kernel": "prefill pass (prep + scan kernels per wave)",
+                     "algorithmic_bytes": bytes_pass, "peak_source": peak_src},
+        "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps * launches_prefill + dsteps,
+        "clocks": clk.summary(),
+        "decode": {"value": DECODE_BYTES / (dec_us_max * 1e-6) / 1e9, "unit": "GB/s",
+                   "us_per_step": dec_us_max, "steps": dsteps,
+                   "workload": "decode_256: 256 seqs x 32 heads, d=128, bf16 q/k/v, fp32 state "
+                               "512 MiB in place (> L2)",
+                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
+                                "frac": dec_gbs / hbm, "traffic": None,
+                                "kernel": "decode_kernel<128,128,bf16>",
+                                "algorithmic_bytes": DECODE_BYTES, "peak_source": peak_src}},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, cores, desc = oracle_sample(seconds_target=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v_cpu, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_kda(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

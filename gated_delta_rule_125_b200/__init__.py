@@ -1,0 +1,194 @@
+"""Kimi Delta Attention (KDA) for NVIDIA B200 -- Python binding of ``libkda.so``.
+
+The functions here only marshal arguments into the C ABI declared in
+``include/kda.h`` (same names); every step of the computation runs in the
+library's CUDA kernels. PyTorch supplies device memory and the current CUDA
+stream. If the library is missing the calls raise -- there is no fallback.
+
+Build the library with ``python -m gated_delta_rule_125_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size", "kda_prefill_launches",
+           "kda_prefill_workspace_min", "kda_status_string", "kda_version", "KDAError",
+           "library_path", "load_library", "KDA_OK", "KDA_ERR_INVALID_ARG",
+           "KDA_ERR_UNSUPPORTED", "KDA_ERR_MISALIGNED", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA",
+           "KDA_ERR_TIMEOUT", "KDA_FLAG_NO_L2NORM", "KDA_FLAG_EXACT"]
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_MISALIGNED = 0, 1, 2, 3
+KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 4, 5, 6
+KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
+KDA_FLAG_NO_L2NORM, KDA_FLAG_EXACT = 0x1, 0x2
+
+EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
+                    "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
+                    "kda_decode_step")
+
+_lib = None
+
+
+def library_path() -> str:
+    return os.environ.get("KDA_LIBRARY",
+                          os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so"))
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s: %s" % (what, kda_status_string(status)))
+        self.status = status
+
+
+def load_library():
+    """Load ``libkda.so`` (raises ``OSError`` if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise OSError("libkda.so not found at %s; build it with "
+                      "`python -m gated_delta_rule_125_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    vp, fp, ip = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    i32, i64, u32, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_size_t
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_version.restype = i32
+    for f in (lib.kda_prefill_workspace_size, lib.kda_prefill_workspace_min):
+        f.argtypes = [i32, i64, i32, i32, i32, i32, ctypes.c_int, i32, u32]
+        f.restype = sz
+    lib.kda_prefill_launches.argtypes = [i32, i64, i32, i32, i32, i32, ctypes.c_int, i32, u32, sz]
+    lib.kda_prefill_launches.restype = i64
+    lib.kda_prefill.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32, i32,
+                                ctypes.c_int, i32, u32, vp, fp, vp, sz, vp]
+    lib.kda_prefill.restype = ctypes.c_int
+    lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
+                                    u32, vp, vp]
+    lib.kda_decode_step.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def kda_status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def kda_version() -> int:
+    return int(load_library().kda_version())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr() or None
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _flags(l2norm, exact):
+    return (0 if l2norm else KDA_FLAG_NO_L2NORM) | (KDA_FLAG_EXACT if exact else 0)
+
+
+def kda_prefill_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype,
+                               chunk=64, l2norm=True, exact=False) -> int:
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    return int(load_library().kda_prefill_workspace_size(num_seqs, total_tokens, max_seqlen, H,
+                                                        dk, dv, code, chunk,
+                                                        _flags(l2norm, exact)))
+
+
+def kda_prefill_workspace_min(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype,
+                              chunk=64, l2norm=True, exact=False) -> int:
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    return int(load_library().kda_prefill_workspace_min(num_seqs, total_tokens, max_seqlen, H,
+                                                       dk, dv, code, chunk,
+                                                       _flags(l2norm, exact)))
+
+
+def kda_prefill_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, workspace_bytes,
+                         chunk=64, l2norm=True, exact=False) -> int:
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_F32
+    return int(load_library().kda_prefill_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                                                  code, chunk, _flags(l2norm, exact),
+                                                  workspace_bytes))
+
+
+def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqlen=None,
+                chunk=64, l2norm=True, exact=False, o=None, S_T=None, workspace=None,
+                stream=None):
+    """Chunkwise KDA prefill (``kda_prefill`` in ``include/kda.h``).
+
+    q, k ``[T,H,dk]``, v ``[T,H,dv]`` (bf16 or fp32), log_alpha ``[T,H,dk]`` fp32,
+    beta ``[T,H]`` fp32, S0 ``[N,H,dk,dv]`` fp32 or None, cu_seqlens ``[N+1]`` int32
+    on the device or None. Returns ``(o [T,H,dv], S_T [N,H,dk,dv])``. Outputs and
+    the workspace are allocated with torch when not given. ``max_seqlen`` (host
+    int) avoids a device-to-host read of ``cu_seqlens``.
+    """
+    lib = load_library()
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        if cu_seqlens is None:
+            max_seqlen = T
+        else:
+            c = cu_seqlens.to("cpu", torch.int64)
+            max_seqlen = int((c[1:] - c[:-1]).max()) if N > 0 else 0
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=dev)
+    if S_T is None:
+        S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    code = _dtype_code(q)
+    flags = _flags(l2norm, exact)
+    if workspace is None:
+        nbytes = lib.kda_prefill_workspace_size(N, T, max_seqlen, H, dk, dv, code, chunk, flags)
+        if nbytes == 0:
+            nbytes = 256
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    rc = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                         _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, code, chunk, flags,
+                         _ptr(o), _ptr(S_T), _ptr(workspace), workspace.numel(),
+                         _stream(stream, dev))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_prefill")
+    return o, S_T
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, S, *, l2norm=True, o=None, stream=None):
+    """One KDA decode step (``kda_decode_step`` in ``include/kda.h``), S updated in place.
+
+    q, k ``[N,H,dk]``, v ``[N,H,dv]``, log_alpha ``[N,H,dk]`` fp32, beta ``[N,H]`` fp32,
+    S ``[N,H,dk,dv]`` fp32. Returns o ``[N,H,dv]``.
+    """
+    lib = load_library()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
+                             N, H, dk, dv, _dtype_code(q), _flags(l2norm, False), _ptr(o),
+                             _stream(stream, q.device))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_decode_step")
+    return o

@@ -1,0 +1,182 @@
+// kda_api.cu -- the extern "C" boundary of libkda.so: argument validation on
+// the host, workspace planning and dispatch to the kernels. Nothing here
+// allocates device memory or synchronises.
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+constexpr float kEps = 1e-6f;  // eps in q / max(||q||, eps)
+constexpr uint32_t kKnownFlags = KDA_FLAG_NO_L2NORM | KDA_FLAG_EXACT;
+
+bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool dims_supported(int32_t dk, int32_t dv) {
+    return (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
+}
+
+// Shape checks shared by the workspace queries and the prefill itself.
+kda_status check_prefill_shape(int32_t num_seqs, int64_t total_tokens, int32_t H, int32_t dk,
+                               int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags) {
+    if (num_seqs < 1 || num_seqs > 65535 || total_tokens < 0 || H < 1 || H > 65535 || dk < 1 ||
+        dv < 1 || chunk < 1)
+        return KDA_ERR_INVALID_ARG;
+    if (flags & ~kKnownFlags) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (!dims_supported(dk, dv) || chunk != kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    if (total_tokens > (int64_t)INT32_MAX * kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+// How the prefill splits into waves for a given workspace.
+struct Plan {
+    int64_t max_chunks;  // chunks of the longest sequence
+    size_t slot_bytes;   // per (chunk, sequence, head)
+    size_t per_wave_chunk;
+    size_t state_bytes;  // running-state carry between waves
+};
+
+Plan make_plan(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
+               int32_t dv) {
+    Plan p;
+    int64_t L = (max_seqlen > 0) ? std::min<int64_t>(max_seqlen, total_tokens) : total_tokens;
+    p.max_chunks = (L + kda::kChunk - 1) / kda::kChunk;
+    p.slot_bytes = kda::simt_slot_bytes(dk);
+    p.per_wave_chunk = (size_t)num_seqs * H * p.slot_bytes;
+    p.state_bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
+    return p;
+}
+
+size_t min_bytes(const Plan &p) {
+    if (p.max_chunks <= 1) return p.per_wave_chunk;
+    return p.state_bytes + p.per_wave_chunk;
+}
+
+constexpr size_t kRecommendedCap = size_t(512) << 20;
+
+// Chunks per wave for a workspace of `bytes` (>= min_bytes(p)).
+int64_t waves_chunks(const Plan &p, size_t bytes) {
+    const size_t single = (size_t)p.max_chunks * p.per_wave_chunk;
+    if (p.max_chunks <= 1 || single <= bytes) return std::max<int64_t>(p.max_chunks, 1);
+    return std::min<int64_t>((int64_t)((bytes - p.state_bytes) / p.per_wave_chunk), INT32_MAX);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: null pointer or invalid size";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: shape, chunk or dtype not implemented";
+        case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED: pointer not 16-byte aligned";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE: workspace missing or too small";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA error while enqueueing";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: bounded device wait gave up";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int32_t kda_version(void) { return 100; }
+
+size_t kda_prefill_workspace_min(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                                 int32_t H, int32_t dk, int32_t dv, kda_dtype dtype,
+                                 int32_t chunk, uint32_t flags) {
+    if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return 0;
+    return min_bytes(make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv));
+}
+
+size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                                  int32_t H, int32_t dk, int32_t dv, kda_dtype dtype,
+                                  int32_t chunk, uint32_t flags) {
+    if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return 0;
+    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv);
+    size_t single = (size_t)std::max<int64_t>(p.max_chunks, 1) * p.per_wave_chunk;
+    if (single <= kRecommendedCap) return single;
+    return std::max(min_bytes(p), p.state_bytes + kRecommendedCap / p.per_wave_chunk * p.per_wave_chunk);
+}
+
+int64_t kda_prefill_launches(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                             int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk,
+                             uint32_t flags, size_t workspace_bytes) {
+    if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return -1;
+    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv);
+    if (workspace_bytes < min_bytes(p)) return -1;
+    const int64_t nw = waves_chunks(p, workspace_bytes);
+    if (p.max_chunks == 0) return 1;
+    const int64_t waves = (p.max_chunks + nw - 1) / nw;
+    return 2 * waves;
+}
+
+kda_status kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, const float *S0, const int32_t *cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                       int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                       void *o, float *S_T, void *workspace, size_t workspace_bytes,
+                       kda_stream_t stream) {
+    kda_status rc = check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags);
+    if (rc != KDA_OK) return rc;
+    if (cu_seqlens == nullptr && num_seqs != 1) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    if (!workspace) return KDA_ERR_WORKSPACE;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+
+    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv);
+    if (workspace_bytes < min_bytes(p)) return KDA_ERR_WORKSPACE;
+
+    kda::PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0;
+    a.cu = cu_seqlens; a.total = total_tokens;
+    a.N = num_seqs; a.H = H; a.dk = dk; a.dv = dv;
+    a.l2norm = (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1;
+    a.eps = kEps;
+    a.o = o; a.S_T = S_T;
+    a.slot_bytes = p.slot_bytes;
+
+    const int64_t nw = waves_chunks(p, workspace_bytes);
+    if (nw >= p.max_chunks) {  // one wave: no state carry needed
+        a.state = nullptr;
+        a.slots = static_cast<char *>(workspace);
+    } else {
+        a.state = static_cast<float *>(workspace);
+        a.slots = static_cast<char *>(workspace) + p.state_bytes;
+    }
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    if (p.max_chunks == 0) {  // only empty sequences: S_T = S0
+        if (kda::simt_prefill_wave(a, 0, 0, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
+        return KDA_OK;
+    }
+    for (int64_t j0 = 0; j0 < p.max_chunks; j0 += nw) {
+        const int n = (int)std::min<int64_t>(nw, p.max_chunks - j0);
+        if (kda::simt_prefill_wave(a, (int)j0, n, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
+                           int32_t dv, kda_dtype dtype, uint32_t flags, void *o,
+                           kda_stream_t stream) {
+    if (N < 1 || H < 1 || dk < 1 || dv < 1 || (int64_t)N * H > INT32_MAX) return KDA_ERR_INVALID_ARG;
+    if (flags & ~kKnownFlags) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    cudaError_t e = kda::decode_step(q, k, v, log_alpha, beta, S, N, H, dk, dv,
+                                     dtype == KDA_DTYPE_BF16, (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1,
+                                     kEps, o, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

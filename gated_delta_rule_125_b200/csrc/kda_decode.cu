@@ -1,0 +1,160 @@
+// kda_decode.cu -- single-token KDA decode step, state updated in place.
+//
+// "[Kimi-2] Kimi Linear：用 KDA 重写长上下文注意力" §5 (recurrent decode:
+// S_(t-1) + current token -> S_t + output) applied to the §3 update
+//     S~ = Diag(alpha) S,  u = beta (v - S~^T k),  S_t = S~ + k u^T,
+//     o  = S_t^T q = S~^T q + (k . q) u
+// with q, k L2-normalised (§6.2).
+//
+// The step is HBM-bound: per (sequence, head) it reads and writes the fp32
+// d_k x d_v state (64 KiB each way at d = 128) and touches < 1.5 KiB of
+// token inputs. One CTA of 256 threads owns one (sequence, head) state:
+// thread (row group, column group) keeps R rows x 4 contiguous columns of S
+// in registers, so every warp access is a coalesced 16-byte-per-lane sweep
+// (read once, evict-first; written once, streaming). The two column sums
+// over d_k (S~^T k and S~^T q) are per-thread partial sums finished through
+// shared memory; nothing else touches HBM.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kDecodeThreads = 256;
+
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+              const float *__restrict__ log_alpha, const float *__restrict__ beta,
+              float *__restrict__ S, T *__restrict__ o, int l2norm, float eps) {
+    constexpr int CG = DV / 4;                // 16-byte column groups per state row
+    constexpr int RPP = kDecodeThreads / CG;  // state rows covered per pass
+    constexpr int R = DK / RPP;               // rows held per thread
+    static_assert(R * RPP == DK && CG * 4 == DV, "shape");
+
+    __shared__ float s_q[DK], s_k[DK], s_a[DK], s_v[DV], s_u[DV];
+    __shared__ float s_red[RPP][CG][8];
+    __shared__ float s_misc[2];  // beta, k.q
+
+    const int unit = blockIdx.x;  // sequence * H + head
+    const int tid = threadIdx.x;
+    const int cg = tid % CG, r0 = tid / CG;
+    float *Su = S + (size_t)unit * DK * DV;
+
+    // 1. Issue the whole state tile load first (R independent 16-byte loads).
+    float4 s[R];
+#pragma unroll
+    for (int m = 0; m < R; ++m)
+        s[m] = __ldcs(reinterpret_cast<const float4 *>(Su + (size_t)(r0 + m * RPP) * DV) + cg);
+
+    // 2. Token inputs while the state is in flight: warp 0 normalises q, k and
+    //    forms k.q; warp 1 exponentiates the gate; warp 2 stages v and beta.
+    const int warp = tid >> 5, lane = tid & 31;
+    if (warp == 0) {
+        float qq = 0.f, kk = 0.f, qk = 0.f;
+        float qv[DK / 32], kv[DK / 32];
+#pragma unroll
+        for (int m = 0; m < DK / 32; ++m) {
+            qv[m] = IO<T>::ld(q + (size_t)unit * DK + lane + 32 * m);
+            kv[m] = IO<T>::ld(k + (size_t)unit * DK + lane + 32 * m);
+            qq += qv[m] * qv[m];
+            kk += kv[m] * kv[m];
+            qk += qv[m] * kv[m];
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            qq += __shfl_xor_sync(0xffffffffu, qq, off);
+            kk += __shfl_xor_sync(0xffffffffu, kk, off);
+            qk += __shfl_xor_sync(0xffffffffu, qk, off);
+        }
+        float iq = 1.f, ik = 1.f;
+        if (l2norm) {
+            iq = 1.f / fmaxf(sqrtf(qq), eps);
+            ik = 1.f / fmaxf(sqrtf(kk), eps);
+        }
+#pragma unroll
+        for (int m = 0; m < DK / 32; ++m) {
+            s_q[lane + 32 * m] = qv[m] * iq;
+            s_k[lane + 32 * m] = kv[m] * ik;
+        }
+        if (lane == 0) s_misc[1] = qk * iq * ik;
+    } else if (warp == 1) {
+        for (int i = lane; i < DK; i += 32) s_a[i] = expf(log_alpha[(size_t)unit * DK + i]);
+    } else if (warp == 2) {
+        for (int j = lane; j < DV; j += 32) s_v[j] = IO<T>::ld(v + (size_t)unit * DV + j);
+        if (lane == 0) s_misc[0] = beta[unit];
+    }
+    __syncthreads();
+
+    // 3. Partial column sums of S~^T k and S~^T q over this thread's rows.
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f), z = y;
+#pragma unroll
+    for (int m = 0; m < R; ++m) {
+        const int i = r0 + m * RPP;
+        const float a = s_a[i], ka = a * s_k[i], qa = a * s_q[i];
+        y.x += ka * s[m].x; y.y += ka * s[m].y; y.z += ka * s[m].z; y.w += ka * s[m].w;
+        z.x += qa * s[m].x; z.y += qa * s[m].y; z.z += qa * s[m].z; z.w += qa * s[m].w;
+    }
+    *reinterpret_cast<float4 *>(&s_red[r0][cg][0]) = y;
+    *reinterpret_cast<float4 *>(&s_red[r0][cg][4]) = z;
+    __syncthreads();
+
+    // 4. Finish the sums per column: u = beta (v - S~^T k), o = S~^T q + (k.q) u.
+    if (tid < DV) {
+        const int j = tid, g = j >> 2, c = j & 3;
+        float yy = 0.f, zz = 0.f;
+#pragma unroll
+        for (int r = 0; r < RPP; ++r) {
+            yy += s_red[r][g][c];
+            zz += s_red[r][g][4 + c];
+        }
+        const float u = s_misc[0] * (s_v[j] - yy);
+        s_u[j] = u;
+        IO<T>::st(o + (size_t)unit * DV + j, zz + s_misc[1] * u);
+    }
+    __syncthreads();
+
+    // 5. S_t = Diag(alpha) S + k u^T, written back once.
+    const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[4 * cg]);
+#pragma unroll
+    for (int m = 0; m < R; ++m) {
+        const int i = r0 + m * RPP;
+        const float a = s_a[i], kk = s_k[i];
+        float4 w;
+        w.x = a * s[m].x + kk * u4.x;
+        w.y = a * s[m].y + kk * u4.y;
+        w.z = a * s[m].z + kk * u4.z;
+        w.w = a * s[m].w + kk * u4.w;
+        __stcs(reinterpret_cast<float4 *>(Su + (size_t)i * DV) + cg, w);
+    }
+}
+
+template <int DK, int DV, typename T>
+cudaError_t launch(const void *q, const void *k, const void *v, const float *la, const float *beta,
+                   float *S, int N, int H, int l2norm, float eps, void *o, cudaStream_t st) {
+    const unsigned units = (unsigned)N * (unsigned)H;
+    decode_kernel<DK, DV, T><<<units, kDecodeThreads, 0, st>>>(
+        (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, eps);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t dispatch(const void *q, const void *k, const void *v, const float *la,
+                     const float *beta, float *S, int N, int H, int dk, int dv, int l2norm,
+                     float eps, void *o, cudaStream_t st) {
+    if (dk == 128 && dv == 128) return launch<128, 128, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
+    if (dk == 128 && dv == 64) return launch<128, 64, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
+    if (dk == 64 && dv == 128) return launch<64, 128, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
+    if (dk == 64 && dv == 64) return launch<64, 64, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
+                        const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
+                        int l2norm, float eps, void *o, cudaStream_t st) {
+    if (bf16) return dispatch<__nv_bfloat16>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, eps, o, st);
+    return dispatch<float>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, eps, o, st);
+}
+
+}  // namespace kda

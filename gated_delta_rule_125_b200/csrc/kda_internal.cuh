@@ -1,0 +1,63 @@
+// kda_internal.cuh -- declarations shared by the libkda translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+constexpr int kChunk = 64;  // chunk length C of the chunkwise prefill
+
+// Element I/O for the two input/output dtypes; arithmetic is always fp32.
+template <typename T> struct IO;
+template <> struct IO<float> {
+    static __device__ __forceinline__ float ld(const float *p) { return *p; }
+    static __device__ __forceinline__ void st(float *p, float x) { *p = x; }
+};
+template <> struct IO<__nv_bfloat16> {
+    static __device__ __forceinline__ float ld(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void st(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+};
+
+// Bounds of sequence s in the packed token axis (cu == nullptr: one sequence).
+__device__ __forceinline__ void seq_bounds(const int32_t *cu, int s, int64_t total, int64_t &bos,
+                                           int64_t &eos) {
+    if (cu) {
+        bos = cu[s];
+        eos = cu[s + 1];
+    } else {
+        bos = 0;
+        eos = total;
+    }
+}
+
+// Parameters of one prefill wave: chunk indices [j0, j0 + nw) of every sequence.
+struct PrefillArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
+    const int32_t *cu;
+    int64_t total;
+    int N, H, dk, dv;
+    int l2norm;
+    float eps;
+    void *o;
+    float *S_T;
+    // workspace
+    float *state;      // running state between waves ([N][H][dk][dv]) or nullptr
+    char *slots;       // per-chunk slots of this wave
+    size_t slot_bytes; // bytes per (chunk, seq, head) slot
+};
+
+// fp32 CUDA-core path (exact arithmetic; any supported shape).
+size_t simt_slot_bytes(int dk);
+cudaError_t simt_prefill_wave(const PrefillArgs &a, int j0, int nw, bool bf16, cudaStream_t st);
+
+// decode step
+cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
+                        const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
+                        int l2norm, float eps, void *o, cudaStream_t st);
+
+}  // namespace kda

@@ -1,0 +1,140 @@
+/*
+ * kda.h -- C ABI of libkda.so, Kimi Delta Attention (KDA) on NVIDIA B200 (sm_100a).
+ *
+ * The operator is the per-head gated delta-rule recurrence
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T q_t,          alpha_t = exp(log_alpha_t) in (0,1]^{d_k},
+ *
+ * with q_t, k_t L2-normalised and an fp32 d_k x d_v state S per (sequence, head).
+ * Sources: "[Kimi-2] Kimi Linear：用 KDA 重写长上下文注意力" (xutianle.me) §3
+ * (boxed update, three-step form), §1 (readout o_t = S_t^T q_t), §5 (chunkwise
+ * prefill and recurrent decode), §6.2 (L2 norm of q, k; d_k = d_v = 128); and
+ * "Kimi Linear — 逐通道的遺忘" (docsaid.org), "KDA：把衰減拆到每個通道".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers are DEVICE pointers unless stated otherwise. The caller owns every
+ *   buffer; the library allocates no device memory and keeps no pointer after
+ *   a call returns.
+ * - Work is enqueued on `stream` and the call returns without synchronising.
+ *   KDA_ERR_CUDA reports a launch error seen at enqueue time; faults during
+ *   execution surface at the caller's next synchronisation.
+ * - Arguments are validated on the host before anything is enqueued; on any
+ *   error nothing is launched and the outputs are untouched.
+ * - Every pointer must be 16-byte aligned (KDA_ERR_MISALIGNED otherwise).
+ *   Tensors are dense row-major with the layouts given below.
+ * - Not checked (undefined behaviour if violated): cu_seqlens monotone with
+ *   cu_seqlens[0] = 0 and cu_seqlens[N] = total_tokens; log_alpha finite and
+ *   <= 0; beta in [0, 1]; outputs not overlapping inputs (except S_T == S0).
+ * - State layout (one layout for prefill S0/S_T and the decode state):
+ *   [N][H][d_k][d_v] fp32, row-major, d_v contiguous (row = key channel).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kda_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* null pointer, bad size or inconsistent sizes */
+    KDA_ERR_UNSUPPORTED = 2, /* valid but not implemented (d_k, d_v, chunk, dtype) */
+    KDA_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
+    KDA_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than the minimum */
+    KDA_ERR_CUDA = 5,        /* CUDA reported an error while enqueueing */
+    KDA_ERR_TIMEOUT = 6      /* reserved: a bounded device-side wait gave up */
+} kda_status;
+
+typedef enum {
+    KDA_DTYPE_F32 = 0, /* q, k, v and o in fp32 */
+    KDA_DTYPE_BF16 = 1 /* q, k, v and o in bf16 (log_alpha, beta, state stay fp32) */
+} kda_dtype;
+
+/* flags */
+#define KDA_FLAG_NO_L2NORM 0x1 /* q, k are used as given (caller already normalised) */
+#define KDA_FLAG_EXACT 0x2     /* fp32 CUDA-core arithmetic even for bf16 inputs */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(kda_status status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int32_t kda_version(void);
+
+/*
+ * Workspace bytes kda_prefill performs best with for this problem. Any
+ * workspace of at least kda_prefill_workspace_min() bytes also works (the
+ * prefill then runs in more waves). Returns 0 if the arguments are invalid.
+ * Arguments as for kda_prefill; max_seqlen <= 0 means "unknown"
+ * (total_tokens is assumed).
+ */
+size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                                  int32_t H, int32_t dk, int32_t dv, kda_dtype dtype,
+                                  int32_t chunk, uint32_t flags);
+size_t kda_prefill_workspace_min(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                                 int32_t H, int32_t dk, int32_t dv, kda_dtype dtype,
+                                 int32_t chunk, uint32_t flags);
+
+/*
+ * Number of kernel launches kda_prefill enqueues for this problem with a
+ * workspace of `workspace_bytes` (for sizing CUDA graphs and for accounting).
+ * Returns -1 if the arguments are invalid or the workspace is too small.
+ */
+int64_t kda_prefill_launches(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                             int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk,
+                             uint32_t flags, size_t workspace_bytes);
+
+/*
+ * Chunkwise-parallel prefill over a packed batch of variable-length sequences
+ * ("[Kimi-2] Kimi Linear" §5: parallel inside a chunk, recurrent between chunks).
+ *
+ *   q, k       [T][H][dk]  dtype         (T = total_tokens, all sequences packed)
+ *   v          [T][H][dv]  dtype
+ *   log_alpha  [T][H][dk]  fp32, <= 0    (per-key-channel log forget gate)
+ *   beta       [T][H]      fp32          (write strength)
+ *   S0         [N][H][dk][dv] fp32 entry states, or NULL for zeros
+ *   cu_seqlens [N+1] int32 (device) token offsets of the N sequences, or NULL
+ *              for one sequence of T tokens (then num_seqs must be 1)
+ *   max_seqlen host upper bound on the sequence lengths (<= 0: unknown)
+ *   chunk      chunk length; 64 is supported
+ *   o          [T][H][dv]  dtype, out: o_t = S_t^T q_t
+ *   S_T        [N][H][dk][dv] fp32 exit states, out, or NULL; may alias S0
+ *   workspace  device scratch of workspace_bytes (>= kda_prefill_workspace_min)
+ *
+ * Supported: dk, dv in {64, 128}; chunk = 64; dtype F32 or BF16. bf16 inputs
+ * run on the tensor cores unless KDA_FLAG_EXACT; fp32 inputs always use fp32
+ * CUDA-core arithmetic. Sequences of length 0 are allowed (S_T = S0).
+ */
+kda_status kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, const float *S0, const int32_t *cu_seqlens,
+                       int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                       int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                       void *o, float *S_T, void *workspace, size_t workspace_bytes,
+                       kda_stream_t stream);
+
+/*
+ * One decode step for N independent sequences, state updated in place
+ * ("[Kimi-2] Kimi Linear" §5: S_(t-1) + current token -> S_t + output).
+ *
+ *   q, k       [N][H][dk]  dtype          v [N][H][dv] dtype
+ *   log_alpha  [N][H][dk]  fp32           beta [N][H] fp32
+ *   S          [N][H][dk][dv] fp32, read and overwritten with S_t
+ *   o          [N][H][dv]  dtype, out
+ *
+ * Supported: dk, dv in {64, 128}; dtype F32 or BF16. Arithmetic is fp32.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                           const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
+                           int32_t dv, kda_dtype dtype, uint32_t flags, void *o,
+                           kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H_ */

@@ -1,0 +1,143 @@
+"""The C-ABI library: it loads, exports every entry point ``include/kda.h``
+declares, and rejects bad arguments on the host before anything is launched.
+
+Calls below pass fake (never dereferenced) addresses, so each must fail
+validation; they are skipped on a machine with a GPU, where a validation bug
+would otherwise launch a kernel on them.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import gated_delta_rule_125_b200 as kda
+from gated_delta_rule_125_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake-pointer calls only without a GPU")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return kda.load_library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kda.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"kda_prefill", "kda_decode_step", "kda_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(kda.EXPORTED_SYMBOLS)
+
+
+def test_status_strings_and_version(lib):
+    for code in range(7):
+        s = kda.kda_status_string(code)
+        assert s.startswith("KDA_")
+    assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
+    assert kda.kda_version() >= 100
+
+
+def test_workspace_queries(lib):
+    f = lib.kda_prefill_workspace_size
+    m = lib.kda_prefill_workspace_min
+    # valid: grows with heads, recommended >= minimum
+    a = f(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
+    b = m(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
+    assert a >= b > 0
+    assert f(1, 8192, 8192, 16, 128, 128, 1, 64, 0) < a
+    # single-chunk problems need no state carry
+    assert m(1, 64, 64, 4, 64, 64, 0, 64, 0) == m(1, 1, 1, 4, 64, 64, 0, 64, 0)
+    # invalid / unsupported -> 0
+    assert f(0, 10, 10, 1, 128, 128, 1, 64, 0) == 0
+    assert f(1, 10, 10, 1, 96, 128, 1, 64, 0) == 0
+    assert f(1, 10, 10, 1, 128, 128, 1, 32, 0) == 0
+    assert f(1, 10, 10, 1, 128, 128, 7, 64, 0) == 0
+    assert f(1, 10, 10, 1, 128, 128, 1, 64, 0x80) == 0
+
+
+A = 0x10000  # fake 16-byte-aligned address, never dereferenced
+
+
+def prefill(lib, **over):
+    args = dict(q=A, k=A, v=A, la=A, beta=A, S0=None, cu=None, N=1, T=128, L=128, H=2, dk=64,
+                dv=64, dt=1, chunk=64, flags=0, o=A, ST=A, ws=A, wsb=1 << 30, stream=None)
+    args.update(over)
+    a = args
+    return lib.kda_prefill(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S0"], a["cu"], a["N"],
+                           a["T"], a["L"], a["H"], a["dk"], a["dv"], a["dt"], a["chunk"],
+                           a["flags"], a["o"], a["ST"], a["ws"], a["wsb"], a["stream"])
+
+
+def decode(lib, **over):
+    a = dict(q=A, k=A, v=A, la=A, beta=A, S=A, N=4, H=2, dk=128, dv=128, dt=1, flags=0, o=A,
+             stream=None)
+    a.update(over)
+    return lib.kda_decode_step(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S"], a["N"],
+                               a["H"], a["dk"], a["dv"], a["dt"], a["flags"], a["o"], a["stream"])
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(beta=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(o=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=3), kda.KDA_ERR_INVALID_ARG),          # several sequences need cu_seqlens
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dv=256), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(dt=5), kda.KDA_ERR_INVALID_ARG),
+    (dict(flags=0x100), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=A + 8), kda.KDA_ERR_MISALIGNED),
+    (dict(la=A + 4), kda.KDA_ERR_MISALIGNED),
+    (dict(S0=A + 2), kda.KDA_ERR_MISALIGNED),
+    (dict(cu=A + 4, N=2), kda.KDA_ERR_MISALIGNED),
+    (dict(ST=A + 12), kda.KDA_ERR_MISALIGNED),
+    (dict(ws=None), kda.KDA_ERR_WORKSPACE),
+    (dict(wsb=1024), kda.KDA_ERR_WORKSPACE),
+])
+def test_prefill_rejects(lib, over, code):
+    assert prefill(lib, **over) == code
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(S=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(H=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dt=2), kda.KDA_ERR_INVALID_ARG),
+    (dict(flags=0x4), kda.KDA_ERR_INVALID_ARG),
+    (dict(v=A + 2), kda.KDA_ERR_MISALIGNED),
+    (dict(S=A + 8), kda.KDA_ERR_MISALIGNED),
+    (dict(o=A + 4), kda.KDA_ERR_MISALIGNED),
+])
+def test_decode_rejects(lib, over, code):
+    assert decode(lib, **over) == code
+
+
+def test_binding_refuses_host_tensors(lib):
+    q = torch.zeros(4, 2, 64)
+    with pytest.raises(ValueError):
+        kda.kda_decode_step(q, q, q, q, torch.zeros(4, 2), torch.zeros(4, 2, 64, 64))
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(kda, "_lib", None)
+    monkeypatch.setenv("KDA_LIBRARY", "/nonexistent/libkda.so")
+    with pytest.raises(OSError):
+        kda.load_library()

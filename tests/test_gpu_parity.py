@@ -1,0 +1,281 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (bf16 q/k/v: max|o - o_ref| <= 2e-2 and relative Frobenius error of
+the final state <= 1e-2; fp32: both <= 1e-4) are the gate of the workloads.
+The oracle always runs on the exact bits the GPU consumed, copied to the host.
+Full-size workloads are checked on sampled (sequence, head) units over their
+whole length -- units are independent, so a sample is an exact check of its
+members.
+"""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_125_b200 as kda
+import kda_inputs as KI
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: (2e-2, 1e-2), torch.float32: (1e-4, 1e-4)}
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    kda.load_library()
+
+
+def host(x):
+    return x.detach().to("cpu", torch.float64).numpy()
+
+
+def rel_fro(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def ref_prefill(inp, heads=None, seqs=None, S0=True):
+    """Oracle on the given (sub)set of heads/sequences. Returns o_ref, S_ref and the index."""
+    cu = inp["cu_seqlens"].cpu().numpy().astype(np.int64)
+    N = len(cu) - 1
+    seqs = list(range(N)) if seqs is None else list(seqs)
+    H = inp["q"].shape[1]
+    heads = list(range(H)) if heads is None else list(heads)
+    tok = np.concatenate([np.arange(cu[s], cu[s + 1]) for s in seqs]) if seqs else np.zeros(0, int)
+    sub_cu = np.cumsum([0] + [cu[s + 1] - cu[s] for s in seqs])
+    hi = torch.tensor(heads)
+    ti = torch.from_numpy(tok)
+    pick = lambda x: host(x.index_select(0, ti.to(x.device)).index_select(1, hi.to(x.device)))
+    S0v = None
+    if S0 and inp.get("S0") is not None:
+        S0v = host(inp["S0"][torch.tensor(seqs).to(DEV)][:, hi.to(DEV)])
+    o_ref, S_ref = oracle.recurrent(pick(inp["q"]), pick(inp["k"]), pick(inp["v"]),
+                                    pick(inp["log_alpha"]), pick(inp["beta"]), S0v, sub_cu)
+    return o_ref, S_ref, ti, hi, seqs
+
+
+def check(o, S_T, inp, dtype, heads=None, seqs=None, label=""):
+    o_ref, S_ref, ti, hi, seqs = ref_prefill(inp, heads, seqs)
+    og = host(o.index_select(0, ti.to(o.device)).index_select(1, hi.to(o.device)))
+    Sg = host(S_T[torch.tensor(seqs).to(DEV)][:, hi.to(DEV)])
+    atol, stol = TOL[dtype]
+    err = float(np.abs(og - o_ref).max()) if og.size else 0.0
+    sf = rel_fro(Sg, S_ref)
+    assert np.isfinite(og).all() and np.isfinite(Sg).all(), label
+    assert err <= atol, "%s: max|o-o_ref| = %.3e > %.1e" % (label, err, atol)
+    assert sf <= stol, "%s: relFro(S_T) = %.3e > %.1e" % (label, sf, stol)
+    return err, sf
+
+
+def make(lengths, H, dk, dv, dtype, seed=0, mu=-3.0, s0=0.1):
+    T = sum(lengths)
+    q, k, v, la, beta = KI.token_inputs(T, H, dk, dv, dtype, DEV, seed, mu)
+    S0 = KI.initial_state(len(lengths), H, dk, dv, s0, DEV, seed)
+    return dict(q=q, k=k, v=v, log_alpha=la, beta=beta, S0=S0,
+                cu_seqlens=KI.cu_from_lengths(lengths, DEV), lengths=list(lengths))
+
+
+def run(inp, **kw):
+    o = torch.full(inp["v"].shape, float("nan"), dtype=inp["v"].dtype, device=DEV)
+    N = len(inp["lengths"])
+    S_T = torch.full((N,) + tuple(inp["S0"].shape[1:]), float("nan"), device=DEV)
+    kda.kda_prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp.get("S0"),
+                    inp["cu_seqlens"], max_seqlen=max(inp["lengths"] + [0]), o=o, S_T=S_T, **kw)
+    torch.cuda.synchronize()
+    return o, S_T
+
+
+# ------------------------------------------------------------ prefill ----
+
+def test_tiny_f32_workload():
+    """B=1, H=2, T=256, d=64, fp32 throughout, S0 = 0 (tolerance 1e-4)."""
+    inp = KI.prefill_workload("tiny_f32", DEV)
+    o, S_T = run(inp)
+    check(o, S_T, inp, torch.float32, label="tiny_f32")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (64, 128), (128, 64)])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 130])
+def test_small_shapes(T, dk, dv, dtype):
+    inp = make([T], 3, dk, dv, dtype, seed=T + dk + dv)
+    o, S_T = run(inp)
+    check(o, S_T, inp, dtype, label="T=%d dk=%d dv=%d %s" % (T, dk, dv, dtype))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_varlen_with_empty_sequences(dtype):
+    lengths = [0, 5, 64, 1, 200, 0, 129]
+    inp = make(lengths, 4, 128, 128, dtype, seed=3)
+    o, S_T = run(inp)
+    check(o, S_T, inp, dtype, label="varlen")
+    # empty sequences return their entry state
+    assert torch.equal(S_T[0], inp["S0"][0]) and torch.equal(S_T[5], inp["S0"][5])
+
+
+def test_varlen_equals_separate_calls():
+    lengths = [70, 1, 191, 64]
+    inp = make(lengths, 2, 128, 128, torch.bfloat16, seed=4)
+    o, S_T = run(inp)
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    for s, n in enumerate(lengths):
+        a, b = cu[s], cu[s + 1]
+        one = dict(q=inp["q"][a:b], k=inp["k"][a:b], v=inp["v"][a:b],
+                   log_alpha=inp["log_alpha"][a:b], beta=inp["beta"][a:b],
+                   S0=inp["S0"][s:s + 1].contiguous(), cu_seqlens=KI.cu_from_lengths([n], DEV),
+                   lengths=[n])
+        o1, S1 = run(one)
+        assert torch.equal(o1, o[a:b]) and torch.equal(S1[0], S_T[s])
+
+
+@pytest.mark.parametrize("t0", [1, 37, 64, 100])
+def test_split_prefill_continuity(t0):
+    """prefill(x[0:T]) == prefill(x[t0:T], S0 = prefill(x[0:t0]).S_T): state across chunk edges."""
+    T = 200
+    inp = make([T], 2, 128, 128, torch.float32, seed=5)
+    o, S_T = run(inp)
+    sl = lambda a, b, S0: dict(q=inp["q"][a:b], k=inp["k"][a:b], v=inp["v"][a:b],
+                               log_alpha=inp["log_alpha"][a:b], beta=inp["beta"][a:b], S0=S0,
+                               cu_seqlens=KI.cu_from_lengths([b - a], DEV), lengths=[b - a])
+    oa, Sa = run(sl(0, t0, inp["S0"]))
+    ob, Sb = run(sl(t0, T, Sa))
+    torch.testing.assert_close(torch.cat([oa, ob]), o, atol=2e-5, rtol=0)
+    torch.testing.assert_close(Sb, S_T, atol=2e-5, rtol=0)
+
+
+def test_multi_wave_matches_single_wave():
+    lengths = [300, 40, 513]
+    inp = make(lengths, 3, 64, 64, torch.bfloat16, seed=6)
+    o1, S1 = run(inp)
+    L = max(lengths)
+    mn = kda.kda_prefill_workspace_min(3, sum(lengths), L, 3, 64, 64, torch.bfloat16)
+    ws = torch.empty(mn + 4096, dtype=torch.uint8, device=DEV)
+    o2, S2 = run(inp, workspace=ws)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    check(o2, S2, inp, torch.bfloat16, label="multi-wave")
+
+
+def test_strong_decay():
+    inp = make([150], 2, 128, 128, torch.float32, seed=7)
+    inp["log_alpha"] = inp["log_alpha"] * 400.0  # ~ -20 per token: exp(+G) would overflow
+    o, S_T = run(inp)
+    check(o, S_T, inp, torch.float32, label="strong decay")
+
+
+def test_no_l2norm_flag():
+    inp = make([100], 2, 64, 64, torch.float32, seed=8)
+    o1, S1 = run(inp)
+    o2, S2 = run(inp, l2norm=False)  # inputs are already unit-norm
+    torch.testing.assert_close(o2, o1, atol=1e-5, rtol=0)
+    torch.testing.assert_close(S2, S1, atol=1e-5, rtol=0)
+
+
+def test_deterministic():
+    inp = make([257, 31], 4, 128, 128, torch.bfloat16, seed=9)
+    o1, S1 = run(inp)
+    o2, S2 = run(inp)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_state_aliasing_in_place():
+    """S_T may alias S0."""
+    inp = make([150, 20], 2, 128, 128, torch.float32, seed=10)
+    o_ref, S_ref = run(inp)
+    S = inp["S0"].clone()
+    kda.kda_prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], S,
+                    inp["cu_seqlens"], max_seqlen=150, S_T=S)
+    torch.cuda.synchronize()
+    assert torch.equal(S, S_ref)
+
+
+# ------------------------------------------------------------- decode ----
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (64, 128), (128, 64)])
+def test_decode_steps(dk, dv, dtype):
+    N, H, steps = 5, 3, 4
+    w = KI.decode_workload(N, H, dk, steps, dtype, DEV, seed=11, s0_std=0.1) if dk == dv else None
+    if w is None:
+        q, k, v, la, beta = KI.token_inputs(steps * N, H, dk, dv, dtype, DEV, 11, -3.0)
+        w = dict(q=q.view(steps, N, H, dk), k=k.view(steps, N, H, dk), v=v.view(steps, N, H, dv),
+                 log_alpha=la.view(steps, N, H, dk), beta=beta.view(steps, N, H),
+                 S0=KI.initial_state(N, H, dk, dv, 0.1, DEV, 11))
+    S = w["S0"].clone()
+    S_ref = host(S)
+    atol, stol = TOL[dtype]
+    for t in range(steps):
+        o = kda.kda_decode_step(w["q"][t], w["k"][t], w["v"][t], w["log_alpha"][t], w["beta"][t], S)
+        torch.cuda.synchronize()
+        o_ref, S_ref = oracle.decode_step(host(w["q"][t]), host(w["k"][t]), host(w["v"][t]),
+                                          host(w["log_alpha"][t]), host(w["beta"][t]), S_ref)
+        assert float(np.abs(host(o) - o_ref).max()) <= atol
+        assert rel_fro(host(S), S_ref) <= stol
+
+
+def test_prefill_then_decode_equals_longer_prefill():
+    """Prefill of T-3 tokens then 3 decode steps == prefill of all T (one state layout)."""
+    T, H = 131, 4
+    inp = make([T], H, 128, 128, torch.float32, seed=12)
+    o_all, S_all = run(inp)
+    m = T - 3
+    part = dict(q=inp["q"][:m], k=inp["k"][:m], v=inp["v"][:m], log_alpha=inp["log_alpha"][:m],
+                beta=inp["beta"][:m], S0=inp["S0"], cu_seqlens=KI.cu_from_lengths([m], DEV),
+                lengths=[m])
+    _, S = run(part)
+    for t in range(m, T):
+        o = kda.kda_decode_step(inp["q"][t:t + 1].contiguous(), inp["k"][t:t + 1].contiguous(),
+                                inp["v"][t:t + 1].contiguous(),
+                                inp["log_alpha"][t:t + 1].contiguous(),
+                                inp["beta"][t:t + 1].contiguous(), S)
+        torch.testing.assert_close(o[0], o_all[t], atol=2e-5, rtol=0)
+    torch.testing.assert_close(S, S_all, atol=2e-5, rtol=0)
+
+
+# ------------------------------------------------ full-size workloads ----
+
+def test_workload_prefill_8k():
+    """B=1, H=32, T=8192, d=128, bf16; every output of heads {0, 17, 31} vs the oracle."""
+    inp = KI.prefill_workload("prefill_8k", DEV)
+    o, S_T = run(inp)
+    check(o, S_T, inp, torch.bfloat16, heads=[0, 17, 31], label="prefill_8k")
+
+
+def test_workload_varlen_16():
+    """16 packed sequences, lengths U[512, 8192]; sampled (sequence, head) units."""
+    inp = KI.prefill_workload("varlen_16", DEV)
+    o, S_T = run(inp)
+    longest = int(np.argmax(inp["lengths"]))
+    check(o, S_T, inp, torch.bfloat16, heads=[3, 30], seqs=[0, longest, 15], label="varlen_16")
+
+
+def test_workload_prefill_1m():
+    """B=1, H=32, T=1,048,576 (long memory); heads {0, 21} over all 1M tokens."""
+    inp = KI.prefill_workload("prefill_1m", DEV)
+    o, S_T = run(inp)
+    check(o, S_T, inp, torch.bfloat16, heads=[0, 21], label="prefill_1m")
+
+
+def test_workload_decode_256():
+    """256 sequences x 32 heads, 1000 in-place steps; sequences {0, 101, 255} vs the oracle."""
+    N, H, d, steps = 256, 32, 128, 1000
+    w = KI.decode_workload(N, H, d, steps, torch.bfloat16, DEV, seed=0, s0_std=0.01)
+    S = w["S0"].clone()
+    seqs = [0, 101, 255]
+    S_ref = host(S[seqs])
+    o_all = torch.empty((steps, N, H, d), dtype=torch.bfloat16, device=DEV)
+    for t in range(steps):
+        kda.kda_decode_step(w["q"][t], w["k"][t], w["v"][t], w["log_alpha"][t], w["beta"][t], S,
+                            o=o_all[t])
+    torch.cuda.synchronize()
+    worst = 0.0
+    for t in range(steps):
+        o_ref, S_ref = oracle.decode_step(host(w["q"][t][seqs]), host(w["k"][t][seqs]),
+                                          host(w["v"][t][seqs]), host(w["log_alpha"][t][seqs]),
+                                          host(w["beta"][t][seqs]), S_ref)
+        worst = max(worst, float(np.abs(host(o_all[t][seqs]) - o_ref).max()))
+    assert worst <= 2e-2
+    assert rel_fro(host(S[seqs]), S_ref) <= 1e-2
