@@ -123,9 +123,10 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
     if (cu_seqlens == nullptr && num_seqs != 1) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
     if (!workspace) return KDA_ERR_WORKSPACE;
-    const void *ptrs[] = {q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace};
+    const void *ptrs[] = {q, k, v, log_alpha, S0, cu_seqlens, o, S_T, workspace};
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(beta) & 3u) return KDA_ERR_MISALIGNED;
 
     Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv);
     if (workspace_bytes < min_bytes(p)) return KDA_ERR_WORKSPACE;
@@ -170,9 +171,10 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, log_alpha, beta, S, o};
+    const void *ptrs[] = {q, k, v, log_alpha, S, o};
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(beta) & 3u) return KDA_ERR_MISALIGNED;
     cudaError_t e = kda::decode_step(q, k, v, log_alpha, beta, S, N, H, dk, dv,
                                      dtype == KDA_DTYPE_BF16, (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1,
                                      kEps, o, reinterpret_cast<cudaStream_t>(stream));

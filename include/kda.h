@@ -22,7 +22,8 @@
  *   execution surface at the caller's next synchronisation.
  * - Arguments are validated on the host before anything is enqueued; on any
  *   error nothing is launched and the outputs are untouched.
- * - Every pointer must be 16-byte aligned (KDA_ERR_MISALIGNED otherwise).
+ * - Every pointer must be 16-byte aligned, except beta (4-byte aligned);
+ *   KDA_ERR_MISALIGNED otherwise.
  *   Tensors are dense row-major with the layouts given below.
  * - Not checked (undefined behaviour if violated): cu_seqlens monotone with
  *   cu_seqlens[0] = 0 and cu_seqlens[N] = total_tokens; log_alpha finite and

@@ -103,6 +103,7 @@ def decode(lib, **over):
     (dict(flags=0x100), kda.KDA_ERR_INVALID_ARG),
     (dict(q=A + 8), kda.KDA_ERR_MISALIGNED),
     (dict(la=A + 4), kda.KDA_ERR_MISALIGNED),
+    (dict(beta=A + 2), kda.KDA_ERR_MISALIGNED),
     (dict(S0=A + 2), kda.KDA_ERR_MISALIGNED),
     (dict(cu=A + 4, N=2), kda.KDA_ERR_MISALIGNED),
     (dict(ST=A + 12), kda.KDA_ERR_MISALIGNED),
@@ -125,6 +126,7 @@ def test_prefill_rejects(lib, over, code):
     (dict(v=A + 2), kda.KDA_ERR_MISALIGNED),
     (dict(S=A + 8), kda.KDA_ERR_MISALIGNED),
     (dict(o=A + 4), kda.KDA_ERR_MISALIGNED),
+    (dict(beta=A + 1), kda.KDA_ERR_MISALIGNED),
 ])
 def test_decode_rejects(lib, over, code):
     assert decode(lib, **over) == code

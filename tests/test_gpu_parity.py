@@ -124,9 +124,10 @@ def test_varlen_equals_separate_calls():
         cu.append(cu[-1] + n)
     for s, n in enumerate(lengths):
         a, b = cu[s], cu[s + 1]
-        one = dict(q=inp["q"][a:b], k=inp["k"][a:b], v=inp["v"][a:b],
-                   log_alpha=inp["log_alpha"][a:b], beta=inp["beta"][a:b],
-                   S0=inp["S0"][s:s + 1].contiguous(), cu_seqlens=KI.cu_from_lengths([n], DEV),
+        # fresh copies: every pointer handed to the library must be 16-byte aligned
+        one = dict(q=inp["q"][a:b].clone(), k=inp["k"][a:b].clone(), v=inp["v"][a:b].clone(),
+                   log_alpha=inp["log_alpha"][a:b].clone(), beta=inp["beta"][a:b].clone(),
+                   S0=inp["S0"][s:s + 1].clone(), cu_seqlens=KI.cu_from_lengths([n], DEV),
                    lengths=[n])
         o1, S1 = run(one)
         assert torch.equal(o1, o[a:b]) and torch.equal(S1[0], S_T[s])
@@ -138,8 +139,9 @@ def test_split_prefill_continuity(t0):
     T = 200
     inp = make([T], 2, 128, 128, torch.float32, seed=5)
     o, S_T = run(inp)
-    sl = lambda a, b, S0: dict(q=inp["q"][a:b], k=inp["k"][a:b], v=inp["v"][a:b],
-                               log_alpha=inp["log_alpha"][a:b], beta=inp["beta"][a:b], S0=S0,
+    sl = lambda a, b, S0: dict(q=inp["q"][a:b].clone(), k=inp["k"][a:b].clone(),
+                               v=inp["v"][a:b].clone(), log_alpha=inp["log_alpha"][a:b].clone(),
+                               beta=inp["beta"][a:b].clone(), S0=S0,
                                cu_seqlens=KI.cu_from_lengths([b - a], DEV), lengths=[b - a])
     oa, Sa = run(sl(0, t0, inp["S0"]))
     ob, Sb = run(sl(t0, T, Sa))
@@ -224,13 +226,12 @@ def test_prefill_then_decode_equals_longer_prefill():
     m = T - 3
     part = dict(q=inp["q"][:m], k=inp["k"][:m], v=inp["v"][:m], log_alpha=inp["log_alpha"][:m],
                 beta=inp["beta"][:m], S0=inp["S0"], cu_seqlens=KI.cu_from_lengths([m], DEV),
-                lengths=[m])
+                lengths=[m])  # prefixes keep the base pointers aligned
     _, S = run(part)
     for t in range(m, T):
-        o = kda.kda_decode_step(inp["q"][t:t + 1].contiguous(), inp["k"][t:t + 1].contiguous(),
-                                inp["v"][t:t + 1].contiguous(),
-                                inp["log_alpha"][t:t + 1].contiguous(),
-                                inp["beta"][t:t + 1].contiguous(), S)
+        o = kda.kda_decode_step(inp["q"][t:t + 1].clone(), inp["k"][t:t + 1].clone(),
+                                inp["v"][t:t + 1].clone(), inp["log_alpha"][t:t + 1].clone(),
+                                inp["beta"][t:t + 1].clone(), S)
         torch.testing.assert_close(o[0], o_all[t], atol=2e-5, rtol=0)
     torch.testing.assert_close(S, S_all, atol=2e-5, rtol=0)
 
