@@ -15,6 +15,7 @@ import os
 import torch
 
 __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size", "kda_prefill_launches",
+           "kda_device_error",
            "kda_prefill_workspace_min", "kda_status_string", "kda_version", "KDAError",
            "library_path", "load_library", "KDA_OK", "KDA_ERR_INVALID_ARG",
            "KDA_ERR_UNSUPPORTED", "KDA_ERR_MISALIGNED", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA",
@@ -27,7 +28,7 @@ KDA_FLAG_NO_L2NORM, KDA_FLAG_EXACT = 0x1, 0x2
 
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
                     "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
-                    "kda_decode_step")
+                    "kda_decode_step", "kda_device_error")
 
 _lib = None
 
@@ -69,6 +70,8 @@ def load_library():
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
                                     u32, vp, vp]
     lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_device_error.argtypes = [ctypes.POINTER(i32), i32]
+    lib.kda_device_error.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -79,6 +82,13 @@ def kda_status_string(status: int) -> str:
 
 def kda_version() -> int:
     return int(load_library().kda_version())
+
+
+def kda_device_error(reset: bool = True) -> int:
+    """Device error word of the current device (0: no bounded wait ran out). Synchronous."""
+    code = ctypes.c_int32(0)
+    load_library().kda_device_error(ctypes.byref(code), int(bool(reset)))
+    return int(code.value)
 
 
 def _dtype_code(t: torch.Tensor) -> int:

@@ -31,40 +31,85 @@ kda_status check_prefill_shape(int32_t num_seqs, int64_t total_tokens, int32_t H
     return KDA_OK;
 }
 
-// How the prefill splits into waves for a given workspace.
+// How the prefill splits into waves for a given workspace. Workspace layout:
+//   [fallback queue: 1 + slots-per-wave ints, 1 KiB aligned]  (tensor-core path)
+//   [state carry: N*H*dk*dv fp32]                             (several waves only)
+//   [slots of one wave]
 struct Plan {
+    bool tc;             // tensor-core path
     int64_t max_chunks;  // chunks of the longest sequence
     size_t slot_bytes;   // per (chunk, sequence, head)
-    size_t per_wave_chunk;
+    size_t units;        // N * H
     size_t state_bytes;  // running-state carry between waves
 };
 
+bool use_tc(kda_dtype dtype, int32_t dk, int32_t dv, uint32_t flags) {
+    return dtype == KDA_DTYPE_BF16 && dk == 128 && dv == 128 && !(flags & KDA_FLAG_EXACT);
+}
+
 Plan make_plan(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
-               int32_t dv) {
+               int32_t dv, kda_dtype dtype, uint32_t flags) {
     Plan p;
+    p.tc = use_tc(dtype, dk, dv, flags);
     int64_t L = (max_seqlen > 0) ? std::min<int64_t>(max_seqlen, total_tokens) : total_tokens;
     p.max_chunks = (L + kda::kChunk - 1) / kda::kChunk;
-    p.slot_bytes = kda::simt_slot_bytes(dk);
-    p.per_wave_chunk = (size_t)num_seqs * H * p.slot_bytes;
+    p.slot_bytes = p.tc ? kda::tc_slot_bytes() : kda::simt_slot_bytes(dk);
+    p.units = (size_t)num_seqs * H;
     p.state_bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
     return p;
 }
 
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t queue_bytes(const Plan &p, int64_t nw) {
+    return p.tc ? round_up(sizeof(int) * (1 + (size_t)nw * p.units), 1024) : 0;
+}
+
+// Bytes needed for waves of nw chunks (several waves: with the state carry).
+size_t bytes_for(const Plan &p, int64_t nw, bool multi) {
+    return queue_bytes(p, nw) + (multi ? round_up(p.state_bytes, 1024) : 0) + (size_t)nw * p.units * p.slot_bytes;
+}
+
 size_t min_bytes(const Plan &p) {
-    if (p.max_chunks <= 1) return p.per_wave_chunk;
-    return p.state_bytes + p.per_wave_chunk;
+    if (p.max_chunks <= 1) return bytes_for(p, 1, false);
+    return bytes_for(p, 1, true);
 }
 
 constexpr size_t kRecommendedCap = size_t(512) << 20;
 
 // Chunks per wave for a workspace of `bytes` (>= min_bytes(p)).
 int64_t waves_chunks(const Plan &p, size_t bytes) {
-    const size_t single = (size_t)p.max_chunks * p.per_wave_chunk;
-    if (p.max_chunks <= 1 || single <= bytes) return std::max<int64_t>(p.max_chunks, 1);
-    return std::min<int64_t>((int64_t)((bytes - p.state_bytes) / p.per_wave_chunk), INT32_MAX);
+    const int64_t all = std::max<int64_t>(p.max_chunks, 1);
+    if (p.max_chunks <= 1 || bytes_for(p, all, false) <= bytes) return all;
+    int64_t lo = 1, hi = all - 1;  // largest nw with bytes_for(nw, multi) <= bytes
+    while (lo < hi) {
+        const int64_t mid = (lo + hi + 1) / 2;
+        if (bytes_for(p, mid, true) <= bytes) lo = mid;
+        else hi = mid - 1;
+    }
+    return std::min<int64_t>(lo, INT32_MAX);
 }
 
 }  // namespace
+
+namespace kda {
+
+__device__ int g_device_error;  // set by kernels whose bounded waits ran out
+
+int *device_error_word() {
+    // One word per device; its address is resolved for the current device.
+    static int *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<int *>(p);
+    }
+    return addr[dev];
+}
+
+}  // namespace kda
 
 extern "C" {
 
@@ -87,29 +132,31 @@ size_t kda_prefill_workspace_min(int32_t num_seqs, int64_t total_tokens, int32_t
                                  int32_t H, int32_t dk, int32_t dv, kda_dtype dtype,
                                  int32_t chunk, uint32_t flags) {
     if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return 0;
-    return min_bytes(make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv));
+    return min_bytes(make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags));
 }
 
 size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
                                   int32_t H, int32_t dk, int32_t dv, kda_dtype dtype,
                                   int32_t chunk, uint32_t flags) {
     if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return 0;
-    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv);
-    size_t single = (size_t)std::max<int64_t>(p.max_chunks, 1) * p.per_wave_chunk;
+    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
+    const int64_t all = std::max<int64_t>(p.max_chunks, 1);
+    const size_t single = bytes_for(p, all, false);
     if (single <= kRecommendedCap) return single;
-    return std::max(min_bytes(p), p.state_bytes + kRecommendedCap / p.per_wave_chunk * p.per_wave_chunk);
+    const int64_t nw = std::max<int64_t>(1, (int64_t)(kRecommendedCap / (p.units * p.slot_bytes)));
+    return std::max(min_bytes(p), bytes_for(p, std::min(nw, all), true));
 }
 
 int64_t kda_prefill_launches(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
                              int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk,
                              uint32_t flags, size_t workspace_bytes) {
     if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return -1;
-    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv);
+    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
     if (workspace_bytes < min_bytes(p)) return -1;
     const int64_t nw = waves_chunks(p, workspace_bytes);
     if (p.max_chunks == 0) return 1;
     const int64_t waves = (p.max_chunks + nw - 1) / nw;
-    return 2 * waves;
+    return (p.tc ? 3 : 2) * waves;  // tensor cores: prep, fallback, scan; else prep, scan
 }
 
 kda_status kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -128,7 +175,7 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
         if (!aligned16(p)) return KDA_ERR_MISALIGNED;
     if (reinterpret_cast<uintptr_t>(beta) & 3u) return KDA_ERR_MISALIGNED;
 
-    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv);
+    Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
     if (workspace_bytes < min_bytes(p)) return KDA_ERR_WORKSPACE;
 
     kda::PrefillArgs a;
@@ -141,25 +188,44 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
     a.slot_bytes = p.slot_bytes;
 
     const int64_t nw = waves_chunks(p, workspace_bytes);
-    if (nw >= p.max_chunks) {  // one wave: no state carry needed
-        a.state = nullptr;
-        a.slots = static_cast<char *>(workspace);
-    } else {
-        a.state = static_cast<float *>(workspace);
-        a.slots = static_cast<char *>(workspace) + p.state_bytes;
-    }
+    const bool multi = nw < p.max_chunks;
+    char *ws = static_cast<char *>(workspace);
+    int *queue = reinterpret_cast<int *>(ws);
+    ws += queue_bytes(p, nw);
+    a.state = multi ? reinterpret_cast<float *>(ws) : nullptr;
+    ws += multi ? round_up(p.state_bytes, 1024) : 0;
+    a.slots = ws;
 
+    int *err = nullptr;
+    if (p.tc && !(err = kda::device_error_word())) return KDA_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == KDA_DTYPE_BF16;
-    if (p.max_chunks == 0) {  // only empty sequences: S_T = S0
-        if (kda::simt_prefill_wave(a, 0, 0, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
-        return KDA_OK;
-    }
+    const int cap = (int)std::min<int64_t>((int64_t)nw * p.units, INT32_MAX);
+    auto wave = [&](int j0, int n) {
+        return p.tc ? kda::tc_prefill_wave(a, j0, n, queue, cap, err, st)
+                    : kda::simt_prefill_wave(a, j0, n, bf16, st);
+    };
+    if (p.max_chunks == 0)  // only empty sequences: S_T = S0
+        return wave(0, 0) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     for (int64_t j0 = 0; j0 < p.max_chunks; j0 += nw) {
         const int n = (int)std::min<int64_t>(nw, p.max_chunks - j0);
-        if (kda::simt_prefill_wave(a, (int)j0, n, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
+        if (wave((int)j0, n) != cudaSuccess) return KDA_ERR_CUDA;
     }
     return KDA_OK;
+}
+
+kda_status kda_device_error(int32_t *code, int32_t reset) {
+    if (!code) return KDA_ERR_INVALID_ARG;
+    int *w = kda::device_error_word();
+    if (!w) return KDA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+    if (reset && v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    *code = v;
+    return v == 0 ? KDA_OK : KDA_ERR_TIMEOUT;
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -55,6 +55,16 @@ struct PrefillArgs {
 size_t simt_slot_bytes(int dk);
 cudaError_t simt_prefill_wave(const PrefillArgs &a, int j0, int nw, bool bf16, cudaStream_t st);
 
+// tensor-core path (bf16, d_k = d_v = 128). `fix` is the fallback queue
+// ([0] = count, then up to fix_cap slot indices); `err` the device error word.
+size_t tc_slot_bytes();
+cudaError_t tc_prefill_wave(const PrefillArgs &a, int j0, int nw, int *fix, int fix_cap, int *err,
+                            cudaStream_t st);
+
+// Address of this device's error word (set by kernels whose bounded waits ran
+// out), or nullptr if it cannot be resolved.
+int *device_error_word();
+
 // decode step
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,

@@ -109,8 +109,10 @@ int64_t kda_prefill_launches(int32_t num_seqs, int64_t total_tokens, int32_t max
  *   workspace  device scratch of workspace_bytes (>= kda_prefill_workspace_min)
  *
  * Supported: dk, dv in {64, 128}; chunk = 64; dtype F32 or BF16. bf16 inputs
- * run on the tensor cores unless KDA_FLAG_EXACT; fp32 inputs always use fp32
- * CUDA-core arithmetic. Sequences of length 0 are allowed (S_T = S0).
+ * with dk = dv = 128 run on the tensor cores (bf16 operands, fp32 accumulation
+ * and state) unless KDA_FLAG_EXACT; every other case uses fp32 CUDA-core
+ * arithmetic. Sequences of length 0 are allowed (S_T = S0). max_seqlen must
+ * not be smaller than any sequence length.
  */
 kda_status kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
                        const float *beta, const float *S0, const int32_t *cu_seqlens,
@@ -118,6 +120,15 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
                        int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
                        void *o, float *S_T, void *workspace, size_t workspace_bytes,
                        kda_stream_t stream);
+
+/*
+ * Reads (and with reset != 0 clears) the calling device's error word, which a
+ * kernel sets when one of its bounded device-side waits (2 s) ran out; the
+ * kernel then abandons its work and the outputs are not valid. Synchronous:
+ * it waits for the device. *code = 0 and KDA_OK when no wait failed, else
+ * the nonzero code and KDA_ERR_TIMEOUT.
+ */
+kda_status kda_device_error(int32_t *code, int32_t reset);
 
 /*
  * One decode step for N independent sequences, state updated in place

@@ -37,6 +37,7 @@ def test_exports_every_declared_symbol(lib):
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(kda.EXPORTED_SYMBOLS)
+    assert "kda_device_error" in names
 
 
 def test_status_strings_and_version(lib):

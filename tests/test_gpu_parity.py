@@ -168,6 +168,34 @@ def test_strong_decay():
     check(o, S_T, inp, torch.float32, label="strong decay")
 
 
+@pytest.mark.parametrize("scale", [400.0, 30.0])
+def test_strong_decay_tensor_core_path(scale):
+    """bf16, d = 128: chunks whose decay range is too large for the factorised
+    Gram go through the exact fallback (every chunk at scale 400, some at 30)."""
+    inp = make([300, 64, 130], 4, 128, 128, torch.bfloat16, seed=13)
+    inp["log_alpha"] = inp["log_alpha"] * scale
+    o, S_T = run(inp)
+    check(o, S_T, inp, torch.bfloat16, label="strong decay bf16 x%g" % scale)
+    assert kda.kda_device_error() == 0
+
+
+def test_tensor_core_matches_exact_path():
+    """The tcgen05 path and the fp32 CUDA-core path agree within the bf16 tolerance."""
+    inp = make([513, 77], 4, 128, 128, torch.bfloat16, seed=14)
+    o1, S1 = run(inp)
+    o2, S2 = run(inp, exact=True)
+    assert float((o1.float() - o2.float()).abs().max()) <= 2e-2
+    assert float((S1 - S2).norm() / S2.norm()) <= 1e-2
+    check(o1, S1, inp, torch.bfloat16, label="tc")
+    check(o2, S2, inp, torch.bfloat16, label="exact")
+
+
+def test_no_device_error_after_runs():
+    inp = make([1000], 8, 128, 128, torch.bfloat16, seed=15)
+    run(inp)
+    assert kda.kda_device_error() == 0
+
+
 def test_no_l2norm_flag():
     inp = make([100], 2, 64, 64, torch.float32, seed=8)
     o1, S1 = run(inp)
