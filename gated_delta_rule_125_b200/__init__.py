@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size", "kda_prefill_launches",
-           "kda_device_error",
+           "kda_device_error", "kda_prefill_noalloc",
            "kda_prefill_workspace_min", "kda_status_string", "kda_version", "KDAError",
            "library_path", "load_library", "KDA_OK", "KDA_ERR_INVALID_ARG",
            "KDA_ERR_UNSUPPORTED", "KDA_ERR_MISALIGNED", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA",
@@ -28,7 +28,7 @@ KDA_FLAG_NO_L2NORM, KDA_FLAG_EXACT = 0x1, 0x2
 
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
                     "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
-                    "kda_decode_step", "kda_device_error")
+                    "kda_decode_step", "kda_device_error", "kda_prefill_noalloc")
 
 _lib = None
 
@@ -70,6 +70,9 @@ def load_library():
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
                                     u32, vp, vp]
     lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32,
+                                        i32, ctypes.c_int, i32, u32, vp, fp, vp]
+    lib.kda_prefill_noalloc.restype = ctypes.c_int
     lib.kda_device_error.argtypes = [ctypes.POINTER(i32), i32]
     lib.kda_device_error.restype = ctypes.c_int
     _lib = lib
@@ -182,6 +185,25 @@ def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqle
                          _stream(stream, dev))
     if rc != KDA_OK:
         raise KDAError(rc, "kda_prefill")
+    return o, S_T
+
+
+def kda_prefill_noalloc(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqlen,
+                        chunk=64, l2norm=True, exact=False, o, S_T, stream=None):
+    """``kda_prefill_noalloc`` in ``include/kda.h``: the prefill with the library's fixed
+    scratch array instead of a workspace, for callers that cannot allocate device
+    memory. Outputs ``o`` and ``S_T`` are the caller's; nothing is allocated here.
+    Calls sharing the array must not overlap on the GPU."""
+    lib = load_library()
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    rc = lib.kda_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                 _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, _dtype_code(q),
+                                 chunk, _flags(l2norm, exact), _ptr(o), _ptr(S_T),
+                                 _stream(stream, q.device))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_prefill_noalloc")
     return o, S_T
 
 

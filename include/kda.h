@@ -122,6 +122,36 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
                        kda_stream_t stream);
 
 /*
+ * kda_prefill without a workspace argument, for callers that cannot allocate
+ * device memory where they run the prefill (a runtime that owns all device
+ * memory through its own pool and forbids library allocations, a plugin whose
+ * host framework hides its allocator, or a serving loop that cannot afford a
+ * cudaMalloc, which may synchronise the device). The pages have no
+ * counterpart to this entry point; it exists only for such callers.
+ *
+ * Same arguments, outputs and results as kda_prefill; the workspace is a
+ * fixed array of KDA_NOALLOC_SCRATCH_BYTES inside the library's device image,
+ * held by every GPU that loads the library until the process exits. Nothing is
+ * allocated: no cudaMalloc, cudaFree or allocating library call.
+ * - Limit: problems whose kda_prefill_workspace_min() exceeds
+ *   KDA_NOALLOC_SCRATCH_BYTES are refused with KDA_ERR_WORKSPACE before
+ *   anything is enqueued (at d_k = d_v = 128: about num_seqs * H <= 240 on the
+ *   tensor-core path; larger batches run as more, smaller waves).
+ * - The first call on a device resolves the array's address on that device
+ *   (with that device current); make that first call before any stream
+ *   capture begins.
+ * - All calls share the one array, which keeps the last call's contents.
+ *   Calls that overlap on the GPU (other streams, other host threads) race on
+ *   it and give wrong results: order them on one stream or synchronise.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                               const float *beta, const float *S0, const int32_t *cu_seqlens,
+                               int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                               int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk,
+                               uint32_t flags, void *o, float *S_T, kda_stream_t stream);
+
+/*
  * Reads (and with reset != 0 clears) the calling device's error word, which a
  * kernel sets when one of its bounded device-side waits (2 s) ran out; the
  * kernel then abandons its work and the outputs are not valid. Synchronous:
