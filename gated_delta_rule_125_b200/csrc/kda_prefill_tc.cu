@@ -23,6 +23,12 @@
 //    products are M=128 tcgen05.mma with fp32 accumulators in TMEM; the fp32
 //    state lives in registers (thread = state row = TMEM lane) and a bf16 copy
 //    in shared memory feeds the next chunk's products.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <mutex>
+
 #include "kda_internal.cuh"
 #include "kda_tc.cuh"
 
@@ -59,44 +65,95 @@ __device__ __forceinline__ void flag_error(int *err, int code) {
 }
 
 // ---------------------------------------------------------------- prep ----
+// Persistent, two CTAs per SM (~84 KB shared memory each), each walking the
+// wave's (chunk, sequence, head) items. q and k stay in registers (coalesced
+// 16-byte loads); log_alpha arrives by one tensor-map TMA box and is turned
+// into G in place; that buffer is then reused for A, X and the solve's
+// scratch. The slot's WQ and T tiles leave by TMA bulk stores; KD, P and D
+// are stored straight from registers.
 constexpr int PT = 256;
-constexpr uint32_t PS_SL = 0;                    // slot staging (66560); WQ first holds [Kg ; Qg]
-constexpr uint32_t PS_GB = 66560;                // K e^-G, K-major 64 x 128 (B of the Gram)
-constexpr uint32_t PS_KGT = PS_GB + 16384;       // K e^G,  MN-major 64 x 128 (A of W^T)
-constexpr uint32_t PS_GF = PS_KGT + 16384;       // fp32 G [64][128]; later X [64][65]
-constexpr uint32_t PS_AF = PS_GF + 33280;        // fp32 A [64][65] (strictly lower, upper blocks scratch)
-constexpr uint32_t PS_SMALL = PS_AF + 16640;     // invq[64] invk[64] beta[64] gl[128]
-constexpr uint32_t PS_BAR = PS_SMALL + 1280;     // 2 mbarriers, tmem base, flags
+constexpr uint32_t PS_LA = 0;                     // log_alpha -> G [64][128] fp32; later A, X
+constexpr uint32_t PS_GA = 34816;                 // [Kg ; Qg] K-major 128 x 128 -> WQ   (34 * 1024)
+constexpr uint32_t PS_GB = PS_GA + 32768;         // K e^-G K-major 64 x 128; later T (8 KB) + R2
+constexpr uint32_t PS_SMALL = PS_GB + 16384;      // invq[64] invk[64] beta[64] eGl[128]
+constexpr uint32_t PS_BAR = PS_SMALL + 1280;      // la, mma barriers; tmem base; flags
 constexpr uint32_t PS_BYTES = PS_BAR + 64;
-constexpr uint32_t PS_ALLOC = PS_BYTES + 1024;   // + alignment slack
+constexpr uint32_t PS_ALLOC = PS_BYTES + 1024;    // + alignment slack
+constexpr int ALD = 65, XLD = 64;                 // row strides of A and X (floats)
+constexpr uint32_t PS_AF = PS_LA, PS_X = PS_LA + 16640;
+constexpr uint32_t PS_T = PS_GB, PS_R2 = PS_GB + 8192;
 
-__global__ void __launch_bounds__(PT, 1)
-prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *__restrict__ la,
-            const float *__restrict__ beta, const int32_t *__restrict__ cu, int64_t total, int H,
-            int N, int j0, int l2norm, float eps, char *__restrict__ slots, int *__restrict__ fix,
-            int fix_cap, int *__restrict__ err) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int jl = blockIdx.x, s = blockIdx.y, h = blockIdx.z;
+struct Item {
+    int64_t t0;
+    int n, h, slot;
+};
+
+// Item `id` of the wave; false if that chunk lies past its sequence's end.
+__device__ __forceinline__ bool decode_item(int id, const int32_t *cu, int64_t total, int H, int N,
+                                            int j0, Item &it) {
+    const int h = id % H, s = (id / H) % N, jl = id / (H * N);
     int64_t bos, eos;
     seq_bounds(cu, s, total, bos, eos);
     const int64_t j = (int64_t)j0 + jl;
-    if (j * C >= eos - bos) return;
-    const int n = (int)((eos - bos - j * C) < C ? (eos - bos - j * C) : C);
-    const int64_t t0 = bos + j * C;
-    const int slot_id = (jl * N + s) * H + h;
-    char *gslot = slots + (size_t)slot_id * SL_BYTES;
+    if (j * C >= eos - bos) return false;
+    it.n = (int)((eos - bos - j * C) < C ? (eos - bos - j * C) : C);
+    it.t0 = bos + j * C;
+    it.h = h;
+    it.slot = id;
+    return true;
+}
 
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+// D (16x8) += A (16x8, row-major) x B (8x8) with tf32 operands, fp32 accumulation.
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// One warp: C[16 x 8] = A[16 x K] B[K x 8] for A(r, k), B(k, n) given as functors;
+// the result is handed back through `out(r, n, value)`.
+template <int K, typename FA, typename FB, typename FO>
+__device__ __forceinline__ void warp_gemm_16x8(int lane, FA A, FB B, FO out) {
+    const int g = lane >> 2, t = lane & 3;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < K / 8; ++ks) {
+        const uint32_t a[4] = {to_tf32(A(g, 8 * ks + t)), to_tf32(A(g + 8, 8 * ks + t)),
+                               to_tf32(A(g, 8 * ks + t + 4)), to_tf32(A(g + 8, 8 * ks + t + 4))};
+        const uint32_t b[2] = {to_tf32(B(8 * ks + t, g)), to_tf32(B(8 * ks + t + 4, g))};
+        mma_tf32(acc, a, b);
+    }
+    out(g, 2 * t, acc[0]);
+    out(g, 2 * t + 1, acc[1]);
+    out(g + 8, 2 * t, acc[2]);
+    out(g + 8, 2 * t + 1, acc[3]);
+}
+
+__global__ void __launch_bounds__(PT, 2)
+prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
+            const __grid_constant__ CUtensorMap tmap_la, const float *__restrict__ beta,
+            const int32_t *__restrict__ cu, int64_t total, int H, int N, int j0, int nw, int l2norm,
+            float eps, char *__restrict__ slots, int *__restrict__ fix, int fix_cap,
+            int *__restrict__ err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint8_t *GA = sm + PS_SL + SL_WQ;
-    uint8_t *GB = sm + PS_GB;
-    uint8_t *KGT = sm + PS_KGT;
-    float *GF = reinterpret_cast<float *>(sm + PS_GF);
+    const int items = nw * N * H;
+    float *G = reinterpret_cast<float *>(sm + PS_LA);
     float *AF = reinterpret_cast<float *>(sm + PS_AF);
+    float *X = reinterpret_cast<float *>(sm + PS_X);
+    float *R2 = reinterpret_cast<float *>(sm + PS_R2);
+    uint8_t *GA = sm + PS_GA;
+    uint8_t *GB = sm + PS_GB;
+    uint8_t *TT = sm + PS_T;
     float *invq = reinterpret_cast<float *>(sm + PS_SMALL);
-    float *invk = invq + 64, *sbeta = invk + 64, *sgl = sbeta + 64;
-    float *Dv = reinterpret_cast<float *>(sm + PS_SL + SL_D);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);
+    float *invk = invq + 64, *sbeta = invk + 64, *eGl = sbeta + 64;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA
     uint32_t *tbase = reinterpret_cast<uint32_t *>(bars + 2);
     int *sflag = reinterpret_cast<int *>(tbase + 1);  // [0] unsafe range, [1] wait failed
 
@@ -111,233 +168,278 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float 
         tmem_alloc(tbase, 128);
         tmem_relinquish();
     }
-    __syncthreads();  // flags and barriers initialised before anyone sets them
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tbase;
+    uint32_t la_phase = 0, mma_phase = 0;
 
-    // 1. G (threads = key channels) | row norms and beta (warps 4..7).
-    if (tid < DK) {
-        const int c = tid;
-        const float *src = la + ((size_t)t0 * H + h) * DK + c;
-        const size_t stride = (size_t)H * DK;
-        float run = 0.f;
-#pragma unroll 8
-        for (int r = 0; r < C; ++r) {
-            run += (r < n) ? __ldg(src + (size_t)r * stride) : 0.f;
-            GF[r * DK + c] = run;
+    for (int id = blockIdx.x; id < items; id += gridDim.x) {
+        Item cur;
+        if (!decode_item(id, cu, total, H, N, j0, cur)) continue;
+        const int n = cur.n;
+        char *gslot = slots + (size_t)cur.slot * SL_BYTES;
+
+        // The previous slot's bulk stores must have left GA / GB before they are rewritten.
+        if (tid == 0) {
+            bulk_wait_read();
+            mbar_arrive_expect_tx(&bars[0], 32768u);
+            tma_load_3d(G, &tmap_la, 0, cur.h, (int)cur.t0, &bars[0]);
         }
-        sgl[c] = run;
-        Dv[c] = expf(run);
-        if (-run > kTau) sflag[0] = 1;
-    } else {
-        const int w = warp - 4;
-        for (int rr = 0; rr < 16; ++rr) {
-            const int r = w * 16 + rr;
-            float sq = 0.f, sk = 0.f;
-            if (r < n) {
-                const size_t off = ((size_t)(t0 + r) * H + h) * DK + lane * 4;
-                const uint2 qv = __ldg(reinterpret_cast<const uint2 *>(q + off));
-                const uint2 kv = __ldg(reinterpret_cast<const uint2 *>(k + off));
-                const uint32_t qw[2] = {qv.x, qv.y}, kw[2] = {kv.x, kv.y};
+        // q and k rows: thread owns chunk c8 = tid & 15 of rows (tid >> 4) + 16 m.
+        const int c8 = tid & 15, rb = tid >> 4;
+        uint4 qraw[4], kraw[4];
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const float a = __uint_as_float(qw[i] << 16), b = __uint_as_float(qw[i] & 0xFFFF0000u);
-                    const float c2 = __uint_as_float(kw[i] << 16), d = __uint_as_float(kw[i] & 0xFFFF0000u);
-                    sq += a * a + b * b;
-                    sk += c2 * c2 + d * d;
-                }
+        for (int m = 0; m < 4; ++m) {
+            const int r = rb + 16 * m;
+            const size_t off = ((size_t)(cur.t0 + r) * H + cur.h) * DK + c8 * 8;
+            qraw[m] = (r < n) ? __ldg(reinterpret_cast<const uint4 *>(q + off)) : make_uint4(0, 0, 0, 0);
+            kraw[m] = (r < n) ? __ldg(reinterpret_cast<const uint4 *>(k + off)) : make_uint4(0, 0, 0, 0);
+        }
+        if (tid < C) sbeta[tid] = (tid < n) ? __ldg(beta + (size_t)(cur.t0 + tid) * H + cur.h) : 0.f;
+
+        // 1a. Row norms: 16 lanes share a row; shuffle-reduce over them.
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            float qf[8], kf[8], sq = 0.f, sk = 0.f;
+            unpack8(qraw[m], qf);
+            unpack8(kraw[m], kf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                sq += qf[e] * qf[e];
+                sk += kf[e] * kf[e];
             }
 #pragma unroll
-            for (int off = 16; off; off >>= 1) {
+            for (int off = 1; off < 16; off <<= 1) {
                 sq += __shfl_xor_sync(0xffffffffu, sq, off);
                 sk += __shfl_xor_sync(0xffffffffu, sk, off);
             }
-            if (lane == 0) {
+            const int r = rb + 16 * m;
+            if (c8 == 0) {
                 const bool live = r < n;
                 invq[r] = !live ? 0.f : (l2norm ? 1.f / fmaxf(sqrtf(sq), eps) : 1.f);
                 invk[r] = !live ? 0.f : (l2norm ? 1.f / fmaxf(sqrtf(sk), eps) : 1.f);
             }
         }
-        const int r = tid - DK;
-        if (r < C) sbeta[r] = r < n ? beta[(size_t)(t0 + r) * H + h] : 0.f;
-    }
-    __syncthreads();
-    const bool safe = sflag[0] == 0;
-
-    // 2. Operands, one (row, 8-channel chunk) item at a time.
-    for (int it = tid; it < C * (DK / 8); it += PT) {
-        const int r = it >> 4, c8 = it & 15;
-        float kf[8], qf[8];
-        if (r < n) {
-            const size_t off = ((size_t)(t0 + r) * H + h) * DK + c8 * 8;
-            load8_bf16(k + off, kf);
-            load8_bf16(q + off, qf);
-        } else {
+        // 1b. G = cumulative sum of log_alpha over rows, in place: thread (channel,
+        //     half) scans 32 rows in registers; the upper half adds the lower total.
+        if (!mbar_wait(&bars[0], la_phase, kWaitNs)) sflag[1] = 1;
+        la_phase ^= 1;
+        {
+            const int c = tid & (DK - 1), half = tid >> 7, r0 = half * 32;
+            float v[32];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) kf[e] = qf[e] = 0.f;
-        }
-        const float ik = invk[r], iq = invq[r];
-        float kg[8], qg[8], kn[8], kd[8];
+            for (int i = 0; i < 32; ++i) v[i] = (r0 + i < n) ? G[(r0 + i) * DK + c] : 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float g = GF[r * DK + c8 * 8 + e];
-            const float ep = __expf(g), en = __expf(-g);
-            const float kk = kf[e] * ik;
-            kg[e] = kk * ep;
-            qg[e] = qf[e] * iq * ep;
-            kn[e] = kk * en;
-            kd[e] = kn[e] * Dv[c8 * 8 + e];
+            for (int i = 1; i < 32; ++i) v[i] += v[i - 1];
+            if (half == 0) eGl[c] = v[31];
+            __syncthreads();
+            const float base = half ? eGl[c] : 0.f;
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) G[(r0 + i) * DK + c] = v[i] + base;
+            if (half == 1) {
+                const float gl = v[31] + base;
+                eGl[c] = expf(gl);
+                reinterpret_cast<float *>(gslot + SL_D)[c] = eGl[c];
+                if (-gl > kTau) sflag[0] = 1;
+            }
         }
-        const uint4 ukg = pack8(kg);
-        *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = ukg;
-        *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = pack8(qg);
-        *reinterpret_cast<uint4 *>(GB + kmaj_chunk(r, c8, 64)) = pack8(kn);
-        *reinterpret_cast<uint4 *>(KGT + mnmaj_chunk(r, c8, 64)) = ukg;
-        *reinterpret_cast<uint4 *>(sm + PS_SL + SL_KD + mnmaj_chunk(r, c8, 64)) = pack8(kd);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tm = *tbase;
+        __syncthreads();
+        const bool safe = sflag[0] == 0;
 
-    if (!safe) {
-        // Decay range too large for e^{-G}: leave the slot to the exact fallback.
+        // 2. Operands for (row, 8-channel chunk): [Kg ; Qg] and K e^-G to smem, Kd to the slot.
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int r = rb + 16 * m;
+            float kf[8], qf[8];
+            unpack8(kraw[m], kf);
+            unpack8(qraw[m], qf);
+            const float ik = invk[r], iq = invq[r];
+            const float4 g0 = *reinterpret_cast<const float4 *>(G + r * DK + c8 * 8);
+            const float4 g1 = *reinterpret_cast<const float4 *>(G + r * DK + c8 * 8 + 4);
+            const float4 d0 = *reinterpret_cast<const float4 *>(eGl + c8 * 8);
+            const float4 d1 = *reinterpret_cast<const float4 *>(eGl + c8 * 8 + 4);
+            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+            float kg[8], qg[8], kn[8], kd[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float ep = __expf(gg[e]), en = __expf(-gg[e]);
+                const float kk = kf[e] * ik;
+                kg[e] = kk * ep;
+                qg[e] = qf[e] * iq * ep;
+                kn[e] = kk * en;
+                kd[e] = kn[e] * dd[e];
+            }
+            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = pack8(kg);
+            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = pack8(qg);
+            *reinterpret_cast<uint4 *>(GB + kmaj_chunk(r, c8, 64)) = pack8(kn);
+            if (safe) *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = pack8(kd);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        if (!safe) {
+            // Decay range too large for e^{-G}: the exact fallback takes this slot.
+            if (tid == 0) {
+                const int pos = atomicAdd(fix, 1);
+                if (pos < fix_cap) fix[1 + pos] = cur.slot;
+                else flag_error(err, 2);
+                sflag[0] = 0;
+            }
+            __syncthreads();
+            continue;
+        }
+
+        // 3. Gram: TMEM cols [0,64) = [Kg ; Qg] (K e^-G)^T.
         if (tid == 0) {
-            const int pos = atomicAdd(fix, 1);
-            if (pos < fix_cap) fix[1 + pos] = slot_id;
-            else flag_error(err, 2);
+            const uint32_t a = smem_u32(GA), b = smem_u32(GB);
+            const uint32_t idg = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int st = 0; st < DK / 16; ++st) mma_bf16(tm, kmaj_desc(a, st, 128), kmaj_desc(b, st, 64), idg, st > 0);
+            mma_commit(&bars[1]);
+        }
+        if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
+        mma_phase ^= 1;
+        tc_fence_after();
+
+        // 4. A (fp32, strictly lower) over the consumed G; P (bf16, lower) to the slot.
+        if (warp < 4) {
+            const int row = warp * 32 + lane;
+            for (int c0 = 0; c0 < C; c0 += 16) {
+                float v[16];
+                tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + c0, v);
+                tmem_wait_ld();
+                if (row < C) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) AF[row * ALD + c0 + i] = (c0 + i < row) ? v[i] : 0.f;
+                } else {
+                    const int r = row - C;
+                    float lo[8], hi[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        lo[i] = (c0 + i <= r) ? v[i] : 0.f;
+                        hi[i] = (c0 + 8 + i <= r) ? v[8 + i] : 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(gslot + SL_P + kmaj_chunk(r, c0 / 8, 64)) = pack8(lo);
+                    *reinterpret_cast<uint4 *>(gslot + SL_P + kmaj_chunk(r, c0 / 8 + 1, 64)) = pack8(hi);
+                }
+            }
+        } else {
+            for (int i = tid - 128; i < C * XLD / 4; i += 128)
+                reinterpret_cast<float4 *>(X)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         tc_fence_before();
         __syncthreads();
-        if (warp == 0) tmem_dealloc(tm, 128);
-        return;
-    }
 
-    // 3. Gram on the tensor cores: TMEM cols [0,64) = [Kg ; Qg] (K e^-G)^T.
-    if (tid == 0) {
-        const uint32_t a = smem_u32(GA), b = smem_u32(GB);
-        const uint32_t id = idesc_bf16(128, 64, false, false);
+        // 5. X = (I + Diag(beta) A)^{-1}: diagonal 16x16 blocks by forward substitution,
+        //    then the 2x2 block recursion with tf32 tensor-core products:
+        //    [X11 0; X21 X22] with X21 = -X22 (Diag(beta_2) A21) X11.
+        if (tid < C) {
+            const int b = tid >> 4, cc = tid & 15;
+            float x[16];
 #pragma unroll
-        for (int st = 0; st < DK / 16; ++st) mma_bf16(tm, kmaj_desc(a, st, 128), kmaj_desc(b, st, 64), id, st > 0);
-        mma_commit(&bars[0]);
-    }
-    if (!mbar_wait(&bars[0], 0, kWaitNs)) sflag[1] = 1;
-    tc_fence_after();
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * b + rr;
+                float acc = 0.f;
+#pragma unroll
+                for (int ii = 0; ii < rr; ++ii) acc += AF[r * ALD + 16 * b + ii] * x[ii];
+                x[rr] = (rr == cc) ? 1.f : (rr > cc ? -sbeta[r] * acc : 0.f);
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * XLD + 16 * b + cc] = x[rr];
+        }
+        __syncthreads();
+        // 16-row level: warps 0, 1 build X[16..31][0..15], X[48..63][32..47] (two 8-column halves each).
+        if (warp < 4) {
+            const int o = (warp >> 1) * 32, nh = (warp & 1) * 8;  // block offset, column half
+            float *Rw = R2 + warp * 128;                          // 16 x 8 scratch per warp
+            warp_gemm_16x8<16>(
+                lane, [&](int r, int kk) { return sbeta[o + 16 + r] * AF[(o + 16 + r) * ALD + o + kk]; },
+                [&](int kk, int nn) { return X[(o + kk) * XLD + o + nh + nn]; },
+                [&](int r, int nn, float v) { Rw[r * 8 + nn] = v; });
+            __syncwarp();
+            warp_gemm_16x8<16>(
+                lane, [&](int r, int kk) { return X[(o + 16 + r) * XLD + o + 16 + kk]; },
+                [&](int kk, int nn) { return Rw[kk * 8 + nn]; },
+                [&](int r, int nn, float v) { X[(o + 16 + r) * XLD + o + nh + nn] = -v; });
+        }
+        __syncthreads();
+        // 32-row level: R2 = (Diag(beta) A)[32..63][0..31] X[0..31][0..31], then X[32..63][0..31] = -X22 R2.
+        {
+            const int mt = warp >> 2, nt = warp & 3;  // 16-row tile, 8-column tile
+            warp_gemm_16x8<32>(
+                lane, [&](int r, int kk) { return sbeta[32 + 16 * mt + r] * AF[(32 + 16 * mt + r) * ALD + kk]; },
+                [&](int kk, int nn) { return X[kk * XLD + 8 * nt + nn]; },
+                [&](int r, int nn, float v) { R2[(16 * mt + r) * 32 + 8 * nt + nn] = v; });
+            __syncthreads();
+            warp_gemm_16x8<32>(
+                lane, [&](int r, int kk) { return X[(32 + 16 * mt + r) * XLD + 32 + kk]; },
+                [&](int kk, int nn) { return R2[kk * 32 + 8 * nt + nn]; },
+                [&](int r, int nn, float v) { X[(32 + 16 * mt + r) * XLD + 8 * nt + nn] = -v; });
+        }
+        __syncthreads();
+        // T = X Diag(beta), lower triangle, bf16: B operand of W^T (smem) and the slot's T tile.
+        for (int e2 = tid; e2 < C * 8; e2 += PT) {
+            const int r = e2 >> 3, cc8 = e2 & 7;
+            float t8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int c = cc8 * 8 + e;
+                t8[e] = (c <= r) ? X[r * XLD + c] * sbeta[c] : 0.f;
+            }
+            *reinterpret_cast<uint4 *>(TT + kmaj_chunk(r, cc8, 64)) = pack8(t8);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
 
-    // 4. A (fp32, strictly lower) to smem; P (bf16, lower incl. diagonal) to the slot.
-    if (warp < 4) {
-        const int row = warp * 32 + lane;
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float v[16];
-            tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + c0, v);
-            tmem_wait_ld();
-            if (row < C) {
+        // 6. W^T = (K e^G)^T T^T: A = rows 0..63 of [Kg ; Qg] read as an MN-major tile
+        //    (64-column blocks 128 rows apart), B = T; TMEM cols [64,128), lane = channel.
+        if (tid == 0) {
+            bulk_s2g(gslot + SL_T, TT, 8192);
+            const uint32_t a = smem_u32(GA), b = smem_u32(TT);
+            const uint32_t idw = idesc_bf16(128, 64, true, false);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) AF[row * 65 + c0 + i] = (c0 + i < row) ? v[i] : 0.f;
-            } else {
-                const int r = row - C;
-                float lo[8], hi[8];
+            for (int st = 0; st < C / 16; ++st)
+                mma_bf16(tm + 64, sdesc(a + st * 16 * 128, 128 * 128, 1024), kmaj_desc(b, st, 64), idw, st > 0);
+            mma_commit(&bars[1]);
+        }
+        if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
+        mma_phase ^= 1;
+        tc_fence_after();
+
+        // 7. W rows into the top half of WQ (its Kg rows are consumed).
+        if (warp < 4) {
+            const int c = warp * 32 + lane;
+            for (int c0 = 0; c0 < C; c0 += 16) {
+                float v[16];
+                tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 64 + c0, v);
+                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    lo[i] = (c0 + i <= r) ? v[i] : 0.f;
-                    hi[i] = (c0 + 8 + i <= r) ? v[8 + i] : 0.f;
-                }
-                *reinterpret_cast<uint4 *>(sm + PS_SL + SL_P + kmaj_chunk(r, c0 / 8, 64)) = pack8(lo);
-                *reinterpret_cast<uint4 *>(sm + PS_SL + SL_P + kmaj_chunk(r, c0 / 8 + 1, 64)) = pack8(hi);
+                for (int i = 0; i < 16; ++i)
+                    *reinterpret_cast<bf16 *>(GA + kmaj_off(c0 + i, c, 128)) = __float2bfloat16_rn(v[i]);
             }
         }
-    }
-    __syncthreads();
-
-    // 5. X = (I + Diag(beta) A)^{-1} by 16x16 blocks; T = X Diag(beta).
-    float *X = GF;  // [64][65]
-    if (tid < C) {
-        // diagonal blocks: column cc of block b by forward substitution
-        const int b = tid >> 4, cc = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            const int r = 16 * b + rr;
-            float acc = 0.f;
-#pragma unroll
-            for (int ii = 0; ii < rr; ++ii) acc += AF[r * 65 + 16 * b + ii] * x[ii];
-            x[rr] = (rr == cc) ? 1.f : (rr > cc ? -sbeta[r] * acc : 0.f);
-        }
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * 65 + 16 * b + cc] = x[rr];
-    }
-    __syncthreads();
-    for (int d = 1; d < 4; ++d) {
-        // R_ij = Diag(beta_i) sum_{k=j}^{i-1} A_ik X_kj  (kept in the unused upper block (j, i) of AF)
-        for (int e = tid; e < (4 - d) * 256; e += PT) {
-            const int jb = e >> 8, ib = jb + d, rr = (e >> 4) & 15, cc = e & 15;
-            const int r = 16 * ib + rr;
-            float acc = 0.f;
-            for (int kb = jb; kb < ib; ++kb)
-#pragma unroll
-                for (int t = 0; t < 16; ++t) acc += AF[r * 65 + 16 * kb + t] * X[(16 * kb + t) * 65 + 16 * jb + cc];
-            AF[(16 * jb + rr) * 65 + 16 * ib + cc] = sbeta[r] * acc;
-        }
+        fence_async_smem();
+        tc_fence_before();
         __syncthreads();
-        // X_ij = -X_ii R_ij
-        for (int e = tid; e < (4 - d) * 256; e += PT) {
-            const int jb = e >> 8, ib = jb + d, rr = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-                acc += X[(16 * ib + rr) * 65 + 16 * ib + t] * AF[(16 * jb + t) * 65 + 16 * ib + cc];
-            X[(16 * ib + rr) * 65 + 16 * jb + cc] = -acc;
-        }
-        __syncthreads();
-    }
-    for (int it = tid; it < C * 8; it += PT) {
-        const int r = it >> 3, c8 = it & 7;
-        float t8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int c = c8 * 8 + e;
-            t8[e] = (c <= r) ? X[r * 65 + c] * sbeta[c] : 0.f;
-        }
-        *reinterpret_cast<uint4 *>(sm + PS_SL + SL_T + kmaj_chunk(r, c8, 64)) = pack8(t8);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
 
-    // 6. W^T = (K e^G)^T T^T on the tensor cores: TMEM cols [64,128), lane = key channel.
+        // 8. WQ leaves in one bulk store; waited for before GA is rewritten.
+        if (tid == 0) {
+            bulk_s2g(gslot + SL_WQ, GA, 32768);
+            bulk_commit();
+        }
+    }
     if (tid == 0) {
-        const uint32_t a = smem_u32(KGT), b = smem_u32(sm + PS_SL + SL_T);
-        const uint32_t id = idesc_bf16(128, 64, true, false);
-#pragma unroll
-        for (int st = 0; st < C / 16; ++st) mma_bf16(tm + 64, mnmaj_desc(a, st, 64), kmaj_desc(b, st, 64), id, st > 0);
-        mma_commit(&bars[1]);
-    }
-    if (!mbar_wait(&bars[1], 0, kWaitNs)) sflag[1] = 1;
-    tc_fence_after();
-
-    // 7. W rows into the top half of WQ (its Kg rows are no longer needed).
-    if (warp < 4) {
-        const int c = warp * 32 + lane;
-        for (int c0 = 0; c0 < C; c0 += 16) {
-            float v[16];
-            tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 64 + c0, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                *reinterpret_cast<bf16 *>(GA + kmaj_off(c0 + i, c, 128)) = __float2bfloat16_rn(v[i]);
-        }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // 8. The assembled slot goes out in one bulk store.
-    if (tid == 0) {
+        bulk_wait_all();
         if (sflag[1]) flag_error(err, 1);
-        bulk_s2g(gslot, sm + PS_SL, SL_USED);
-        bulk_commit();
-        bulk_wait_read();
     }
+    tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 128);
 }
@@ -470,31 +572,34 @@ fix_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *
 
 // ---------------------------------------------------------------- scan ----
 constexpr int ST = 128;
-// shared memory (bytes): two slot buffers, then V, S (bf16), U (bf16), barriers
-constexpr uint32_t SB_WQ = 0, SB_KD = 32768, SB_TT = 49152, SB_PP = 65536, SB_D = 81920, SB_BYTES = 82944;
-constexpr uint32_t SS_V = 2 * SB_BYTES;          // [64 (i)][64 (j)] MN-major
-constexpr uint32_t SS_S = SS_V + 8192;           // [128 (c)][64 (j)] MN-major
-constexpr uint32_t SS_U = SS_S + 16384;          // [64 (r)][64 (j)] MN-major
+// Per chunk buffer (bytes): the slot's tiles plus this CTA's V tile. T is
+// followed by the zero half of [0 ; P], so "T then zeros" is the 128-row A
+// operand of X = T V (its lower 64 output rows are zero and unused).
+constexpr uint32_t SB_WQ = 0, SB_KD = 32768, SB_T = 49152, SB_PP = 57344, SB_V = 73728, SB_D = 81920;
+constexpr uint32_t SB_BYTES = 82944;
+constexpr uint32_t SS_S = 2 * SB_BYTES;          // [128 (c)][64 (j)] MN-major bf16 state
+constexpr uint32_t SS_U = SS_S + 16384;          // [64 (r)][64 (j)] MN-major bf16 pseudo-values
 constexpr uint32_t SS_BAR = SS_U + 8192;         // full[2], bU, bS, tmem base, flag
 constexpr uint32_t SS_BYTES = SS_BAR + 64;
 constexpr uint32_t SS_ALLOC = SS_BYTES + 1024;
-constexpr uint32_t SLOT_COPY_BYTES = 32768 + 16384 + 2 * 8192 + 8192 + 512;
-// TMEM columns: X (two buffers), Y, Z
-constexpr uint32_t TM_X0 = 0, TM_X1 = 64, TM_Y = 128, TM_Z = 192;
+constexpr uint32_t CHUNK_COPY_BYTES = 32768 + 16384 + 8192 + 8192 + 512 + 8192;
+// TMEM columns: X and Y double-buffered, Z
+constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = 256;
 
-__device__ __forceinline__ void issue_slot_copy(uint8_t *buf, const char *g, uint64_t *bar) {
-    mbar_arrive_expect_tx(bar, SLOT_COPY_BYTES);
+__device__ __forceinline__ void issue_chunk_copy(uint8_t *buf, const char *g, const void *tmap_v, int vx,
+                                                 int vy, int vz, uint64_t *bar) {
+    mbar_arrive_expect_tx(bar, CHUNK_COPY_BYTES);
     bulk_g2s(buf + SB_WQ, g + SL_WQ, 32768, bar);
     bulk_g2s(buf + SB_KD, g + SL_KD, 16384, bar);
-    bulk_g2s(buf + SB_TT, g + SL_T, 8192, bar);
-    bulk_g2s(buf + SB_TT + 8192, g + SL_T, 8192, bar);
+    bulk_g2s(buf + SB_T, g + SL_T, 8192, bar);
     bulk_g2s(buf + SB_PP + 8192, g + SL_P, 8192, bar);
     bulk_g2s(buf + SB_D, g + SL_D, 512, bar);
+    tma_load_3d(buf + SB_V, tmap_v, vx, vy, vz, bar);  // 64 tokens x 64 columns of v, SW128
 }
 
 __global__ void __launch_bounds__(ST, 1)
-scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t total, int H, int N,
-            int j0, int nw, const char *__restrict__ slots, const float *__restrict__ S0,
+scan_kernel(const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ cu, int64_t total,
+            int H, int N, int j0, int nw, const char *__restrict__ slots, const float *__restrict__ S0,
             float *__restrict__ state, float *__restrict__ S_T, bf16 *__restrict__ o,
             int *__restrict__ err) {
     extern __shared__ uint8_t smem_raw[];
@@ -509,7 +614,7 @@ scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t 
     const int nj = jend - j0 > 0 ? jend - j0 : 0;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint8_t *sV = sm + SS_V, *sS = sm + SS_S, *sU = sm + SS_U;
+    uint8_t *sS = sm + SS_S, *sU = sm + SS_U;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SS_BAR);  // full0, full1, bU, bS
     uint32_t *tbase = reinterpret_cast<uint32_t *>(bars + 4);
     int *sfail = reinterpret_cast<int *>(tbase + 1);
@@ -522,14 +627,12 @@ scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t 
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(tbase, 256);
+        tmem_alloc(tbase, 512);
         tmem_relinquish();
     }
-    // Rows 0..63 of both [0 ; P] operand buffers stay zero.
-    for (int i = tid; i < 2 * 512; i += ST) {
-        uint8_t *b = sm + (i >> 9) * SB_BYTES + SB_PP;
-        reinterpret_cast<uint4 *>(b)[i & 511] = make_uint4(0, 0, 0, 0);
-    }
+    // Rows 0..63 of both [0 ; P] tiles stay zero.
+    for (int i = tid; i < 2 * 512; i += ST)
+        reinterpret_cast<uint4 *>(sm + (i >> 9) * SB_BYTES + SB_PP)[i & 511] = make_uint4(0, 0, 0, 0);
     // Entry state: S0 (or zeros) on the first wave, else the carry.
     float Sr[DVT];
     {
@@ -551,67 +654,68 @@ scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t 
         }
     };
     store_state_bf16();
-    // V rows of chunk jj (zeros past the sequence end): 4 x 16 bytes per thread.
-    uint4 vreg[4];
-    auto load_v = [&](int jj) {
-        const int nn = (int)((len - (int64_t)jj * C) < C ? (len - (int64_t)jj * C) : C);
-        const int64_t tt = bos + (int64_t)jj * C;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int qi = tid + ST * m, i = qi >> 3, c8 = qi & 7;
-            vreg[m] = (i < nn) ? __ldg(reinterpret_cast<const uint4 *>(v + ((size_t)(tt + i) * H + h) * DV + jv * DVT + c8 * 8))
-                               : make_uint4(0, 0, 0, 0);
-        }
+    auto copy_chunk = [&](int jj, int b) {
+        const char *g = slots + ((size_t)((jj - j0) * N + s) * H + h) * SL_BYTES;
+        issue_chunk_copy(sm + b * SB_BYTES, g, &tmap_v, jv * DVT, h, (int)(bos + (int64_t)jj * C), &bars[b]);
     };
-    auto store_v = [&]() {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int qi = tid + ST * m, i = qi >> 3, c8 = qi & 7;
-            *reinterpret_cast<uint4 *>(sV + mnmaj_chunk(i, c8, C)) = vreg[m];
-        }
-    };
-    auto slot_ptr = [&](int jj) {
-        return slots + ((size_t)((jj - j0) * N + s) * H + h) * SL_BYTES;
-    };
-    if (nj > 0) {
-        if (tid == 0) issue_slot_copy(sm, slot_ptr(j0), &bars[0]);
-        load_v(j0);
-        store_v();
-    }
+    if (nj > 0 && tid == 0) copy_chunk(j0, 0);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tbase;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t id128 = idesc_bf16(128, DVT, false, true);    // K-major A, MN-major B
-    const uint32_t idKd = idesc_bf16(128, DVT, true, true);      // MN-major A (Kd^T)
-    bool ok = true;
+    const uint32_t id128 = idesc_bf16(128, DVT, false, true);  // K-major A, MN-major B
+    const uint32_t idKd = idesc_bf16(128, DVT, true, true);    // MN-major A (Kd^T)
 
     if (nj > 0 && tid == 0) {
-        // X(j0) = [T ; T] V
         if (!mbar_wait(&bars[0], 0, kWaitNs)) *sfail = 1;
-        const uint32_t a = smem_u32(sm + SB_TT), b = smem_u32(sV);
+        const uint32_t a = smem_u32(sm + SB_T), bv = smem_u32(sm + SB_V);
 #pragma unroll
-        for (int st = 0; st < C / 16; ++st) mma_bf16(tm + TM_X0, kmaj_desc(a, st, 128), mnmaj_desc(b, st, C), id128, st > 0);
+        for (int st = 0; st < C / 16; ++st) mma_bf16(tm + TM_X, kmaj_desc(a, st, 128), mnmaj_desc(bv, st, C), id128, st > 0);
     }
 
+    // O = rows 64..127 of Y (buffer yb) for chunk jj -> o (warps 2, 3).
+    auto store_o = [&](int jj, uint32_t yb) {
+        const int nn = (int)((len - (int64_t)jj * C) < C ? (len - (int64_t)jj * C) : C);
+        const int64_t tt = bos + (int64_t)jj * C;
+        const int r = c - 64;
+#pragma unroll
+        for (int c0 = 0; c0 < DVT; c0 += 16) {
+            float yv[16];
+            tmem_ld16(tm + TM_Y + yb + lane_base + c0, yv);
+            tmem_wait_ld();
+            if (r < nn) {
+                bf16 *dst = o + ((size_t)(tt + r) * H + h) * DV + jv * DVT + c0;
+                float lo[8], hi[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    lo[e] = yv[e];
+                    hi[e] = yv[8 + e];
+                }
+                reinterpret_cast<uint4 *>(dst)[0] = pack8(lo);
+                reinterpret_cast<uint4 *>(dst)[1] = pack8(hi);
+            }
+        }
+    };
+
+    bool ok = true;
     for (int it = 0; it < nj && ok; ++it) {
         const int jj = j0 + it, b = it & 1;
         uint8_t *buf = sm + b * SB_BYTES;
-        const int nn = (int)((len - (int64_t)jj * C) < C ? (len - (int64_t)jj * C) : C);
-        const int64_t tt = bos + (int64_t)jj * C;
-        const uint32_t tmX = tm + ((it & 1) ? TM_X1 : TM_X0);
-        // Y = [W ; Q e^G] S ; prefetch the next slot
+        const uint32_t xb = (uint32_t)b * 64, yb = (uint32_t)b * 64;
+        // Y = [W ; Q e^G] S ; prefetch the next chunk
         if (tid == 0) {
             if (!mbar_wait(&bars[b], (it >> 1) & 1, kWaitNs)) *sfail = 1;
-            if (it + 1 < nj) issue_slot_copy(sm + (b ^ 1) * SB_BYTES, slot_ptr(jj + 1), &bars[b ^ 1]);
+            if (it + 1 < nj) copy_chunk(jj + 1, b ^ 1);
             const uint32_t a = smem_u32(buf + SB_WQ), bs = smem_u32(sS);
 #pragma unroll
-            for (int st = 0; st < DK / 16; ++st) mma_bf16(tm + TM_Y, kmaj_desc(a, st, 128), mnmaj_desc(bs, st, DK), id128, st > 0);
+            for (int st = 0; st < DK / 16; ++st)
+                mma_bf16(tm + TM_Y + yb, kmaj_desc(a, st, 128), mnmaj_desc(bs, st, DK), id128, st > 0);
             mma_commit(&bars[2]);
         }
-        if (it + 1 < nj) load_v(jj + 1);
+        // Output of the previous chunk while Y computes.
+        if (warp >= 2 && it > 0) store_o(jj - 1, yb ^ 64);
         if (!mbar_wait(&bars[2], it & 1, kWaitNs)) *sfail = 1;
         tc_fence_after();
         // U = X - Y (rows 0..63 live in lanes 0..63: warps 0 and 1)
@@ -620,8 +724,8 @@ scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t 
 #pragma unroll
             for (int c0 = 0; c0 < DVT; c0 += 16) {
                 float xv[16], yv[16];
-                tmem_ld16(tmX + lane_base + c0, xv);
-                tmem_ld16(tm + TM_Y + lane_base + c0, yv);
+                tmem_ld16(tm + TM_X + xb + lane_base + c0, xv);
+                tmem_ld16(tm + TM_Y + yb + lane_base + c0, yv);
                 tmem_wait_ld();
                 float lo[8], hi[8];
 #pragma unroll
@@ -633,27 +737,28 @@ scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t 
                 *reinterpret_cast<uint4 *>(sU + mnmaj_chunk(r, c0 / 8 + 1, C)) = pack8(hi);
             }
         }
-        if (it + 1 < nj) store_v();
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // O: Y += [0 ; P] U ; Z = Kd^T U ; then X(j+1) = [T ; T] V(j+1)
+        // O: Y += [0 ; P] U ; Z = Kd^T U ; then X(j+1) = T(j+1) V(j+1)
         if (tid == 0) {
             const uint32_t bu = smem_u32(sU);
             const uint32_t ap = smem_u32(buf + SB_PP), ak = smem_u32(buf + SB_KD);
 #pragma unroll
-            for (int st = 0; st < C / 16; ++st) mma_bf16(tm + TM_Y, kmaj_desc(ap, st, 128), mnmaj_desc(bu, st, C), id128, 1);
+            for (int st = 0; st < C / 16; ++st)
+                mma_bf16(tm + TM_Y + yb, kmaj_desc(ap, st, 128), mnmaj_desc(bu, st, C), id128, 1);
 #pragma unroll
-            for (int st = 0; st < C / 16; ++st) mma_bf16(tm + TM_Z, mnmaj_desc(ak, st, C), mnmaj_desc(bu, st, C), idKd, st > 0);
+            for (int st = 0; st < C / 16; ++st)
+                mma_bf16(tm + TM_Z, mnmaj_desc(ak, st, C), mnmaj_desc(bu, st, C), idKd, st > 0);
             mma_commit(&bars[3]);
             if (it + 1 < nj) {
                 uint8_t *nbuf = sm + (b ^ 1) * SB_BYTES;
                 if (!mbar_wait(&bars[b ^ 1], ((it + 1) >> 1) & 1, kWaitNs)) *sfail = 1;
-                const uint32_t a = smem_u32(nbuf + SB_TT), bv = smem_u32(sV);
-                const uint32_t tmXn = tm + ((it & 1) ? TM_X0 : TM_X1);
+                const uint32_t a = smem_u32(nbuf + SB_T), bv = smem_u32(nbuf + SB_V);
 #pragma unroll
-                for (int st = 0; st < C / 16; ++st) mma_bf16(tmXn, kmaj_desc(a, st, 128), mnmaj_desc(bv, st, C), id128, st > 0);
+                for (int st = 0; st < C / 16; ++st)
+                    mma_bf16(tm + TM_X + (xb ^ 64), kmaj_desc(a, st, 128), mnmaj_desc(bv, st, C), id128, st > 0);
             }
         }
         if (!mbar_wait(&bars[3], it & 1, kWaitNs)) *sfail = 1;
@@ -672,36 +777,14 @@ scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t 
             }
             store_state_bf16();
         }
-        // O rows live in lanes 64..127 (warps 2, 3)
-        if (warp >= 2) {
-            const int r = c - 64;
-#pragma unroll
-            for (int c0 = 0; c0 < DVT; c0 += 16) {
-                float yv[16];
-                tmem_ld16(tm + TM_Y + lane_base + c0, yv);
-                tmem_wait_ld();
-                if (r < nn) {
-                    bf16 *dst = o + ((size_t)(tt + r) * H + h) * DV + jv * DVT + c0;
-                    float lo[8], hi[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        lo[e] = yv[e];
-                        hi[e] = yv[8 + e];
-                    }
-                    reinterpret_cast<uint4 *>(dst)[0] = pack8(lo);
-                    reinterpret_cast<uint4 *>(dst)[1] = pack8(hi);
-                }
-            }
-        }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         ok = (*sfail == 0);
     }
-    if (!ok) {
-        if (tid == 0) flag_error(err, 1);
-    }
+    if (ok && nj > 0 && warp >= 2) store_o(j0 + nj - 1, (uint32_t)((nj - 1) & 1) * 64);
+    if (!ok && tid == 0) flag_error(err, 1);
 
     // Exit: final state when the sequence ended in this wave, else the carry.
     float *Sout = (jend == nch) ? S_T : state;
@@ -713,7 +796,54 @@ scan_kernel(const bf16 *__restrict__ v, const int32_t *__restrict__ cu, int64_t 
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 256);
+    if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// cuTensorMapEncodeTiled, resolved once through the runtime (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// v viewed as [T][H][DV] bf16; a box is 64 columns x 1 head x 64 tokens, SW128.
+bool make_v_map(CUtensorMap *m, const void *v, int64_t total, int H) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)DV, (cuuint64_t)H, (cuuint64_t)total};
+    const cuuint64_t strides[2] = {(cuuint64_t)DV * 2, (cuuint64_t)H * DV * 2};
+    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(v), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q, k or log_alpha viewed as [T][H][128]; a box is 128 channels x 1 head x 64 tokens.
+bool make_row_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int64_t total, int H) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)total};
+    const cuuint64_t strides[2] = {(cuuint64_t)DK * esize, (cuuint64_t)H * DK * esize};
+    const cuuint32_t box[3] = {(cuuint32_t)DK, 1, (cuuint32_t)C};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
 }
 
 }  // namespace
@@ -728,20 +858,29 @@ cudaError_t tc_prefill_wave(const PrefillArgs &a, int j0, int nw, int *fix, int 
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS_ALLOC);
     if (e != cudaSuccess) return e;
+    CUtensorMap vmap;
+    memset(&vmap, 0, sizeof(vmap));
+    if (a.total > 0 && !make_v_map(&vmap, a.v, a.total, a.H)) return cudaErrorInvalidValue;
+    const int sms = sm_count();
     if (nw > 0) {
+        CUtensorMap lamap;
+        if (!make_row_map(&lamap, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.total, a.H))
+            return cudaErrorInvalidValue;
         e = cudaMemsetAsync(fix, 0, sizeof(int), st);
         if (e != cudaSuccess) return e;
-        prep_kernel<<<dim3(nw, a.N, a.H), PT, PS_ALLOC, st>>>(
-            (const bf16 *)a.q, (const bf16 *)a.k, a.log_alpha, a.beta, a.cu, a.total, a.H, a.N, j0,
-            a.l2norm, a.eps, a.slots, fix, fix_cap, err);
+        const int items = nw * a.N * a.H;
+        const int grid = items < 2 * sms ? items : 2 * sms;
+        prep_kernel<<<grid, PT, PS_ALLOC, st>>>((const bf16 *)a.q, (const bf16 *)a.k, lamap, a.beta, a.cu,
+                                                a.total, a.H, a.N, j0, nw, a.l2norm, a.eps, a.slots, fix,
+                                                fix_cap, err);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        fix_kernel<<<148, FT, FS_BYTES, st>>>((const bf16 *)a.q, (const bf16 *)a.k, a.log_alpha, a.beta,
+        fix_kernel<<<sms, FT, FS_BYTES, st>>>((const bf16 *)a.q, (const bf16 *)a.k, a.log_alpha, a.beta,
                                               a.cu, a.total, a.H, a.N, j0, a.l2norm, a.eps, a.slots,
                                               fix, fix_cap);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     scan_kernel<<<dim3(DV / DVT, a.N, a.H), ST, SS_ALLOC, st>>>(
-        (const bf16 *)a.v, a.cu, a.total, a.H, a.N, j0, nw, a.slots, a.S0, a.state, a.S_T, (bf16 *)a.o, err);
+        vmap, a.cu, a.total, a.H, a.N, j0, nw, a.slots, a.S0, a.state, a.S_T, (bf16 *)a.o, err);
     return cudaGetLastError();
 }
 
