@@ -76,6 +76,11 @@ size_t min_bytes(const Plan &p) {
 }
 
 constexpr size_t kRecommendedCap = size_t(512) << 20;
+// Tensor-core path: a wave's slots are sized to stay resident in L2 (126 MB)
+// between the prep kernel that writes them and the scan that reads them, with
+// at least 16 chunks per wave so the state carry between waves stays cheap.
+constexpr size_t kL2SlotBudget = size_t(48) << 20;
+constexpr int64_t kMinWaveChunks = 16;
 
 // Chunks per wave for a workspace of `bytes` (>= min_bytes(p)).
 int64_t waves_chunks(const Plan &p, size_t bytes) {
@@ -141,6 +146,11 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
     if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return 0;
     Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
     const int64_t all = std::max<int64_t>(p.max_chunks, 1);
+    if (p.tc) {
+        int64_t nw = std::max<int64_t>(kMinWaveChunks, (int64_t)(kL2SlotBudget / (p.units * p.slot_bytes)));
+        nw = std::min(nw, all);
+        return bytes_for(p, nw, nw < all);
+    }
     const size_t single = bytes_for(p, all, false);
     if (single <= kRecommendedCap) return single;
     const int64_t nw = std::max<int64_t>(1, (int64_t)(kRecommendedCap / (p.units * p.slot_bytes)));

@@ -47,7 +47,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every device-side wait 
 
 // ---------------------------------------------------------------- slot ----
 // One slot per (chunk, sequence, head), bytes (every tile 1024-byte aligned):
-//   WQ [W ; Q e^G]   128 x 128 bf16, K-major SW128      (A operand of [W;Qg] S)
+//   WQ [Q e^G ; W]   128 x 128 bf16, K-major SW128      (A operand of [Qg;W] S)
 //   KD K e^{Gl-G}    64 (r) x 128 (c) bf16, MN-major     (A operand of Kd^T U)
 //   T                64 x 64 bf16, K-major               (A operand of T V)
 //   P                64 x 64 bf16, K-major               (A operand of P U)
@@ -73,7 +73,7 @@ __device__ __forceinline__ void flag_error(int *err, int code) {
 // are stored straight from registers.
 constexpr int PT = 256;
 constexpr uint32_t PS_LA = 0;                     // log_alpha -> G [64][128] fp32; later A, X
-constexpr uint32_t PS_GA = 34816;                 // [Kg ; Qg] K-major 128 x 128 -> WQ   (34 * 1024)
+constexpr uint32_t PS_GA = 34816;                 // [Qg ; Kg] K-major 128 x 128 -> WQ   (34 * 1024)
 constexpr uint32_t PS_GB = PS_GA + 32768;         // K e^-G K-major 64 x 128; later T (8 KB) + R2
 constexpr uint32_t PS_SMALL = PS_GB + 16384;      // invq[64] invk[64] beta[64] eGl[128]
 constexpr uint32_t PS_BAR = PS_SMALL + 1280;      // la, mma barriers; tmem base; flags
@@ -248,7 +248,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         __syncthreads();
         const bool safe = sflag[0] == 0;
 
-        // 2. Operands for (row, 8-channel chunk): [Kg ; Qg] and K e^-G to smem, Kd to the slot.
+        // 2. Operands for (row, 8-channel chunk): [Qg ; Kg] and K e^-G to smem, Kd to the slot.
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const int r = rb + 16 * m;
@@ -272,8 +272,8 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                 kn[e] = kk * en;
                 kd[e] = kn[e] * dd[e];
             }
-            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = pack8(kg);
-            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = pack8(qg);
+            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = pack8(qg);
+            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = pack8(kg);
             *reinterpret_cast<uint4 *>(GB + kmaj_chunk(r, c8, 64)) = pack8(kn);
             if (safe) *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = pack8(kd);
         }
@@ -294,7 +294,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
             continue;
         }
 
-        // 3. Gram: TMEM cols [0,64) = [Kg ; Qg] (K e^-G)^T.
+        // 3. Gram: TMEM cols [0,64) = [Qg ; Kg] (K e^-G)^T = [P ; A] before masking.
         if (tid == 0) {
             const uint32_t a = smem_u32(GA), b = smem_u32(GB);
             const uint32_t idg = idesc_bf16(128, 64, false, false);
@@ -306,18 +306,20 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         mma_phase ^= 1;
         tc_fence_after();
 
-        // 4. A (fp32, strictly lower) over the consumed G; P (bf16, lower) to the slot.
+        // 4. P (bf16, lower incl. diagonal; TMEM lanes 0..63) to the slot; A (fp32,
+        //    strictly lower; lanes 64..127) over the consumed G.
         if (warp < 4) {
             const int row = warp * 32 + lane;
             for (int c0 = 0; c0 < C; c0 += 16) {
                 float v[16];
                 tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + c0, v);
                 tmem_wait_ld();
-                if (row < C) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) AF[row * ALD + c0 + i] = (c0 + i < row) ? v[i] : 0.f;
-                } else {
+                if (row >= C) {
                     const int r = row - C;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) AF[r * ALD + c0 + i] = (c0 + i < r) ? v[i] : 0.f;
+                } else {
+                    const int r = row;
                     float lo[8], hi[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
@@ -398,7 +400,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         __syncthreads();
         tc_fence_after();
 
-        // 6. W^T = (K e^G)^T T^T: A = rows 0..63 of [Kg ; Qg] read as an MN-major tile
+        // 6. W^T = (K e^G)^T T^T: A = rows 64..127 of [Qg ; Kg] read as an MN-major tile
         //    (64-column blocks 128 rows apart), B = T; TMEM cols [64,128), lane = channel.
         if (tid == 0) {
             bulk_s2g(gslot + SL_T, TT, 8192);
@@ -406,14 +408,15 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
             const uint32_t idw = idesc_bf16(128, 64, true, false);
 #pragma unroll
             for (int st = 0; st < C / 16; ++st)
-                mma_bf16(tm + 64, sdesc(a + st * 16 * 128, 128 * 128, 1024), kmaj_desc(b, st, 64), idw, st > 0);
+                mma_bf16(tm + 64, sdesc(a + 64 * 128 + st * 16 * 128, 128 * 128, 1024), kmaj_desc(b, st, 64), idw,
+                         st > 0);
             mma_commit(&bars[1]);
         }
         if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
         mma_phase ^= 1;
         tc_fence_after();
 
-        // 7. W rows into the top half of WQ (its Kg rows are consumed).
+        // 7. W rows into the lower half of WQ = [Qg ; W] (its Kg rows are consumed).
         if (warp < 4) {
             const int c = warp * 32 + lane;
             for (int c0 = 0; c0 < C; c0 += 16) {
@@ -422,7 +425,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    *reinterpret_cast<bf16 *>(GA + kmaj_off(c0 + i, c, 128)) = __float2bfloat16_rn(v[i]);
+                    *reinterpret_cast<bf16 *>(GA + kmaj_off(64 + c0 + i, c, 128)) = __float2bfloat16_rn(v[i]);
             }
         }
         fence_async_smem();
@@ -541,12 +544,12 @@ fix_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *
             }
         }
         __syncthreads();
-        // Q e^G -> WQ rows 64..127; K e^{Gl-G} -> KD; D; K e^G kept in sK
+        // Q e^G -> WQ rows 0..63; K e^{Gl-G} -> KD; D; K e^G kept in sK
         for (int idx = tid; idx < C * DK; idx += FT) {
             const int r = idx / DK, c = idx % DK;
             const float gg = sG[r * FLD + c], gl = sG[(C - 1) * FLD + c];
             const float ex = expf(gg);
-            *reinterpret_cast<bf16 *>(g + SL_WQ + kmaj_off(64 + r, c, 128)) = __float2bfloat16_rn(sQ[r * FLD + c] * ex);
+            *reinterpret_cast<bf16 *>(g + SL_WQ + kmaj_off(r, c, 128)) = __float2bfloat16_rn(sQ[r * FLD + c] * ex);
             *reinterpret_cast<bf16 *>(g + SL_KD + mnmaj_off(r, c, 64)) = __float2bfloat16_rn(sK[r * FLD + c] * expf(gl - gg));
         }
         for (int c = tid; c < DK; c += FT) reinterpret_cast<float *>(g + SL_D)[c] = expf(sG[(C - 1) * FLD + c]);
@@ -560,7 +563,7 @@ fix_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *
             const int r = idx / DK, c = idx % DK;
             float acc = 0.f;
             for (int i = 0; i <= r; ++i) acc += sT[r * (C + 1) + i] * sK[i * FLD + c];
-            *reinterpret_cast<bf16 *>(g + SL_WQ + kmaj_off(r, c, 128)) = __float2bfloat16_rn(acc);
+            *reinterpret_cast<bf16 *>(g + SL_WQ + kmaj_off(64 + r, c, 128)) = __float2bfloat16_rn(acc);
         }
         for (int idx = tid; idx < C * C; idx += FT) {
             const int r = idx / C, c = idx % C;
@@ -571,31 +574,26 @@ fix_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *
 }
 
 // ---------------------------------------------------------------- scan ----
-constexpr int ST = 128;
-// Per chunk buffer (bytes): the slot's tiles plus this CTA's V tile. T is
-// followed by the zero half of [0 ; P], so "T then zeros" is the 128-row A
-// operand of X = T V (its lower 64 output rows are zero and unused).
-constexpr uint32_t SB_WQ = 0, SB_KD = 32768, SB_T = 49152, SB_PP = 57344, SB_V = 73728, SB_D = 81920;
-constexpr uint32_t SB_BYTES = 82944;
-constexpr uint32_t SS_S = 2 * SB_BYTES;          // [128 (c)][64 (j)] MN-major bf16 state
+// The big tiles of a chunk (WQ = [Q e^G ; W], K e^{Gl-G}) are triple-buffered
+// and fetched two chunks ahead; the small ones (T, P, the V tile, e^{Gl}) are
+// double-buffered, one chunk ahead. Every product is an M = 128 tcgen05.mma;
+// the 128-row A operands of T V and P U take the 64 rows next to T (before)
+// and P (after) as filler whose output rows are never read, so no zero
+// padding is stored. TMEM lanes: 0..63 hold O = Q e^G S + P U, 64..127 hold
+// W S and T V (their difference is U); Z = Kd^T U fills all 128 lanes.
+constexpr int ST = 160;  // warps 0..3: TMEM-lane epilogues; warp 4: copy and MMA issue
+constexpr uint32_t SA_WQ = 0, SA_KD = 32768, SA_BYTES = 49152;                 // x3
+constexpr uint32_t SB_T = 0, SB_P = 8192, SB_V = 16384, SB_D = 24576, SB_BYTES = 25600;  // x2
+constexpr uint32_t SS_A = 0;
+constexpr uint32_t SS_B = 3 * SA_BYTES;          // T of B0 is preceded by the last A buffer
+constexpr uint32_t SS_S = SS_B + 2 * SB_BYTES;   // [128 (c)][64 (j)] MN-major bf16 state
 constexpr uint32_t SS_U = SS_S + 16384;          // [64 (r)][64 (j)] MN-major bf16 pseudo-values
-constexpr uint32_t SS_BAR = SS_U + 8192;         // full[2], bU, bS, tmem base, flag
-constexpr uint32_t SS_BYTES = SS_BAR + 64;
+constexpr uint32_t SS_BAR = SS_U + 8192;         // fullA[3] fullB[2] bU bS uready sready, tmem base, flag
+constexpr uint32_t SS_BYTES = SS_BAR + 96;
 constexpr uint32_t SS_ALLOC = SS_BYTES + 1024;
-constexpr uint32_t CHUNK_COPY_BYTES = 32768 + 16384 + 8192 + 8192 + 512 + 8192;
+constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 8192 + 512;
 // TMEM columns: X and Y double-buffered, Z
 constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = 256;
-
-__device__ __forceinline__ void issue_chunk_copy(uint8_t *buf, const char *g, const void *tmap_v, int vx,
-                                                 int vy, int vz, uint64_t *bar) {
-    mbar_arrive_expect_tx(bar, CHUNK_COPY_BYTES);
-    bulk_g2s(buf + SB_WQ, g + SL_WQ, 32768, bar);
-    bulk_g2s(buf + SB_KD, g + SL_KD, 16384, bar);
-    bulk_g2s(buf + SB_T, g + SL_T, 8192, bar);
-    bulk_g2s(buf + SB_PP + 8192, g + SL_P, 8192, bar);
-    bulk_g2s(buf + SB_D, g + SL_D, 512, bar);
-    tma_load_3d(buf + SB_V, tmap_v, vx, vy, vz, bar);  // 64 tokens x 64 columns of v, SW128
-}
 
 __global__ void __launch_bounds__(ST, 1)
 scan_kernel(const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ cu, int64_t total,
@@ -615,14 +613,18 @@ scan_kernel(const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restric
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t *sS = sm + SS_S, *sU = sm + SS_U;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SS_BAR);  // full0, full1, bU, bS
-    uint32_t *tbase = reinterpret_cast<uint32_t *>(bars + 4);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SS_BAR);
+    uint64_t *fullA = bars, *fullB = bars + 3, *bU = bars + 5, *bS = bars + 6, *uready = bars + 7,
+             *sready = bars + 8;
+    uint32_t *tbase = reinterpret_cast<uint32_t *>(bars + 9);
     int *sfail = reinterpret_cast<int *>(tbase + 1);
     const size_t sofs = ((size_t)s * H + h) * DK * DV + (size_t)jv * DVT;
-    const int c = tid;  // state row owned by this thread (= TMEM lane)
+    const int c = tid;  // epilogue threads: state row owned (= TMEM lane)
 
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
+        mbar_init(uready, 64);   // the 64 threads of warps 2, 3
+        mbar_init(sready, 128);  // the 128 epilogue threads
         *sfail = 0;
         fence_barrier_init();
     }
@@ -630,20 +632,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restric
         tmem_alloc(tbase, 512);
         tmem_relinquish();
     }
-    // Rows 0..63 of both [0 ; P] tiles stay zero.
-    for (int i = tid; i < 2 * 512; i += ST)
-        reinterpret_cast<uint4 *>(sm + (i >> 9) * SB_BYTES + SB_PP)[i & 511] = make_uint4(0, 0, 0, 0);
-    // Entry state: S0 (or zeros) on the first wave, else the carry.
     float Sr[DVT];
-    {
-        const float *Sin = (j0 == 0) ? S0 : state;
-#pragma unroll
-        for (int q4 = 0; q4 < DVT / 4; ++q4) {
-            float4 x = Sin ? *reinterpret_cast<const float4 *>(Sin + sofs + (size_t)c * DV + 4 * q4)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-            Sr[4 * q4] = x.x; Sr[4 * q4 + 1] = x.y; Sr[4 * q4 + 2] = x.z; Sr[4 * q4 + 3] = x.w;
-        }
-    }
     auto store_state_bf16 = [&]() {
 #pragma unroll
         for (int c8 = 0; c8 < DVT / 8; ++c8) {
@@ -653,149 +642,192 @@ scan_kernel(const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restric
             *reinterpret_cast<uint4 *>(sS + mnmaj_chunk(c, c8, DK)) = pack8(x);
         }
     };
-    store_state_bf16();
-    auto copy_chunk = [&](int jj, int b) {
-        const char *g = slots + ((size_t)((jj - j0) * N + s) * H + h) * SL_BYTES;
-        issue_chunk_copy(sm + b * SB_BYTES, g, &tmap_v, jv * DVT, h, (int)(bos + (int64_t)jj * C), &bars[b]);
+    if (tid < 128) {
+        // Entry state: S0 (or zeros) on the first wave, else the carry.
+        const float *Sin = (j0 == 0) ? S0 : state;
+#pragma unroll
+        for (int q4 = 0; q4 < DVT / 4; ++q4) {
+            float4 x = Sin ? *reinterpret_cast<const float4 *>(Sin + sofs + (size_t)c * DV + 4 * q4)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            Sr[4 * q4] = x.x; Sr[4 * q4 + 1] = x.y; Sr[4 * q4 + 2] = x.z; Sr[4 * q4 + 3] = x.w;
+        }
+        store_state_bf16();
+    }
+    auto slot_of = [&](int jj) { return slots + ((size_t)((jj - j0) * N + s) * H + h) * SL_BYTES; };
+    auto copy_a = [&](int jj) {  // big tiles of chunk jj -> A buffer (jj - j0) % 3
+        const int ab = (jj - j0) % 3;
+        uint8_t *buf = sm + SS_A + ab * SA_BYTES;
+        const char *g = slot_of(jj);
+        mbar_arrive_expect_tx(&fullA[ab], COPY_A);
+        bulk_g2s(buf + SA_WQ, g + SL_WQ, 32768, &fullA[ab]);
+        bulk_g2s(buf + SA_KD, g + SL_KD, 16384, &fullA[ab]);
     };
-    if (nj > 0 && tid == 0) copy_chunk(j0, 0);
+    auto copy_b = [&](int jj) {  // small tiles and the V box of chunk jj -> B buffer (jj - j0) % 2
+        const int bb = (jj - j0) & 1;
+        uint8_t *buf = sm + SS_B + bb * SB_BYTES;
+        const char *g = slot_of(jj);
+        mbar_arrive_expect_tx(&fullB[bb], COPY_B);
+        bulk_g2s(buf + SB_T, g + SL_T, 8192, &fullB[bb]);
+        bulk_g2s(buf + SB_P, g + SL_P, 8192, &fullB[bb]);
+        bulk_g2s(buf + SB_D, g + SL_D, 512, &fullB[bb]);
+        tma_load_3d(buf + SB_V, &tmap_v, jv * DVT, h, (int)(bos + (int64_t)jj * C), &fullB[bb]);
+    };
+    if (nj > 0 && tid == 128) {
+        copy_a(j0);
+        if (nj > 1) copy_a(j0 + 1);
+        copy_b(j0);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tbase;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t id128 = idesc_bf16(128, DVT, false, true);  // K-major A, MN-major B
-    const uint32_t idKd = idesc_bf16(128, DVT, true, true);    // MN-major A (Kd^T)
 
-    if (nj > 0 && tid == 0) {
-        if (!mbar_wait(&bars[0], 0, kWaitNs)) *sfail = 1;
-        const uint32_t a = smem_u32(sm + SB_T), bv = smem_u32(sm + SB_V);
-#pragma unroll
-        for (int st = 0; st < C / 16; ++st) mma_bf16(tm + TM_X, kmaj_desc(a, st, 128), mnmaj_desc(bv, st, C), id128, st > 0);
-    }
-
-    // O = rows 64..127 of Y (buffer yb) for chunk jj -> o (warps 2, 3).
-    auto store_o = [&](int jj, uint32_t yb) {
-        const int nn = (int)((len - (int64_t)jj * C) < C ? (len - (int64_t)jj * C) : C);
-        const int64_t tt = bos + (int64_t)jj * C;
-        const int r = c - 64;
-#pragma unroll
-        for (int c0 = 0; c0 < DVT; c0 += 16) {
-            float yv[16];
-            tmem_ld16(tm + TM_Y + yb + lane_base + c0, yv);
-            tmem_wait_ld();
-            if (r < nn) {
-                bf16 *dst = o + ((size_t)(tt + r) * H + h) * DV + jv * DVT + c0;
-                float lo[8], hi[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    lo[e] = yv[e];
-                    hi[e] = yv[8 + e];
-                }
-                reinterpret_cast<uint4 *>(dst)[0] = pack8(lo);
-                reinterpret_cast<uint4 *>(dst)[1] = pack8(hi);
-            }
-        }
-    };
-
-    bool ok = true;
-    for (int it = 0; it < nj && ok; ++it) {
-        const int jj = j0 + it, b = it & 1;
-        uint8_t *buf = sm + b * SB_BYTES;
-        const uint32_t xb = (uint32_t)b * 64, yb = (uint32_t)b * 64;
-        // Y = [W ; Q e^G] S ; prefetch the next chunk
-        if (tid == 0) {
-            if (!mbar_wait(&bars[b], (it >> 1) & 1, kWaitNs)) *sfail = 1;
-            if (it + 1 < nj) copy_chunk(jj + 1, b ^ 1);
-            const uint32_t a = smem_u32(buf + SB_WQ), bs = smem_u32(sS);
-#pragma unroll
-            for (int st = 0; st < DK / 16; ++st)
-                mma_bf16(tm + TM_Y + yb, kmaj_desc(a, st, 128), mnmaj_desc(bs, st, DK), id128, st > 0);
-            mma_commit(&bars[2]);
-        }
-        // Output of the previous chunk while Y computes.
-        if (warp >= 2 && it > 0) store_o(jj - 1, yb ^ 64);
-        if (!mbar_wait(&bars[2], it & 1, kWaitNs)) *sfail = 1;
-        tc_fence_after();
-        // U = X - Y (rows 0..63 live in lanes 0..63: warps 0 and 1)
-        if (warp < 2) {
-            const int r = c;
-#pragma unroll
-            for (int c0 = 0; c0 < DVT; c0 += 16) {
-                float xv[16], yv[16];
-                tmem_ld16(tm + TM_X + xb + lane_base + c0, xv);
-                tmem_ld16(tm + TM_Y + yb + lane_base + c0, yv);
-                tmem_wait_ld();
-                float lo[8], hi[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    lo[e] = xv[e] - yv[e];
-                    hi[e] = xv[8 + e] - yv[8 + e];
-                }
-                *reinterpret_cast<uint4 *>(sU + mnmaj_chunk(r, c0 / 8, C)) = pack8(lo);
-                *reinterpret_cast<uint4 *>(sU + mnmaj_chunk(r, c0 / 8 + 1, C)) = pack8(hi);
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // O: Y += [0 ; P] U ; Z = Kd^T U ; then X(j+1) = T(j+1) V(j+1)
-        if (tid == 0) {
-            const uint32_t bu = smem_u32(sU);
-            const uint32_t ap = smem_u32(buf + SB_PP), ak = smem_u32(buf + SB_KD);
-#pragma unroll
-            for (int st = 0; st < C / 16; ++st)
-                mma_bf16(tm + TM_Y + yb, kmaj_desc(ap, st, 128), mnmaj_desc(bu, st, C), id128, 1);
-#pragma unroll
-            for (int st = 0; st < C / 16; ++st)
-                mma_bf16(tm + TM_Z, mnmaj_desc(ak, st, C), mnmaj_desc(bu, st, C), idKd, st > 0);
-            mma_commit(&bars[3]);
-            if (it + 1 < nj) {
-                uint8_t *nbuf = sm + (b ^ 1) * SB_BYTES;
-                if (!mbar_wait(&bars[b ^ 1], ((it + 1) >> 1) & 1, kWaitNs)) *sfail = 1;
-                const uint32_t a = smem_u32(nbuf + SB_T), bv = smem_u32(nbuf + SB_V);
+    if (warp == 4) {
+        // ---------------- copy and MMA issue (one thread) ----------------
+        if (lane == 0 && nj > 0) {
+            const uint32_t id128 = idesc_bf16(128, DVT, false, true);  // K-major A, MN-major B
+            const uint32_t idKd = idesc_bf16(128, DVT, true, true);    // MN-major A (Kd^T)
+            // Descriptors of buffer 0; buffer i is i strides further (16-byte units).
+            const uint64_t dWQ = sdesc(smem_u32(sm + SS_A + SA_WQ), 16, 1024);
+            const uint64_t dKD = sdesc(smem_u32(sm + SS_A + SA_KD), C * 128, 1024);
+            // "T then filler": 128 rows starting 64 rows before T (output rows 0..63 unused)
+            const uint64_t dTf = sdesc(smem_u32(sm + SS_B + SB_T) - 8192, 16, 1024);
+            // "P then filler": rows 64..127 read the V tile after P (output rows unused)
+            const uint64_t dP = sdesc(smem_u32(sm + SS_B + SB_P), 16, 1024);
+            const uint64_t dV = sdesc(smem_u32(sm + SS_B + SB_V), C * 128, 1024);
+            const uint64_t dS = sdesc(smem_u32(sS), DK * 128, 1024), dU = sdesc(smem_u32(sU), C * 128, 1024);
+            constexpr uint64_t kA = SA_BYTES >> 4, kB = SB_BYTES >> 4;
+            auto issue_x = [&](int bb, uint32_t xb) {
 #pragma unroll
                 for (int st = 0; st < C / 16; ++st)
-                    mma_bf16(tm + TM_X + (xb ^ 64), kmaj_desc(a, st, 128), mnmaj_desc(bv, st, C), id128, st > 0);
+                    mma_bf16(tm + TM_X + xb, dTf + bb * kB + kmaj_step(st, 128), dV + bb * kB + mnmaj_step(st), id128,
+                             st > 0);
+            };
+            if (!mbar_wait(&fullB[0], 0, kWaitNs)) *sfail = 1;
+            issue_x(0, 0);
+            for (int it = 0; it < nj; ++it) {
+                const int jj = j0 + it, ab = it % 3, bb = it & 1;
+                const uint32_t yb = (uint32_t)bb * 64;
+                bool good = mbar_wait(&fullA[ab], (it / 3) & 1, kWaitNs);
+                if (it > 0) good = good && mbar_wait(sready, (it - 1) & 1, kWaitNs);  // S(jj) in smem
+                tc_fence_after();
+                if (it + 2 < nj) copy_a(jj + 2);
+                if (it + 1 < nj) copy_b(jj + 1);
+                // Y = [Q e^G ; W] S
+                const uint64_t dWQa = dWQ + ab * kA, dKDa = dKD + ab * kA, dPb = dP + bb * kB;
+#pragma unroll
+                for (int st = 0; st < DK / 16; ++st)
+                    mma_bf16(tm + TM_Y + yb, dWQa + kmaj_step(st, 128), dS + mnmaj_step(st), id128, st > 0);
+                mma_commit(bU);
+                good = good && mbar_wait(uready, it & 1, kWaitNs);  // U(jj) in smem
+                tc_fence_after();
+                // O: Y += [P ; filler] U ;  Z = Kd^T U
+#pragma unroll
+                for (int st = 0; st < C / 16; ++st)
+                    mma_bf16(tm + TM_Y + yb, dPb + kmaj_step(st, 128), dU + mnmaj_step(st), id128, 1);
+#pragma unroll
+                for (int st = 0; st < C / 16; ++st)
+                    mma_bf16(tm + TM_Z, dKDa + mnmaj_step(st), dU + mnmaj_step(st), idKd, st > 0);
+                mma_commit(bS);
+                if (it + 1 < nj) {
+                    good = good && mbar_wait(&fullB[bb ^ 1], ((it + 1) >> 1) & 1, kWaitNs);
+                    issue_x(bb ^ 1, yb ^ 64);
+                }
+                if (!good) {
+                    *sfail = 1;
+                    break;
+                }
             }
         }
-        if (!mbar_wait(&bars[3], it & 1, kWaitNs)) *sfail = 1;
-        if (!mbar_wait(&bars[b], (it >> 1) & 1, kWaitNs)) *sfail = 1;  // D of this chunk
-        tc_fence_after();
-        // S' = Diag(e^{G_last}) S + Z   (row c)
-        {
-            const float dc = reinterpret_cast<const float *>(buf + SB_D)[c];
+    } else {
+        // ---------------- epilogues (TMEM lane = thread) ----------------
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        for (int it = 0; it < nj; ++it) {
+            const int jj = j0 + it, bb = it & 1;
+            const uint32_t xb = (uint32_t)bb * 64, yb = (uint32_t)bb * 64;
+            const uint8_t *bbuf = sm + SS_B + bb * SB_BYTES;
+            bool good = true;
+            if (warp >= 2) {
+                // U = T V - W S for rows r = lane - 64 (TMEM lanes 64..127)
+                good = mbar_wait(bU, it & 1, kWaitNs);
+                tc_fence_after();
+                const int r = c - 64;
 #pragma unroll
-            for (int c0 = 0; c0 < DVT; c0 += 16) {
-                float zv[16];
-                tmem_ld16(tm + TM_Z + lane_base + c0, zv);
+                for (int c0 = 0; c0 < DVT; c0 += 32) {
+                    float xv[32], yv[32];
+                    tmem_ld32(tm + TM_X + xb + lane_base + c0, xv);
+                    tmem_ld32(tm + TM_Y + yb + lane_base + c0, yv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        float u8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) u8[e] = xv[q8 * 8 + e] - yv[q8 * 8 + e];
+                        *reinterpret_cast<uint4 *>(sU + mnmaj_chunk(r, c0 / 8 + q8, C)) = pack8(u8);
+                    }
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(uready);
+            }
+            // S' = Diag(e^{G_last}) S + Z  (row c); needs Z(jj) and e^{Gl} of the chunk
+            good = mbar_wait(bS, it & 1, kWaitNs) && good;
+            good = mbar_wait(&fullB[bb], (it >> 1) & 1, kWaitNs) && good;
+            tc_fence_after();
+            const float dc = reinterpret_cast<const float *>(bbuf + SB_D)[c];
+#pragma unroll
+            for (int c0 = 0; c0 < DVT; c0 += 32) {
+                float zv[32];
+                tmem_ld32(tm + TM_Z + lane_base + c0, zv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) Sr[c0 + e] = dc * Sr[c0 + e] + zv[e];
+                for (int e = 0; e < 32; ++e) Sr[c0 + e] = dc * Sr[c0 + e] + zv[e];
             }
             store_state_bf16();
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(sready);
+            // O(jj) = rows 0..63 of Y, complete with Z: warps 0, 1 store it
+            if (warp < 2) {
+                const int nn = (int)((len - (int64_t)jj * C) < C ? (len - (int64_t)jj * C) : C);
+                const int64_t tt = bos + (int64_t)jj * C;
+#pragma unroll
+                for (int c0 = 0; c0 < DVT; c0 += 32) {
+                    float yv[32];
+                    tmem_ld32(tm + TM_Y + yb + lane_base + c0, yv);
+                    tmem_wait_ld();
+                    if (c < nn) {
+                        bf16 *dst = o + ((size_t)(tt + c) * H + h) * DV + jv * DVT + c0;
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            float o8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) o8[e] = yv[q8 * 8 + e];
+                            reinterpret_cast<uint4 *>(dst)[q8] = pack8(o8);
+                        }
+                    }
+                }
+            }
+            if (!good) {
+                *sfail = 1;
+                break;
+            }
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        ok = (*sfail == 0);
     }
-    if (ok && nj > 0 && warp >= 2) store_o(j0 + nj - 1, (uint32_t)((nj - 1) & 1) * 64);
+    tc_fence_before();
+    __syncthreads();
+    const bool ok = (*sfail == 0);
     if (!ok && tid == 0) flag_error(err, 1);
 
     // Exit: final state when the sequence ended in this wave, else the carry.
     float *Sout = (jend == nch) ? S_T : state;
-    if (Sout && ok) {
+    if (Sout && ok && tid < 128) {
 #pragma unroll
         for (int q4 = 0; q4 < DVT / 4; ++q4)
             *reinterpret_cast<float4 *>(Sout + sofs + (size_t)c * DV + 4 * q4) =
                 make_float4(Sr[4 * q4], Sr[4 * q4 + 1], Sr[4 * q4 + 2], Sr[4 * q4 + 3]);
     }
-    tc_fence_before();
-    __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
 }
 

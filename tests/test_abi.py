@@ -51,11 +51,14 @@ def test_status_strings_and_version(lib):
 def test_workspace_queries(lib):
     f = lib.kda_prefill_workspace_size
     m = lib.kda_prefill_workspace_min
-    # valid: grows with heads, recommended >= minimum
+    # valid: recommended >= minimum; the exact (fp32) path's minimum grows with heads
     a = f(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
     b = m(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
     assert a >= b > 0
-    assert f(1, 8192, 8192, 16, 128, 128, 1, 64, 0) < a
+    assert m(1, 8192, 8192, 16, 128, 128, 0, 64, 0) < m(1, 8192, 8192, 32, 128, 128, 0, 64, 0)
+    # tensor-core path: waves sized for L2, never more than the whole problem needs
+    assert f(1, 640, 640, 32, 128, 128, 1, 64, 0) <= f(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
+    assert lib.kda_prefill_launches(1, 8192, 8192, 32, 128, 128, 1, 64, 0, a) >= 3
     # single-chunk problems need no state carry
     assert m(1, 64, 64, 4, 64, 64, 0, 64, 0) == m(1, 1, 1, 4, 64, 64, 0, 64, 0)
     # invalid / unsupported -> 0
