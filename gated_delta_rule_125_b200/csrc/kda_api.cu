@@ -62,17 +62,27 @@ Plan make_plan(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t queue_bytes(const Plan &p, int64_t nw) {
-    return p.tc ? round_up(sizeof(int) * (1 + (size_t)nw * p.units), 1024) : 0;
+    return p.tc ? round_up(sizeof(int) * (2 + (size_t)nw * p.units), 1024) : 0;
 }
 
-// Bytes needed for waves of nw chunks (several waves: with the state carry).
+// One wave buffer: its fallback queue (tensor-core path) and its slots.
+size_t wave_buffer_bytes(const Plan &p, int64_t nw) {
+    return round_up(queue_bytes(p, nw) + (size_t)nw * p.units * p.slot_bytes, 1024);
+}
+
+// Bytes needed for waves of nw chunks. Several waves need the state carry and,
+// on the tensor-core path, two wave buffers (the next wave's prep overlaps the
+// current wave's scan).
 size_t bytes_for(const Plan &p, int64_t nw, bool multi) {
-    return queue_bytes(p, nw) + (multi ? round_up(p.state_bytes, 1024) : 0) + (size_t)nw * p.units * p.slot_bytes;
+    const size_t nbuf = (multi && p.tc) ? 2 : 1;
+    return nbuf * wave_buffer_bytes(p, nw) + (multi ? round_up(p.state_bytes, 1024) : 0);
 }
 
+// The smaller of one wave holding every chunk and the smallest multi-wave plan.
 size_t min_bytes(const Plan &p) {
-    if (p.max_chunks <= 1) return bytes_for(p, 1, false);
-    return bytes_for(p, 1, true);
+    const size_t single = bytes_for(p, std::max<int64_t>(p.max_chunks, 1), false);
+    if (p.max_chunks <= 1) return single;
+    return std::min(single, bytes_for(p, 1, true));
 }
 
 constexpr size_t kRecommendedCap = size_t(512) << 20;
@@ -147,7 +157,9 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
     Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
     const int64_t all = std::max<int64_t>(p.max_chunks, 1);
     if (p.tc) {
-        int64_t nw = std::max<int64_t>(kMinWaveChunks, (int64_t)(kL2SlotBudget / (p.units * p.slot_bytes)));
+        if (bytes_for(p, all, false) <= kL2SlotBudget) return bytes_for(p, all, false);
+        // two wave buffers share the L2 budget
+        int64_t nw = std::max<int64_t>(kMinWaveChunks, (int64_t)(kL2SlotBudget / (2 * p.units * p.slot_bytes)));
         nw = std::min(nw, all);
         return bytes_for(p, nw, nw < all);
     }
@@ -166,7 +178,7 @@ int64_t kda_prefill_launches(int32_t num_seqs, int64_t total_tokens, int32_t max
     const int64_t nw = waves_chunks(p, workspace_bytes);
     if (p.max_chunks == 0) return 1;
     const int64_t waves = (p.max_chunks + nw - 1) / nw;
-    return (p.tc ? 3 : 2) * waves;  // tensor cores: prep, fallback, scan; else prep, scan
+    return (p.tc ? 3 : 2) * waves;  // tensor cores: prep, fallback, scan per wave; else prep, scan
 }
 
 kda_status kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -199,27 +211,30 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
 
     const int64_t nw = waves_chunks(p, workspace_bytes);
     const bool multi = nw < p.max_chunks;
-    char *ws = static_cast<char *>(workspace);
-    int *queue = reinterpret_cast<int *>(ws);
-    ws += queue_bytes(p, nw);
-    a.state = multi ? reinterpret_cast<float *>(ws) : nullptr;
-    ws += multi ? round_up(p.state_bytes, 1024) : 0;
-    a.slots = ws;
-
-    int *err = nullptr;
-    if (p.tc && !(err = kda::device_error_word())) return KDA_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char *ws = static_cast<char *>(workspace);
+
+    if (p.tc) {
+        int *err = kda::device_error_word();
+        if (!err) return KDA_ERR_CUDA;
+        const size_t bb = wave_buffer_bytes(p, nw), qb = queue_bytes(p, nw);
+        char *slots[2] = {ws + qb, ws + bb + qb};
+        int *queue[2] = {reinterpret_cast<int *>(ws), reinterpret_cast<int *>(ws + bb)};
+        a.state = multi ? reinterpret_cast<float *>(ws + 2 * bb) : nullptr;
+        a.slots = slots[0];
+        const int cap = (int)std::min<int64_t>((int64_t)nw * p.units, INT32_MAX);
+        return kda::tc_prefill(a, p.max_chunks, (int)nw, slots, queue, cap, err, st) == cudaSuccess
+                   ? KDA_OK
+                   : KDA_ERR_CUDA;
+    }
+    a.state = multi ? reinterpret_cast<float *>(ws) : nullptr;
+    a.slots = ws + (multi ? round_up(p.state_bytes, 1024) : 0);
     const bool bf16 = dtype == KDA_DTYPE_BF16;
-    const int cap = (int)std::min<int64_t>((int64_t)nw * p.units, INT32_MAX);
-    auto wave = [&](int j0, int n) {
-        return p.tc ? kda::tc_prefill_wave(a, j0, n, queue, cap, err, st)
-                    : kda::simt_prefill_wave(a, j0, n, bf16, st);
-    };
     if (p.max_chunks == 0)  // only empty sequences: S_T = S0
-        return wave(0, 0) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+        return kda::simt_prefill_wave(a, 0, 0, bf16, st) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     for (int64_t j0 = 0; j0 < p.max_chunks; j0 += nw) {
         const int n = (int)std::min<int64_t>(nw, p.max_chunks - j0);
-        if (wave((int)j0, n) != cudaSuccess) return KDA_ERR_CUDA;
+        if (kda::simt_prefill_wave(a, (int)j0, n, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
     }
     return KDA_OK;
 }

@@ -55,11 +55,14 @@ struct PrefillArgs {
 size_t simt_slot_bytes(int dk);
 cudaError_t simt_prefill_wave(const PrefillArgs &a, int j0, int nw, bool bf16, cudaStream_t st);
 
-// tensor-core path (bf16, d_k = d_v = 128). `fix` is the fallback queue
-// ([0] = count, then up to fix_cap slot indices); `err` the device error word.
+// tensor-core path (bf16, d_k = d_v = 128). The prefill runs in waves of `nw`
+// chunks; with several waves, wave buffers 0 and 1 alternate and the prep of
+// the next wave overlaps the scan of the current one on an internal stream.
+// Each buffer has its slots and a queue ([0] fallback count, [1] item counter,
+// then up to `cap` fallback entries); `err` is the device error word.
 size_t tc_slot_bytes();
-cudaError_t tc_prefill_wave(const PrefillArgs &a, int j0, int nw, int *fix, int fix_cap, int *err,
-                            cudaStream_t st);
+cudaError_t tc_prefill(const PrefillArgs &a, int64_t max_chunks, int nw, char *const buf_slots[2],
+                       int *const buf_queue[2], int cap, int *err, cudaStream_t st);
 
 // Address of this device's error word (set by kernels whose bounded waits ran
 // out), or nullptr if it cannot be resolved.

@@ -79,8 +79,8 @@ constexpr uint32_t PS_SMALL = PS_GB + 16384;      // invq[64] invk[64] beta[64] 
 constexpr uint32_t PS_BAR = PS_SMALL + 1280;      // la, mma barriers; tmem base; flags
 constexpr uint32_t PS_BYTES = PS_BAR + 64;
 constexpr uint32_t PS_ALLOC = PS_BYTES + 1024;    // + alignment slack
-constexpr int ALD = 65, XLD = 64;                 // row strides of A and X (floats)
-constexpr uint32_t PS_AF = PS_LA, PS_X = PS_LA + 16640;
+constexpr int ALD = 68, XLD = 64;                 // row strides of A and X (floats)
+constexpr uint32_t PS_AF = PS_LA, PS_X = PS_LA + 17408;
 constexpr uint32_t PS_T = PS_GB, PS_R2 = PS_GB + 8192;
 
 struct Item {
@@ -155,7 +155,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     float *invk = invq + 64, *sbeta = invk + 64, *eGl = sbeta + 64;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA
     uint32_t *tbase = reinterpret_cast<uint32_t *>(bars + 2);
-    int *sflag = reinterpret_cast<int *>(tbase + 1);  // [0] unsafe range, [1] wait failed
+    int *sflag = reinterpret_cast<int *>(tbase + 1);  // [0] unsafe range, [1] wait failed, [2] next item
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
@@ -165,7 +165,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(tbase, 128);
+        tmem_alloc(tbase, 256);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -173,30 +173,47 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     tc_fence_after();
     const uint32_t tm = *tbase;
     uint32_t la_phase = 0, mma_phase = 0;
+    const int c8 = tid & 15, rb = tid >> 4;  // thread's 16-byte channel chunk and first row
 
-    for (int id = blockIdx.x; id < items; id += gridDim.x) {
-        Item cur;
-        if (!decode_item(id, cu, total, H, N, j0, cur)) continue;
-        const int n = cur.n;
-        char *gslot = slots + (size_t)cur.slot * SL_BYTES;
-
-        // The previous slot's bulk stores must have left GA / GB before they are rewritten.
+    // Items are claimed from a counter (fix[1]) so that CTAs that start late, e.g.
+    // while another kernel holds SMs, simply find no work left. Thread 0 claims.
+    auto claim = [&]() {
+        Item tmp;
+        int i = atomicAdd(&fix[1], 1);
+        while (i < items && !decode_item(i, cu, total, H, N, j0, tmp)) i = atomicAdd(&fix[1], 1);
+        return i;
+    };
+    // Inputs of an item: log_alpha by one TMA box (thread 0), q and k rows into
+    // registers (rows rb + 16 m, chunk c8), beta into a register (threads < 64).
+    uint4 qraw[4], kraw[4];
+    float bnext = 0.f;
+    auto fetch = [&](const Item &it) {
         if (tid == 0) {
-            bulk_wait_read();
             mbar_arrive_expect_tx(&bars[0], 32768u);
-            tma_load_3d(G, &tmap_la, 0, cur.h, (int)cur.t0, &bars[0]);
+            tma_load_3d(G, &tmap_la, 0, it.h, (int)it.t0, &bars[0]);
         }
-        // q and k rows: thread owns chunk c8 = tid & 15 of rows (tid >> 4) + 16 m.
-        const int c8 = tid & 15, rb = tid >> 4;
-        uint4 qraw[4], kraw[4];
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const int r = rb + 16 * m;
-            const size_t off = ((size_t)(cur.t0 + r) * H + cur.h) * DK + c8 * 8;
-            qraw[m] = (r < n) ? __ldg(reinterpret_cast<const uint4 *>(q + off)) : make_uint4(0, 0, 0, 0);
-            kraw[m] = (r < n) ? __ldg(reinterpret_cast<const uint4 *>(k + off)) : make_uint4(0, 0, 0, 0);
+            const size_t off = ((size_t)(it.t0 + r) * H + it.h) * DK + c8 * 8;
+            qraw[m] = (r < it.n) ? __ldg(reinterpret_cast<const uint4 *>(q + off)) : make_uint4(0, 0, 0, 0);
+            kraw[m] = (r < it.n) ? __ldg(reinterpret_cast<const uint4 *>(k + off)) : make_uint4(0, 0, 0, 0);
         }
-        if (tid < C) sbeta[tid] = (tid < n) ? __ldg(beta + (size_t)(cur.t0 + tid) * H + cur.h) : 0.f;
+        bnext = (tid < it.n) ? __ldg(beta + (size_t)(it.t0 + tid) * H + it.h) : 0.f;
+    };
+
+    if (tid == 0) sflag[2] = claim();
+    __syncthreads();
+    Item cur;
+    int id = sflag[2];
+    if (id < items) {
+        decode_item(id, cu, total, H, N, j0, cur);
+        fetch(cur);
+    }
+    while (id < items) {
+        const int n = cur.n;
+        char *gslot = slots + (size_t)cur.slot * SL_BYTES;
+        if (tid < C) sbeta[tid] = bnext;
 
         // 1a. Row norms: 16 lanes share a row; shuffle-reduce over them.
 #pragma unroll
@@ -245,9 +262,12 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                 if (-gl > kTau) sflag[0] = 1;
             }
         }
+        // GA / GB are rewritten next: the previous slot's bulk stores must have read them.
+        if (tid == 0) bulk_wait_read();
         __syncthreads();
         const bool safe = sflag[0] == 0;
 
+        if (tid == 0) sflag[2] = claim();  // next item, read by all after the sync below
         // 2. Operands for (row, 8-channel chunk): [Qg ; Kg] and K e^-G to smem, Kd to the slot.
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -282,15 +302,21 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         __syncthreads();
         tc_fence_after();
 
+        Item nxt;
+        const int nid = sflag[2];
+        if (nid < items) decode_item(nid, cu, total, H, N, j0, nxt);
         if (!safe) {
             // Decay range too large for e^{-G}: the exact fallback takes this slot.
             if (tid == 0) {
                 const int pos = atomicAdd(fix, 1);
-                if (pos < fix_cap) fix[1 + pos] = cur.slot;
+                if (pos < fix_cap) fix[2 + pos] = cur.slot;
                 else flag_error(err, 2);
                 sflag[0] = 0;
             }
             __syncthreads();
+            if (nid < items) fetch(nxt);
+            id = nid;
+            cur = nxt;
             continue;
         }
 
@@ -317,7 +343,10 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                 if (row >= C) {
                     const int r = row - C;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) AF[r * ALD + c0 + i] = (c0 + i < r) ? v[i] : 0.f;
+                    for (int i4 = 0; i4 < 4; ++i4)
+                        *reinterpret_cast<float4 *>(AF + r * ALD + c0 + 4 * i4) =
+                            make_float4((c0 + 4 * i4 + 0 < r) ? v[4 * i4 + 0] : 0.f, (c0 + 4 * i4 + 1 < r) ? v[4 * i4 + 1] : 0.f,
+                                        (c0 + 4 * i4 + 2 < r) ? v[4 * i4 + 2] : 0.f, (c0 + 4 * i4 + 3 < r) ? v[4 * i4 + 3] : 0.f);
                 } else {
                     const int r = row;
                     float lo[8], hi[8];
@@ -355,7 +384,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
             for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * XLD + 16 * b + cc] = x[rr];
         }
         __syncthreads();
-        // 16-row level: warps 0, 1 build X[16..31][0..15], X[48..63][32..47] (two 8-column halves each).
+        // 16-row level: warps 0, 1 build X[16..31][0..15], warps 2, 3 X[48..63][32..47] (8-column halves).
         if (warp < 4) {
             const int o = (warp >> 1) * 32, nh = (warp & 1) * 8;  // block offset, column half
             float *Rw = R2 + warp * 128;                          // 16 x 8 scratch per warp
@@ -384,7 +413,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                 [&](int r, int nn, float v) { X[(32 + 16 * mt + r) * XLD + 8 * nt + nn] = -v; });
         }
         __syncthreads();
-        // T = X Diag(beta), lower triangle, bf16: B operand of W^T (smem) and the slot's T tile.
+        // T = X Diag(beta), lower triangle, bf16: A operand of W (smem) and the slot's T tile.
         for (int e2 = tid; e2 < C * 8; e2 += PT) {
             const int r = e2 >> 3, cc8 = e2 & 7;
             float t8[8];
@@ -400,32 +429,41 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         __syncthreads();
         tc_fence_after();
 
-        // 6. W^T = (K e^G)^T T^T: A = rows 64..127 of [Qg ; Kg] read as an MN-major tile
-        //    (64-column blocks 128 rows apart), B = T; TMEM cols [64,128), lane = channel.
+        // 6. W = T (K e^G): M = 64 MMA, A = T (K-major), B = rows 64..127 of [Qg ; Kg] read as
+        //    an MN-major tile (64-column blocks 128 rows apart); TMEM cols [64,192), M=64 layout:
+        //    row r in lane (r % 16) + 32 (r / 16).
         if (tid == 0) {
             bulk_s2g(gslot + SL_T, TT, 8192);
-            const uint32_t a = smem_u32(GA), b = smem_u32(TT);
-            const uint32_t idw = idesc_bf16(128, 64, true, false);
+            const uint32_t a = smem_u32(TT), b = smem_u32(GA);
+            const uint32_t idw = idesc_bf16(64, 128, false, true);
 #pragma unroll
             for (int st = 0; st < C / 16; ++st)
-                mma_bf16(tm + 64, sdesc(a + 64 * 128 + st * 16 * 128, 128 * 128, 1024), kmaj_desc(b, st, 64), idw,
+                mma_bf16(tm + 64, kmaj_desc(a, st, 64), sdesc(b + 64 * 128 + st * 16 * 128, 128 * 128, 1024), idw,
                          st > 0);
             mma_commit(&bars[1]);
         }
+        // The log_alpha buffer (A, X) is consumed: fetch the next item's inputs now.
+        if (nid < items) fetch(nxt);
         if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
         mma_phase ^= 1;
         tc_fence_after();
 
-        // 7. W rows into the lower half of WQ = [Qg ; W] (its Kg rows are consumed).
+        // 7. W rows (16-byte chunks) into the lower half of WQ = [Qg ; W] (its Kg rows are consumed).
         if (warp < 4) {
-            const int c = warp * 32 + lane;
-            for (int c0 = 0; c0 < C; c0 += 16) {
-                float v[16];
-                tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + 64 + c0, v);
+            const int r = 16 * warp + (lane & 15);
+            for (int c0 = 0; c0 < DK; c0 += 32) {
+                float v[32];
+                tmem_ld32(tm + 64 + ((uint32_t)(warp * 32) << 16) + c0, v);
                 tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    *reinterpret_cast<bf16 *>(GA + kmaj_off(64 + c0 + i, c, 128)) = __float2bfloat16_rn(v[i]);
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        float w8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) w8[e] = v[q8 * 8 + e];
+                        *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c0 / 8 + q8, 128)) = pack8(w8);
+                    }
+                }
             }
         }
         fence_async_smem();
@@ -437,6 +475,8 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
             bulk_s2g(gslot + SL_WQ, GA, 32768);
             bulk_commit();
         }
+        id = nid;
+        cur = nxt;
     }
     if (tid == 0) {
         bulk_wait_all();
@@ -444,7 +484,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 128);
+    if (warp == 0) tmem_dealloc(tm, 256);
 }
 
 // ----------------------------------------------------------------- fix ----
@@ -464,7 +504,7 @@ fix_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int count = min(fix[0], fix_cap);
     for (int e = blockIdx.x; e < count; e += gridDim.x) {
-        const int slot_id = fix[1 + e];
+        const int slot_id = fix[2 + e];
         const int h = slot_id % H, s = (slot_id / H) % N, jl = slot_id / (H * N);
         int64_t bos, eos;
         seq_bounds(cu, s, total, bos, eos);
@@ -878,42 +918,104 @@ int sm_count() {
     return n;
 }
 
-}  // namespace
-
-size_t tc_slot_bytes() { return SL_BYTES; }
-
-cudaError_t tc_prefill_wave(const PrefillArgs &a, int j0, int nw, int *fix, int fix_cap, int *err,
-                            cudaStream_t st) {
+cudaError_t set_attributes() {
     cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PS_ALLOC);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FS_BYTES);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS_ALLOC);
+    return e;
+}
+
+// Prep (+ exact fallback) of chunks [j0, j0 + nw) into `slots`; `queue` = [fallback count,
+// item counter, fallback entries...].
+cudaError_t tc_prep(const PrefillArgs &a, int j0, int nw, char *slots, int *queue, int cap, int *err,
+                    cudaStream_t st) {
+    CUtensorMap lamap;
+    if (!make_row_map(&lamap, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.total, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(queue, 0, 2 * sizeof(int), st);
     if (e != cudaSuccess) return e;
+    const int sms = sm_count();
+    const int items = nw * a.N * a.H;
+    const int grid = items < 2 * sms ? items : 2 * sms;
+    prep_kernel<<<grid, PT, PS_ALLOC, st>>>((const bf16 *)a.q, (const bf16 *)a.k, lamap, a.beta, a.cu, a.total,
+                                            a.H, a.N, j0, nw, a.l2norm, a.eps, slots, queue, cap, err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    fix_kernel<<<sms, FT, FS_BYTES, st>>>((const bf16 *)a.q, (const bf16 *)a.k, a.log_alpha, a.beta, a.cu,
+                                          a.total, a.H, a.N, j0, a.l2norm, a.eps, slots, queue, cap);
+    return cudaGetLastError();
+}
+
+cudaError_t tc_scan(const PrefillArgs &a, int j0, int nw, const char *slots, int *err, cudaStream_t st) {
     CUtensorMap vmap;
     memset(&vmap, 0, sizeof(vmap));
     if (a.total > 0 && !make_v_map(&vmap, a.v, a.total, a.H)) return cudaErrorInvalidValue;
-    const int sms = sm_count();
-    if (nw > 0) {
-        CUtensorMap lamap;
-        if (!make_row_map(&lamap, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.total, a.H))
-            return cudaErrorInvalidValue;
-        e = cudaMemsetAsync(fix, 0, sizeof(int), st);
-        if (e != cudaSuccess) return e;
-        const int items = nw * a.N * a.H;
-        const int grid = items < 2 * sms ? items : 2 * sms;
-        prep_kernel<<<grid, PT, PS_ALLOC, st>>>((const bf16 *)a.q, (const bf16 *)a.k, lamap, a.beta, a.cu,
-                                                a.total, a.H, a.N, j0, nw, a.l2norm, a.eps, a.slots, fix,
-                                                fix_cap, err);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        fix_kernel<<<sms, FT, FS_BYTES, st>>>((const bf16 *)a.q, (const bf16 *)a.k, a.log_alpha, a.beta,
-                                              a.cu, a.total, a.H, a.N, j0, a.l2norm, a.eps, a.slots,
-                                              fix, fix_cap);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    scan_kernel<<<dim3(DV / DVT, a.N, a.H), ST, SS_ALLOC, st>>>(
-        vmap, a.cu, a.total, a.H, a.N, j0, nw, a.slots, a.S0, a.state, a.S_T, (bf16 *)a.o, err);
+    scan_kernel<<<dim3(DV / DVT, a.N, a.H), ST, SS_ALLOC, st>>>(vmap, a.cu, a.total, a.H, a.N, j0, nw, slots,
+                                                                a.S0, a.state, a.S_T, (bf16 *)a.o, err);
     return cudaGetLastError();
+}
+
+// Per-device side stream and events for overlapping the prep of wave w+1 with
+// the scan of wave w. Created on first use and kept for the process lifetime;
+// the enqueue sequence of a call holds the mutex so that calls from several
+// host threads do not interleave their use of the shared events.
+struct Overlap {
+    cudaStream_t side = nullptr;
+    cudaEvent_t start = nullptr, prep[2] = {nullptr, nullptr}, scan[2] = {nullptr, nullptr};
+    bool ok = false;
+};
+std::mutex g_overlap_mu;
+Overlap g_overlap[64];
+
+Overlap *overlap_for_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    Overlap &o = g_overlap[dev];
+    if (!o.ok) {
+        const unsigned f = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&o.side, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&o.start, f) != cudaSuccess ||
+            cudaEventCreateWithFlags(&o.prep[0], f) != cudaSuccess ||
+            cudaEventCreateWithFlags(&o.prep[1], f) != cudaSuccess ||
+            cudaEventCreateWithFlags(&o.scan[0], f) != cudaSuccess ||
+            cudaEventCreateWithFlags(&o.scan[1], f) != cudaSuccess)
+            return nullptr;
+        o.ok = true;
+    }
+    return &o;
+}
+
+}  // namespace
+
+size_t tc_slot_bytes() { return SL_BYTES; }
+
+cudaError_t tc_prefill(const PrefillArgs &a, int64_t max_chunks, int nw, char *const buf_slots[2],
+                       int *const buf_queue[2], int cap, int *err, cudaStream_t st) {
+    cudaError_t e = set_attributes();
+    if (e != cudaSuccess) return e;
+    if (max_chunks == 0) return tc_scan(a, 0, 0, buf_slots[0], err, st);  // only empty sequences
+    if (nw >= max_chunks) {  // one wave: everything on the caller's stream
+        if ((e = tc_prep(a, 0, (int)max_chunks, buf_slots[0], buf_queue[0], cap, err, st)) != cudaSuccess) return e;
+        return tc_scan(a, 0, (int)max_chunks, buf_slots[0], err, st);
+    }
+    std::lock_guard<std::mutex> lock(g_overlap_mu);
+    Overlap *ov = overlap_for_device();
+    if (!ov) return cudaErrorInitializationError;
+    if ((e = cudaEventRecord(ov->start, st)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(ov->side, ov->start, 0)) != cudaSuccess) return e;
+    int w = 0;
+    for (int64_t j0 = 0; j0 < max_chunks; j0 += nw, ++w) {
+        const int n = (int)((max_chunks - j0) < nw ? (max_chunks - j0) : nw);
+        const int b = w & 1;
+        if (w >= 2 && (e = cudaStreamWaitEvent(ov->side, ov->scan[b], 0)) != cudaSuccess) return e;
+        if ((e = tc_prep(a, (int)j0, n, buf_slots[b], buf_queue[b], cap, err, ov->side)) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(ov->prep[b], ov->side)) != cudaSuccess) return e;
+        if ((e = cudaStreamWaitEvent(st, ov->prep[b], 0)) != cudaSuccess) return e;
+        if ((e = tc_scan(a, (int)j0, n, buf_slots[b], err, st)) != cudaSuccess) return e;
+        if ((e = cudaEventRecord(ov->scan[b], st)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace kda

@@ -135,8 +135,9 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
  * allocated: no cudaMalloc, cudaFree or allocating library call.
  * - Limit: problems whose kda_prefill_workspace_min() exceeds
  *   KDA_NOALLOC_SCRATCH_BYTES are refused with KDA_ERR_WORKSPACE before
- *   anything is enqueued (at d_k = d_v = 128: about num_seqs * H <= 240 on the
- *   tensor-core path; larger batches run as more, smaller waves).
+ *   anything is enqueued (at d_k = d_v = 128 on the tensor-core path: any
+ *   problem whose chunks all fit one wave, else about num_seqs * H <= 160;
+ *   larger problems run as more, smaller waves).
  * - The first call on a device resolves the array's address on that device
  *   (with that device current); make that first call before any stream
  *   capture begins.
