@@ -31,16 +31,20 @@ kda_status check_prefill_shape(int32_t num_seqs, int64_t total_tokens, int32_t H
     return KDA_OK;
 }
 
-// How the prefill splits into waves for a given workspace. Workspace layout:
-//   [fallback queue: 1 + slots-per-wave ints, 1 KiB aligned]  (tensor-core path)
-//   [state carry: N*H*dk*dv fp32]                             (several waves only)
-//   [slots of one wave]
+// How the prefill uses its workspace.
+// CUDA-core path: it runs in waves of chunks; workspace = [state carry: N*H*dk*dv
+// fp32 (several waves only)][slots of one wave].
+// Tensor-core path: one persistent kernel; workspace = the schedule tables and
+// a ring of R slots for each of `streams` streams (more slots: the chunk
+// preparation runs further ahead of the scan).
 struct Plan {
     bool tc;             // tensor-core path
     int64_t max_chunks;  // chunks of the longest sequence
-    size_t slot_bytes;   // per (chunk, sequence, head)
+    size_t slot_bytes;   // per (chunk, sequence, head), CUDA-core path
     size_t units;        // N * H
-    size_t state_bytes;  // running-state carry between waves
+    size_t state_bytes;  // running-state carry between waves, CUDA-core path
+    int streams;         // tensor-core path: scan streams
+    int64_t max_len;     // tensor-core path: bound on a stream's chunk count
 };
 
 bool use_tc(kda_dtype dtype, int32_t dk, int32_t dv, uint32_t flags) {
@@ -53,44 +57,39 @@ Plan make_plan(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32
     p.tc = use_tc(dtype, dk, dv, flags);
     int64_t L = (max_seqlen > 0) ? std::min<int64_t>(max_seqlen, total_tokens) : total_tokens;
     p.max_chunks = (L + kda::kChunk - 1) / kda::kChunk;
-    p.slot_bytes = p.tc ? kda::tc_slot_bytes() : kda::simt_slot_bytes(dk);
+    p.slot_bytes = kda::simt_slot_bytes(dk);
     p.units = (size_t)num_seqs * H;
     p.state_bytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
+    p.streams = (int)std::min<size_t>(p.units, (size_t)kda::kTcMaxStreams);
+    p.max_len = (int64_t)((p.units + p.streams - 1) / p.streams) * std::max<int64_t>(p.max_chunks, 1);
     return p;
 }
 
+// Tensor-core path: recommended and smallest ring (slots per stream).
+constexpr int64_t kRingMin = 4;
+int tc_ring(const Plan &p, int64_t want) {
+    return (int)std::max<int64_t>(1, std::min<int64_t>({want, (int64_t)kda::tc_max_ring(), p.max_len}));
+}
+size_t tc_bytes(const Plan &p, int R) { return kda::tc_workspace_bytes((long long)p.units, p.streams, R); }
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t queue_bytes(const Plan &p, int64_t nw) {
-    return p.tc ? round_up(sizeof(int) * (2 + (size_t)nw * p.units), 1024) : 0;
-}
-
-// One wave buffer: its fallback queue (tensor-core path) and its slots.
-size_t wave_buffer_bytes(const Plan &p, int64_t nw) {
-    return round_up(queue_bytes(p, nw) + (size_t)nw * p.units * p.slot_bytes, 1024);
-}
-
-// Bytes needed for waves of nw chunks. Several waves need the state carry and,
-// on the tensor-core path, two wave buffers (the next wave's prep overlaps the
-// current wave's scan).
+// CUDA-core path: bytes needed for waves of nw chunks (several waves also
+// need the state carry).
 size_t bytes_for(const Plan &p, int64_t nw, bool multi) {
-    const size_t nbuf = (multi && p.tc) ? 2 : 1;
-    return nbuf * wave_buffer_bytes(p, nw) + (multi ? round_up(p.state_bytes, 1024) : 0);
+    return round_up((size_t)nw * p.units * p.slot_bytes, 1024) + (multi ? round_up(p.state_bytes, 1024) : 0);
 }
 
-// The smaller of one wave holding every chunk and the smallest multi-wave plan.
+// CUDA-core path: the smaller of one wave holding every chunk and the smallest
+// multi-wave plan. Tensor-core path: the smallest ring.
 size_t min_bytes(const Plan &p) {
+    if (p.tc) return tc_bytes(p, tc_ring(p, kRingMin));
     const size_t single = bytes_for(p, std::max<int64_t>(p.max_chunks, 1), false);
     if (p.max_chunks <= 1) return single;
     return std::min(single, bytes_for(p, 1, true));
 }
 
 constexpr size_t kRecommendedCap = size_t(512) << 20;
-// Tensor-core path: a wave's slots are sized to stay resident in L2 (126 MB)
-// between the prep kernel that writes them and the scan that reads them, with
-// at least 16 chunks per wave so the state carry between waves stays cheap.
-constexpr size_t kL2SlotBudget = size_t(48) << 20;
-constexpr int64_t kMinWaveChunks = 16;
 
 // Chunks per wave for a workspace of `bytes` (>= min_bytes(p)).
 int64_t waves_chunks(const Plan &p, size_t bytes) {
@@ -156,13 +155,7 @@ size_t kda_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
     if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return 0;
     Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
     const int64_t all = std::max<int64_t>(p.max_chunks, 1);
-    if (p.tc) {
-        if (bytes_for(p, all, false) <= kL2SlotBudget) return bytes_for(p, all, false);
-        // two wave buffers share the L2 budget
-        int64_t nw = std::max<int64_t>(kMinWaveChunks, (int64_t)(kL2SlotBudget / (2 * p.units * p.slot_bytes)));
-        nw = std::min(nw, all);
-        return bytes_for(p, nw, nw < all);
-    }
+    if (p.tc) return tc_bytes(p, tc_ring(p, kda::tc_max_ring()));
     const size_t single = bytes_for(p, all, false);
     if (single <= kRecommendedCap) return single;
     const int64_t nw = std::max<int64_t>(1, (int64_t)(kRecommendedCap / (p.units * p.slot_bytes)));
@@ -175,10 +168,11 @@ int64_t kda_prefill_launches(int32_t num_seqs, int64_t total_tokens, int32_t max
     if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return -1;
     Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
     if (workspace_bytes < min_bytes(p)) return -1;
+    if (p.tc) return 2;  // planning kernel + persistent prefill kernel
     const int64_t nw = waves_chunks(p, workspace_bytes);
     if (p.max_chunks == 0) return 1;
     const int64_t waves = (p.max_chunks + nw - 1) / nw;
-    return (p.tc ? 3 : 2) * waves;  // tensor cores: prep, fallback, scan per wave; else prep, scan
+    return 2 * waves;  // prep, scan per wave
 }
 
 kda_status kda_prefill(const void *q, const void *k, const void *v, const float *log_alpha,
@@ -209,24 +203,18 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
     a.o = o; a.S_T = S_T;
     a.slot_bytes = p.slot_bytes;
 
-    const int64_t nw = waves_chunks(p, workspace_bytes);
-    const bool multi = nw < p.max_chunks;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
 
     if (p.tc) {
         int *err = kda::device_error_word();
         if (!err) return KDA_ERR_CUDA;
-        const size_t bb = wave_buffer_bytes(p, nw), qb = queue_bytes(p, nw);
-        char *slots[2] = {ws + qb, ws + bb + qb};
-        int *queue[2] = {reinterpret_cast<int *>(ws), reinterpret_cast<int *>(ws + bb)};
-        a.state = multi ? reinterpret_cast<float *>(ws + 2 * bb) : nullptr;
-        a.slots = slots[0];
-        const int cap = (int)std::min<int64_t>((int64_t)nw * p.units, INT32_MAX);
-        return kda::tc_prefill(a, p.max_chunks, (int)nw, slots, queue, cap, err, st) == cudaSuccess
-                   ? KDA_OK
-                   : KDA_ERR_CUDA;
+        a.state = nullptr;
+        a.slots = nullptr;
+        return kda::tc_prefill(a, ws, workspace_bytes, p.streams, err, st) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
     }
+    const int64_t nw = waves_chunks(p, workspace_bytes);
+    const bool multi = nw < p.max_chunks;
     a.state = multi ? reinterpret_cast<float *>(ws) : nullptr;
     a.slots = ws + (multi ? round_up(p.state_bytes, 1024) : 0);
     const bool bf16 = dtype == KDA_DTYPE_BF16;

@@ -55,14 +55,15 @@ struct PrefillArgs {
 size_t simt_slot_bytes(int dk);
 cudaError_t simt_prefill_wave(const PrefillArgs &a, int j0, int nw, bool bf16, cudaStream_t st);
 
-// tensor-core path (bf16, d_k = d_v = 128). The prefill runs in waves of `nw`
-// chunks; with several waves, wave buffers 0 and 1 alternate and the prep of
-// the next wave overlaps the scan of the current one on an internal stream.
-// Each buffer has its slots and a queue ([0] fallback count, [1] item counter,
-// then up to `cap` fallback entries); `err` is the device error word.
-size_t tc_slot_bytes();
-cudaError_t tc_prefill(const PrefillArgs &a, int64_t max_chunks, int nw, char *const buf_slots[2],
-                       int *const buf_queue[2], int cap, int *err, cudaStream_t st);
+// tensor-core path (bf16, d_k = d_v = 128): one planning kernel and one
+// persistent cooperative kernel. The (sequence, head) units are dealt to
+// `ns` <= kTcMaxStreams streams, each scanned by two CTAs and fed through a
+// ring of R slots in the workspace; R follows from the workspace size.
+constexpr int kTcMaxStreams = 32;
+size_t tc_workspace_bytes(long long NH, int ns, int R);   // NH = N * H units
+int tc_ring_slots(long long NH, int ns, size_t bytes);   // R for a workspace (capped)
+int tc_max_ring();
+cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, int *err, cudaStream_t st);
 
 // Address of this device's error word (set by kernels whose bounded waits ran
 // out), or nullptr if it cannot be resolved.

@@ -4,25 +4,30 @@
 // Math ("[Kimi-2] Kimi Linear：用 KDA 重写长上下文注意力" §5, the UT transform and the
 // inter-/intra-chunk split; §3 for the per-token update it rearranges). Per chunk
 // with entry state S, G = cumulative sum of log_alpha over the chunk's rows:
-//   Gram:  [A ; P] = [K e^G ; Q e^G] (K e^-G)^T      (masked: A strictly lower, P lower)
+//   Gram:  [P ; A] = [Q e^G ; K e^G] (K e^-G)^T      (masked: P lower, A strictly lower)
 //   solve: T = (I + Diag(beta) A)^{-1} Diag(beta),   W = T (K e^G)
 //   scan:  U = T V - W S,  O = (Q e^G) S + P U,  S' = Diag(e^{G_last}) S + (K e^{G_last-G})^T U
 //
-// Two kernels per wave of chunks, plus an exact fallback:
-//  * prep_kernel (one CTA per chunk x head, all chunks of the wave in parallel):
-//    L2 norm, G, the exponentiated operands, the Gram on the tensor cores
-//    (one M=128 tcgen05.mma stacking K e^G over Q e^G), the 64x64 triangular
-//    solve on the CUDA cores (16x16 blocks), W^T = (K e^G)^T T^T on the tensor
-//    cores, and the whole workspace slot assembled in shared memory in the
-//    scan's operand layout and written with one TMA bulk store.
-//    The factorisation e^{G_r - G_i} = e^{G_r} e^{-G_i} needs e^{-G} to stay
-//    finite; chunks whose decay range exceeds kTau are queued instead.
-//  * fix_kernel: recomputes queued chunks in fp32 with element-wise exponents.
-//  * scan_kernel (one CTA per sequence x head x 64-column tile of d_v): the
-//    slot of chunk j+1 arrives by TMA bulk copy while chunk j computes; all
-//    products are M=128 tcgen05.mma with fp32 accumulators in TMEM; the fp32
-//    state lives in registers (thread = state row = TMEM lane) and a bf16 copy
-//    in shared memory feeds the next chunk's products.
+// One persistent kernel per call, after a one-CTA planning kernel:
+//  * The (sequence, head) units are dealt round-robin to NS streams. Scan
+//    CTAs 2 st and 2 st + 1 walk stream st's units chunk by chunk, each for 64
+//    of the 128 state columns; the fp32 state stays on chip for a whole unit.
+//    All products are M = 128 tcgen05.mma with fp32 accumulators in TMEM.
+//  * Every other CTA runs two prep engines of 256 threads. An engine claims
+//    the next (stream, position) item in a global order, computes that
+//    chunk's operands (L2 norm, G, the Gram on the tensor cores, the 64 x 64
+//    triangular solve, W on the tensor cores) and publishes them in the
+//    stream's ring of R slots in the workspace (L2-resident).
+//  * Ring handshake: a slot carries a ready generation (set by the engine
+//    with a gpu-scope release after its stores completed) and a release count
+//    (two per generation, one from each scan CTA of the stream once the
+//    slot's bytes are in its shared memory). The kernel is launched
+//    cooperatively, so scan and prep CTAs are co-resident and these waits
+//    always end; each is bounded all the same (2 s), and one that runs out
+//    sets the device error word and an abort flag that ends the others.
+//  * The factorisation e^{G_r - G_i} = e^{G_r} e^{-G_i} needs e^{-G} finite:
+//    for a chunk whose decay range exceeds kTau the engine builds P and A with
+//    element-wise exponents (all <= 1) instead of the Gram MMA.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <string.h>
@@ -41,65 +46,236 @@ using bf16 = __nv_bfloat16;
 constexpr int C = kChunk;  // 64
 constexpr int DK = 128;
 constexpr int DV = 128;
-constexpr int DVT = 64;                    // state columns per scan CTA
-constexpr float kTau = 60.f;               // largest per-chunk decay range for the factorised Gram
+constexpr int DVT = 64;                      // state columns per scan CTA
+constexpr float kTau = 60.f;                 // largest per-chunk decay range for the factorised Gram
 constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every device-side wait (2 s)
+constexpr int kThreads = 512;                // per CTA: two prep engines, or one scan CTA
+constexpr int kMaxRing = 16;                 // ring slots per stream, upper bound (~34 MB at 32 streams)
 
 // ---------------------------------------------------------------- slot ----
-// One slot per (chunk, sequence, head), bytes (every tile 1024-byte aligned):
+// One ring slot per item, bytes (every tile 1024-byte aligned):
 //   WQ [Q e^G ; W]   128 x 128 bf16, K-major SW128      (A operand of [Qg;W] S)
 //   KD K e^{Gl-G}    64 (r) x 128 (c) bf16, MN-major     (A operand of Kd^T U)
 //   T                64 x 64 bf16, K-major               (A operand of T V)
 //   P                64 x 64 bf16, K-major               (A operand of P U)
 //   D  e^{G_last}    128 fp32
 constexpr uint32_t SL_WQ = 0, SL_KD = 32768, SL_T = 49152, SL_P = 57344, SL_D = 65536;
-constexpr uint32_t SL_USED = 66048, SL_BYTES = 66560;
+constexpr uint32_t SL_BYTES = 66560;
 
-__device__ __forceinline__ void load8_bf16(const bf16 *p, float (&x)[8]) {
-    unpack8(__ldg(reinterpret_cast<const uint4 *>(p)), x);
-}
+// ----------------------------------------------------------- workspace ----
+// [header 256 B][L: int64 per stream][order: int32 per stream] (1 KiB)
+// [ustart: int64 per unit][nch: int32 per unit] (1 KiB aligned)
+// [ready: int32 x kMaxStreams*kMaxRing][freed: same][ring: NS*R slots]
+struct Hdr {
+    unsigned long long claim;  // next item to claim
+    long long total;           // items over all streams
+    long long maxlen;          // positions of the longest stream
+    int uniform;               // every stream has the same length
+    int abort_flag;            // a bounded wait of this call gave up
+};
+constexpr size_t WS_L = 256, WS_ORDER = 768, WS_USTART = 1024;
+constexpr size_t kFlagInts = (size_t)kTcMaxStreams * kMaxRing;
 
-// Records a device-side failure (first one wins) for kda_device_error().
+__host__ __device__ inline size_t ru1024(size_t x) { return (x + 1023) & ~size_t(1023); }
+__host__ __device__ inline size_t ws_nch(long long NH) { return WS_USTART + 8 * (size_t)NH; }
+__host__ __device__ inline size_t ws_flags(long long NH) { return ru1024(ws_nch(NH) + 4 * (size_t)NH); }
+__host__ __device__ inline size_t ws_ring(long long NH) { return ws_flags(NH) + 2 * kFlagInts * sizeof(int); }
+
+struct FusedParams {
+    CUtensorMap tmap_la;  // log_alpha [T][H][128] fp32, box 128 x 1 x 64
+    CUtensorMap tmap_v;   // v [T][H][128] bf16, box 64 x 1 x 64, SW128
+    const bf16 *q, *k;
+    const float *beta, *S0;
+    const int32_t *cu;
+    float *S_T;
+    bf16 *o;
+    char *ws;
+    int *err;
+    long long total;  // tokens
+    int N, H, ns, R, l2norm;
+    float eps;
+};
+
 __device__ __forceinline__ void flag_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
+// A bounded wait gave up: record it and make every other wait of the call end.
+__device__ __forceinline__ void fail_call(const FusedParams &P) {
+    Hdr *hd = reinterpret_cast<Hdr *>(P.ws);
+    atomicExch(&hd->abort_flag, 1);
+    flag_error(P.err, 1);
+}
+// Wait until *flag >= target (gpu-scope acquire); false on abort or after kWaitNs.
+__device__ __forceinline__ bool wait_flag_geq(const int *flag, int target, const int *abort_flag) {
+    if (ld_acquire_gpu(flag) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(100);
+        if (ld_acquire_gpu(flag) >= target) return true;
+        if (ld_relaxed_gpu(abort_flag) || globaltimer_ns() - t0 > kWaitNs) return false;
+    }
+}
+
+// --------------------------------------------------------------- plan ----
+// One CTA: chunks per unit, each unit's first position in its stream (units
+// st, st + NS, ... in order), stream lengths L, the streams ordered by
+// decreasing length, and zeroed counters and ring flags.
+constexpr int PLAN_T = 1024;
+__global__ void __launch_bounds__(PLAN_T)
+plan_kernel(const int32_t *__restrict__ cu, long long total, int N, int H, int ns, char *__restrict__ ws) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long NH = (long long)N * H;
+    Hdr *hd = reinterpret_cast<Hdr *>(ws);
+    long long *L = reinterpret_cast<long long *>(ws + WS_L);
+    int *order = reinterpret_cast<int *>(ws + WS_ORDER);
+    long long *ustart = reinterpret_cast<long long *>(ws + WS_USTART);
+    int *nch = reinterpret_cast<int *>(ws + ws_nch(NH));
+    int *flags = reinterpret_cast<int *>(ws + ws_flags(NH));
+    for (long long u = tid; u < NH; u += PLAN_T) {
+        int64_t bos, eos;
+        seq_bounds(cu, (int)(u / H), total, bos, eos);
+        nch[u] = (int)((eos - bos + C - 1) / C);
+    }
+    for (size_t i = tid; i < 2 * kFlagInts; i += PLAN_T) flags[i] = 0;
+    __syncthreads();
+    // one warp per stream: lanes own contiguous runs of the stream's units
+    for (int st = warp; st < ns; st += PLAN_T / 32) {
+        const long long K = (NH - st + ns - 1) / ns;
+        const long long per = (K + 31) / 32, k0 = lane * per, k1 = (k0 + per < K) ? k0 + per : K;
+        long long sum = 0;
+        for (long long kk = k0; kk < k1; ++kk) sum += nch[st + kk * ns];
+        long long incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        long long acc = incl - sum;
+        for (long long kk = k0; kk < k1; ++kk) {
+            ustart[st + kk * ns] = acc;
+            acc += nch[st + kk * ns];
+        }
+        if (lane == 31) L[st] = incl;
+    }
+    __syncthreads();
+    if (tid < ns) {
+        int rank = 0;
+        for (int j = 0; j < ns; ++j) rank += (L[j] > L[tid]) || (L[j] == L[tid] && j < tid);
+        order[rank] = tid;
+    }
+    if (tid == 0) {
+        long long tot = 0, mx = 0, mn = L[0];
+        for (int j = 0; j < ns; ++j) {
+            tot += L[j];
+            mx = L[j] > mx ? L[j] : mx;
+            mn = L[j] < mn ? L[j] : mn;
+        }
+        hd->claim = 0;
+        hd->total = tot;
+        hd->maxlen = mx;
+        hd->uniform = (mx == mn);
+        hd->abort_flag = 0;
+    }
+}
+
+// ------------------------------------------------------ shared memory ----
+// Prep engine (one per 256 threads, two per CTA):
+constexpr int PT = 256;
+constexpr uint32_t PS_LA = 0;                  // log_alpha -> G [64][128] fp32; later A/X, R2, T
+constexpr uint32_t PS_GA = 32768;              // [Qg ; Kg] K-major 128 x 128 -> WQ
+constexpr uint32_t PS_GB = PS_GA + 32768;      // q of the next item, then K e^-G (K-major 64 x 128)
+constexpr uint32_t PS_KS = PS_GB + 16384;      // k of the next item (K-major 64 x 128)
+constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[64] eGl[128]
+constexpr uint32_t PS_BAR = PS_SMALL + 1280;   // la, mma barriers; 3 item records; flags
+constexpr uint32_t PS_BYTES = PS_BAR + 128;
+constexpr uint32_t PS_STRIDE = 100352;         // engine 1 starts here (1024-aligned)
+constexpr int ALD = 68;                        // row stride of A / X (floats)
+constexpr uint32_t PS_AF = PS_LA;              // A, then X in place: 64 x 68 fp32
+constexpr uint32_t PS_R2 = PS_LA + 17408;      // solve scratch, 4 KB
+constexpr uint32_t PS_T = PS_LA + 21504;       // T, 64 x 64 bf16 K-major (1024-aligned)
+static_assert(PS_BYTES <= PS_STRIDE, "prep engine layout");
+
+// Scan CTA: the tiles of a chunk from its ring slot: A (WQ, KD) double-buffered,
+// B (T, P, e^{Gl}) triple-buffered; the V tile, an input independent of the
+// prep, in a ring of four loaded ahead by its own thread.
+constexpr uint32_t SA_WQ = 0, SA_KD = 32768, SA_BYTES = 49152;             // x2
+constexpr uint32_t SB_T = 0, SB_P = 8192, SB_D = 16384, SB_BYTES = 17408;  // x3
+constexpr uint32_t SV_BYTES = 8192;                                        // x4
+constexpr uint32_t SS_A = 0;
+constexpr uint32_t SS_B = 2 * SA_BYTES;         // T of B0 is preceded by the last A buffer
+constexpr uint32_t SS_V = SS_B + 3 * SB_BYTES;
+constexpr uint32_t SS_S = SS_V + 4 * SV_BYTES;  // [128 (c)][64 (j)] MN-major bf16 state
+constexpr uint32_t SS_U = SS_S + 16384;         // [64 (r)][64 (j)] MN-major bf16 pseudo-values
+constexpr uint32_t SS_BAR = SS_U + 8192;        // 24 mbarriers
+constexpr uint32_t SS_BYTES = SS_BAR + 256;
+constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 512;
+// scan mbarrier indices
+constexpr int MB_FULLA = 0, MB_FULLB = 2, MB_FULLV = 5, MB_EMPTYA = 9, MB_EMPTYB = 11, MB_EMPTYV = 14,
+              MB_U = 18, MB_S = 19, MB_O = 20, MB_UREADY = 21, MB_SREADY = 22, MB_FIN = 23, MB_COUNT = 24;
+constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = 256;  // scan TMEM columns (X, Y double-buffered)
+
+// Per-CTA control block after both layouts.
+struct Ctrl {
+    uint32_t tbase;
+    int uniform;
+    long long total, maxlen;
+    long long L[kTcMaxStreams];
+    int order[kTcMaxStreams];
+};
+constexpr uint32_t CTRL_OFF = SS_BYTES > 2 * PS_STRIDE ? SS_BYTES : 2 * PS_STRIDE;
+constexpr uint32_t SMEM_ALLOC = CTRL_OFF + 512 + 1024;  // + alignment slack
+static_assert(2 * PS_STRIDE <= CTRL_OFF, "prep engines overlap the control block");
+static_assert(sizeof(Ctrl) <= 512, "control block");
 
 // ---------------------------------------------------------------- prep ----
-// Persistent, two CTAs per SM (~84 KB shared memory each), each walking the
-// wave's (chunk, sequence, head) items. q and k stay in registers (coalesced
-// 16-byte loads); log_alpha arrives by one tensor-map TMA box and is turned
-// into G in place; that buffer is then reused for A, X and the solve's
-// scratch. The slot's WQ and T tiles leave by TMA bulk stores; KD, P and D
-// are stored straight from registers.
-constexpr int PT = 256;
-constexpr uint32_t PS_LA = 0;                     // log_alpha -> G [64][128] fp32; later A, X
-constexpr uint32_t PS_GA = 34816;                 // [Qg ; Kg] K-major 128 x 128 -> WQ   (34 * 1024)
-constexpr uint32_t PS_GB = PS_GA + 32768;         // K e^-G K-major 64 x 128; later T (8 KB) + R2
-constexpr uint32_t PS_SMALL = PS_GB + 16384;      // invq[64] invk[64] beta[64] eGl[128]
-constexpr uint32_t PS_BAR = PS_SMALL + 1280;      // la, mma barriers; tmem base; flags
-constexpr uint32_t PS_BYTES = PS_BAR + 64;
-constexpr uint32_t PS_ALLOC = PS_BYTES + 1024;    // + alignment slack
-constexpr int ALD = 68, XLD = 64;                 // row strides of A and X (floats)
-constexpr uint32_t PS_AF = PS_LA, PS_X = PS_LA + 17408;
-constexpr uint32_t PS_T = PS_GB, PS_R2 = PS_GB + 8192;
-
-struct Item {
-    int64_t t0;
-    int n, h, slot;
+struct ItemS {
+    long long t0, p;  // first token; position in the stream
+    int n, h, st, valid;
 };
 
-// Item `id` of the wave; false if that chunk lies past its sequence's end.
-__device__ __forceinline__ bool decode_item(int id, const int32_t *cu, int64_t total, int H, int N,
-                                            int j0, Item &it) {
-    const int h = id % H, s = (id / H) % N, jl = id / (H * N);
+// Item g of the global claim order: position-major over the streams still
+// running at that position, longest streams first.
+__device__ bool map_item(unsigned long long g, const FusedParams &P, const Ctrl *ctl, ItemS &it) {
+    if ((long long)g >= ctl->total) return false;
+    const int ns = P.ns;
+    long long p;
+    int i;
+    if (ctl->uniform) {
+        p = (long long)(g / (unsigned long long)ns);
+        i = (int)(g % (unsigned long long)ns);
+    } else {
+        // largest p with sum_st min(L_st, p) <= g
+        long long lo = 0, hi = ctl->maxlen - 1;
+        while (lo < hi) {
+            const long long mid = (lo + hi + 1) >> 1;
+            long long s = 0;
+            for (int t = 0; t < ns; ++t) s += ctl->L[t] < mid ? ctl->L[t] : mid;
+            if (s <= (long long)g) lo = mid;
+            else hi = mid - 1;
+        }
+        p = lo;
+        long long s = 0;
+        for (int t = 0; t < ns; ++t) s += ctl->L[t] < p ? ctl->L[t] : p;
+        i = (int)((long long)g - s);
+    }
+    const int st = ctl->order[i];
+    const long long NH = (long long)P.N * P.H;
+    const long long *ustart = reinterpret_cast<const long long *>(P.ws + WS_USTART);
+    long long lo = 0, hi = (NH - st + ns - 1) / ns - 1;  // last unit of the stream starting at or before p
+    while (lo < hi) {
+        const long long mid = (lo + hi + 1) >> 1;
+        if (ustart[st + mid * ns] <= p) lo = mid;
+        else hi = mid - 1;
+    }
+    const long long u = st + lo * ns;
+    const long long j = p - ustart[u];
     int64_t bos, eos;
-    seq_bounds(cu, s, total, bos, eos);
-    const int64_t j = (int64_t)j0 + jl;
-    if (j * C >= eos - bos) return false;
-    it.n = (int)((eos - bos - j * C) < C ? (eos - bos - j * C) : C);
+    seq_bounds(P.cu, (int)(u / P.H), P.total, bos, eos);
     it.t0 = bos + j * C;
-    it.h = h;
-    it.slot = id;
+    it.n = (int)((eos - it.t0) < C ? (eos - it.t0) : C);
+    it.h = (int)(u % P.H);
+    it.st = st;
+    it.p = p;
     return true;
 }
 
@@ -134,206 +310,278 @@ __device__ __forceinline__ void warp_gemm_16x8(int lane, FA A, FB B, FO out) {
     out(g + 8, 2 * t + 1, acc[3]);
 }
 
-__global__ void __launch_bounds__(PT, 2)
-prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
-            const __grid_constant__ CUtensorMap tmap_la, const float *__restrict__ beta,
-            const int32_t *__restrict__ cu, int64_t total, int H, int N, int j0, int nw, int l2norm,
-            float eps, char *__restrict__ slots, int *__restrict__ fix, int fix_cap,
-            int *__restrict__ err) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int items = nw * N * H;
+// Prep engine e (threads 256 e .. 256 e + 255) with its shared memory `sm` and
+// TMEM columns [tm, tm + 256). Named barriers 1 + e (the engine) and 3 + 2e,
+// 4 + 2e (warp pairs of the solve).
+__device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ctl, int e, uint8_t *sm,
+                                            uint32_t tm) {
+    const int tid = (int)threadIdx.x - PT * e, warp = tid >> 5, lane = tid & 31;
+    const uint32_t bar_id = 1 + e;
+    const int H = P.H, R = P.R;
     float *G = reinterpret_cast<float *>(sm + PS_LA);
     float *AF = reinterpret_cast<float *>(sm + PS_AF);
-    float *X = reinterpret_cast<float *>(sm + PS_X);
     float *R2 = reinterpret_cast<float *>(sm + PS_R2);
+    uint8_t *TT = sm + PS_T;
     uint8_t *GA = sm + PS_GA;
     uint8_t *GB = sm + PS_GB;
-    uint8_t *TT = sm + PS_T;
+    uint8_t *KS = sm + PS_KS;
     float *invq = reinterpret_cast<float *>(sm + PS_SMALL);
     float *invk = invq + 64, *sbeta = invk + 64, *eGl = sbeta + 64;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA
-    uint32_t *tbase = reinterpret_cast<uint32_t *>(bars + 2);
-    int *sflag = reinterpret_cast<int *>(tbase + 1);  // [0] unsafe range, [1] wait failed, [2] next item
-
-    if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
-        sflag[0] = 0;
-        sflag[1] = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tbase, 256);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tm = *tbase;
+    // Item records of iterations it (current), it + 1 (claimed during the Gram)
+    // and it - 1 (published by the store thread) in entries it % 3, ...
+    ItemS *sitem = reinterpret_cast<ItemS *>(bars + 2);
+    int *sflag = reinterpret_cast<int *>(sitem + 3);  // [0] unsafe range, [1] a wait failed
+    Hdr *hd = reinterpret_cast<Hdr *>(P.ws);
+    const long long NH = (long long)P.N * H;
+    int *ready = reinterpret_cast<int *>(P.ws + ws_flags(NH));
+    int *freed = ready + kFlagInts;
+    char *ring = P.ws + ws_ring(NH);
+    auto sync = [&]() { bar_sync(bar_id, PT); };
     uint32_t la_phase = 0, mma_phase = 0;
     const int c8 = tid & 15, rb = tid >> 4;  // thread's 16-byte channel chunk and first row
 
-    // Items are claimed from a counter (fix[1]) so that CTAs that start late, e.g.
-    // while another kernel holds SMs, simply find no work left. Thread 0 claims.
-    auto claim = [&]() {
-        Item tmp;
-        int i = atomicAdd(&fix[1], 1);
-        while (i < items && !decode_item(i, cu, total, H, N, j0, tmp)) i = atomicAdd(&fix[1], 1);
-        return i;
+    auto slot_index = [&](const ItemS &it) { return it.st * R + (int)(it.p % R); };
+    // Thread 128 issues the slot's bulk stores (bulk groups belong to the issuing
+    // thread) and the log_alpha boxes, and publishes each item: after the item's
+    // generic slot stores (ordered before it by the engine's barriers) and its
+    // bulk stores completed, one gpu-scope release of the slot's ready generation.
+    // The previous item is published during the Gram, or at once if the current
+    // item has to wait for its slot (that wait may depend on the previous item).
+    // Thread 160 claims items.
+    constexpr int kStoreTid = 128, kClaimTid = 160;
+    bool slot_ok = false;       // store thread: the current item's slot is known to be free
+    bool prev_pending = false;  // store thread: the previous item is not yet published
+    bool la_pending = false;    // store thread: a log_alpha box is in flight
+    auto publish_prev = [&](const ItemS &pv) {
+        if (!prev_pending) return;
+        bulk_wait_all();
+        fence_proxy_async_global();
+        st_release_gpu(&ready[slot_index(pv)], (int)(pv.p / R) + 1);
+        prev_pending = false;
     };
-    // Inputs of an item: log_alpha by one TMA box (thread 0), q and k rows into
-    // registers (rows rb + 16 m, chunk c8), beta into a register (threads < 64).
-    uint4 qraw[4], kraw[4];
+    auto slot_free = [&](const ItemS &it) {
+        return ld_acquire_gpu(&freed[slot_index(it)]) >= 2 * (int)(it.p / R);
+    };
+    auto claim = [&](ItemS &it) {
+        it.valid = 0;
+        if (ld_relaxed_gpu(&hd->abort_flag)) return;
+        it.valid = map_item(atomicAdd(&hd->claim, 1ull), P, ctl, it) ? 1 : 0;
+    };
+    auto fetch_la = [&](const ItemS &it) {  // store thread: log_alpha rows by one TMA box
+        mbar_arrive_expect_tx(&bars[0], 32768u);
+        tma_load_3d(G, &P.tmap_la, 0, it.h, (int)it.t0, &bars[0]);
+        la_pending = true;
+    };
+    // q and k rows rb + 16 m, chunk c8, by cp.async into GB / KS at the chunk's
+    // place in a K-major SW128 64 x 128 tile (the thread reads back exactly what
+    // it copied; K e^-G later overwrites q in place); rows past the sequence
+    // are zero-filled. beta into a register (threads < 64).
     float bnext = 0.f;
-    auto fetch = [&](const Item &it) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bars[0], 32768u);
-            tma_load_3d(G, &tmap_la, 0, it.h, (int)it.t0, &bars[0]);
-        }
+    auto fetch_qk = [&](const ItemS &it) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const int r = rb + 16 * m;
-            const size_t off = ((size_t)(it.t0 + r) * H + it.h) * DK + c8 * 8;
-            qraw[m] = (r < it.n) ? __ldg(reinterpret_cast<const uint4 *>(q + off)) : make_uint4(0, 0, 0, 0);
-            kraw[m] = (r < it.n) ? __ldg(reinterpret_cast<const uint4 *>(k + off)) : make_uint4(0, 0, 0, 0);
+            const size_t off = ((size_t)(it.t0 + (r < it.n ? r : 0)) * H + it.h) * DK + c8 * 8;
+            const uint32_t bytes = r < it.n ? 16u : 0u;
+            cp_async16(GB + kmaj_chunk(r, c8, 64), P.q + off, bytes);
+            cp_async16(KS + kmaj_chunk(r, c8, 64), P.k + off, bytes);
         }
-        bnext = (tid < it.n) ? __ldg(beta + (size_t)(it.t0 + tid) * H + it.h) : 0.f;
+        cp_async_commit();
+        bnext = (tid < it.n) ? __ldg(P.beta + (size_t)(it.t0 + tid) * H + it.h) : 0.f;
     };
 
-    if (tid == 0) sflag[2] = claim();
-    __syncthreads();
-    Item cur;
-    int id = sflag[2];
-    if (id < items) {
-        decode_item(id, cu, total, H, N, j0, cur);
-        fetch(cur);
-    }
-    while (id < items) {
+    if (tid == kClaimTid) claim(sitem[0]);
+    sync();
+    if (tid == kStoreTid && sitem[0].valid) fetch_la(sitem[0]);
+    if (sitem[0].valid) fetch_qk(sitem[0]);
+    bool failed = false;
+    int iter = 0;
+    for (; sitem[iter % 3].valid; ++iter) {
+        const ItemS &cur = sitem[iter % 3];
+        ItemS &next = sitem[(iter + 1) % 3];
+        const ItemS &prev = sitem[(iter + 2) % 3];
         const int n = cur.n;
-        char *gslot = slots + (size_t)cur.slot * SL_BYTES;
+        char *gslot = ring + (size_t)slot_index(cur) * SL_BYTES;
         if (tid < C) sbeta[tid] = bnext;
+        if (tid == kStoreTid) {
+            bulk_wait_read();  // the previous item's bulk stores no longer read GA
+            // This item's slot is written below: both scan CTAs of the stream must
+            // have released its previous generation.
+            if (!slot_ok) {
+                publish_prev(prev);
+                if (!wait_flag_geq(&freed[slot_index(cur)], 2 * (int)(cur.p / R), &hd->abort_flag)) sflag[1] = 1;
+            }
+            slot_ok = false;
+        }
 
         // 1a. Row norms: 16 lanes share a row; shuffle-reduce over them.
+        cp_async_wait_all();  // this thread's q, k chunks
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
+            const int r = rb + 16 * m;
             float qf[8], kf[8], sq = 0.f, sk = 0.f;
-            unpack8(qraw[m], qf);
-            unpack8(kraw[m], kf);
+            unpack8(*reinterpret_cast<const uint4 *>(GB + kmaj_chunk(r, c8, 64)), qf);
+            unpack8(*reinterpret_cast<const uint4 *>(KS + kmaj_chunk(r, c8, 64)), kf);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                sq += qf[e] * qf[e];
-                sk += kf[e] * kf[e];
+            for (int i = 0; i < 8; ++i) {
+                sq += qf[i] * qf[i];
+                sk += kf[i] * kf[i];
             }
 #pragma unroll
             for (int off = 1; off < 16; off <<= 1) {
                 sq += __shfl_xor_sync(0xffffffffu, sq, off);
                 sk += __shfl_xor_sync(0xffffffffu, sk, off);
             }
-            const int r = rb + 16 * m;
             if (c8 == 0) {
                 const bool live = r < n;
-                invq[r] = !live ? 0.f : (l2norm ? 1.f / fmaxf(sqrtf(sq), eps) : 1.f);
-                invk[r] = !live ? 0.f : (l2norm ? 1.f / fmaxf(sqrtf(sk), eps) : 1.f);
+                invq[r] = !live ? 0.f : (P.l2norm ? 1.f / fmaxf(sqrtf(sq), P.eps) : 1.f);
+                invk[r] = !live ? 0.f : (P.l2norm ? 1.f / fmaxf(sqrtf(sk), P.eps) : 1.f);
             }
         }
-        // 1b. G = cumulative sum of log_alpha over rows, in place: thread (channel,
-        //     half) scans 32 rows in registers; the upper half adds the lower total.
-        if (!mbar_wait(&bars[0], la_phase, kWaitNs)) sflag[1] = 1;
+        // 1b. G = cumulative sum of log_alpha over the rows, in place: one thread per channel.
+        if (tid < DK) {
+            if (!mbar_wait(&bars[0], la_phase, kWaitNs)) sflag[1] = 1;
+            const int c = tid;
+            float run = 0.f;
+#pragma unroll
+            for (int r0 = 0; r0 < C; r0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = (r0 + i < n) ? G[(r0 + i) * DK + c] : 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    run += v[i];
+                    G[(r0 + i) * DK + c] = run;
+                }
+            }
+            eGl[c] = expf(run);
+            if (-run > kTau) sflag[0] = 1;
+        }
         la_phase ^= 1;
-        {
-            const int c = tid & (DK - 1), half = tid >> 7, r0 = half * 32;
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = (r0 + i < n) ? G[(r0 + i) * DK + c] : 0.f;
-#pragma unroll
-            for (int i = 1; i < 32; ++i) v[i] += v[i - 1];
-            if (half == 0) eGl[c] = v[31];
-            __syncthreads();
-            const float base = half ? eGl[c] : 0.f;
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) G[(r0 + i) * DK + c] = v[i] + base;
-            if (half == 1) {
-                const float gl = v[31] + base;
-                eGl[c] = expf(gl);
-                reinterpret_cast<float *>(gslot + SL_D)[c] = eGl[c];
-                if (-gl > kTau) sflag[0] = 1;
-            }
+        sync();
+        if (sflag[1]) {
+            failed = true;
+            break;
         }
-        // GA / GB are rewritten next: the previous slot's bulk stores must have read them.
-        if (tid == 0) bulk_wait_read();
-        __syncthreads();
+        if (tid == kStoreTid) la_pending = false;
         const bool safe = sflag[0] == 0;
 
-        if (tid == 0) sflag[2] = claim();  // next item, read by all after the sync below
-        // 2. Operands for (row, 8-channel chunk): [Qg ; Kg] and K e^-G to smem, Kd to the slot.
+        // 2. Operands for (row, 8-channel chunk): [Qg ; Kg] to GA, K e^-G to GB (over q),
+        //    Kd to the slot, one channel pair at a time (packed as soon as computed).
+        //    Unsafe range: [Q ; K] without exponents (the element-wise Gram needs them).
+        if (safe) {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int r = rb + 16 * m;
-            float kf[8], qf[8];
-            unpack8(kraw[m], kf);
-            unpack8(qraw[m], qf);
-            const float ik = invk[r], iq = invq[r];
-            const float4 g0 = *reinterpret_cast<const float4 *>(G + r * DK + c8 * 8);
-            const float4 g1 = *reinterpret_cast<const float4 *>(G + r * DK + c8 * 8 + 4);
-            const float4 d0 = *reinterpret_cast<const float4 *>(eGl + c8 * 8);
-            const float4 d1 = *reinterpret_cast<const float4 *>(eGl + c8 * 8 + 4);
-            const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            const float dd[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-            float kg[8], qg[8], kn[8], kd[8];
+            for (int m = 0; m < 4; ++m) {
+                const int r = rb + 16 * m;
+                const float ik = invk[r], iq = invq[r];
+                const uint4 qv = *reinterpret_cast<const uint4 *>(GB + kmaj_chunk(r, c8, 64));
+                const uint4 kv = *reinterpret_cast<const uint4 *>(KS + kmaj_chunk(r, c8, 64));
+                const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+                const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+                uint32_t pq[4], pk[4], pn[4], pd[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float ep = __expf(gg[e]), en = __expf(-gg[e]);
-                const float kk = kf[e] * ik;
-                kg[e] = kk * ep;
-                qg[e] = qf[e] * iq * ep;
-                kn[e] = kk * en;
-                kd[e] = kn[e] * dd[e];
+                for (int w = 0; w < 4; ++w) {
+                    const float2 g = *reinterpret_cast<const float2 *>(G + r * DK + c8 * 8 + 2 * w);
+                    const float2 d = *reinterpret_cast<const float2 *>(eGl + c8 * 8 + 2 * w);
+                    const float k0 = __uint_as_float(kw[w] << 16) * ik, k1 = __uint_as_float(kw[w] & 0xFFFF0000u) * ik;
+                    const float q0 = __uint_as_float(qw[w] << 16) * iq, q1 = __uint_as_float(qw[w] & 0xFFFF0000u) * iq;
+                    const float ep0 = __expf(g.x), ep1 = __expf(g.y);
+                    const float n0 = k0 * __expf(-g.x), n1 = k1 * __expf(-g.y);
+                    pq[w] = pack_bf16(q0 * ep0, q1 * ep1);
+                    pk[w] = pack_bf16(k0 * ep0, k1 * ep1);
+                    pn[w] = pack_bf16(n0, n1);
+                    pd[w] = pack_bf16(n0 * d.x, n1 * d.y);
+                }
+                *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
+                *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4 *>(GB + kmaj_chunk(r, c8, 64)) = make_uint4(pn[0], pn[1], pn[2], pn[3]);
+                *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = make_uint4(pd[0], pd[1], pd[2], pd[3]);
             }
-            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = pack8(qg);
-            *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = pack8(kg);
-            *reinterpret_cast<uint4 *>(GB + kmaj_chunk(r, c8, 64)) = pack8(kn);
-            if (safe) *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = pack8(kd);
+        } else {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int r = rb + 16 * m;
+                float kf[8], qf[8], kd[8];
+                unpack8(*reinterpret_cast<const uint4 *>(KS + kmaj_chunk(r, c8, 64)), kf);
+                unpack8(*reinterpret_cast<const uint4 *>(GB + kmaj_chunk(r, c8, 64)), qf);
+                const float ik = invk[r], iq = invq[r];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    kf[i] *= ik;
+                    qf[i] *= iq;
+                    kd[i] = kf[i] * __expf(G[(C - 1) * DK + c8 * 8 + i] - G[r * DK + c8 * 8 + i]);
+                }
+                *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = pack8(qf);
+                *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = pack8(kf);
+                *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = pack8(kd);
+            }
         }
+        if (tid < DK) reinterpret_cast<float *>(gslot + SL_D)[tid] = eGl[tid];
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        sync();
         tc_fence_after();
-
-        Item nxt;
-        const int nid = sflag[2];
-        if (nid < items) decode_item(nid, cu, total, H, N, j0, nxt);
-        if (!safe) {
-            // Decay range too large for e^{-G}: the exact fallback takes this slot.
-            if (tid == 0) {
-                const int pos = atomicAdd(fix, 1);
-                if (pos < fix_cap) fix[2 + pos] = cur.slot;
-                else flag_error(err, 2);
-                sflag[0] = 0;
-            }
-            __syncthreads();
-            if (nid < items) fetch(nxt);
-            id = nid;
-            cur = nxt;
-            continue;
-        }
 
         // 3. Gram: TMEM cols [0,64) = [Qg ; Kg] (K e^-G)^T = [P ; A] before masking.
-        if (tid == 0) {
-            const uint32_t a = smem_u32(GA), b = smem_u32(GB);
-            const uint32_t idg = idesc_bf16(128, 64, false, false);
+        if (safe) {
+            if (tid == 0) {
+                const uint32_t a = smem_u32(GA), b = smem_u32(GB);
+                const uint32_t idg = idesc_bf16(128, 64, false, false);
 #pragma unroll
-            for (int st = 0; st < DK / 16; ++st) mma_bf16(tm, kmaj_desc(a, st, 128), kmaj_desc(b, st, 64), idg, st > 0);
-            mma_commit(&bars[1]);
+                for (int s8 = 0; s8 < DK / 16; ++s8)
+                    mma_bf16(tm, kmaj_desc(a, s8, 128), kmaj_desc(b, s8, 64), idg, s8 > 0);
+                mma_commit(&bars[1]);
+            }
+            if (tid == kClaimTid) claim(next);
+            if (tid == kStoreTid) publish_prev(prev);
+            if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
+            mma_phase ^= 1;
+            tc_fence_after();
+        } else {
+            // Element-wise: row `row` of [Q ; K] against rows i of K, exponents G_r - G_i <= 0.
+            const int row = (warp & 3) * 32 + lane, r = row & (C - 1);
+            const bool isq = row < C;
+            for (int i0 = (warp >> 2) * 32; i0 < (warp >> 2) * 32 + 32; i0 += 16) {
+                float acc[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+                for (int c = 0; c < DK; ++c) {
+                    const float gr = G[r * DK + c];
+                    const float xr = __bfloat162float(*reinterpret_cast<const bf16 *>(GA + kmaj_off(row, c, 128)));
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int ii = i0 + i;
+                        const float ki = __bfloat162float(*reinterpret_cast<const bf16 *>(GA + kmaj_off(64 + ii, c, 128)));
+                        const bool keep = isq ? (ii <= r) : (ii < r);
+                        acc[i] += keep ? xr * ki * __expf(gr - G[ii * DK + c]) : 0.f;
+                    }
+                }
+                tmem_st16(tm + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)i0, acc);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            sync();
+            tc_fence_after();
+            // [Q ; K] -> [Q e^G ; K e^G] in place for the W product.
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int rr = rb + 16 * m, r2 = rr & (C - 1);
+                float x[8];
+                unpack8(*reinterpret_cast<const uint4 *>(GA + kmaj_chunk(rr, c8, 128)), x);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) x[i] *= __expf(G[r2 * DK + c8 * 8 + i]);
+                *reinterpret_cast<uint4 *>(GA + kmaj_chunk(rr, c8, 128)) = pack8(x);
+            }
+            fence_async_smem();
+            if (tid == kClaimTid) claim(next);
+            if (tid == kStoreTid) publish_prev(prev);
+            sync();  // G is overwritten by A below
         }
-        if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
-        mma_phase ^= 1;
-        tc_fence_after();
+        if (tid == 0) sflag[0] = 0;
 
         // 4. P (bf16, lower incl. diagonal; TMEM lanes 0..63) to the slot; A (fp32,
-        //    strictly lower; lanes 64..127) over the consumed G.
+        //    strictly lower, zero elsewhere; lanes 64..127) over the consumed G.
         if (warp < 4) {
             const int row = warp * 32 + lane;
             for (int c0 = 0; c0 < C; c0 += 16) {
@@ -359,94 +607,109 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                     *reinterpret_cast<uint4 *>(gslot + SL_P + kmaj_chunk(r, c0 / 8 + 1, 64)) = pack8(hi);
                 }
             }
-        } else {
-            for (int i = tid - 128; i < C * XLD / 4; i += 128)
-                reinterpret_cast<float4 *>(X)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         tc_fence_before();
-        __syncthreads();
+        sync();
+        // The next item is known (claimed during the Gram): its q, k rows load into
+        // GB (free: the Gram has consumed K e^-G) and KS while this item finishes,
+        // and the store thread checks its slot.
+        if (next.valid) fetch_qk(next);
+        if (tid == kStoreTid && next.valid) slot_ok = slot_free(next);
 
-        // 5. X = (I + Diag(beta) A)^{-1}: diagonal 16x16 blocks by forward substitution,
-        //    then the 2x2 block recursion with tf32 tensor-core products:
-        //    [X11 0; X21 X22] with X21 = -X22 (Diag(beta_2) A21) X11.
-        if (tid < C) {
-            const int b = tid >> 4, cc = tid & 15;
+        // 5. In place, AF (A) becomes X = (I + Diag(beta) A)^{-1}: diagonal 16x16 blocks by
+        //    forward substitution, then the 2x2 block recursion with tf32 tensor-core products:
+        //    [X11 0; X21 X22] with X21 = -X22 (Diag(beta_2) A21) X11, written over A21 once
+        //    A21 is consumed.
+        {
             float x[16];
+            const int b = tid >> 4, cc = tid & 15;
+            if (tid < C) {
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * b + rr;
-                float acc = 0.f;
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int r = 16 * b + rr;
+                    float acc = 0.f;
 #pragma unroll
-                for (int ii = 0; ii < rr; ++ii) acc += AF[r * ALD + 16 * b + ii] * x[ii];
-                x[rr] = (rr == cc) ? 1.f : (rr > cc ? -sbeta[r] * acc : 0.f);
+                    for (int ii = 0; ii < rr; ++ii) acc += AF[r * ALD + 16 * b + ii] * x[ii];
+                    x[rr] = (rr == cc) ? 1.f : (rr > cc ? -sbeta[r] * acc : 0.f);
+                }
             }
+            sync();  // every diagonal block of A has been read
+            if (tid < C) {
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * XLD + 16 * b + cc] = x[rr];
+                for (int rr = 0; rr < 16; ++rr) AF[(16 * b + rr) * ALD + 16 * b + cc] = x[rr];
+            }
         }
-        __syncthreads();
+        sync();
         // 16-row level: warps 0, 1 build X[16..31][0..15], warps 2, 3 X[48..63][32..47] (8-column halves).
         if (warp < 4) {
             const int o = (warp >> 1) * 32, nh = (warp & 1) * 8;  // block offset, column half
             float *Rw = R2 + warp * 128;                          // 16 x 8 scratch per warp
             warp_gemm_16x8<16>(
                 lane, [&](int r, int kk) { return sbeta[o + 16 + r] * AF[(o + 16 + r) * ALD + o + kk]; },
-                [&](int kk, int nn) { return X[(o + kk) * XLD + o + nh + nn]; },
+                [&](int kk, int nn) { return AF[(o + kk) * ALD + o + nh + nn]; },
                 [&](int r, int nn, float v) { Rw[r * 8 + nn] = v; });
-            __syncwarp();
+            bar_sync(3 + 2 * e + (warp >> 1), 64);  // both column halves have read A21
             warp_gemm_16x8<16>(
-                lane, [&](int r, int kk) { return X[(o + 16 + r) * XLD + o + 16 + kk]; },
+                lane, [&](int r, int kk) { return AF[(o + 16 + r) * ALD + o + 16 + kk]; },
                 [&](int kk, int nn) { return Rw[kk * 8 + nn]; },
-                [&](int r, int nn, float v) { X[(o + 16 + r) * XLD + o + nh + nn] = -v; });
+                [&](int r, int nn, float v) { AF[(o + 16 + r) * ALD + o + nh + nn] = -v; });
         }
-        __syncthreads();
+        sync();
         // 32-row level: R2 = (Diag(beta) A)[32..63][0..31] X[0..31][0..31], then X[32..63][0..31] = -X22 R2.
         {
             const int mt = warp >> 2, nt = warp & 3;  // 16-row tile, 8-column tile
             warp_gemm_16x8<32>(
                 lane, [&](int r, int kk) { return sbeta[32 + 16 * mt + r] * AF[(32 + 16 * mt + r) * ALD + kk]; },
-                [&](int kk, int nn) { return X[kk * XLD + 8 * nt + nn]; },
+                [&](int kk, int nn) { return AF[kk * ALD + 8 * nt + nn]; },
                 [&](int r, int nn, float v) { R2[(16 * mt + r) * 32 + 8 * nt + nn] = v; });
-            __syncthreads();
+            sync();
             warp_gemm_16x8<32>(
-                lane, [&](int r, int kk) { return X[(32 + 16 * mt + r) * XLD + 32 + kk]; },
+                lane, [&](int r, int kk) { return AF[(32 + 16 * mt + r) * ALD + 32 + kk]; },
                 [&](int kk, int nn) { return R2[kk * 32 + 8 * nt + nn]; },
-                [&](int r, int nn, float v) { X[(32 + 16 * mt + r) * XLD + 8 * nt + nn] = -v; });
+                [&](int r, int nn, float v) { AF[(32 + 16 * mt + r) * ALD + 8 * nt + nn] = -v; });
         }
-        __syncthreads();
+        sync();
         // T = X Diag(beta), lower triangle, bf16: A operand of W (smem) and the slot's T tile.
         for (int e2 = tid; e2 < C * 8; e2 += PT) {
             const int r = e2 >> 3, cc8 = e2 & 7;
             float t8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int c = cc8 * 8 + e;
-                t8[e] = (c <= r) ? X[r * XLD + c] * sbeta[c] : 0.f;
+            for (int i = 0; i < 8; ++i) {
+                const int c = cc8 * 8 + i;
+                t8[i] = (c <= r) ? AF[r * ALD + c] * sbeta[c] : 0.f;
             }
             *reinterpret_cast<uint4 *>(TT + kmaj_chunk(r, cc8, 64)) = pack8(t8);
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        sync();
         tc_fence_after();
 
         // 6. W = T (K e^G): M = 64 MMA, A = T (K-major), B = rows 64..127 of [Qg ; Kg] read as
         //    an MN-major tile (64-column blocks 128 rows apart); TMEM cols [64,192), M=64 layout:
         //    row r in lane (r % 16) + 32 (r / 16).
-        if (tid == 0) {
+        if (tid == kStoreTid) {
             bulk_s2g(gslot + SL_T, TT, 8192);
+            bulk_commit();
+        }
+        if (tid == 0) {
             const uint32_t a = smem_u32(TT), b = smem_u32(GA);
             const uint32_t idw = idesc_bf16(64, 128, false, true);
 #pragma unroll
-            for (int st = 0; st < C / 16; ++st)
-                mma_bf16(tm + 64, kmaj_desc(a, st, 64), sdesc(b + 64 * 128 + st * 16 * 128, 128 * 128, 1024), idw,
-                         st > 0);
+            for (int s4 = 0; s4 < C / 16; ++s4)
+                mma_bf16(tm + 64, kmaj_desc(a, s4, 64), sdesc(b + 64 * 128 + s4 * 16 * 128, 128 * 128, 1024), idw,
+                         s4 > 0);
             mma_commit(&bars[1]);
         }
-        // The log_alpha buffer (A, X) is consumed: fetch the next item's inputs now.
-        if (nid < items) fetch(nxt);
         if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
         mma_phase ^= 1;
         tc_fence_after();
+        // T has been read by the MMA and, once the bulk store has read it too, the
+        // log_alpha region is free for the next item's box.
+        if (tid == kStoreTid && next.valid) {
+            bulk_wait_read();
+            fetch_la(next);
+        }
 
         // 7. W rows (16-byte chunks) into the lower half of WQ = [Qg ; W] (its Kg rows are consumed).
         if (warp < 4) {
@@ -460,7 +723,7 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
                     for (int q8 = 0; q8 < 4; ++q8) {
                         float w8[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) w8[e] = v[q8 * 8 + e];
+                        for (int i = 0; i < 8; ++i) w8[i] = v[q8 * 8 + i];
                         *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c0 / 8 + q8, 128)) = pack8(w8);
                     }
                 }
@@ -468,406 +731,347 @@ prep_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k,
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        sync();
 
-        // 8. WQ leaves in one bulk store; waited for before GA is rewritten.
-        if (tid == 0) {
+        // 8. WQ leaves in one bulk store; the slot is published once it completed.
+        if (tid == kStoreTid) {
             bulk_s2g(gslot + SL_WQ, GA, 32768);
             bulk_commit();
+            prev_pending = true;  // `cur` is the previous item of the next iteration
         }
-        id = nid;
-        cur = nxt;
     }
-    if (tid == 0) {
+    // Publish the last item (after a failed wait: settle what is in flight).
+    cp_async_wait_all();
+    if (tid == kStoreTid) {
         bulk_wait_all();
-        if (sflag[1]) flag_error(err, 1);
+        if (!failed && !sflag[1]) publish_prev(sitem[(iter + 2) % 3]);  // the last item
+        if (la_pending) mbar_wait(&bars[0], la_phase ^ (failed ? 1u : 0u), kWaitNs);
     }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 256);
+    sync();
+    if (tid == 0 && (failed || sflag[1])) fail_call(P);
 }
-
-// ----------------------------------------------------------------- fix ----
-// Exact fallback for queued chunks: element-wise exponents e^{G_r - G_i} <= 1.
-constexpr int FT = 256;
-constexpr int FLD = DK + 1;
-constexpr size_t FS_BYTES = (size_t)(3 * C * FLD + 3 * C * (C + 1) + C) * 4;
-
-__global__ void __launch_bounds__(FT)
-fix_kernel(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const float *__restrict__ la,
-           const float *__restrict__ beta, const int32_t *__restrict__ cu, int64_t total, int H, int N,
-           int j0, int l2norm, float eps, char *__restrict__ slots, const int *__restrict__ fix,
-           int fix_cap) {
-    extern __shared__ float fsm[];
-    float *sK = fsm, *sQ = sK + C * FLD, *sG = sQ + C * FLD;
-    float *sA = sG + C * FLD, *sP = sA + C * (C + 1), *sT = sP + C * (C + 1), *sB = sT + C * (C + 1);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int count = min(fix[0], fix_cap);
-    for (int e = blockIdx.x; e < count; e += gridDim.x) {
-        const int slot_id = fix[2 + e];
-        const int h = slot_id % H, s = (slot_id / H) % N, jl = slot_id / (H * N);
-        int64_t bos, eos;
-        seq_bounds(cu, s, total, bos, eos);
-        const int64_t j = (int64_t)j0 + jl;
-        const int n = (int)((eos - bos - j * C) < C ? (eos - bos - j * C) : C);
-        const int64_t t0 = bos + j * C;
-        uint8_t *g = reinterpret_cast<uint8_t *>(slots + (size_t)slot_id * SL_BYTES);
-        __syncthreads();
-        for (int idx = tid; idx < C * DK; idx += FT) {
-            const int r = idx / DK, c = idx % DK;
-            float kv = 0.f, qv = 0.f, lv = 0.f;
-            if (r < n) {
-                const size_t off = ((size_t)(t0 + r) * H + h) * DK + c;
-                kv = __bfloat162float(k[off]);
-                qv = __bfloat162float(q[off]);
-                lv = la[off];
-            }
-            sK[r * FLD + c] = kv;
-            sQ[r * FLD + c] = qv;
-            sG[r * FLD + c] = lv;
-        }
-        if (tid < C) sB[tid] = tid < n ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
-        __syncthreads();
-        if (l2norm) {
-            for (int r = warp; r < C; r += FT / 32) {
-                float a = 0.f, b = 0.f;
-                for (int c = lane; c < DK; c += 32) {
-                    a += sK[r * FLD + c] * sK[r * FLD + c];
-                    b += sQ[r * FLD + c] * sQ[r * FLD + c];
-                }
-#pragma unroll
-                for (int off = 16; off; off >>= 1) {
-                    a += __shfl_xor_sync(0xffffffffu, a, off);
-                    b += __shfl_xor_sync(0xffffffffu, b, off);
-                }
-                const float ia = 1.f / fmaxf(sqrtf(a), eps), ib = 1.f / fmaxf(sqrtf(b), eps);
-                for (int c = lane; c < DK; c += 32) {
-                    sK[r * FLD + c] *= ia;
-                    sQ[r * FLD + c] *= ib;
-                }
-            }
-        }
-        if (tid < DK) {
-            float run = 0.f;
-            for (int r = 0; r < C; ++r) {
-                run += sG[r * FLD + tid];
-                sG[r * FLD + tid] = run;
-            }
-        }
-        __syncthreads();
-        for (int p = tid; p < C * C; p += FT) {
-            const int r = p / C, i = p % C;
-            float a = 0.f, pp = 0.f;
-            if (i <= r)
-                for (int c = 0; c < DK; ++c) {
-                    const float ex = expf(sG[r * FLD + c] - sG[i * FLD + c]);
-                    const float ki = sK[i * FLD + c] * ex;
-                    a += sK[r * FLD + c] * ki;
-                    pp += sQ[r * FLD + c] * ki;
-                }
-            sA[r * (C + 1) + i] = (i < r) ? a : 0.f;
-            sP[r * (C + 1) + i] = pp;
-        }
-        __syncthreads();
-        if (tid < C) {
-            const int c = tid;
-            for (int r = 0; r < C; ++r) {
-                float val = 0.f;
-                if (r == c) {
-                    val = sB[c];
-                } else if (r > c) {
-                    float acc = 0.f;
-                    for (int i = c; i < r; ++i) acc += sA[r * (C + 1) + i] * sT[i * (C + 1) + c];
-                    val = -sB[r] * acc;
-                }
-                sT[r * (C + 1) + c] = val;
-            }
-        }
-        __syncthreads();
-        // Q e^G -> WQ rows 0..63; K e^{Gl-G} -> KD; D; K e^G kept in sK
-        for (int idx = tid; idx < C * DK; idx += FT) {
-            const int r = idx / DK, c = idx % DK;
-            const float gg = sG[r * FLD + c], gl = sG[(C - 1) * FLD + c];
-            const float ex = expf(gg);
-            *reinterpret_cast<bf16 *>(g + SL_WQ + kmaj_off(r, c, 128)) = __float2bfloat16_rn(sQ[r * FLD + c] * ex);
-            *reinterpret_cast<bf16 *>(g + SL_KD + mnmaj_off(r, c, 64)) = __float2bfloat16_rn(sK[r * FLD + c] * expf(gl - gg));
-        }
-        for (int c = tid; c < DK; c += FT) reinterpret_cast<float *>(g + SL_D)[c] = expf(sG[(C - 1) * FLD + c]);
-        __syncthreads();
-        for (int idx = tid; idx < C * DK; idx += FT) {
-            const int r = idx / DK, c = idx % DK;
-            sK[r * FLD + c] *= expf(sG[r * FLD + c]);
-        }
-        __syncthreads();
-        for (int idx = tid; idx < C * DK; idx += FT) {
-            const int r = idx / DK, c = idx % DK;
-            float acc = 0.f;
-            for (int i = 0; i <= r; ++i) acc += sT[r * (C + 1) + i] * sK[i * FLD + c];
-            *reinterpret_cast<bf16 *>(g + SL_WQ + kmaj_off(64 + r, c, 128)) = __float2bfloat16_rn(acc);
-        }
-        for (int idx = tid; idx < C * C; idx += FT) {
-            const int r = idx / C, c = idx % C;
-            *reinterpret_cast<bf16 *>(g + SL_T + kmaj_off(r, c, 64)) = __float2bfloat16_rn(sT[r * (C + 1) + c]);
-            *reinterpret_cast<bf16 *>(g + SL_P + kmaj_off(r, c, 64)) = __float2bfloat16_rn(sP[r * (C + 1) + c]);
-        }
-    }
-}
-
 // ---------------------------------------------------------------- scan ----
-// The big tiles of a chunk (WQ = [Q e^G ; W], K e^{Gl-G}) are triple-buffered
-// and fetched two chunks ahead; the small ones (T, P, the V tile, e^{Gl}) are
-// double-buffered, one chunk ahead. Every product is an M = 128 tcgen05.mma;
-// the 128-row A operands of T V and P U take the 64 rows next to T (before)
-// and P (after) as filler whose output rows are never read, so no zero
-// padding is stored. TMEM lanes: 0..63 hold O = Q e^G S + P U, 64..127 hold
-// W S and T V (their difference is U); Z = Kd^T U fills all 128 lanes.
-constexpr int ST = 160;  // warps 0..3: TMEM-lane epilogues; warp 4: copy and MMA issue
-constexpr uint32_t SA_WQ = 0, SA_KD = 32768, SA_BYTES = 49152;                 // x3
-constexpr uint32_t SB_T = 0, SB_P = 8192, SB_V = 16384, SB_D = 24576, SB_BYTES = 25600;  // x2
-constexpr uint32_t SS_A = 0;
-constexpr uint32_t SS_B = 3 * SA_BYTES;          // T of B0 is preceded by the last A buffer
-constexpr uint32_t SS_S = SS_B + 2 * SB_BYTES;   // [128 (c)][64 (j)] MN-major bf16 state
-constexpr uint32_t SS_U = SS_S + 16384;          // [64 (r)][64 (j)] MN-major bf16 pseudo-values
-constexpr uint32_t SS_BAR = SS_U + 8192;         // fullA[3] fullB[2] bU bS uready sready, tmem base, flag
-constexpr uint32_t SS_BYTES = SS_BAR + 96;
-constexpr uint32_t SS_ALLOC = SS_BYTES + 1024;
-constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 8192 + 512;
-// TMEM columns: X and Y double-buffered, Z
-constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = 256;
-
-__global__ void __launch_bounds__(ST, 1)
-scan_kernel(const __grid_constant__ CUtensorMap tmap_v, const int32_t *__restrict__ cu, int64_t total,
-            int H, int N, int j0, int nw, const char *__restrict__ slots, const float *__restrict__ S0,
-            float *__restrict__ state, float *__restrict__ S_T, bf16 *__restrict__ o,
-            int *__restrict__ err) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int jv = blockIdx.x, s = blockIdx.y, h = blockIdx.z;
-    int64_t bos, eos;
-    seq_bounds(cu, s, total, bos, eos);
-    const int64_t len = eos - bos;
-    const int nch = (int)((len + C - 1) / C);
-    if (j0 >= nch && !(nch == 0 && j0 == 0)) return;
-    const int jend = min(j0 + nw, nch);
-    const int nj = jend - j0 > 0 ? jend - j0 : 0;
-
+// Scan CTA for stream st, state columns [64 jv, 64 jv + 64). Warps 0..7:
+// TMEM-lane epilogues (warp w: lanes 32 (w % 4) .., columns 32 (w / 4) ..);
+// warp 8: MMA issue; warp 9: copies. TMEM lanes 0..63 hold O = Q e^G S + P U,
+// 64..127 hold W S and T V (their difference is U); Z = Kd^T U fills all 128.
+// The 128-row A operands of T V and P U take the 64 rows next to T (before) and
+// P (after) as filler whose output rows are never read.
+__device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uint32_t tm, int st, int jv) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ns = P.ns, R = P.R, H = P.H;
+    const long long NH = (long long)P.N * H;
+    const long long K = (NH - st + ns - 1) / ns;  // units of this stream
+    const long long L = reinterpret_cast<const long long *>(P.ws + WS_L)[st];
+    Hdr *hd = reinterpret_cast<Hdr *>(P.ws);
+    const int *ready = reinterpret_cast<const int *>(P.ws + ws_flags(NH));
+    int *freed = const_cast<int *>(ready) + kFlagInts;
+    const char *ring = P.ws + ws_ring(NH);
     uint8_t *sS = sm + SS_S, *sU = sm + SS_U;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SS_BAR);
-    uint64_t *fullA = bars, *fullB = bars + 3, *bU = bars + 5, *bS = bars + 6, *uready = bars + 7,
-             *sready = bars + 8;
-    uint32_t *tbase = reinterpret_cast<uint32_t *>(bars + 9);
-    int *sfail = reinterpret_cast<int *>(tbase + 1);
-    const size_t sofs = ((size_t)s * H + h) * DK * DV + (size_t)jv * DVT;
-    const int c = tid;  // epilogue threads: state row owned (= TMEM lane)
+    uint64_t *fullA = bars + MB_FULLA, *fullB = bars + MB_FULLB, *fullV = bars + MB_FULLV, *emptyA = bars + MB_EMPTYA,
+             *emptyB = bars + MB_EMPTYB, *emptyV = bars + MB_EMPTYV, *bU = bars + MB_U, *bS = bars + MB_S,
+             *bO = bars + MB_O, *uready = bars + MB_UREADY, *sready = bars + MB_SREADY, *bFin = bars + MB_FIN;
+    auto unit_bounds = [&](long long kk, int &s, int &h, int64_t &bos, int64_t &eos) {
+        const long long u = st + kk * ns;
+        s = (int)(u / H);
+        h = (int)(u % H);
+        seq_bounds(P.cu, s, P.total, bos, eos);
+    };
 
-    if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
-        mbar_init(uready, 64);   // the 64 threads of warps 2, 3
-        mbar_init(sready, 128);  // the 128 epilogue threads
-        *sfail = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tbase, 512);
-        tmem_relinquish();
-    }
-    float Sr[DVT];
-    auto store_state_bf16 = [&]() {
-#pragma unroll
-        for (int c8 = 0; c8 < DVT / 8; ++c8) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = Sr[c8 * 8 + e];
-            *reinterpret_cast<uint4 *>(sS + mnmaj_chunk(c, c8, DK)) = pack8(x);
-        }
-    };
-    if (tid < 128) {
-        // Entry state: S0 (or zeros) on the first wave, else the carry.
-        const float *Sin = (j0 == 0) ? S0 : state;
-#pragma unroll
-        for (int q4 = 0; q4 < DVT / 4; ++q4) {
-            float4 x = Sin ? *reinterpret_cast<const float4 *>(Sin + sofs + (size_t)c * DV + 4 * q4)
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-            Sr[4 * q4] = x.x; Sr[4 * q4 + 1] = x.y; Sr[4 * q4 + 2] = x.z; Sr[4 * q4 + 3] = x.w;
-        }
-        store_state_bf16();
-    }
-    auto slot_of = [&](int jj) { return slots + ((size_t)((jj - j0) * N + s) * H + h) * SL_BYTES; };
-    auto copy_a = [&](int jj) {  // big tiles of chunk jj -> A buffer (jj - j0) % 3
-        const int ab = (jj - j0) % 3;
-        uint8_t *buf = sm + SS_A + ab * SA_BYTES;
-        const char *g = slot_of(jj);
-        mbar_arrive_expect_tx(&fullA[ab], COPY_A);
-        bulk_g2s(buf + SA_WQ, g + SL_WQ, 32768, &fullA[ab]);
-        bulk_g2s(buf + SA_KD, g + SL_KD, 16384, &fullA[ab]);
-    };
-    auto copy_b = [&](int jj) {  // small tiles and the V box of chunk jj -> B buffer (jj - j0) % 2
-        const int bb = (jj - j0) & 1;
-        uint8_t *buf = sm + SS_B + bb * SB_BYTES;
-        const char *g = slot_of(jj);
-        mbar_arrive_expect_tx(&fullB[bb], COPY_B);
-        bulk_g2s(buf + SB_T, g + SL_T, 8192, &fullB[bb]);
-        bulk_g2s(buf + SB_P, g + SL_P, 8192, &fullB[bb]);
-        bulk_g2s(buf + SB_D, g + SL_D, 512, &fullB[bb]);
-        tma_load_3d(buf + SB_V, &tmap_v, jv * DVT, h, (int)(bos + (int64_t)jj * C), &fullB[bb]);
-    };
-    if (nj > 0 && tid == 128) {
-        copy_a(j0);
-        if (nj > 1) copy_a(j0 + 1);
-        copy_b(j0);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tm = *tbase;
-
-    if (warp == 4) {
-        // ---------------- copy and MMA issue (one thread) ----------------
-        if (lane == 0 && nj > 0) {
-            const uint32_t id128 = idesc_bf16(128, DVT, false, true);  // K-major A, MN-major B
-            const uint32_t idKd = idesc_bf16(128, DVT, true, true);    // MN-major A (Kd^T)
-            // Descriptors of buffer 0; buffer i is i strides further (16-byte units).
-            const uint64_t dWQ = sdesc(smem_u32(sm + SS_A + SA_WQ), 16, 1024);
-            const uint64_t dKD = sdesc(smem_u32(sm + SS_A + SA_KD), C * 128, 1024);
-            // "T then filler": 128 rows starting 64 rows before T (output rows 0..63 unused)
-            const uint64_t dTf = sdesc(smem_u32(sm + SS_B + SB_T) - 8192, 16, 1024);
-            // "P then filler": rows 64..127 read the V tile after P (output rows unused)
-            const uint64_t dP = sdesc(smem_u32(sm + SS_B + SB_P), 16, 1024);
-            const uint64_t dV = sdesc(smem_u32(sm + SS_B + SB_V), C * 128, 1024);
-            const uint64_t dS = sdesc(smem_u32(sS), DK * 128, 1024), dU = sdesc(smem_u32(sU), C * 128, 1024);
-            constexpr uint64_t kA = SA_BYTES >> 4, kB = SB_BYTES >> 4;
-            auto issue_x = [&](int bb, uint32_t xb) {
-#pragma unroll
-                for (int st = 0; st < C / 16; ++st)
-                    mma_bf16(tm + TM_X + xb, dTf + bb * kB + kmaj_step(st, 128), dV + bb * kB + mnmaj_step(st), id128,
-                             st > 0);
-            };
-            if (!mbar_wait(&fullB[0], 0, kWaitNs)) *sfail = 1;
-            issue_x(0, 0);
-            for (int it = 0; it < nj; ++it) {
-                const int jj = j0 + it, ab = it % 3, bb = it & 1;
-                const uint32_t yb = (uint32_t)bb * 64;
-                bool good = mbar_wait(&fullA[ab], (it / 3) & 1, kWaitNs);
-                if (it > 0) good = good && mbar_wait(sready, (it - 1) & 1, kWaitNs);  // S(jj) in smem
-                tc_fence_after();
-                if (it + 2 < nj) copy_a(jj + 2);
-                if (it + 1 < nj) copy_b(jj + 1);
-                // Y = [Q e^G ; W] S
-                const uint64_t dWQa = dWQ + ab * kA, dKDa = dKD + ab * kA, dPb = dP + bb * kB;
-#pragma unroll
-                for (int st = 0; st < DK / 16; ++st)
-                    mma_bf16(tm + TM_Y + yb, dWQa + kmaj_step(st, 128), dS + mnmaj_step(st), id128, st > 0);
-                mma_commit(bU);
-                good = good && mbar_wait(uready, it & 1, kWaitNs);  // U(jj) in smem
-                tc_fence_after();
-                // O: Y += [P ; filler] U ;  Z = Kd^T U
-#pragma unroll
-                for (int st = 0; st < C / 16; ++st)
-                    mma_bf16(tm + TM_Y + yb, dPb + kmaj_step(st, 128), dU + mnmaj_step(st), id128, 1);
-#pragma unroll
-                for (int st = 0; st < C / 16; ++st)
-                    mma_bf16(tm + TM_Z, dKDa + mnmaj_step(st), dU + mnmaj_step(st), idKd, st > 0);
-                mma_commit(bS);
-                if (it + 1 < nj) {
-                    good = good && mbar_wait(&fullB[bb ^ 1], ((it + 1) >> 1) & 1, kWaitNs);
-                    issue_x(bb ^ 1, yb ^ 64);
-                }
-                if (!good) {
-                    *sfail = 1;
-                    break;
-                }
+    if (warp == 9) {
+        // ---------------- ring-slot copies (one thread) ----------------
+        if (lane != 0) return;
+        long long p = 0;
+        bool ok = true;
+        for (long long kk = 0; kk < K && ok; ++kk) {
+            int s, h;
+            int64_t bos, eos;
+            unit_bounds(kk, s, h, bos, eos);
+            const long long nch = (eos - bos + C - 1) / C;
+            for (long long j = 0; j < nch; ++j, ++p) {
+                const int ab = (int)(p & 1), bb = (int)(p % 3);
+                if (p >= 2) ok = mbar_wait(&emptyA[ab], (uint32_t)((p / 2 - 1) & 1), kWaitNs);
+                if (ok && p >= 3) ok = mbar_wait(&emptyB[bb], (uint32_t)((p / 3 - 1) & 1), kWaitNs);
+                const int slot = st * R + (int)(p % R);
+                if (ok) ok = wait_flag_geq(&ready[slot], (int)(p / R) + 1, &hd->abort_flag);
+                if (!ok) break;
+                fence_proxy_async_global();
+                const char *g = ring + (size_t)slot * SL_BYTES;
+                uint8_t *A = sm + SS_A + ab * SA_BYTES, *B = sm + SS_B + bb * SB_BYTES;
+                mbar_arrive_expect_tx(&fullA[ab], COPY_A);
+                bulk_g2s(A + SA_WQ, g + SL_WQ, 32768, &fullA[ab]);
+                bulk_g2s(A + SA_KD, g + SL_KD, 16384, &fullA[ab]);
+                mbar_arrive_expect_tx(&fullB[bb], COPY_B);
+                bulk_g2s(B + SB_T, g + SL_T, 8192, &fullB[bb]);
+                bulk_g2s(B + SB_P, g + SL_P, 8192, &fullB[bb]);
+                bulk_g2s(B + SB_D, g + SL_D, 512, &fullB[bb]);
             }
         }
-    } else {
-        // ---------------- epilogues (TMEM lane = thread) ----------------
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        for (int it = 0; it < nj; ++it) {
-            const int jj = j0 + it, bb = it & 1;
-            const uint32_t xb = (uint32_t)bb * 64, yb = (uint32_t)bb * 64;
-            const uint8_t *bbuf = sm + SS_B + bb * SB_BYTES;
-            bool good = true;
-            if (warp >= 2) {
-                // U = T V - W S for rows r = lane - 64 (TMEM lanes 64..127)
-                good = mbar_wait(bU, it & 1, kWaitNs);
+        // Settle the copies still in flight (consumed ones return at once).
+        for (long long q = (p > 2 ? p - 2 : 0); q < p; ++q) mbar_wait(&fullA[q & 1], (uint32_t)((q / 2) & 1), kWaitNs);
+        for (long long q = (p > 3 ? p - 3 : 0); q < p; ++q) mbar_wait(&fullB[q % 3], (uint32_t)((q / 3) & 1), kWaitNs);
+        if (!ok) fail_call(P);
+        return;
+    }
+    if (warp == 10) {
+        // ---------------- V tiles (one thread), ahead of the ring ----------------
+        if (lane != 0) return;
+        long long p = 0;
+        bool ok = true;
+        for (long long kk = 0; kk < K && ok; ++kk) {
+            int s, h;
+            int64_t bos, eos;
+            unit_bounds(kk, s, h, bos, eos);
+            const long long nch = (eos - bos + C - 1) / C;
+            for (long long j = 0; j < nch; ++j, ++p) {
+                const int vb = (int)(p & 3);
+                if (p >= 4) ok = mbar_wait(&emptyV[vb], (uint32_t)((p / 4 - 1) & 1), kWaitNs);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&fullV[vb], SV_BYTES);
+                tma_load_3d(sm + SS_V + vb * SV_BYTES, &P.tmap_v, jv * DVT, h, (int)(bos + j * C), &fullV[vb]);
+            }
+        }
+        for (long long q = (p > 4 ? p - 4 : 0); q < p; ++q) mbar_wait(&fullV[q & 3], (uint32_t)((q / 4) & 1), kWaitNs);
+        if (!ok) fail_call(P);
+        return;
+    }
+    if (warp == 8) {
+        // ---------------- MMA issue (one thread) ----------------
+        if (lane != 0) return;
+        const uint32_t id128 = idesc_bf16(128, DVT, false, true);  // K-major A, MN-major B
+        const uint32_t idKd = idesc_bf16(128, DVT, true, true);    // MN-major A (Kd^T)
+        // Descriptors of buffer 0; buffer i is i strides further (16-byte units).
+        const uint64_t dWQ = sdesc(smem_u32(sm + SS_A + SA_WQ), 16, 1024);
+        const uint64_t dKD = sdesc(smem_u32(sm + SS_A + SA_KD), C * 128, 1024);
+        const uint64_t dTf = sdesc(smem_u32(sm + SS_B + SB_T) - 8192, 16, 1024);  // filler, then T
+        const uint64_t dP = sdesc(smem_u32(sm + SS_B + SB_P), 16, 1024);          // P, then filler
+        const uint64_t dV = sdesc(smem_u32(sm + SS_V), C * 128, 1024);
+        const uint64_t dS = sdesc(smem_u32(sS), DK * 128, 1024), dU = sdesc(smem_u32(sU), C * 128, 1024);
+        constexpr uint64_t kA = SA_BYTES >> 4, kB = SB_BYTES >> 4, kV = SV_BYTES >> 4;
+        // X[q & 1] = [filler ; T] V of position q, once its T and V tiles are in.
+        auto issue_x = [&](long long q) {
+            const int bb = (int)(q % 3), vb = (int)(q & 3);
+            if (!(mbar_wait(&fullB[bb], (uint32_t)((q / 3) & 1), kWaitNs) &&
+                  mbar_wait(&fullV[vb], (uint32_t)((q >> 2) & 1), kWaitNs)))
+                return false;
+            tc_fence_after();
+#pragma unroll
+            for (int s4 = 0; s4 < C / 16; ++s4)
+                mma_bf16(tm + TM_X + (uint32_t)(q & 1) * 64, dTf + bb * kB + kmaj_step(s4, 128), dV + vb * kV + mnmaj_step(s4),
+                         id128, s4 > 0);
+            mma_commit(&emptyV[vb]);
+            return true;
+        };
+        bool ok = true;
+        if (L > 0) ok = issue_x(0);
+        for (long long p = 0; p < L && ok; ++p) {
+            const int ab = (int)(p & 1), bb = (int)(p % 3);
+            const uint32_t yb = (uint32_t)ab * 64;
+            ok = mbar_wait(&fullA[ab], (uint32_t)((p >> 1) & 1), kWaitNs);
+            if (!ok) break;
+            // Both tile groups of position p are in shared memory: release the ring slot.
+            fence_proxy_async_global();
+            red_release_gpu_add(&freed[st * R + (int)(p % R)], 1);
+            ok = mbar_wait(sready, (uint32_t)(p & 1), kWaitNs);  // S(p) in smem
+            if (!ok) break;
+            if (p >= 1) mbar_arrive(&emptyB[(p - 1) % 3]);  // e^{Gl} of p-1 has been read
+            tc_fence_after();
+            // Y = [Q e^G ; W] S
+            const uint64_t dWQa = dWQ + ab * kA, dKDa = dKD + ab * kA, dPb = dP + bb * kB;
+#pragma unroll
+            for (int s8 = 0; s8 < DK / 16; ++s8)
+                mma_bf16(tm + TM_Y + yb, dWQa + kmaj_step(s8, 128), dS + mnmaj_step(s8), id128, s8 > 0);
+            mma_commit(bU);
+            // T V of the next position runs while U(p) is formed.
+            if (p + 1 < L && !(ok = issue_x(p + 1))) break;
+            ok = mbar_wait(uready, (uint32_t)(p & 1), kWaitNs);  // U(p) in smem
+            if (!ok) break;
+            tc_fence_after();
+            // Z = Kd^T U first (the state chain), then O: Y += [P ; filler] U
+#pragma unroll
+            for (int s4 = 0; s4 < C / 16; ++s4)
+                mma_bf16(tm + TM_Z, dKDa + mnmaj_step(s4), dU + mnmaj_step(s4), idKd, s4 > 0);
+            mma_commit(bS);
+#pragma unroll
+            for (int s4 = 0; s4 < C / 16; ++s4)
+                mma_bf16(tm + TM_Y + yb, dPb + kmaj_step(s4, 128), dU + mnmaj_step(s4), id128, 1);
+            mma_commit(bO);
+            mma_commit(&emptyA[ab]);
+            mma_commit(&emptyB[bb]);
+        }
+        mma_commit(bFin);  // every MMA of this CTA completes before TMEM is freed
+        if (!mbar_wait(bFin, 0, kWaitNs)) ok = false;
+        if (!ok) fail_call(P);
+        return;
+    }
+    if (warp >= 8) return;  // warps 11..15 idle
+
+    // ---------------- epilogues (TMEM lane = state row c) ----------------
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int c = q4 * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16, col = (uint32_t)(hf * 32);
+    float Sr[32];
+    auto load_state = [&](const float *src, size_t sofs) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 x = src ? *reinterpret_cast<const float4 *>(src + sofs + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            Sr[4 * q] = x.x;
+            Sr[4 * q + 1] = x.y;
+            Sr[4 * q + 2] = x.z;
+            Sr[4 * q + 3] = x.w;
+        }
+    };
+    auto store_state = [&](float *dst, size_t sofs) {
+        if (!dst) return;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(dst + sofs + 4 * q) = make_float4(Sr[4 * q], Sr[4 * q + 1], Sr[4 * q + 2], Sr[4 * q + 3]);
+    };
+    auto state_to_smem = [&]() {  // bf16 copy: B operand of the next chunk's products
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+            float x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) x[i] = Sr[q8 * 8 + i];
+            *reinterpret_cast<uint4 *>(sS + mnmaj_chunk(c, hf * 4 + q8, DK)) = pack8(x);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        mbar_arrive(sready);
+    };
+    bool ok = true;
+    long long p = 0;
+    for (long long kk = 0; kk < K && ok; ++kk) {
+        int s, h;
+        int64_t bos, eos;
+        unit_bounds(kk, s, h, bos, eos);
+        const long long len = eos - bos, nch = (len + C - 1) / C;
+        const size_t sofs = ((size_t)((long long)s * H + h) * DK + c) * DV + jv * DVT + hf * 32;
+        load_state(P.S0, sofs);
+        if (nch == 0) {
+            store_state(P.S_T, sofs);
+            continue;
+        }
+        state_to_smem();
+        for (long long j = 0; j < nch; ++j, ++p) {
+            const int bb = (int)(p & 1);
+            const uint32_t xy = (uint32_t)bb * 64;
+            const uint32_t par = (uint32_t)(p & 1);
+            if (q4 >= 2) {
+                // U = T V - W S for rows r = c - 64 (TMEM lanes 64..127)
+                ok = __all_sync(0xffffffffu, mbar_wait(bU, par, kWaitNs));
+                if (!ok) break;
                 tc_fence_after();
-                const int r = c - 64;
+                float xv[32], yv[32];
+                tmem_ld32(tm + TM_X + xy + lane_base + col, xv);
+                tmem_ld32(tm + TM_Y + xy + lane_base + col, yv);
+                tmem_wait_ld();
 #pragma unroll
-                for (int c0 = 0; c0 < DVT; c0 += 32) {
-                    float xv[32], yv[32];
-                    tmem_ld32(tm + TM_X + xb + lane_base + c0, xv);
-                    tmem_ld32(tm + TM_Y + yb + lane_base + c0, yv);
-                    tmem_wait_ld();
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    float u8[8];
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        float u8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) u8[e] = xv[q8 * 8 + e] - yv[q8 * 8 + e];
-                        *reinterpret_cast<uint4 *>(sU + mnmaj_chunk(r, c0 / 8 + q8, C)) = pack8(u8);
-                    }
+                    for (int i = 0; i < 8; ++i) u8[i] = xv[q8 * 8 + i] - yv[q8 * 8 + i];
+                    *reinterpret_cast<uint4 *>(sU + mnmaj_chunk(c - 64, hf * 4 + q8, C)) = pack8(u8);
                 }
                 fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(uready);
             }
-            // S' = Diag(e^{G_last}) S + Z  (row c); needs Z(jj) and e^{Gl} of the chunk
-            good = mbar_wait(bS, it & 1, kWaitNs) && good;
-            good = mbar_wait(&fullB[bb], (it >> 1) & 1, kWaitNs) && good;
+            // S' = Diag(e^{G_last}) S + Z  (row c)
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(bS, par, kWaitNs) && mbar_wait(&fullB[p % 3], (uint32_t)((p / 3) & 1), kWaitNs));
+            if (!ok) break;
             tc_fence_after();
-            const float dc = reinterpret_cast<const float *>(bbuf + SB_D)[c];
-#pragma unroll
-            for (int c0 = 0; c0 < DVT; c0 += 32) {
+            const float dc = reinterpret_cast<const float *>(sm + SS_B + (p % 3) * SB_BYTES + SB_D)[c];
+            {
                 float zv[32];
-                tmem_ld32(tm + TM_Z + lane_base + c0, zv);
+                tmem_ld32(tm + TM_Z + lane_base + col, zv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) Sr[c0 + e] = dc * Sr[c0 + e] + zv[e];
+                for (int i = 0; i < 32; ++i) Sr[i] = dc * Sr[i] + zv[i];
             }
-            store_state_bf16();
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(sready);
-            // O(jj) = rows 0..63 of Y, complete with Z: warps 0, 1 store it
-            if (warp < 2) {
-                const int nn = (int)((len - (int64_t)jj * C) < C ? (len - (int64_t)jj * C) : C);
-                const int64_t tt = bos + (int64_t)jj * C;
+            if (j + 1 < nch) state_to_smem();
+            // O = rows 0..63 of Y once P U is added (TMEM lanes 0..63)
+            if (q4 < 2) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bO, par, kWaitNs));
+                if (!ok) break;
+                tc_fence_after();
+                const long long nn = (len - j * C) < C ? (len - j * C) : C;
+                float yv[32];
+                tmem_ld32(tm + TM_Y + xy + lane_base + col, yv);
+                tmem_wait_ld();
+                if (c < nn) {
+                    bf16 *dst = P.o + ((size_t)(bos + j * C + c) * H + h) * DV + jv * DVT + hf * 32;
 #pragma unroll
-                for (int c0 = 0; c0 < DVT; c0 += 32) {
-                    float yv[32];
-                    tmem_ld32(tm + TM_Y + yb + lane_base + c0, yv);
-                    tmem_wait_ld();
-                    if (c < nn) {
-                        bf16 *dst = o + ((size_t)(tt + c) * H + h) * DV + jv * DVT + c0;
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        float o8[8];
 #pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
-                            float o8[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) o8[e] = yv[q8 * 8 + e];
-                            reinterpret_cast<uint4 *>(dst)[q8] = pack8(o8);
-                        }
+                        for (int i = 0; i < 8; ++i) o8[i] = yv[q8 * 8 + i];
+                        reinterpret_cast<uint4 *>(dst)[q8] = pack8(o8);
                     }
                 }
-            }
-            if (!good) {
-                *sfail = 1;
-                break;
+                tc_fence_before();
             }
         }
+        if (ok) store_state(P.S_T, sofs);
+    }
+    if (!ok) fail_call(P);
+}
+
+// ----------------------------------------------------------- the kernel ----
+__global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constant__ FusedParams P) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Ctrl *ctl = reinterpret_cast<Ctrl *>(sm + CTRL_OFF);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const bool scan = (int)blockIdx.x < 2 * P.ns;
+    if (tid == 0) {
+        if (scan) {
+            uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SS_BAR);
+            for (int i = 0; i < MB_COUNT; ++i) {
+                uint32_t count = 1;
+                if (i >= MB_EMPTYB && i < MB_EMPTYB + 3) count = 2;  // MMA commit + e^{Gl} read
+                if (i == MB_UREADY) count = 128;  // epilogue threads of TMEM lanes 64..127
+                if (i == MB_SREADY) count = 256;  // all epilogue threads
+                mbar_init(&bars[i], count);
+            }
+        } else {
+            for (int e = 0; e < 2; ++e) {
+                uint64_t *bars = reinterpret_cast<uint64_t *>(sm + e * PS_STRIDE + PS_BAR);
+                mbar_init(&bars[0], 1);
+                mbar_init(&bars[1], 1);
+                int *sflag = reinterpret_cast<int *>(reinterpret_cast<ItemS *>(bars + 2) + 3);
+                sflag[0] = 0;
+                sflag[1] = 0;
+            }
+        }
+        fence_barrier_init();
+    }
+    if (!scan) {
+        const Hdr *hd = reinterpret_cast<const Hdr *>(P.ws);
+        if (tid < P.ns) {
+            ctl->L[tid] = reinterpret_cast<const long long *>(P.ws + WS_L)[tid];
+            ctl->order[tid] = reinterpret_cast<const int *>(P.ws + WS_ORDER)[tid];
+        }
+        if (tid == 64) {
+            ctl->total = hd->total;
+            ctl->maxlen = hd->maxlen;
+            ctl->uniform = hd->uniform;
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(&ctl->tbase, 512);
+        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
-    const bool ok = (*sfail == 0);
-    if (!ok && tid == 0) flag_error(err, 1);
-
-    // Exit: final state when the sequence ended in this wave, else the carry.
-    float *Sout = (jend == nch) ? S_T : state;
-    if (Sout && ok && tid < 128) {
-#pragma unroll
-        for (int q4 = 0; q4 < DVT / 4; ++q4)
-            *reinterpret_cast<float4 *>(Sout + sofs + (size_t)c * DV + 4 * q4) =
-                make_float4(Sr[4 * q4], Sr[4 * q4 + 1], Sr[4 * q4 + 2], Sr[4 * q4 + 3]);
-    }
+    tc_fence_after();
+    const uint32_t tm = ctl->tbase;
+    if (scan) scan_role(P, sm, tm, blockIdx.x >> 1, blockIdx.x & 1);
+    else prep_engine(P, ctl, tid >> 8, sm + (tid >> 8) * PS_STRIDE, tm + 256u * (uint32_t)(tid >> 8));
+    tc_fence_before();
+    __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
 }
 
@@ -898,124 +1102,89 @@ bool make_v_map(CUtensorMap *m, const void *v, int64_t total, int H) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// q, k or log_alpha viewed as [T][H][128]; a box is 128 channels x 1 head x 64 tokens.
-bool make_row_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int64_t total, int H) {
+// log_alpha viewed as [T][H][128] fp32; a box is 128 channels x 1 head x 64 tokens.
+bool make_la_map(CUtensorMap *m, const void *base, int64_t total, int H) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)total};
-    const cuuint64_t strides[2] = {(cuuint64_t)DK * esize, (cuuint64_t)H * DK * esize};
+    const cuuint64_t strides[2] = {(cuuint64_t)DK * 4, (cuuint64_t)H * DK * 4};
     const cuuint32_t box[3] = {(cuuint32_t)DK, 1, (cuuint32_t)C};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-    return n;
-}
-
-cudaError_t set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PS_ALLOC);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(fix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FS_BYTES);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SS_ALLOC);
-    return e;
-}
-
-// Prep (+ exact fallback) of chunks [j0, j0 + nw) into `slots`; `queue` = [fallback count,
-// item counter, fallback entries...].
-cudaError_t tc_prep(const PrefillArgs &a, int j0, int nw, char *slots, int *queue, int cap, int *err,
-                    cudaStream_t st) {
-    CUtensorMap lamap;
-    if (!make_row_map(&lamap, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.total, a.H))
-        return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(queue, 0, 2 * sizeof(int), st);
-    if (e != cudaSuccess) return e;
-    const int sms = sm_count();
-    const int items = nw * a.N * a.H;
-    const int grid = items < 2 * sms ? items : 2 * sms;
-    prep_kernel<<<grid, PT, PS_ALLOC, st>>>((const bf16 *)a.q, (const bf16 *)a.k, lamap, a.beta, a.cu, a.total,
-                                            a.H, a.N, j0, nw, a.l2norm, a.eps, slots, queue, cap, err);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    fix_kernel<<<sms, FT, FS_BYTES, st>>>((const bf16 *)a.q, (const bf16 *)a.k, a.log_alpha, a.beta, a.cu,
-                                          a.total, a.H, a.N, j0, a.l2norm, a.eps, slots, queue, cap);
-    return cudaGetLastError();
-}
-
-cudaError_t tc_scan(const PrefillArgs &a, int j0, int nw, const char *slots, int *err, cudaStream_t st) {
-    CUtensorMap vmap;
-    memset(&vmap, 0, sizeof(vmap));
-    if (a.total > 0 && !make_v_map(&vmap, a.v, a.total, a.H)) return cudaErrorInvalidValue;
-    scan_kernel<<<dim3(DV / DVT, a.N, a.H), ST, SS_ALLOC, st>>>(vmap, a.cu, a.total, a.H, a.N, j0, nw, slots,
-                                                                a.S0, a.state, a.S_T, (bf16 *)a.o, err);
-    return cudaGetLastError();
-}
-
-// Per-device side stream and events for overlapping the prep of wave w+1 with
-// the scan of wave w. Created on first use and kept for the process lifetime;
-// the enqueue sequence of a call holds the mutex so that calls from several
-// host threads do not interleave their use of the shared events.
-struct Overlap {
-    cudaStream_t side = nullptr;
-    cudaEvent_t start = nullptr, prep[2] = {nullptr, nullptr}, scan[2] = {nullptr, nullptr};
-    bool ok = false;
-};
-std::mutex g_overlap_mu;
-Overlap g_overlap[64];
-
-Overlap *overlap_for_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    Overlap &o = g_overlap[dev];
-    if (!o.ok) {
-        const unsigned f = cudaEventDisableTiming;
-        if (cudaStreamCreateWithFlags(&o.side, cudaStreamNonBlocking) != cudaSuccess ||
-            cudaEventCreateWithFlags(&o.start, f) != cudaSuccess ||
-            cudaEventCreateWithFlags(&o.prep[0], f) != cudaSuccess ||
-            cudaEventCreateWithFlags(&o.prep[1], f) != cudaSuccess ||
-            cudaEventCreateWithFlags(&o.scan[0], f) != cudaSuccess ||
-            cudaEventCreateWithFlags(&o.scan[1], f) != cudaSuccess)
-            return nullptr;
-        o.ok = true;
-    }
-    return &o;
 }
 
 }  // namespace
 
-size_t tc_slot_bytes() { return SL_BYTES; }
+size_t tc_workspace_bytes(long long NH, int ns, int R) {
+    return ws_ring(NH) + (size_t)ns * (size_t)R * SL_BYTES;
+}
 
-cudaError_t tc_prefill(const PrefillArgs &a, int64_t max_chunks, int nw, char *const buf_slots[2],
-                       int *const buf_queue[2], int cap, int *err, cudaStream_t st) {
-    cudaError_t e = set_attributes();
-    if (e != cudaSuccess) return e;
-    if (max_chunks == 0) return tc_scan(a, 0, 0, buf_slots[0], err, st);  // only empty sequences
-    if (nw >= max_chunks) {  // one wave: everything on the caller's stream
-        if ((e = tc_prep(a, 0, (int)max_chunks, buf_slots[0], buf_queue[0], cap, err, st)) != cudaSuccess) return e;
-        return tc_scan(a, 0, (int)max_chunks, buf_slots[0], err, st);
-    }
-    std::lock_guard<std::mutex> lock(g_overlap_mu);
-    Overlap *ov = overlap_for_device();
-    if (!ov) return cudaErrorInitializationError;
-    if ((e = cudaEventRecord(ov->start, st)) != cudaSuccess) return e;
-    if ((e = cudaStreamWaitEvent(ov->side, ov->start, 0)) != cudaSuccess) return e;
-    int w = 0;
-    for (int64_t j0 = 0; j0 < max_chunks; j0 += nw, ++w) {
-        const int n = (int)((max_chunks - j0) < nw ? (max_chunks - j0) : nw);
-        const int b = w & 1;
-        if (w >= 2 && (e = cudaStreamWaitEvent(ov->side, ov->scan[b], 0)) != cudaSuccess) return e;
-        if ((e = tc_prep(a, (int)j0, n, buf_slots[b], buf_queue[b], cap, err, ov->side)) != cudaSuccess) return e;
-        if ((e = cudaEventRecord(ov->prep[b], ov->side)) != cudaSuccess) return e;
-        if ((e = cudaStreamWaitEvent(st, ov->prep[b], 0)) != cudaSuccess) return e;
-        if ((e = tc_scan(a, (int)j0, n, buf_slots[b], err, st)) != cudaSuccess) return e;
-        if ((e = cudaEventRecord(ov->scan[b], st)) != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+int tc_ring_slots(long long NH, int ns, size_t bytes) {
+    const size_t base = ws_ring(NH);
+    if (ns < 1 || bytes < base) return 0;
+    const size_t r = (bytes - base) / ((size_t)ns * SL_BYTES);
+    return (int)(r < (size_t)kMaxRing ? r : (size_t)kMaxRing);
+}
+
+int tc_max_ring() { return kMaxRing; }
+
+cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, int *err, cudaStream_t st) {
+    cudaError_t e;
+    // Per device (context): cheap enough to set on every call.
+    if ((e = cudaFuncSetAttribute(fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC)) !=
+        cudaSuccess)
+        return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_kernel, kThreads, SMEM_ALLOC)) != cudaSuccess)
+        return e;
+    const int grid = per_sm * sms;
+    // At least two prep CTAs beside the scan CTAs.
+    if (2 * ns + 2 > grid) ns = (grid - 2) / 2;
+    if (ns < 1) return cudaErrorLaunchOutOfResources;
+    const long long NH = (long long)a.N * a.H;
+    const int R = tc_ring_slots(NH, ns, ws_bytes);
+    if (R < 1) return cudaErrorInvalidValue;
+
+    FusedParams P;
+    memset(&P, 0, sizeof(P));
+    if (a.total > 0 && (!make_la_map(&P.tmap_la, a.log_alpha, a.total, a.H) || !make_v_map(&P.tmap_v, a.v, a.total, a.H)))
+        return cudaErrorInvalidValue;
+    P.q = static_cast<const bf16 *>(a.q);
+    P.k = static_cast<const bf16 *>(a.k);
+    P.beta = a.beta;
+    P.S0 = a.S0;
+    P.cu = a.cu;
+    P.S_T = a.S_T;
+    P.o = static_cast<bf16 *>(a.o);
+    P.ws = ws;
+    P.err = err;
+    P.total = a.total;
+    P.N = a.N;
+    P.H = a.H;
+    P.ns = ns;
+    P.R = R;
+    P.l2norm = a.l2norm;
+    P.eps = a.eps;
+
+    plan_kernel<<<1, PLAN_T, 0, st>>>(a.cu, a.total, a.N, a.H, ns, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_ALLOC;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fused_kernel, P);
 }
 
 }  // namespace kda

@@ -71,7 +71,8 @@ int32_t kda_version(void);
 /*
  * Workspace bytes kda_prefill performs best with for this problem. Any
  * workspace of at least kda_prefill_workspace_min() bytes also works (the
- * prefill then runs in more waves). Returns 0 if the arguments are invalid.
+ * CUDA-core path then runs in more waves; the tensor-core path keeps fewer
+ * prepared chunks in flight). Returns 0 if the arguments are invalid.
  * Arguments as for kda_prefill; max_seqlen <= 0 means "unknown"
  * (total_tokens is assumed).
  */
@@ -135,9 +136,9 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
  * allocated: no cudaMalloc, cudaFree or allocating library call.
  * - Limit: problems whose kda_prefill_workspace_min() exceeds
  *   KDA_NOALLOC_SCRATCH_BYTES are refused with KDA_ERR_WORKSPACE before
- *   anything is enqueued (at d_k = d_v = 128 on the tensor-core path: any
- *   problem whose chunks all fit one wave, else about num_seqs * H <= 160;
- *   larger problems run as more, smaller waves).
+ *   anything is enqueued. On the tensor-core path (bf16, d_k = d_v = 128)
+ *   the minimum is about 8.5 MB plus 12 bytes per (sequence, head), so every
+ *   practical problem fits; on the CUDA-core path it grows with num_seqs * H.
  * - The first call on a device resolves the array's address on that device
  *   (with that device current); make that first call before any stream
  *   capture begins.

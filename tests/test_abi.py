@@ -56,9 +56,15 @@ def test_workspace_queries(lib):
     b = m(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
     assert a >= b > 0
     assert m(1, 8192, 8192, 16, 128, 128, 0, 64, 0) < m(1, 8192, 8192, 32, 128, 128, 0, 64, 0)
-    # tensor-core path: waves sized for L2, never more than the whole problem needs
-    assert f(1, 640, 640, 32, 128, 128, 1, 64, 0) <= f(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
-    assert lib.kda_prefill_launches(1, 8192, 8192, 32, 128, 128, 1, 64, 0, a) >= 3
+    # tensor-core path: a planning launch and one persistent launch; the ring of
+    # each stream holds at most its chunks and at most 16 slots, so a short
+    # problem needs less and a long one no more than a 16-chunk problem
+    assert lib.kda_prefill_launches(1, 8192, 8192, 32, 128, 128, 1, 64, 0, a) == 2
+    assert lib.kda_prefill_launches(1, 8192, 8192, 32, 128, 128, 1, 64, 0, b) == 2
+    assert lib.kda_prefill_launches(1, 8192, 8192, 32, 128, 128, 1, 64, 0, b - 1) == -1
+    assert f(1, 128, 128, 32, 128, 128, 1, 64, 0) < f(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
+    assert f(1, 1024, 1024, 32, 128, 128, 1, 64, 0) == a == f(1, 1 << 20, 1 << 20, 32, 128, 128, 1, 64, 0)
+    assert m(1, 1 << 20, 1 << 20, 32, 128, 128, 1, 64, 0) == b < a
     # single-chunk problems need no state carry
     assert m(1, 64, 64, 4, 64, 64, 0, 64, 0) == m(1, 1, 1, 4, 64, 64, 0, 64, 0)
     # invalid / unsupported -> 0

@@ -161,6 +161,25 @@ def test_multi_wave_matches_single_wave():
     check(o2, S2, inp, torch.bfloat16, label="multi-wave")
 
 
+def test_tensor_core_ring_sizes_and_many_units():
+    """bf16, d = 128 with more (sequence, head) units than scan streams (72 over
+    32: streams of 2 or 3 units of different lengths) and empty, one-token and
+    ragged sequences. The smallest workspace (fewest ring slots per stream)
+    gives bit-identical results to the recommended one; both match the oracle."""
+    lengths = [0, 130, 1, 64, 700, 0, 65, 257]
+    H = 9
+    inp = make(lengths, H, 128, 128, torch.bfloat16, seed=21)
+    o1, S1 = run(inp)
+    mn = kda.kda_prefill_workspace_min(len(lengths), sum(lengths), max(lengths), H, 128, 128,
+                                       torch.bfloat16)
+    ws = torch.empty(mn, dtype=torch.uint8, device=DEV)
+    o2, S2 = run(inp, workspace=ws)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    check(o1, S1, inp, torch.bfloat16, label="tc streams")
+    assert torch.equal(S1[0], inp["S0"][0]) and torch.equal(S1[5], inp["S0"][5])
+    assert kda.kda_device_error() == 0
+
+
 def test_strong_decay():
     inp = make([150], 2, 128, 128, torch.float32, seed=7)
     inp["log_alpha"] = inp["log_alpha"] * 400.0  # ~ -20 per token: exp(+G) would overflow
