@@ -185,8 +185,8 @@ constexpr uint32_t PS_LA = 0;                  // log_alpha -> G [64][128] fp32;
 constexpr uint32_t PS_GA = 32768;              // [Qg ; Kg] K-major 128 x 128 -> WQ
 constexpr uint32_t PS_GB = PS_GA + 32768;      // q of the next item, then K e^-G (K-major 64 x 128)
 constexpr uint32_t PS_KS = PS_GB + 16384;      // k of the next item (K-major 64 x 128)
-constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[64] eGl[128]
-constexpr uint32_t PS_BAR = PS_SMALL + 1280;   // la, mma barriers; 3 item records; flags
+constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[2][64] eGl[128]
+constexpr uint32_t PS_BAR = PS_SMALL + 1536;   // la, mma barriers; 3 item records; flags
 constexpr uint32_t PS_BYTES = PS_BAR + 128;
 constexpr uint32_t PS_STRIDE = 100352;         // engine 1 starts here (1024-aligned)
 constexpr int ALD = 68;                        // row stride of A / X (floats)
@@ -206,7 +206,7 @@ constexpr uint32_t SS_B = 2 * SA_BYTES;         // T of B0 is preceded by the la
 constexpr uint32_t SS_V = SS_B + 3 * SB_BYTES;
 constexpr uint32_t SS_S = SS_V + 4 * SV_BYTES;  // [128 (c)][64 (j)] MN-major bf16 state
 constexpr uint32_t SS_U = SS_S + 16384;         // [64 (r)][64 (j)] MN-major bf16 pseudo-values
-constexpr uint32_t SS_BAR = SS_U + 8192;        // 24 mbarriers
+constexpr uint32_t SS_BAR = SS_U + 8192;        // 24 mbarriers, then the consumed-position counter
 constexpr uint32_t SS_BYTES = SS_BAR + 256;
 constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 512;
 // scan mbarrier indices
@@ -326,7 +326,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     uint8_t *GB = sm + PS_GB;
     uint8_t *KS = sm + PS_KS;
     float *invq = reinterpret_cast<float *>(sm + PS_SMALL);
-    float *invk = invq + 64, *sbeta = invk + 64, *eGl = sbeta + 64;
+    float *invk = invq + 64, *sbeta2 = invk + 64, *eGl = sbeta2 + 128;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA
     // Item records of iterations it (current), it + 1 (claimed during the Gram)
     // and it - 1 (published by the store thread) in entries it % 3, ...
@@ -342,14 +342,14 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     const int c8 = tid & 15, rb = tid >> 4;  // thread's 16-byte channel chunk and first row
 
     auto slot_index = [&](const ItemS &it) { return it.st * R + (int)(it.p % R); };
-    // Thread 128 issues the slot's bulk stores (bulk groups belong to the issuing
-    // thread) and the log_alpha boxes, and publishes each item: after the item's
-    // generic slot stores (ordered before it by the engine's barriers) and its
-    // bulk stores completed, one gpu-scope release of the slot's ready generation.
-    // The previous item is published during the Gram, or at once if the current
-    // item has to wait for its slot (that wait may depend on the previous item).
-    // Thread 160 claims items.
-    constexpr int kStoreTid = 128, kClaimTid = 160;
+    // Thread 128 claims items, issues the slot's bulk stores (bulk groups belong
+    // to the issuing thread) and the log_alpha boxes, and publishes each item:
+    // after the item's generic slot stores (ordered before it by the engine's
+    // barriers) and its bulk stores completed, one gpu-scope release of the
+    // slot's ready generation. The previous item is published during the Gram
+    // (warps 4..7 are idle there), or at once if the current item has to wait
+    // for its slot (that wait may depend on the previous item).
+    constexpr int kStoreTid = 128;
     bool slot_ok = false;       // store thread: the current item's slot is known to be free
     bool prev_pending = false;  // store thread: the previous item is not yet published
     bool la_pending = false;    // store thread: a log_alpha box is in flight
@@ -375,10 +375,9 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     };
     // q and k rows rb + 16 m, chunk c8, by cp.async into GB / KS at the chunk's
     // place in a K-major SW128 64 x 128 tile (the thread reads back exactly what
-    // it copied; K e^-G later overwrites q in place); rows past the sequence
-    // are zero-filled. beta into a register (threads < 64).
-    float bnext = 0.f;
-    auto fetch_qk = [&](const ItemS &it) {
+    // it copied; K e^-G later overwrites q in place); beta of row `tid` (threads
+    // < 64) into sbeta2[buf]. Rows past the sequence are zero-filled.
+    auto fetch_qk = [&](const ItemS &it, int buf) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
             const int r = rb + 16 * m;
@@ -387,14 +386,16 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             cp_async16(GB + kmaj_chunk(r, c8, 64), P.q + off, bytes);
             cp_async16(KS + kmaj_chunk(r, c8, 64), P.k + off, bytes);
         }
+        if (tid < C)
+            cp_async4(sbeta2 + buf * 64 + tid, P.beta + (size_t)(it.t0 + (tid < it.n ? tid : 0)) * H + it.h,
+                      tid < it.n ? 4u : 0u);
         cp_async_commit();
-        bnext = (tid < it.n) ? __ldg(P.beta + (size_t)(it.t0 + tid) * H + it.h) : 0.f;
     };
 
-    if (tid == kClaimTid) claim(sitem[0]);
+    if (tid == kStoreTid) claim(sitem[0]);
     sync();
     if (tid == kStoreTid && sitem[0].valid) fetch_la(sitem[0]);
-    if (sitem[0].valid) fetch_qk(sitem[0]);
+    if (sitem[0].valid) fetch_qk(sitem[0], 0);
     bool failed = false;
     int iter = 0;
     for (; sitem[iter % 3].valid; ++iter) {
@@ -403,7 +404,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         const ItemS &prev = sitem[(iter + 2) % 3];
         const int n = cur.n;
         char *gslot = ring + (size_t)slot_index(cur) * SL_BYTES;
-        if (tid < C) sbeta[tid] = bnext;
+        const float *sbeta = sbeta2 + (iter & 1) * 64;
         if (tid == kStoreTid) {
             bulk_wait_read();  // the previous item's bulk stores no longer read GA
             // This item's slot is written below: both scan CTAs of the stream must
@@ -415,31 +416,11 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             slot_ok = false;
         }
 
-        // 1a. Row norms: 16 lanes share a row; shuffle-reduce over them.
-        cp_async_wait_all();  // this thread's q, k chunks
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int r = rb + 16 * m;
-            float qf[8], kf[8], sq = 0.f, sk = 0.f;
-            unpack8(*reinterpret_cast<const uint4 *>(GB + kmaj_chunk(r, c8, 64)), qf);
-            unpack8(*reinterpret_cast<const uint4 *>(KS + kmaj_chunk(r, c8, 64)), kf);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                sq += qf[i] * qf[i];
-                sk += kf[i] * kf[i];
-            }
-#pragma unroll
-            for (int off = 1; off < 16; off <<= 1) {
-                sq += __shfl_xor_sync(0xffffffffu, sq, off);
-                sk += __shfl_xor_sync(0xffffffffu, sk, off);
-            }
-            if (c8 == 0) {
-                const bool live = r < n;
-                invq[r] = !live ? 0.f : (P.l2norm ? 1.f / fmaxf(sqrtf(sq), P.eps) : 1.f);
-                invk[r] = !live ? 0.f : (P.l2norm ? 1.f / fmaxf(sqrtf(sk), P.eps) : 1.f);
-            }
-        }
-        // 1b. G = cumulative sum of log_alpha over the rows, in place: one thread per channel.
+        // 1. Warps 0..3: G = cumulative sum of log_alpha over the rows, in place, one
+        //    thread per channel. Warps 4..7: the row norms of q (threads 128..191) and
+        //    k (192..255), one row per thread, from the chunks every thread copied.
+        cp_async_wait_all();  // this thread's q, k chunks and beta
+        sync();
         if (tid < DK) {
             if (!mbar_wait(&bars[0], la_phase, kWaitNs)) sflag[1] = 1;
             const int c = tid;
@@ -457,6 +438,20 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             }
             eGl[c] = expf(run);
             if (-run > kTau) sflag[0] = 1;
+        } else {
+            const int r = tid & (C - 1);
+            const uint8_t *src = (tid < 192) ? GB : KS;
+            float ss = 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 16; ++cc) {
+                float x[8];
+                unpack8(*reinterpret_cast<const uint4 *>(src + kmaj_chunk(r, cc, 64)), x);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+            }
+            // 1 / max(||x||, eps) = rsqrt(max(||x||^2, eps^2))
+            const float inv = (r >= n) ? 0.f : (P.l2norm ? rsqrtf(fmaxf(ss, P.eps * P.eps)) : 1.f);
+            ((tid < 192) ? invq : invk)[r] = inv;
         }
         la_phase ^= 1;
         sync();
@@ -533,8 +528,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     mma_bf16(tm, kmaj_desc(a, s8, 128), kmaj_desc(b, s8, 64), idg, s8 > 0);
                 mma_commit(&bars[1]);
             }
-            if (tid == kClaimTid) claim(next);
-            if (tid == kStoreTid) publish_prev(prev);
+            if (tid == kStoreTid) claim(next);
             if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
             mma_phase ^= 1;
             tc_fence_after();
@@ -574,8 +568,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(rr, c8, 128)) = pack8(x);
             }
             fence_async_smem();
-            if (tid == kClaimTid) claim(next);
-            if (tid == kStoreTid) publish_prev(prev);
+            if (tid == kStoreTid) claim(next);
             sync();  // G is overwritten by A below
         }
         if (tid == 0) sflag[0] = 0;
@@ -607,14 +600,16 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     *reinterpret_cast<uint4 *>(gslot + SL_P + kmaj_chunk(r, c0 / 8 + 1, 64)) = pack8(hi);
                 }
             }
+        } else if (tid == kStoreTid) {
+            publish_prev(prev);  // warps 4..7 are idle in this phase
         }
         tc_fence_before();
         sync();
         // The next item is known (claimed during the Gram): its q, k rows load into
         // GB (free: the Gram has consumed K e^-G) and KS while this item finishes,
         // and the store thread checks its slot.
-        if (next.valid) fetch_qk(next);
-        if (tid == kStoreTid && next.valid) slot_ok = slot_free(next);
+        if (next.valid) fetch_qk(next, (iter + 1) & 1);
+        if (tid == kStoreTid && next.valid) slot_ok = slot_free(next);  // warp 4 is idle in the next phase
 
         // 5. In place, AF (A) becomes X = (I + Diag(beta) A)^{-1}: diagonal 16x16 blocks by
         //    forward substitution, then the 2x2 block recursion with tf32 tensor-core products:
@@ -753,7 +748,8 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
 // ---------------------------------------------------------------- scan ----
 // Scan CTA for stream st, state columns [64 jv, 64 jv + 64). Warps 0..7:
 // TMEM-lane epilogues (warp w: lanes 32 (w % 4) .., columns 32 (w / 4) ..);
-// warp 8: MMA issue; warp 9: copies. TMEM lanes 0..63 hold O = Q e^G S + P U,
+// warp 8: MMA issue; warp 9: ring-slot copies; warp 10: V copies; warp 11: slot
+// release. TMEM lanes 0..63 hold O = Q e^G S + P U,
 // 64..127 hold W S and T V (their difference is U); Z = Kd^T U fills all 128.
 // The 128-row A operands of T V and P U take the 64 rows next to T (before) and
 // P (after) as filler whose output rows are never read.
@@ -814,6 +810,35 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         if (!ok) fail_call(P);
         return;
     }
+    // Positions whose tiles are in shared memory (written by the MMA thread).
+    volatile long long *consumed = reinterpret_cast<volatile long long *>(bars + MB_COUNT);
+    if (warp == 11) {
+        // ---------------- ring-slot release (one thread) ----------------
+        // Both scan CTAs of the stream release each slot once its tiles are in
+        // their shared memory; the gpu-scope release (with the proxy fence it
+        // needs) stays off the MMA thread.
+        if (lane != 0) return;
+        bool ok = true;
+        for (long long p = 0; p < L && ok;) {
+            long long upto = *consumed;
+            if (upto <= p) {
+                const uint64_t t0 = globaltimer_ns();
+                while ((upto = *consumed) <= p) {
+                    __nanosleep(64);
+                    if (ld_relaxed_gpu(&hd->abort_flag) || globaltimer_ns() - t0 > kWaitNs) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok) break;
+            }
+            __threadfence_block();
+            fence_proxy_async_global();
+            for (; p < upto; ++p) red_release_gpu_add(&freed[st * R + (int)(p % R)], 1);
+        }
+        if (!ok) fail_call(P);
+        return;
+    }
     if (warp == 10) {
         // ---------------- V tiles (one thread), ahead of the ring ----------------
         if (lane != 0) return;
@@ -870,9 +895,10 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             const uint32_t yb = (uint32_t)ab * 64;
             ok = mbar_wait(&fullA[ab], (uint32_t)((p >> 1) & 1), kWaitNs);
             if (!ok) break;
-            // Both tile groups of position p are in shared memory: release the ring slot.
-            fence_proxy_async_global();
-            red_release_gpu_add(&freed[st * R + (int)(p % R)], 1);
+            // Both tile groups of position p are in shared memory (B was waited for
+            // with X(p)): its ring slot can be released.
+            __threadfence_block();
+            *consumed = p + 1;
             ok = mbar_wait(sready, (uint32_t)(p & 1), kWaitNs);  // S(p) in smem
             if (!ok) break;
             if (p >= 1) mbar_arrive(&emptyB[(p - 1) % 3]);  // e^{Gl} of p-1 has been read
@@ -905,7 +931,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         if (!ok) fail_call(P);
         return;
     }
-    if (warp >= 8) return;  // warps 11..15 idle
+    if (warp >= 8) return;  // warps 12..15 idle
 
     // ---------------- epilogues (TMEM lane = state row c) ----------------
     const int q4 = warp & 3, hf = warp >> 2;
@@ -1036,6 +1062,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
                 if (i == MB_SREADY) count = 256;  // all epilogue threads
                 mbar_init(&bars[i], count);
             }
+            *reinterpret_cast<long long *>(bars + MB_COUNT) = 0;
         } else {
             for (int e = 0; e < 2; ++e) {
                 uint64_t *bars = reinterpret_cast<uint64_t *>(sm + e * PS_STRIDE + PS_BAR);

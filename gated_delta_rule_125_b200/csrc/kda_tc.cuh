@@ -284,6 +284,11 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc, uin
                  "r"(src_bytes)
                  : "memory");
 }
+// 4-byte asynchronous copy global -> shared (cp.async through L1).
+__device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
