@@ -18,8 +18,10 @@ sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -182,6 +184,27 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------- kda ----
 
+PREFILL_SOURCES = ["gated_delta_rule_125_b200/csrc/kda_prefill_tc.cu", "gated_delta_rule_125_b200/csrc/kda_tc.cuh"]
+DECODE_SOURCES = ["gated_delta_rule_125_b200/csrc/kda_decode.cu"]
+
+
+def profiled_traffic(profile, sources):
+    """DRAM bytes (read + write) per launch from a committed ncu summary under
+    profiles/, or None when the summary is missing or the kernel's sources have
+    changed since it was taken (the summary records their sha256)."""
+    root = os.path.dirname(os.path.abspath(__file__))
+    try:
+        txt = open(os.path.join(root, "profiles", profile)).read()
+        blob = b"".join(open(os.path.join(root, f), "rb").read() for f in sources)
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*(\d+)", txt)
+    h = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    if not m or not h or hashlib.sha256(blob).hexdigest() != h.group(1):
+        return None
+    return int(m.group(1))
+
+
 def run_kda(args, world, rank, local):
     import gated_delta_rule_125_b200 as kda
     dev = torch.device("cuda", local)
@@ -283,8 +306,9 @@ def run_kda(args, world, rank, local):
                    "l2": "inputs 404 MB > 126 MB L2 (no flush)",
                    "parallelism": "independent batch per GPU" if world > 1 else "1 GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
-                     "kernel": "prefill pass (prep + scan kernels per wave)",
+                     "frac": achieved / hbm,
+                     "traffic": profiled_traffic("fused_kernel_prefill_8k.md", PREFILL_SOURCES),
+                     "kernel": "kda_prefill = plan_kernel + persistent fused_kernel (timed together)",
                      "algorithmic_bytes": bytes_pass, "peak_source": peak_src},
         "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -295,7 +319,8 @@ def run_kda(args, world, rank, local):
                    "workload": "decode_256: 256 seqs x 32 heads, d=128, bf16 q/k/v, fp32 state "
                                "512 MiB in place (> L2)",
                    "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
-                                "frac": dec_gbs / hbm, "traffic": None,
+                                "frac": dec_gbs / hbm,
+                                "traffic": profiled_traffic("decode_kernel_decode_256.md", DECODE_SOURCES),
                                 "kernel": "decode_kernel<128,128,bf16>",
                                 "algorithmic_bytes": DECODE_BYTES, "peak_source": peak_src}},
     }

@@ -34,7 +34,8 @@ __device__ __forceinline__ void seq_bounds(const int32_t *cu, int s, int64_t tot
     }
 }
 
-// Parameters of one prefill wave: chunk indices [j0, j0 + nw) of every sequence.
+// Parameters of a prefill call (the CUDA-core path runs it in waves: chunk
+// indices [j0, j0 + nw) of every sequence per wave).
 struct PrefillArgs {
     const void *q, *k, *v;
     const float *log_alpha, *beta, *S0;

@@ -13,8 +13,8 @@
 // The array is file-scope, 256-byte aligned and kNoAllocScratchBytes large;
 // every GPU that loads the library holds it until the process exits. Every
 // call shares it and it keeps the last call's contents. The prefill needs no
-// part of it to start at zero except the fallback-queue counter, which the
-// kernels' host code clears on the stream before each wave. Calls that overlap
+// part of it to start at zero except its counters and ring flags, which the
+// prefill's own planning kernel clears at the start of every call. Calls that overlap
 // on the GPU (different streams, or several host threads) race on the array
 // and give wrong results; the caller must order them.
 #include <mutex>

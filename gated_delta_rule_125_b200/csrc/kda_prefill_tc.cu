@@ -575,11 +575,12 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
 
         // 4. P (bf16, lower incl. diagonal; TMEM lanes 0..63) to the slot; A (fp32,
         //    strictly lower, zero elsewhere; lanes 64..127) over the consumed G.
-        if (warp < 4) {
-            const int row = warp * 32 + lane;
-            for (int c0 = 0; c0 < C; c0 += 16) {
+        //    Warps w and w + 4 share TMEM lanes 32 (w % 4) .. and take 32 columns each.
+        {
+            const int row = (warp & 3) * 32 + lane;
+            for (int c0 = (warp >> 2) * 32; c0 < (warp >> 2) * 32 + 32; c0 += 16) {
                 float v[16];
-                tmem_ld16(tm + ((uint32_t)(warp * 32) << 16) + c0, v);
+                tmem_ld16(tm + ((uint32_t)((warp & 3) * 32) << 16) + c0, v);
                 tmem_wait_ld();
                 if (row >= C) {
                     const int r = row - C;
@@ -600,8 +601,6 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     *reinterpret_cast<uint4 *>(gslot + SL_P + kmaj_chunk(r, c0 / 8 + 1, 64)) = pack8(hi);
                 }
             }
-        } else if (tid == kStoreTid) {
-            publish_prev(prev);  // warps 4..7 are idle in this phase
         }
         tc_fence_before();
         sync();
@@ -609,7 +608,10 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         // GB (free: the Gram has consumed K e^-G) and KS while this item finishes,
         // and the store thread checks its slot.
         if (next.valid) fetch_qk(next, (iter + 1) & 1);
-        if (tid == kStoreTid && next.valid) slot_ok = slot_free(next);  // warp 4 is idle in the next phase
+        if (tid == kStoreTid) {  // warp 4 is idle in the diagonal-block solve below
+            publish_prev(prev);
+            if (next.valid) slot_ok = slot_free(next);
+        }
 
         // 5. In place, AF (A) becomes X = (I + Diag(beta) A)^{-1}: diagonal 16x16 blocks by
         //    forward substitution, then the 2x2 block recursion with tf32 tensor-core products:
@@ -707,11 +709,12 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         }
 
         // 7. W rows (16-byte chunks) into the lower half of WQ = [Qg ; W] (its Kg rows are consumed).
-        if (warp < 4) {
-            const int r = 16 * warp + (lane & 15);
-            for (int c0 = 0; c0 < DK; c0 += 32) {
+        //    Warps w and w + 4 share TMEM lanes 32 (w % 4) .. and take 64 columns each.
+        {
+            const int r = 16 * (warp & 3) + (lane & 15);
+            for (int c0 = (warp >> 2) * 64; c0 < (warp >> 2) * 64 + 64; c0 += 32) {
                 float v[32];
-                tmem_ld32(tm + 64 + ((uint32_t)(warp * 32) << 16) + c0, v);
+                tmem_ld32(tm + 64 + ((uint32_t)((warp & 3) * 32) << 16) + c0, v);
                 tmem_wait_ld();
                 if (lane < 16) {
 #pragma unroll
@@ -728,11 +731,14 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         tc_fence_before();
         sync();
 
-        // 8. WQ leaves in one bulk store; the slot is published once it completed.
+        // 8. WQ leaves in one bulk store; the slot is published once it completed:
+        //    the engine's first item at once (the scan is waiting for the first
+        //    positions), later ones during the next item.
         if (tid == kStoreTid) {
             bulk_s2g(gslot + SL_WQ, GA, 32768);
             bulk_commit();
             prev_pending = true;  // `cur` is the previous item of the next iteration
+            if (iter == 0) publish_prev(cur);
         }
     }
     // Publish the last item (after a failed wait: settle what is in flight).
