@@ -43,6 +43,8 @@ DEC_N, DEC_STEPS_POOL = 256, 64
 #   + o 32*128*2 = 49,280 B; plus S0 read and S_T written (2 MiB each at H=32).
 PREFILL_BYTES_PER_TOKEN = 3 * H * D * 2 + H * D * 4 + H * 4 + H * D * 2
 PREFILL_STATE_BYTES = 2 * H * D * D * 4
+# the Gated DeltaNet form: one fp32 gate per (token, head) instead of d_k
+GDN_BYTES_PER_TOKEN = 3 * H * D * 2 + H * 4 + H * 4 + H * D * 2
 # decode per step: state read + write, q,k,v bf16, log_alpha fp32, beta fp32, o bf16
 DECODE_BYTES = DEC_N * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
 
@@ -243,6 +245,27 @@ def run_kda(args, world, rank, local):
     bytes_pass = T8K * PREFILL_BYTES_PER_TOKEN + PREFILL_STATE_BYTES
     achieved = bytes_pass / (ms * 1e-3) / 1e9
 
+    # ---- the Gated DeltaNet form of the same workload: one gate per (token, head)
+    gdn = KI.prefill_workload("gdn_8k", dev, seed=rank)
+
+    def prefill_gdn():
+        kda.kda_prefill(gdn["q"], gdn["k"], gdn["v"], gdn["log_alpha"], gdn["beta"], gdn["S0"], cu,
+                        max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
+
+    for _ in range(args.warmup):
+        prefill_gdn()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        prefill_gdn()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    gdn_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    gdn_bytes = T8K * GDN_BYTES_PER_TOKEN + PREFILL_STATE_BYTES
+    gdn_gbs = gdn_bytes / (ev0.elapsed_time(ev1) / args.steps * 1e-3) / 1e9
+    del gdn
+
     # ---- end to end through the C ABI: pinned host inputs -> device -> host
     h_in = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v", "log_alpha", "beta", "S0")}
     h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -312,8 +335,15 @@ def run_kda(args, world, rank, local):
                      "algorithmic_bytes": bytes_pass, "peak_source": peak_src},
         "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": args.steps * launches_prefill + dsteps,
+        "gpu_launches": 2 * args.steps * launches_prefill + dsteps,
         "clocks": clk.summary(),
+        "gdn": {"value": world * T8K / (gdn_ms * 1e-3), "unit": "tokens/s", "ms_per_step": gdn_ms,
+                "workload": "gdn_8k: prefill_8k with one forget gate per (token, head) "
+                            "(log_alpha [T][H], the Gated DeltaNet form)",
+                "roofline": {"bound": "hbm", "achieved": gdn_gbs, "peak": hbm, "unit": "GB/s",
+                             "frac": gdn_gbs / hbm, "traffic": None,
+                             "kernel": "kda_prefill with KDA_FLAG_SCALAR_GATE (timed like the main line)",
+                             "algorithmic_bytes": gdn_bytes, "peak_source": peak_src}},
         "decode": {"value": DECODE_BYTES / (dec_us_max * 1e-6) / 1e9, "unit": "GB/s",
                    "us_per_step": dec_us_max, "steps": dsteps,
                    "workload": "decode_256: 256 seqs x 32 heads, d=128, bf16 q/k/v, fp32 state "

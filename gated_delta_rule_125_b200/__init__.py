@@ -19,12 +19,12 @@ __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size", "kda_
            "kda_prefill_workspace_min", "kda_status_string", "kda_version", "KDAError",
            "library_path", "load_library", "KDA_OK", "KDA_ERR_INVALID_ARG",
            "KDA_ERR_UNSUPPORTED", "KDA_ERR_MISALIGNED", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA",
-           "KDA_ERR_TIMEOUT", "KDA_FLAG_NO_L2NORM", "KDA_FLAG_EXACT"]
+           "KDA_ERR_TIMEOUT", "KDA_FLAG_NO_L2NORM", "KDA_FLAG_EXACT", "KDA_FLAG_SCALAR_GATE"]
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_MISALIGNED = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 4, 5, 6
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
-KDA_FLAG_NO_L2NORM, KDA_FLAG_EXACT = 0x1, 0x2
+KDA_FLAG_NO_L2NORM, KDA_FLAG_EXACT, KDA_FLAG_SCALAR_GATE = 0x1, 0x2, 0x4
 
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
                     "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
@@ -118,8 +118,9 @@ def _stream(stream, device):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _flags(l2norm, exact):
-    return (0 if l2norm else KDA_FLAG_NO_L2NORM) | (KDA_FLAG_EXACT if exact else 0)
+def _flags(l2norm, exact, scalar_gate=False):
+    return ((0 if l2norm else KDA_FLAG_NO_L2NORM) | (KDA_FLAG_EXACT if exact else 0) |
+            (KDA_FLAG_SCALAR_GATE if scalar_gate else 0))
 
 
 def kda_prefill_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype,
@@ -151,8 +152,8 @@ def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqle
                 stream=None):
     """Chunkwise KDA prefill (``kda_prefill`` in ``include/kda.h``).
 
-    q, k ``[T,H,dk]``, v ``[T,H,dv]`` (bf16 or fp32), log_alpha ``[T,H,dk]`` fp32,
-    beta ``[T,H]`` fp32, S0 ``[N,H,dk,dv]`` fp32 or None, cu_seqlens ``[N+1]`` int32
+    q, k ``[T,H,dk]``, v ``[T,H,dv]`` (bf16 or fp32), log_alpha ``[T,H,dk]`` fp32
+    (or ``[T,H]``: one gate per token and head, the Gated DeltaNet form), beta ``[T,H]`` fp32, S0 ``[N,H,dk,dv]`` fp32 or None, cu_seqlens ``[N+1]`` int32
     on the device or None. Returns ``(o [T,H,dv], S_T [N,H,dk,dv])``. Outputs and
     the workspace are allocated with torch when not given. ``max_seqlen`` (host
     int) avoids a device-to-host read of ``cu_seqlens``.
@@ -173,7 +174,7 @@ def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqle
     if S_T is None:
         S_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     code = _dtype_code(q)
-    flags = _flags(l2norm, exact)
+    flags = _flags(l2norm, exact, log_alpha.dim() == 2)
     if workspace is None:
         nbytes = lib.kda_prefill_workspace_size(N, T, max_seqlen, H, dk, dv, code, chunk, flags)
         if nbytes == 0:
@@ -200,7 +201,7 @@ def kda_prefill_noalloc(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, m
     N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
     rc = lib.kda_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
                                  _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, _dtype_code(q),
-                                 chunk, _flags(l2norm, exact), _ptr(o), _ptr(S_T),
+                                 chunk, _flags(l2norm, exact, log_alpha.dim() == 2), _ptr(o), _ptr(S_T),
                                  _stream(stream, q.device))
     if rc != KDA_OK:
         raise KDAError(rc, "kda_prefill_noalloc")
@@ -210,7 +211,8 @@ def kda_prefill_noalloc(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, m
 def kda_decode_step(q, k, v, log_alpha, beta, S, *, l2norm=True, o=None, stream=None):
     """One KDA decode step (``kda_decode_step`` in ``include/kda.h``), S updated in place.
 
-    q, k ``[N,H,dk]``, v ``[N,H,dv]``, log_alpha ``[N,H,dk]`` fp32, beta ``[N,H]`` fp32,
+    q, k ``[N,H,dk]``, v ``[N,H,dv]``, log_alpha ``[N,H,dk]`` (or ``[N,H]``, one gate per
+    head) fp32, beta ``[N,H]`` fp32,
     S ``[N,H,dk,dv]`` fp32. Returns o ``[N,H,dv]``.
     """
     lib = load_library()
@@ -219,7 +221,7 @@ def kda_decode_step(q, k, v, log_alpha, beta, S, *, l2norm=True, o=None, stream=
     if o is None:
         o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
     rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
-                             N, H, dk, dv, _dtype_code(q), _flags(l2norm, False), _ptr(o),
+                             N, H, dk, dv, _dtype_code(q), _flags(l2norm, False, log_alpha.dim() == 2), _ptr(o),
                              _stream(stream, q.device))
     if rc != KDA_OK:
         raise KDAError(rc, "kda_decode_step")

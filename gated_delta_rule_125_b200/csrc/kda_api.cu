@@ -10,9 +10,14 @@
 namespace {
 
 constexpr float kEps = 1e-6f;  // eps in q / max(||q||, eps)
-constexpr uint32_t kKnownFlags = KDA_FLAG_NO_L2NORM | KDA_FLAG_EXACT;
+constexpr uint32_t kKnownFlags = KDA_FLAG_NO_L2NORM | KDA_FLAG_EXACT | KDA_FLAG_SCALAR_GATE;
 
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// log_alpha: 16 bytes (tensor-map rows), or 4 with one gate per (token, head).
+bool gate_aligned(const void *p, uint32_t flags) {
+    return (flags & KDA_FLAG_SCALAR_GATE) ? (reinterpret_cast<uintptr_t>(p) & 3u) == 0 : aligned16(p);
+}
 
 bool dims_supported(int32_t dk, int32_t dv) {
     return (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
@@ -186,10 +191,11 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
     if (cu_seqlens == nullptr && num_seqs != 1) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
     if (!workspace) return KDA_ERR_WORKSPACE;
-    const void *ptrs[] = {q, k, v, log_alpha, S0, cu_seqlens, o, S_T, workspace};
+    const void *ptrs[] = {q, k, v, S0, cu_seqlens, o, S_T, workspace};
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_MISALIGNED;
     if (reinterpret_cast<uintptr_t>(beta) & 3u) return KDA_ERR_MISALIGNED;
+    if (!gate_aligned(log_alpha, flags)) return KDA_ERR_MISALIGNED;
 
     Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
     if (workspace_bytes < min_bytes(p)) return KDA_ERR_WORKSPACE;
@@ -199,6 +205,7 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
     a.cu = cu_seqlens; a.total = total_tokens;
     a.N = num_seqs; a.H = H; a.dk = dk; a.dv = dv;
     a.l2norm = (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1;
+    a.la_scalar = (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0;
     a.eps = kEps;
     a.o = o; a.S_T = S_T;
     a.slot_bytes = p.slot_bytes;
@@ -250,13 +257,15 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, log_alpha, S, o};
+    const void *ptrs[] = {q, k, v, S, o};
     for (const void *p : ptrs)
         if (!aligned16(p)) return KDA_ERR_MISALIGNED;
     if (reinterpret_cast<uintptr_t>(beta) & 3u) return KDA_ERR_MISALIGNED;
+    if (!gate_aligned(log_alpha, flags)) return KDA_ERR_MISALIGNED;
     cudaError_t e = kda::decode_step(q, k, v, log_alpha, beta, S, N, H, dk, dv,
                                      dtype == KDA_DTYPE_BF16, (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1,
-                                     kEps, o, reinterpret_cast<cudaStream_t>(stream));
+                                     (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0, kEps, o,
+                                     reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

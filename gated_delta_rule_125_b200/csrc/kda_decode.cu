@@ -25,7 +25,7 @@ template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ S, T *__restrict__ o, int l2norm, float eps) {
+              float *__restrict__ S, T *__restrict__ o, int l2norm, int la_scalar, float eps) {
     constexpr int CG = DV / 4;                // 16-byte column groups per state row
     constexpr int RPP = kDecodeThreads / CG;  // state rows covered per pass
     constexpr int R = DK / RPP;               // rows held per thread
@@ -78,7 +78,8 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         }
         if (lane == 0) s_misc[1] = qk * iq * ik;
     } else if (warp == 1) {
-        for (int i = lane; i < DK; i += 32) s_a[i] = expf(log_alpha[(size_t)unit * DK + i]);
+        for (int i = lane; i < DK; i += 32)
+            s_a[i] = expf(la_scalar ? log_alpha[unit] : log_alpha[(size_t)unit * DK + i]);
     } else if (warp == 2) {
         for (int j = lane; j < DV; j += 32) s_v[j] = IO<T>::ld(v + (size_t)unit * DV + j);
         if (lane == 0) s_misc[0] = beta[unit];
@@ -130,21 +131,21 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
 
 template <int DK, int DV, typename T>
 cudaError_t launch(const void *q, const void *k, const void *v, const float *la, const float *beta,
-                   float *S, int N, int H, int l2norm, float eps, void *o, cudaStream_t st) {
+                   float *S, int N, int H, int l2norm, int la_scalar, float eps, void *o, cudaStream_t st) {
     const unsigned units = (unsigned)N * (unsigned)H;
     decode_kernel<DK, DV, T><<<units, kDecodeThreads, 0, st>>>(
-        (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, eps);
+        (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps);
     return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t dispatch(const void *q, const void *k, const void *v, const float *la,
                      const float *beta, float *S, int N, int H, int dk, int dv, int l2norm,
-                     float eps, void *o, cudaStream_t st) {
-    if (dk == 128 && dv == 128) return launch<128, 128, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
-    if (dk == 128 && dv == 64) return launch<128, 64, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
-    if (dk == 64 && dv == 128) return launch<64, 128, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
-    if (dk == 64 && dv == 64) return launch<64, 64, T>(q, k, v, la, beta, S, N, H, l2norm, eps, o, st);
+                     int la_scalar, float eps, void *o, cudaStream_t st) {
+    if (dk == 128 && dv == 128) return launch<128, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
+    if (dk == 128 && dv == 64) return launch<128, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
+    if (dk == 64 && dv == 128) return launch<64, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
+    if (dk == 64 && dv == 64) return launch<64, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
     return cudaErrorInvalidValue;
 }
 
@@ -152,9 +153,9 @@ cudaError_t dispatch(const void *q, const void *k, const void *v, const float *l
 
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
-                        int l2norm, float eps, void *o, cudaStream_t st) {
-    if (bf16) return dispatch<__nv_bfloat16>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, eps, o, st);
-    return dispatch<float>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, eps, o, st);
+                        int l2norm, int la_scalar, float eps, void *o, cudaStream_t st) {
+    if (bf16) return dispatch<__nv_bfloat16>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, o, st);
+    return dispatch<float>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, o, st);
 }
 
 }  // namespace kda

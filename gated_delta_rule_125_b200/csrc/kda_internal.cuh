@@ -43,6 +43,7 @@ struct PrefillArgs {
     int64_t total;
     int N, H, dk, dv;
     int l2norm;
+    int la_scalar;  // log_alpha is [T][H] (one gate per token and head)
     float eps;
     void *o;
     float *S_T;
@@ -73,6 +74,6 @@ int *device_error_word();
 // decode step
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
-                        int l2norm, float eps, void *o, cudaStream_t st);
+                        int l2norm, int la_scalar, float eps, void *o, cudaStream_t st);
 
 }  // namespace kda

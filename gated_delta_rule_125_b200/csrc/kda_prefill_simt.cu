@@ -49,7 +49,7 @@ template <int DK, typename T>
 __global__ void __launch_bounds__(kThreads)
 prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
             const float *__restrict__ beta, const int32_t *__restrict__ cu, int64_t total, int H,
-            int N, int j0, int l2norm, float eps, char *__restrict__ slots, size_t slot_bytes) {
+            int N, int j0, int l2norm, int la_scalar, float eps, char *__restrict__ slots, size_t slot_bytes) {
     constexpr int LD = DK + 1;  // padded row stride: rows i, i+1 fall in different banks
     const int jl = blockIdx.x, s = blockIdx.y, h = blockIdx.z;
     int64_t bos, eos;
@@ -79,7 +79,7 @@ prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__res
             const size_t off = ((size_t)(t0 + r) * H + h) * DK + c;
             kv = IO<T>::ld(k + off);
             qv = IO<T>::ld(q + off);
-            lv = la[off];
+            lv = la_scalar ? la[(size_t)(t0 + r) * H + h] : la[off];
         }
         sK[r * LD + c] = kv;
         sQ[r * LD + c] = qv;
@@ -310,7 +310,7 @@ cudaError_t wave(const PrefillArgs &a, int j0, int nw, cudaStream_t st) {
         dim3 gp(nw, a.N, a.H);
         prep_kernel<DK, T><<<gp, kThreads, prep_smem<DK>(), st>>>(
             (const T *)a.q, (const T *)a.k, a.log_alpha, a.beta, a.cu, a.total, a.H, a.N, j0,
-            a.l2norm, a.eps, a.slots, a.slot_bytes);
+            a.l2norm, a.la_scalar, a.eps, a.slots, a.slot_bytes);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }

@@ -86,13 +86,14 @@ struct FusedParams {
     CUtensorMap tmap_v;   // v [T][H][128] bf16, box 64 x 1 x 64, SW128
     const bf16 *q, *k;
     const float *beta, *S0;
+    const float *la;  // log_alpha, read directly when it is one gate per (token, head)
     const int32_t *cu;
     float *S_T;
     bf16 *o;
     char *ws;
     int *err;
     long long total;  // tokens
-    int N, H, ns, R, l2norm;
+    int N, H, ns, R, l2norm, la_scalar;
     float eps;
 };
 
@@ -185,10 +186,10 @@ constexpr uint32_t PS_LA = 0;                  // log_alpha -> G [64][128] fp32;
 constexpr uint32_t PS_GA = 32768;              // [Qg ; Kg] K-major 128 x 128 -> WQ
 constexpr uint32_t PS_GB = PS_GA + 32768;      // q of the next item, then K e^-G (K-major 64 x 128)
 constexpr uint32_t PS_KS = PS_GB + 16384;      // k of the next item (K-major 64 x 128)
-constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[2][64] eGl[128]
-constexpr uint32_t PS_BAR = PS_SMALL + 1536;   // la, mma barriers; 3 item records; flags
+constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[2][64] eGl[128] gate[2][64]
+constexpr uint32_t PS_BAR = PS_SMALL + 2048;   // la, mma barriers; 3 item records; flags
 constexpr uint32_t PS_BYTES = PS_BAR + 128;
-constexpr uint32_t PS_STRIDE = 100352;         // engine 1 starts here (1024-aligned)
+constexpr uint32_t PS_STRIDE = 101376;         // engine 1 starts here (1024-aligned)
 constexpr int ALD = 68;                        // row stride of A / X (floats)
 constexpr uint32_t PS_AF = PS_LA;              // A, then X in place: 64 x 68 fp32
 constexpr uint32_t PS_R2 = PS_LA + 17408;      // solve scratch, 4 KB
@@ -326,7 +327,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     uint8_t *GB = sm + PS_GB;
     uint8_t *KS = sm + PS_KS;
     float *invq = reinterpret_cast<float *>(sm + PS_SMALL);
-    float *invk = invq + 64, *sbeta2 = invk + 64, *eGl = sbeta2 + 128;
+    float *invk = invq + 64, *sbeta2 = invk + 64, *eGl = sbeta2 + 128, *sgate2 = eGl + 128;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA
     // Item records of iterations it (current), it + 1 (claimed during the Gram)
     // and it - 1 (published by the store thread) in entries it % 3, ...
@@ -369,6 +370,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         it.valid = map_item(atomicAdd(&hd->claim, 1ull), P, ctl, it) ? 1 : 0;
     };
     auto fetch_la = [&](const ItemS &it) {  // store thread: log_alpha rows by one TMA box
+        if (P.la_scalar) return;             // one gate per row: with q, k below
         mbar_arrive_expect_tx(&bars[0], 32768u);
         tma_load_3d(G, &P.tmap_la, 0, it.h, (int)it.t0, &bars[0]);
         la_pending = true;
@@ -376,7 +378,8 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     // q and k rows rb + 16 m, chunk c8, by cp.async into GB / KS at the chunk's
     // place in a K-major SW128 64 x 128 tile (the thread reads back exactly what
     // it copied; K e^-G later overwrites q in place); beta of row `tid` (threads
-    // < 64) into sbeta2[buf]. Rows past the sequence are zero-filled.
+    // < 64) into sbeta2[buf], and with a scalar gate log_alpha of row `tid` into
+    // sgate2[buf]. Rows past the sequence are zero-filled.
     auto fetch_qk = [&](const ItemS &it, int buf) {
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -386,9 +389,11 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             cp_async16(GB + kmaj_chunk(r, c8, 64), P.q + off, bytes);
             cp_async16(KS + kmaj_chunk(r, c8, 64), P.k + off, bytes);
         }
-        if (tid < C)
-            cp_async4(sbeta2 + buf * 64 + tid, P.beta + (size_t)(it.t0 + (tid < it.n ? tid : 0)) * H + it.h,
-                      tid < it.n ? 4u : 0u);
+        if (tid < C) {
+            const size_t row = (size_t)(it.t0 + (tid < it.n ? tid : 0)) * H + it.h;
+            cp_async4(sbeta2 + buf * 64 + tid, P.beta + row, tid < it.n ? 4u : 0u);
+            if (P.la_scalar) cp_async4(sgate2 + buf * 64 + tid, P.la + row, tid < it.n ? 4u : 0u);
+        }
         cp_async_commit();
     };
 
@@ -422,14 +427,16 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         cp_async_wait_all();  // this thread's q, k chunks and beta
         sync();
         if (tid < DK) {
-            if (!mbar_wait(&bars[0], la_phase, kWaitNs)) sflag[1] = 1;
+            const float *sgate = sgate2 + (iter & 1) * 64;
+            if (!P.la_scalar && !mbar_wait(&bars[0], la_phase, kWaitNs)) sflag[1] = 1;
             const int c = tid;
             float run = 0.f;
 #pragma unroll
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float v[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = (r0 + i < n) ? G[(r0 + i) * DK + c] : 0.f;
+                for (int i = 0; i < 16; ++i)
+                    v[i] = (r0 + i < n) ? (P.la_scalar ? sgate[r0 + i] : G[(r0 + i) * DK + c]) : 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     run += v[i];
@@ -453,7 +460,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             const float inv = (r >= n) ? 0.f : (P.l2norm ? rsqrtf(fmaxf(ss, P.eps * P.eps)) : 1.f);
             ((tid < 192) ? invq : invk)[r] = inv;
         }
-        la_phase ^= 1;
+        if (!P.la_scalar) la_phase ^= 1;
         sync();
         if (sflag[1]) {
             failed = true;
@@ -1184,8 +1191,11 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
 
     FusedParams P;
     memset(&P, 0, sizeof(P));
-    if (a.total > 0 && (!make_la_map(&P.tmap_la, a.log_alpha, a.total, a.H) || !make_v_map(&P.tmap_v, a.v, a.total, a.H)))
+    if (a.total > 0 && ((!a.la_scalar && !make_la_map(&P.tmap_la, a.log_alpha, a.total, a.H)) ||
+                        !make_v_map(&P.tmap_v, a.v, a.total, a.H)))
         return cudaErrorInvalidValue;
+    P.la = a.log_alpha;
+    P.la_scalar = a.la_scalar;
     P.q = static_cast<const bf16 *>(a.q);
     P.k = static_cast<const bf16 *>(a.k);
     P.beta = a.beta;

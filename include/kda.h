@@ -22,8 +22,8 @@
  *   execution surface at the caller's next synchronisation.
  * - Arguments are validated on the host before anything is enqueued; on any
  *   error nothing is launched and the outputs are untouched.
- * - Every pointer must be 16-byte aligned, except beta (4-byte aligned);
- *   KDA_ERR_MISALIGNED otherwise.
+ * - Every pointer must be 16-byte aligned, except beta and, with
+ *   KDA_FLAG_SCALAR_GATE, log_alpha (4-byte aligned); KDA_ERR_MISALIGNED otherwise.
  *   Tensors are dense row-major with the layouts given below.
  * - Not checked (undefined behaviour if violated): cu_seqlens monotone with
  *   cu_seqlens[0] = 0 and cu_seqlens[N] = total_tokens; log_alpha finite and
@@ -61,6 +61,11 @@ typedef enum {
 /* flags */
 #define KDA_FLAG_NO_L2NORM 0x1 /* q, k are used as given (caller already normalised) */
 #define KDA_FLAG_EXACT 0x2     /* fp32 CUDA-core arithmetic even for bf16 inputs */
+/* Gated DeltaNet form ("[Kimi-2] Kimi Linear" §3): one forget gate per (token, head),
+ * S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T, i.e. the KDA update with
+ * alpha_t broadcast over the d_k channels. log_alpha is then [T][H] (prefill) or [N][H]
+ * (decode) fp32 instead of [..][H][dk]. */
+#define KDA_FLAG_SCALAR_GATE 0x4
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *kda_status_string(kda_status status);
@@ -98,7 +103,8 @@ int64_t kda_prefill_launches(int32_t num_seqs, int64_t total_tokens, int32_t max
  *
  *   q, k       [T][H][dk]  dtype         (T = total_tokens, all sequences packed)
  *   v          [T][H][dv]  dtype
- *   log_alpha  [T][H][dk]  fp32, <= 0    (per-key-channel log forget gate)
+ *   log_alpha  [T][H][dk]  fp32, <= 0    (per-key-channel log forget gate;
+ *                                         [T][H] with KDA_FLAG_SCALAR_GATE)
  *   beta       [T][H]      fp32          (write strength)
  *   S0         [N][H][dk][dv] fp32 entry states, or NULL for zeros
  *   cu_seqlens [N+1] int32 (device) token offsets of the N sequences, or NULL
@@ -167,7 +173,7 @@ kda_status kda_device_error(int32_t *code, int32_t reset);
  * ("[Kimi-2] Kimi Linear" §5: S_(t-1) + current token -> S_t + output).
  *
  *   q, k       [N][H][dk]  dtype          v [N][H][dv] dtype
- *   log_alpha  [N][H][dk]  fp32           beta [N][H] fp32
+ *   log_alpha  [N][H][dk]  fp32 ([N][H] with KDA_FLAG_SCALAR_GATE)   beta [N][H] fp32
  *   S          [N][H][dk][dv] fp32, read and overwritten with S_t
  *   o          [N][H][dv]  dtype, out
  *

@@ -23,7 +23,7 @@ import torch.nn.functional as F
 
 _BLOCK = 1 << 16  # tokens drawn per generator call (bounds fp32 temporaries)
 
-_IDS = {"q": 1, "k": 2, "v": 3, "beta": 4, "log_alpha": 5, "S0": 6, "len": 7}
+_IDS = {"q": 1, "k": 2, "v": 3, "beta": 4, "log_alpha": 5, "S0": 6, "len": 7, "log_alpha_scalar": 8}
 
 
 def _gen(device, seed, name, block=0):
@@ -73,6 +73,16 @@ def token_inputs(T, H, dk, dv, dtype=torch.bfloat16, device="cpu", seed=0, mu=-3
     return q, k, v, la, beta
 
 
+def scalar_gates(T, H, device="cpu", seed=0, mu=-3.0):
+    """log_alpha [T,H] fp32 = -softplus(N(mu, 1)): one forget gate per (token, head),
+    the Gated DeltaNet form; same distribution as the per-channel gates."""
+    la = torch.empty((T, H), dtype=torch.float32, device=device)
+    for b, t0 in enumerate(range(0, T, _BLOCK)):
+        n = min(_BLOCK, T - t0)
+        la[t0:t0 + n] = -F.softplus(_normal((n, H), device, seed, "log_alpha_scalar", b) + mu)
+    return la
+
+
 def initial_state(N, H, dk, dv, std, device="cpu", seed=0):
     """S0 [N,H,dk,dv] fp32 drawn N(0, std^2); zeros when ``std`` is 0 or None."""
     if not std:
@@ -88,6 +98,8 @@ WORKLOADS = {
                       s0_std=0.0),
     "prefill_1m": dict(lengths=[1 << 20], H=32, d=128, dtype="bf16", mu=-4.0, s0_std=0.0),
     "decode_256": dict(N=256, H=32, d=128, dtype="bf16", mu=-3.0, s0_std=0.01, steps=1000),
+    # Gated DeltaNet form of prefill_8k: one gate per (token, head)
+    "gdn_8k": dict(lengths=[8192], H=32, d=128, dtype="bf16", mu=-3.0, s0_std=0.01, scalar_gate=True),
 }
 
 
@@ -111,6 +123,8 @@ def prefill_workload(name, device="cpu", seed=0, lengths=None, heads=None):
     T = sum(lengths)
     q, k, v, la, beta = token_inputs(T, H, w["d"], w["d"], torch_dtype(w["dtype"]), device,
                                      seed, w["mu"])
+    if w.get("scalar_gate"):
+        la = scalar_gates(T, H, device, seed, w["mu"])
     S0 = initial_state(len(lengths), H, w["d"], w["d"], w["s0_std"], device, seed)
     return dict(q=q, k=k, v=v, log_alpha=la, beta=beta, S0=S0,
                 cu_seqlens=cu_from_lengths(lengths, device), lengths=lengths)

@@ -15,6 +15,9 @@ Functions and the passages they follow (pages cited by title and section):
   source's comment.
 * :func:`decode_step` -- one token of the recurrence on a resident state,
   §5 ("S_(t-1) + current token -> S_t + output").
+* :func:`output_gate` -- the layer's output step after the recurrence, §6 and
+  §6.3 (and "Kimi Linear — 逐通道的遺忘", 其他零件): head-wise RMSNorm of o_t,
+  then a product with a sigmoid gate computed from the input.
 
 Arrays are ``numpy`` (any real dtype; converted to fp64). Layouts::
 
@@ -145,3 +148,19 @@ def decode_step(q, k, v, log_alpha, beta, S, l2norm=True, eps=1e-6):
     if rc:
         raise RuntimeError("kda_oracle_decode_step failed (%d)" % rc)
     return o, Snew
+
+
+def output_gate(o, g, w, eps=1e-6):
+    """Head-wise RMSNorm and sigmoid output gate, per (token, head) over the d_v
+    channels: ``y = o / sqrt(mean(o^2) + eps) * w * sigmoid(g)``.
+
+    o, g ``[..., dv]`` (g is the gate's pre-activation), w ``[dv]`` (one weight
+    vector shared by the heads). The pages give no epsilon and do not say
+    whether the weight is per head; this reads both as the plainest choice
+    (a caller-chosen epsilon, one weight vector of d_v). fp64 numpy.
+    """
+    o = np.asarray(o, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
+    return o / rms * w / (1.0 + np.exp(-g))

@@ -73,6 +73,9 @@ def test_workspace_queries(lib):
     assert f(1, 10, 10, 1, 128, 128, 1, 32, 0) == 0
     assert f(1, 10, 10, 1, 128, 128, 7, 64, 0) == 0
     assert f(1, 10, 10, 1, 128, 128, 1, 64, 0x80) == 0
+    # the scalar-gate flag (log_alpha [T][H]) is a known flag
+    assert f(1, 8192, 8192, 32, 128, 128, 1, 64, kda.KDA_FLAG_SCALAR_GATE) > 0
+    assert f(1, 10, 10, 1, 64, 64, 0, 64, kda.KDA_FLAG_SCALAR_GATE | kda.KDA_FLAG_EXACT) > 0
 
 
 A = 0x10000  # fake 16-byte-aligned address, never dereferenced
@@ -132,7 +135,7 @@ def test_prefill_rejects(lib, over, code):
     (dict(H=-1), kda.KDA_ERR_INVALID_ARG),
     (dict(dk=32), kda.KDA_ERR_UNSUPPORTED),
     (dict(dt=2), kda.KDA_ERR_INVALID_ARG),
-    (dict(flags=0x4), kda.KDA_ERR_INVALID_ARG),
+    (dict(flags=0x8), kda.KDA_ERR_INVALID_ARG),
     (dict(v=A + 2), kda.KDA_ERR_MISALIGNED),
     (dict(S=A + 8), kda.KDA_ERR_MISALIGNED),
     (dict(o=A + 4), kda.KDA_ERR_MISALIGNED),

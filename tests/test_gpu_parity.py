@@ -327,3 +327,69 @@ def test_workload_decode_256():
         worst = max(worst, float(np.abs(host(o_all[t][seqs]) - o_ref).max()))
     assert worst <= 2e-2
     assert rel_fro(host(S[seqs]), S_ref) <= 1e-2
+
+
+# ------------------------------------------------- scalar gate (GDN) ----
+# KDA_FLAG_SCALAR_GATE: log_alpha [T,H], one gate per (token, head), the Gated
+# DeltaNet form of page "[Kimi-2] Kimi Linear" §3. The oracle is the KDA
+# recurrence with that gate broadcast over d_k (the reduction the oracle pin
+# `pin_gdn_special_case` checks against the explicit GDN matrices).
+
+def _with_scalar_gate(inp, seed):
+    T, H = inp["beta"].shape
+    g = KI.scalar_gates(T, H, DEV, seed)
+    dk = inp["q"].shape[-1]
+    gdn = dict(inp, log_alpha=g)
+    expanded = dict(inp, log_alpha=g[:, :, None].expand(T, H, dk).contiguous())
+    return gdn, expanded
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64), (torch.bfloat16, 64)])
+def test_scalar_gate_prefill(dtype, d):
+    """Both prefill paths: the scalar-gate call equals the per-channel call with the
+    gate broadcast (bit for bit), and both match the oracle; varlen with empty and
+    ragged sequences."""
+    inp = make([0, 130, 1, 257, 64], 3, d, d, dtype, seed=31)
+    gdn, expanded = _with_scalar_gate(inp, 31)
+    o1, S1 = run(gdn)
+    o2, S2 = run(expanded)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    check(o1, S1, expanded, dtype, label="scalar gate %s d=%d" % (dtype, d))
+
+
+def test_scalar_gate_strong_decay_tensor_core_path():
+    """Scalar gates large enough that every chunk takes the element-wise Gram."""
+    inp = make([300, 64, 130], 4, 128, 128, torch.bfloat16, seed=33)
+    gdn, expanded = _with_scalar_gate(inp, 33)
+    gdn["log_alpha"] = gdn["log_alpha"] * 400.0
+    expanded["log_alpha"] = expanded["log_alpha"] * 400.0
+    o, S_T = run(gdn)
+    check(o, S_T, expanded, torch.bfloat16, label="scalar gate strong decay")
+    assert kda.kda_device_error() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_scalar_gate_decode(dtype):
+    N, H, d, steps = 5, 3, 128, 4
+    w = KI.decode_workload(N, H, d, steps, dtype, DEV, seed=35, s0_std=0.1)
+    g = KI.scalar_gates(steps * N, H, DEV, 35).view(steps, N, H)
+    S = w["S0"].clone()
+    S_ref = host(S)
+    atol, stol = TOL[dtype]
+    for t in range(steps):
+        o = kda.kda_decode_step(w["q"][t], w["k"][t], w["v"][t], g[t], w["beta"][t], S)
+        torch.cuda.synchronize()
+        la = host(g[t])[:, :, None].repeat(d, axis=2)
+        o_ref, S_ref = oracle.decode_step(host(w["q"][t]), host(w["k"][t]), host(w["v"][t]), la,
+                                          host(w["beta"][t]), S_ref)
+        assert float(np.abs(host(o) - o_ref).max()) <= atol
+        assert rel_fro(host(S), S_ref) <= stol
+
+
+def test_workload_gdn_8k():
+    """The Gated DeltaNet form of prefill_8k; every output of heads {3, 30} vs the oracle."""
+    inp = KI.prefill_workload("gdn_8k", DEV)
+    o, S_T = run(inp)
+    T, H = inp["beta"].shape
+    expanded = dict(inp, log_alpha=inp["log_alpha"][:, :, None].expand(T, H, 128).contiguous())
+    check(o, S_T, expanded, torch.bfloat16, heads=[3, 30], label="gdn_8k")

@@ -360,3 +360,82 @@ def test_pins_catch_planted_mistakes(name, tmp_path):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, "planted mistake %r passed every pin" % name
+
+
+# ------------------------------------------------ output gate (§6.3) ----
+# oracle.output_gate: head-wise RMSNorm of o_t, then a sigmoid gate ("[Kimi-2]
+# Kimi Linear" §6 and §6.3). Pinned to hand arithmetic and to properties the
+# definition fixes; each planted mistake below must fail at least one pin.
+
+def og_pin_worked_example(f):
+    # o = (3, 4): mean square 12.5; w = (2, 1); g = (0, ln 3): sigmoid = (1/2, 3/4).
+    # y = (3 * 2 * 1/2, 4 * 1 * 3/4) / sqrt(12.5) = (3, 3) / sqrt(12.5).
+    y = f(np.array([[3.0, 4.0]]), np.array([[0.0, np.log(3.0)]]), np.array([2.0, 1.0]), 0.0)
+    np.testing.assert_allclose(y, [[3.0 / np.sqrt(12.5), 3.0 / np.sqrt(12.5)]], rtol=1e-14)
+
+
+def og_pin_unit_rms(f):
+    # w = 1 and a saturated gate leave the RMSNorm, whose mean square is 1 (eps = 0).
+    o = np.random.default_rng(1).normal(size=(5, 3, 16)) * 7.0
+    y = f(o, np.full_like(o, 60.0), np.ones(16), 0.0)
+    np.testing.assert_allclose(np.mean(y * y, axis=-1), 1.0, rtol=1e-12)
+
+
+def og_pin_scale_invariance(f):
+    rng = np.random.default_rng(2)
+    o, g, w = rng.normal(size=(4, 2, 8)), rng.normal(size=(4, 2, 8)), rng.normal(size=8)
+    np.testing.assert_allclose(f(3.5 * o, g, w, 0.0), f(o, g, w, 0.0), rtol=1e-12)
+
+
+def og_pin_heads_independent(f):
+    # head-wise: a head's output does not depend on the other heads' values
+    rng = np.random.default_rng(3)
+    o, g, w = rng.normal(size=(4, 2, 8)), rng.normal(size=(4, 2, 8)), rng.normal(size=8)
+    o2 = o.copy()
+    o2[:, 1] *= 100.0
+    np.testing.assert_allclose(f(o2, g, w, 1e-6)[:, 0], f(o, g, w, 1e-6)[:, 0], rtol=1e-14)
+
+
+def og_pin_zero_row(f):
+    # eps keeps an all-zero row finite (and zero)
+    y = f(np.zeros((2, 8)), np.zeros((2, 8)), np.ones(8), 1e-6)
+    assert np.all(y == 0.0)
+
+
+OG_PINS = [og_pin_worked_example, og_pin_unit_rms, og_pin_scale_invariance,
+           og_pin_heads_independent, og_pin_zero_row]
+
+
+@pytest.mark.parametrize("pin", OG_PINS, ids=lambda p: p.__name__)
+def test_output_gate_pin(pin):
+    pin(oracle.output_gate)
+
+
+def _og_mutant(kind):
+    def f(o, g, w, eps):
+        o, g, w = (np.asarray(x, dtype=np.float64) for x in (o, g, w))
+        ms = np.mean(o * o, axis=-1, keepdims=True)
+        if kind == "sum_not_mean":
+            ms = np.sum(o * o, axis=-1, keepdims=True)
+        if kind == "across_heads":
+            ms = np.mean(o * o, axis=(-2, -1), keepdims=True) if o.ndim > 2 else ms
+        if kind == "no_eps":
+            eps = 0.0
+        gate = np.tanh(g) if kind == "tanh_gate" else 1.0 / (1.0 + np.exp(-g))
+        if kind == "no_weight":
+            w = np.ones_like(w)
+        with np.errstate(invalid="ignore", divide="ignore"):
+            return o / np.sqrt(ms + eps) * w * gate
+    return f
+
+
+@pytest.mark.parametrize("kind", ["sum_not_mean", "across_heads", "no_eps", "tanh_gate", "no_weight"])
+def test_output_gate_pins_catch_planted_mistakes(kind):
+    f = _og_mutant(kind)
+    failed = 0
+    for pin in OG_PINS:
+        try:
+            pin(f)
+        except AssertionError:
+            failed += 1
+    assert failed > 0, kind
