@@ -266,6 +266,30 @@ def run_kda(args, world, rank, local):
     gdn_gbs = gdn_bytes / (ev0.elapsed_time(ev1) / args.steps * 1e-3) / 1e9
     del gdn
 
+    # ---- the same workload with the layer's output step fused (RMSNorm + sigmoid gate)
+    g_gen = torch.Generator(device=dev)
+    g_gen.manual_seed(1000 + rank)
+    og = (torch.randn((T8K, H, D), generator=g_gen, device=dev).to(torch.bfloat16),
+          1.0 + 0.1 * torch.randn((D,), generator=g_gen, device=dev), 1e-6)
+
+    def prefill_gated():
+        kda.kda_prefill(q, k, v, la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws,
+                        out_gate=og)
+
+    for _ in range(args.warmup):
+        prefill_gated()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        prefill_gated()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    og_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    og_bytes = T8K * (PREFILL_BYTES_PER_TOKEN + H * D * 2) + PREFILL_STATE_BYTES
+    og_gbs = og_bytes / (ev0.elapsed_time(ev1) / args.steps * 1e-3) / 1e9
+    del og
+
     # ---- end to end through the C ABI: pinned host inputs -> device -> host
     h_in = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v", "log_alpha", "beta", "S0")}
     h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -335,7 +359,7 @@ def run_kda(args, world, rank, local):
                      "algorithmic_bytes": bytes_pass, "peak_source": peak_src},
         "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps * launches_prefill + dsteps,
+        "gpu_launches": 3 * args.steps * launches_prefill + dsteps,
         "clocks": clk.summary(),
         "gdn": {"value": world * T8K / (gdn_ms * 1e-3), "unit": "tokens/s", "ms_per_step": gdn_ms,
                 "workload": "gdn_8k: prefill_8k with one forget gate per (token, head) "
@@ -344,6 +368,13 @@ def run_kda(args, world, rank, local):
                              "frac": gdn_gbs / hbm, "traffic": None,
                              "kernel": "kda_prefill with KDA_FLAG_SCALAR_GATE (timed like the main line)",
                              "algorithmic_bytes": gdn_bytes, "peak_source": peak_src}},
+        "output_gate": {"value": world * T8K / (og_ms * 1e-3), "unit": "tokens/s", "ms_per_step": og_ms,
+                        "workload": "prefill_8k with the output step fused: RMSNorm over d_v and "
+                                    "a sigmoid gate [T][H][d_v] bf16 (page section 6.3)",
+                        "roofline": {"bound": "hbm", "achieved": og_gbs, "peak": hbm, "unit": "GB/s",
+                                     "frac": og_gbs / hbm, "traffic": None,
+                                     "kernel": "kda_prefill_ex with a kda_output_gate",
+                                     "algorithmic_bytes": og_bytes, "peak_source": peak_src}},
         "decode": {"value": DECODE_BYTES / (dec_us_max * 1e-6) / 1e9, "unit": "GB/s",
                    "us_per_step": dec_us_max, "steps": dsteps,
                    "workload": "decode_256: 256 seqs x 32 heads, d=128, bf16 q/k/v, fp32 state "

@@ -28,7 +28,13 @@ KDA_FLAG_NO_L2NORM, KDA_FLAG_EXACT, KDA_FLAG_SCALAR_GATE = 0x1, 0x2, 0x4
 
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
                     "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
-                    "kda_decode_step", "kda_device_error", "kda_prefill_noalloc")
+                    "kda_prefill_ex", "kda_decode_step", "kda_decode_step_ex", "kda_device_error",
+                    "kda_prefill_noalloc")
+
+
+class OutputGate(ctypes.Structure):
+    """``kda_output_gate``: the fused output step (RMSNorm over d_v, sigmoid gate)."""
+    _fields_ = [("gate", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 _lib = None
 
@@ -70,6 +76,13 @@ def load_library():
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
                                     u32, vp, vp]
     lib.kda_decode_step.restype = ctypes.c_int
+    og = ctypes.POINTER(OutputGate)
+    lib.kda_prefill_ex.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32, i32,
+                                   ctypes.c_int, i32, u32, og, vp, fp, vp, sz, vp]
+    lib.kda_prefill_ex.restype = ctypes.c_int
+    lib.kda_decode_step_ex.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
+                                       u32, og, vp, vp]
+    lib.kda_decode_step_ex.restype = ctypes.c_int
     lib.kda_prefill_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32,
                                         i32, ctypes.c_int, i32, u32, vp, fp, vp]
     lib.kda_prefill_noalloc.restype = ctypes.c_int
@@ -112,6 +125,14 @@ def _ptr(t):
     return t.data_ptr() or None
 
 
+def _out_gate(out_gate):
+    """(gate, weight, eps) -> a ``kda_output_gate`` (None -> NULL)."""
+    if out_gate is None:
+        return None
+    g, w, eps = out_gate
+    return ctypes.byref(OutputGate(_ptr(g), _ptr(w), float(eps)))
+
+
 def _stream(stream, device):
     if stream is None:
         stream = torch.cuda.current_stream(device)
@@ -149,14 +170,16 @@ def kda_prefill_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, w
 
 def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqlen=None,
                 chunk=64, l2norm=True, exact=False, o=None, S_T=None, workspace=None,
-                stream=None):
+                out_gate=None, stream=None):
     """Chunkwise KDA prefill (``kda_prefill`` in ``include/kda.h``).
 
     q, k ``[T,H,dk]``, v ``[T,H,dv]`` (bf16 or fp32), log_alpha ``[T,H,dk]`` fp32
     (or ``[T,H]``: one gate per token and head, the Gated DeltaNet form), beta ``[T,H]`` fp32, S0 ``[N,H,dk,dv]`` fp32 or None, cu_seqlens ``[N+1]`` int32
     on the device or None. Returns ``(o [T,H,dv], S_T [N,H,dk,dv])``. Outputs and
     the workspace are allocated with torch when not given. ``max_seqlen`` (host
-    int) avoids a device-to-host read of ``cu_seqlens``.
+    int) avoids a device-to-host read of ``cu_seqlens``. ``out_gate = (gate
+    [T,H,dv] (dtype of q), weight [dv] fp32, eps)`` fuses the layer's output step
+    (``kda_prefill_ex``): o <- RMSNorm(o) * weight * sigmoid(gate).
     """
     lib = load_library()
     T, H, dk = q.shape
@@ -180,10 +203,10 @@ def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqle
         if nbytes == 0:
             nbytes = 256
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    rc = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                         _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, code, chunk, flags,
-                         _ptr(o), _ptr(S_T), _ptr(workspace), workspace.numel(),
-                         _stream(stream, dev))
+    rc = lib.kda_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                            _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, code, chunk, flags,
+                            _out_gate(out_gate), _ptr(o), _ptr(S_T), _ptr(workspace),
+                            workspace.numel(), _stream(stream, dev))
     if rc != KDA_OK:
         raise KDAError(rc, "kda_prefill")
     return o, S_T
@@ -208,7 +231,8 @@ def kda_prefill_noalloc(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, m
     return o, S_T
 
 
-def kda_decode_step(q, k, v, log_alpha, beta, S, *, l2norm=True, o=None, stream=None):
+def kda_decode_step(q, k, v, log_alpha, beta, S, *, l2norm=True, o=None, out_gate=None,
+                    stream=None):
     """One KDA decode step (``kda_decode_step`` in ``include/kda.h``), S updated in place.
 
     q, k ``[N,H,dk]``, v ``[N,H,dv]``, log_alpha ``[N,H,dk]`` (or ``[N,H]``, one gate per
@@ -220,9 +244,9 @@ def kda_decode_step(q, k, v, log_alpha, beta, S, *, l2norm=True, o=None, stream=
     dv = v.shape[-1]
     if o is None:
         o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
-    rc = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
-                             N, H, dk, dv, _dtype_code(q), _flags(l2norm, False, log_alpha.dim() == 2), _ptr(o),
-                             _stream(stream, q.device))
+    rc = lib.kda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
+                                N, H, dk, dv, _dtype_code(q), _flags(l2norm, False, log_alpha.dim() == 2),
+                                _out_gate(out_gate), _ptr(o), _stream(stream, q.device))
     if rc != KDA_OK:
         raise KDAError(rc, "kda_decode_step")
     return o

@@ -19,6 +19,14 @@ bool gate_aligned(const void *p, uint32_t flags) {
     return (flags & KDA_FLAG_SCALAR_GATE) ? (reinterpret_cast<uintptr_t>(p) & 3u) == 0 : aligned16(p);
 }
 
+// The fused output step's arguments (nullptr: none).
+kda_status check_output_gate(const kda_output_gate *g, bool any_tokens) {
+    if (!g) return KDA_OK;
+    if (!(g->eps > 0.f) || (any_tokens && (!g->gate || !g->weight))) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(g->gate) || (reinterpret_cast<uintptr_t>(g->weight) & 3u)) return KDA_ERR_MISALIGNED;
+    return KDA_OK;
+}
+
 bool dims_supported(int32_t dk, int32_t dv) {
     return (dk == 64 || dk == 128) && (dv == 64 || dv == 128);
 }
@@ -186,8 +194,20 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
                        int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
                        void *o, float *S_T, void *workspace, size_t workspace_bytes,
                        kda_stream_t stream) {
+    return kda_prefill_ex(q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, total_tokens,
+                          max_seqlen, H, dk, dv, dtype, chunk, flags, nullptr, o, S_T, workspace,
+                          workspace_bytes, stream);
+}
+
+kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *S0, const int32_t *cu_seqlens,
+                          int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                          int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                          const kda_output_gate *out_gate, void *o, float *S_T, void *workspace,
+                          size_t workspace_bytes, kda_stream_t stream) {
     kda_status rc = check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags);
     if (rc != KDA_OK) return rc;
+    if ((rc = check_output_gate(out_gate, total_tokens > 0)) != KDA_OK) return rc;
     if (cu_seqlens == nullptr && num_seqs != 1) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
     if (!workspace) return KDA_ERR_WORKSPACE;
@@ -207,6 +227,9 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
     a.l2norm = (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1;
     a.la_scalar = (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0;
     a.eps = kEps;
+    a.og_gate = out_gate ? out_gate->gate : nullptr;
+    a.og_w = out_gate ? out_gate->weight : nullptr;
+    a.og_eps = out_gate ? out_gate->eps : 0.f;
     a.o = o; a.S_T = S_T;
     a.slot_bytes = p.slot_bytes;
 
@@ -231,6 +254,7 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
         const int n = (int)std::min<int64_t>(nw, p.max_chunks - j0);
         if (kda::simt_prefill_wave(a, (int)j0, n, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
     }
+    if (a.og_gate && total_tokens > 0 && kda::simt_output_gate(a, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
 }
 
@@ -252,6 +276,14 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
                            const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
                            int32_t dv, kda_dtype dtype, uint32_t flags, void *o,
                            kda_stream_t stream) {
+    return kda_decode_step_ex(q, k, v, log_alpha, beta, S, N, H, dk, dv, dtype, flags, nullptr, o,
+                              stream);
+}
+
+kda_status kda_decode_step_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
+                              int32_t dv, kda_dtype dtype, uint32_t flags,
+                              const kda_output_gate *out_gate, void *o, kda_stream_t stream) {
     if (N < 1 || H < 1 || dk < 1 || dv < 1 || (int64_t)N * H > INT32_MAX) return KDA_ERR_INVALID_ARG;
     if (flags & ~kKnownFlags) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
@@ -262,10 +294,14 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
         if (!aligned16(p)) return KDA_ERR_MISALIGNED;
     if (reinterpret_cast<uintptr_t>(beta) & 3u) return KDA_ERR_MISALIGNED;
     if (!gate_aligned(log_alpha, flags)) return KDA_ERR_MISALIGNED;
+    const kda_status rc = check_output_gate(out_gate, true);
+    if (rc != KDA_OK) return rc;
     cudaError_t e = kda::decode_step(q, k, v, log_alpha, beta, S, N, H, dk, dv,
                                      dtype == KDA_DTYPE_BF16, (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1,
-                                     (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0, kEps, o,
-                                     reinterpret_cast<cudaStream_t>(stream));
+                                     (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0, kEps,
+                                     out_gate ? out_gate->gate : nullptr,
+                                     out_gate ? out_gate->weight : nullptr, out_gate ? out_gate->eps : 0.f,
+                                     o, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

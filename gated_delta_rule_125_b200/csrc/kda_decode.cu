@@ -25,7 +25,8 @@ template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
-              float *__restrict__ S, T *__restrict__ o, int l2norm, int la_scalar, float eps) {
+              float *__restrict__ S, T *__restrict__ o, int l2norm, int la_scalar, float eps,
+              const T *__restrict__ og_gate, const float *__restrict__ og_w, float og_eps) {
     constexpr int CG = DV / 4;                // 16-byte column groups per state row
     constexpr int RPP = kDecodeThreads / CG;  // state rows covered per pass
     constexpr int R = DK / RPP;               // rows held per thread
@@ -34,6 +35,7 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
     __shared__ float s_q[DK], s_k[DK], s_a[DK], s_v[DV], s_u[DV];
     __shared__ float s_red[RPP][CG][8];
     __shared__ float s_misc[2];  // beta, k.q
+    __shared__ float s_o[DV], s_gss[DV / 32];  // fused output step: o, per-warp sums of o^2
 
     const int unit = blockIdx.x;  // sequence * H + head
     const int tid = threadIdx.x;
@@ -110,9 +112,29 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         }
         const float u = s_misc[0] * (s_v[j] - yy);
         s_u[j] = u;
-        IO<T>::st(o + (size_t)unit * DV + j, zz + s_misc[1] * u);
+        const float oj = zz + s_misc[1] * u;
+        if (og_gate) {
+            // fused output step: keep o_j for the head's RMSNorm (sum of squares per warp)
+            s_o[j] = oj;
+            float ss = oj * oj;
+#pragma unroll
+            for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            if ((j & 31) == 0) s_gss[j >> 5] = ss;
+        } else {
+            IO<T>::st(o + (size_t)unit * DV + j, oj);
+        }
     }
     __syncthreads();
+    // 4b. Fused output step: o <- o / sqrt(mean(o^2) + eps) * w * sigmoid(gate).
+    if (og_gate && tid < DV) {
+        const int j = tid;
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < DV / 32; ++w) tot += s_gss[w];
+        const float gv = IO<T>::ld(og_gate + (size_t)unit * DV + j);
+        const float y = s_o[j] * rsqrtf(tot / DV + og_eps) * og_w[j] / (1.f + __expf(-gv));
+        IO<T>::st(o + (size_t)unit * DV + j, y);
+    }
 
     // 5. S_t = Diag(alpha) S + k u^T, written back once.
     const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[4 * cg]);
@@ -131,21 +153,24 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
 
 template <int DK, int DV, typename T>
 cudaError_t launch(const void *q, const void *k, const void *v, const float *la, const float *beta,
-                   float *S, int N, int H, int l2norm, int la_scalar, float eps, void *o, cudaStream_t st) {
+                   float *S, int N, int H, int l2norm, int la_scalar, float eps, const void *og_gate,
+                   const float *og_w, float og_eps, void *o, cudaStream_t st) {
     const unsigned units = (unsigned)N * (unsigned)H;
     decode_kernel<DK, DV, T><<<units, kDecodeThreads, 0, st>>>(
-        (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps);
+        (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps,
+        (const T *)og_gate, og_w, og_eps);
     return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t dispatch(const void *q, const void *k, const void *v, const float *la,
                      const float *beta, float *S, int N, int H, int dk, int dv, int l2norm,
-                     int la_scalar, float eps, void *o, cudaStream_t st) {
-    if (dk == 128 && dv == 128) return launch<128, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
-    if (dk == 128 && dv == 64) return launch<128, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
-    if (dk == 64 && dv == 128) return launch<64, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
-    if (dk == 64 && dv == 64) return launch<64, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, o, st);
+                     int la_scalar, float eps, const void *og, const float *ow, float oe, void *o,
+                     cudaStream_t st) {
+    if (dk == 128 && dv == 128) return launch<128, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
+    if (dk == 128 && dv == 64) return launch<128, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
+    if (dk == 64 && dv == 128) return launch<64, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
+    if (dk == 64 && dv == 64) return launch<64, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
     return cudaErrorInvalidValue;
 }
 
@@ -153,9 +178,12 @@ cudaError_t dispatch(const void *q, const void *k, const void *v, const float *l
 
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
-                        int l2norm, int la_scalar, float eps, void *o, cudaStream_t st) {
-    if (bf16) return dispatch<__nv_bfloat16>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, o, st);
-    return dispatch<float>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, o, st);
+                        int l2norm, int la_scalar, float eps, const void *og_gate, const float *og_w,
+                        float og_eps, void *o, cudaStream_t st) {
+    if (bf16)
+        return dispatch<__nv_bfloat16>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, og_gate, og_w,
+                                       og_eps, o, st);
+    return dispatch<float>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, og_gate, og_w, og_eps, o, st);
 }
 
 }  // namespace kda

@@ -45,6 +45,10 @@ struct PrefillArgs {
     int l2norm;
     int la_scalar;  // log_alpha is [T][H] (one gate per token and head)
     float eps;
+    // fused output step (og_gate == nullptr: none): o <- RMSNorm(o) * og_w * sigmoid(og_gate)
+    const void *og_gate;
+    const float *og_w;
+    float og_eps;
     void *o;
     float *S_T;
     // workspace
@@ -74,6 +78,9 @@ int *device_error_word();
 // decode step
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
-                        int l2norm, int la_scalar, float eps, void *o, cudaStream_t st);
+                        int l2norm, int la_scalar, float eps, const void *og_gate, const float *og_w,
+                        float og_eps, void *o, cudaStream_t st);
+// fp32 CUDA-core path: the output step applied to o in place after the prefill.
+cudaError_t simt_output_gate(const PrefillArgs &a, bool bf16, cudaStream_t st);
 
 }  // namespace kda

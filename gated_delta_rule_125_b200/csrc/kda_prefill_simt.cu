@@ -325,6 +325,46 @@ cudaError_t wave(const PrefillArgs &a, int j0, int nw, cudaStream_t st) {
 
 size_t simt_slot_bytes(int dk) { return dk == 64 ? Slot<64>::BYTES : Slot<128>::BYTES; }
 
+// Output step after the fp32 prefill, in place on o: one warp per (token, head)
+// row, o <- o / sqrt(mean(o^2) + eps) * w * sigmoid(gate) over the DV channels.
+template <int DV, typename T>
+__global__ void __launch_bounds__(256)
+output_gate_kernel(T *__restrict__ o, const T *__restrict__ gate, const float *__restrict__ w, float eps,
+                   int64_t rows) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float x[DV / 32], ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < DV / 32; ++i) {
+        x[i] = IO<T>::ld(o + row * DV + lane + 32 * i);
+        ss += x[i] * x[i];
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float r = rsqrtf(ss / DV + eps);
+#pragma unroll
+    for (int i = 0; i < DV / 32; ++i) {
+        const int c = lane + 32 * i;
+        const float g = IO<T>::ld(gate + row * DV + c);
+        IO<T>::st(o + row * DV + c, x[i] * r * w[c] / (1.f + __expf(-g)));
+    }
+}
+
+template <int DV, typename T>
+cudaError_t output_gate(const PrefillArgs &a, cudaStream_t st) {
+    const int64_t rows = a.total * a.H;
+    output_gate_kernel<DV, T><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+        (T *)a.o, (const T *)a.og_gate, a.og_w, a.og_eps, rows);
+    return cudaGetLastError();
+}
+
+cudaError_t simt_output_gate(const PrefillArgs &a, bool bf16, cudaStream_t st) {
+    if (a.dv == 128) return bf16 ? output_gate<128, __nv_bfloat16>(a, st) : output_gate<128, float>(a, st);
+    if (a.dv == 64) return bf16 ? output_gate<64, __nv_bfloat16>(a, st) : output_gate<64, float>(a, st);
+    return cudaErrorInvalidValue;
+}
+
 cudaError_t simt_prefill_wave(const PrefillArgs &a, int j0, int nw, bool bf16, cudaStream_t st) {
     if (a.dk == 128) return bf16 ? wave<128, __nv_bfloat16>(a, j0, nw, st) : wave<128, float>(a, j0, nw, st);
     if (a.dk == 64) return bf16 ? wave<64, __nv_bfloat16>(a, j0, nw, st) : wave<64, float>(a, j0, nw, st);

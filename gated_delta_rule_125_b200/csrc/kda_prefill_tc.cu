@@ -65,7 +65,9 @@ constexpr uint32_t SL_BYTES = 66560;
 // ----------------------------------------------------------- workspace ----
 // [header 256 B][L: int64 per stream][order: int32 per stream] (1 KiB)
 // [ustart: int64 per unit][nch: int32 per unit] (1 KiB aligned)
-// [ready: int32 x kMaxStreams*kMaxRing][freed: same][ring: NS*R slots]
+// [ready: int32 x kMaxStreams*kMaxRing][freed: same]
+// [output-step exchange: per scan CTA, 2 x 64 words (row sum of squares, position tag)]
+// [ring: NS*R slots]
 struct Hdr {
     unsigned long long claim;  // next item to claim
     long long total;           // items over all streams
@@ -79,7 +81,9 @@ constexpr size_t kFlagInts = (size_t)kTcMaxStreams * kMaxRing;
 __host__ __device__ inline size_t ru1024(size_t x) { return (x + 1023) & ~size_t(1023); }
 __host__ __device__ inline size_t ws_nch(long long NH) { return WS_USTART + 8 * (size_t)NH; }
 __host__ __device__ inline size_t ws_flags(long long NH) { return ru1024(ws_nch(NH) + 4 * (size_t)NH); }
-__host__ __device__ inline size_t ws_ring(long long NH) { return ws_flags(NH) + 2 * kFlagInts * sizeof(int); }
+__host__ __device__ inline size_t ws_xch(long long NH) { return ws_flags(NH) + 2 * kFlagInts * sizeof(int); }
+constexpr size_t kXchWords = (size_t)kTcMaxStreams * 2 * 2 * 64;
+__host__ __device__ inline size_t ws_ring(long long NH) { return ru1024(ws_xch(NH) + kXchWords * 8); }
 
 struct FusedParams {
     CUtensorMap tmap_la;  // log_alpha [T][H][128] fp32, box 128 x 1 x 64
@@ -90,6 +94,9 @@ struct FusedParams {
     const int32_t *cu;
     float *S_T;
     bf16 *o;
+    const bf16 *og_gate;  // fused output step (nullptr: none)
+    const float *og_w;
+    float og_eps;
     char *ws;
     int *err;
     long long total;  // tokens
@@ -107,11 +114,13 @@ __device__ __forceinline__ void fail_call(const FusedParams &P) {
     flag_error(P.err, 1);
 }
 // Wait until *flag >= target (gpu-scope acquire); false on abort or after kWaitNs.
-__device__ __forceinline__ bool wait_flag_geq(const int *flag, int target, const int *abort_flag) {
+// Polls every `sleep_ns` (0: back to back, for waits expected to be short).
+__device__ __forceinline__ bool wait_flag_geq(const int *flag, int target, const int *abort_flag,
+                                              unsigned sleep_ns = 100) {
     if (ld_acquire_gpu(flag) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        __nanosleep(100);
+        if (sleep_ns) __nanosleep(sleep_ns);
         if (ld_acquire_gpu(flag) >= target) return true;
         if (ld_relaxed_gpu(abort_flag) || globaltimer_ns() - t0 > kWaitNs) return false;
     }
@@ -138,6 +147,7 @@ plan_kernel(const int32_t *__restrict__ cu, long long total, int N, int H, int n
         nch[u] = (int)((eos - bos + C - 1) / C);
     }
     for (size_t i = tid; i < 2 * kFlagInts; i += PLAN_T) flags[i] = 0;
+    for (size_t i = tid; i < kXchWords; i += PLAN_T) reinterpret_cast<unsigned long long *>(ws + ws_xch(NH))[i] = 0;
     __syncthreads();
     // one warp per stream: lanes own contiguous runs of the stream's units
     for (int st = warp; st < ns; st += PLAN_T / 32) {
@@ -207,13 +217,16 @@ constexpr uint32_t SS_B = 2 * SA_BYTES;         // T of B0 is preceded by the la
 constexpr uint32_t SS_V = SS_B + 3 * SB_BYTES;
 constexpr uint32_t SS_S = SS_V + 4 * SV_BYTES;  // [128 (c)][64 (j)] MN-major bf16 state
 constexpr uint32_t SS_U = SS_S + 16384;         // [64 (r)][64 (j)] MN-major bf16 pseudo-values
-constexpr uint32_t SS_BAR = SS_U + 8192;        // 24 mbarriers, then the consumed-position counter
-constexpr uint32_t SS_BYTES = SS_BAR + 256;
+constexpr uint32_t SS_BAR = SS_U + 8192;        // 31 mbarriers, the consumed-position counter, a flag
+constexpr uint32_t SS_OGW = SS_BAR + 512;       // output-step weights of this CTA's 64 columns
+constexpr uint32_t SS_BYTES = SS_OGW + 256;
 constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 512;
 // scan mbarrier indices
 constexpr int MB_FULLA = 0, MB_FULLB = 2, MB_FULLV = 5, MB_EMPTYA = 9, MB_EMPTYB = 11, MB_EMPTYV = 14,
-              MB_U = 18, MB_S = 19, MB_O = 20, MB_UREADY = 21, MB_SREADY = 22, MB_FIN = 23, MB_COUNT = 24;
-constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = 256;  // scan TMEM columns (X, Y double-buffered)
+              MB_U = 18, MB_S = 19, MB_O = 20, MB_UREADY = 24, MB_SREADY = 25, MB_FIN = 26, MB_OREADY = 27,
+              MB_COUNT = 31;  // MB_O and MB_OREADY: one barrier per Y buffer
+constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = 384;  // scan TMEM columns: X x2, Y x4, Z
+constexpr int NY = 4;                                  // Y buffers: the O epilogue may lag NY - 1 chunks
 
 // Per-CTA control block after both layouts.
 struct Ctrl {
@@ -226,6 +239,8 @@ struct Ctrl {
 constexpr uint32_t CTRL_OFF = SS_BYTES > 2 * PS_STRIDE ? SS_BYTES : 2 * PS_STRIDE;
 constexpr uint32_t SMEM_ALLOC = CTRL_OFF + 512 + 1024;  // + alignment slack
 static_assert(2 * PS_STRIDE <= CTRL_OFF, "prep engines overlap the control block");
+static_assert(MB_O + NY == MB_UREADY && MB_OREADY + NY == MB_COUNT, "scan barrier indices");
+static_assert(MB_COUNT * 8 + 16 <= SS_OGW - SS_BAR, "scan barrier area");
 static_assert(sizeof(Ctrl) <= 512, "control block");
 
 // ---------------------------------------------------------------- prep ----
@@ -762,7 +777,9 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
 // Scan CTA for stream st, state columns [64 jv, 64 jv + 64). Warps 0..7:
 // TMEM-lane epilogues (warp w: lanes 32 (w % 4) .., columns 32 (w / 4) ..);
 // warp 8: MMA issue; warp 9: ring-slot copies; warp 10: V copies; warp 11: slot
-// release. TMEM lanes 0..63 hold O = Q e^G S + P U,
+// release; warps 12, 13: O rows to HBM (with the fused output step: RMSNorm over
+// the row's 128 columns, the two scan CTAs of a stream exchanging their halves'
+// sums of squares, and the sigmoid gate). TMEM lanes 0..63 hold O = Q e^G S + P U,
 // 64..127 hold W S and T V (their difference is U); Z = Kd^T U fills all 128.
 // The 128-row A operands of T V and P U take the 64 rows next to T (before) and
 // P (after) as filler whose output rows are never read.
@@ -780,7 +797,8 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SS_BAR);
     uint64_t *fullA = bars + MB_FULLA, *fullB = bars + MB_FULLB, *fullV = bars + MB_FULLV, *emptyA = bars + MB_EMPTYA,
              *emptyB = bars + MB_EMPTYB, *emptyV = bars + MB_EMPTYV, *bU = bars + MB_U, *bS = bars + MB_S,
-             *bO = bars + MB_O, *uready = bars + MB_UREADY, *sready = bars + MB_SREADY, *bFin = bars + MB_FIN;
+             *bO = bars + MB_O, *uready = bars + MB_UREADY, *sready = bars + MB_SREADY, *bFin = bars + MB_FIN,
+             *oready = bars + MB_OREADY;
     auto unit_bounds = [&](long long kk, int &s, int &h, int64_t &bos, int64_t &eos) {
         const long long u = st + kk * ns;
         s = (int)(u / H);
@@ -905,14 +923,17 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         if (L > 0) ok = issue_x(0);
         for (long long p = 0; p < L && ok; ++p) {
             const int ab = (int)(p & 1), bb = (int)(p % 3);
-            const uint32_t yb = (uint32_t)ab * 64;
+            const uint32_t yb = (uint32_t)(p % NY) * 64;
             ok = mbar_wait(&fullA[ab], (uint32_t)((p >> 1) & 1), kWaitNs);
             if (!ok) break;
             // Both tile groups of position p are in shared memory (B was waited for
             // with X(p)): its ring slot can be released.
             __threadfence_block();
             *consumed = p + 1;
-            ok = mbar_wait(sready, (uint32_t)(p & 1), kWaitNs);  // S(p) in smem
+            // S(p) in smem, and O(p - NY) read out of Y[p % NY] (one barrier per Y buffer: it
+            // completes for positions p % NY, p % NY + NY, ... and so never runs two ahead)
+            ok = mbar_wait(sready, (uint32_t)(p & 1), kWaitNs) &&
+                 (p < NY || mbar_wait(&oready[p % NY], (uint32_t)((p / NY + 1) & 1), kWaitNs));
             if (!ok) break;
             if (p >= 1) mbar_arrive(&emptyB[(p - 1) % 3]);  // e^{Gl} of p-1 has been read
             tc_fence_after();
@@ -935,7 +956,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
 #pragma unroll
             for (int s4 = 0; s4 < C / 16; ++s4)
                 mma_bf16(tm + TM_Y + yb, dPb + kmaj_step(s4, 128), dU + mnmaj_step(s4), id128, 1);
-            mma_commit(bO);
+            mma_commit(&bO[p % NY]);
             mma_commit(&emptyA[ab]);
             mma_commit(&emptyB[bb]);
         }
@@ -944,7 +965,103 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         if (!ok) fail_call(P);
         return;
     }
-    if (warp >= 8) return;  // warps 12..15 idle
+    if (warp == 12 || warp == 13) {
+        // ---------------- O rows (warps 12, 13: TMEM lanes 0..63) ----------------
+        // With the fused output step, a row's RMSNorm needs the partner CTA's 64
+        // columns: each thread publishes its row's sum of squares with the position
+        // as tag in one 8-byte word and polls the partner's word for the same row
+        // (two words per row alternate by position parity; a word is rewritten two
+        // positions later, after its reader has moved past it).
+        const int c = (warp & 3) * 32 + lane;  // chunk row
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const bool gated = P.og_gate != nullptr;
+        float *sw = reinterpret_cast<float *>(sm + SS_OGW);
+        unsigned long long *xw = reinterpret_cast<unsigned long long *>(P.ws + ws_xch(NH));
+        if (gated) {
+            sw[c] = P.og_w[jv * DVT + c];
+            bar_sync(7, 64);
+        }
+        bool ok = true;
+        long long p = 0;
+        for (long long kk = 0; kk < K && ok; ++kk) {
+            int s, h;
+            int64_t bos, eos;
+            unit_bounds(kk, s, h, bos, eos);
+            const long long len = eos - bos, nch = (len + C - 1) / C;
+            for (long long j = 0; j < nch; ++j, ++p) {
+                const uint32_t ybuf = tm + TM_Y + (uint32_t)(p % NY) * 64 + lane_base;
+                // one bO barrier per Y buffer: it completes for positions p % NY, p % NY + NY, ...
+                // (the MMA thread may run up to NY - 1 positions ahead of these warps)
+                ok = __all_sync(0xffffffffu, mbar_wait(&bO[p % NY], (uint32_t)((p / NY) & 1), kWaitNs));
+                if (!ok) break;
+                tc_fence_after();
+                const long long nn = (len - j * C) < C ? (len - j * C) : C;
+                const int64_t t = bos + j * C + c;
+                const bf16 *grow = gated ? P.og_gate + ((size_t)t * H + h) * DV + jv * DVT : nullptr;
+                // this row's 64 gate pre-activations, loaded while the exchange runs
+                uint4 graw[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    graw[i] = (gated && c < nn) ? __ldg(reinterpret_cast<const uint4 *>(grow) + i) : make_uint4(0, 0, 0, 0);
+                float scale = 1.f;
+                if (gated) {
+                    float ss = 0.f;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        float y[32];
+                        tmem_ld32(ybuf + half * 32, y);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ss += y[i] * y[i];
+                    }
+                    const unsigned long long tag = (unsigned long long)(p + 1) << 32;
+                    st_relaxed_gpu_u64(&xw[((st * 2 + jv) * 2 + (p & 1)) * 64 + c], tag | __float_as_uint(ss));
+                    const unsigned long long *pw = &xw[((st * 2 + (jv ^ 1)) * 2 + (p & 1)) * 64 + c];
+                    unsigned long long got = ld_relaxed_gpu_u64(pw);
+                    if ((got >> 32) != (tag >> 32)) {
+                        const uint64_t t0 = globaltimer_ns();
+                        while (((got = ld_relaxed_gpu_u64(pw)) >> 32) != (tag >> 32))
+                            if (globaltimer_ns() - t0 > kWaitNs || ld_relaxed_gpu(&hd->abort_flag)) break;
+                    }
+                    ok = __all_sync(0xffffffffu, (got >> 32) == (tag >> 32));
+                    if (!ok) break;
+                    scale = rsqrtf((ss + __uint_as_float((uint32_t)got)) * (1.f / DV) + P.og_eps);
+                }
+                bf16 *dst = P.o + ((size_t)t * H + h) * DV + jv * DVT;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float y[32];
+                    tmem_ld32(ybuf + half * 32, y);
+                    tmem_wait_ld();
+                    if (c < nn) {
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8) {
+                            float o8[8];
+                            if (gated) {
+                                float g8[8];
+                                unpack8(graw[half * 4 + q8], g8);
+                                const float4 w0 = *reinterpret_cast<const float4 *>(sw + half * 32 + q8 * 8);
+                                const float4 w1 = *reinterpret_cast<const float4 *>(sw + half * 32 + q8 * 8 + 4);
+                                const float w8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)  // y * scale * w * sigmoid(g)
+                                    o8[i] = __fdividef(y[q8 * 8 + i] * scale * w8[i], 1.f + __expf(-g8[i]));
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) o8[i] = y[q8 * 8 + i];
+                            }
+                            reinterpret_cast<uint4 *>(dst)[half * 4 + q8] = pack8(o8);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&oready[p % NY]);  // Y[p % NY] may be overwritten (by Y(p + NY))
+            }
+        }
+        if (!ok) fail_call(P);
+        return;
+    }
+    if (warp >= 8) return;  // warps 14, 15 idle
 
     // ---------------- epilogues (TMEM lane = state row c) ----------------
     const int q4 = warp & 3, hf = warp >> 2;
@@ -994,8 +1111,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         }
         state_to_smem();
         for (long long j = 0; j < nch; ++j, ++p) {
-            const int bb = (int)(p & 1);
-            const uint32_t xy = (uint32_t)bb * 64;
+            const uint32_t xb = (uint32_t)(p & 1) * 64, yb = (uint32_t)(p % NY) * 64;
             const uint32_t par = (uint32_t)(p & 1);
             if (q4 >= 2) {
                 // U = T V - W S for rows r = c - 64 (TMEM lanes 64..127)
@@ -1003,8 +1119,8 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 if (!ok) break;
                 tc_fence_after();
                 float xv[32], yv[32];
-                tmem_ld32(tm + TM_X + xy + lane_base + col, xv);
-                tmem_ld32(tm + TM_Y + xy + lane_base + col, yv);
+                tmem_ld32(tm + TM_X + xb + lane_base + col, xv);
+                tmem_ld32(tm + TM_Y + yb + lane_base + col, yv);
                 tmem_wait_ld();
 #pragma unroll
                 for (int q8 = 0; q8 < 4; ++q8) {
@@ -1031,27 +1147,6 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 for (int i = 0; i < 32; ++i) Sr[i] = dc * Sr[i] + zv[i];
             }
             if (j + 1 < nch) state_to_smem();
-            // O = rows 0..63 of Y once P U is added (TMEM lanes 0..63)
-            if (q4 < 2) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bO, par, kWaitNs));
-                if (!ok) break;
-                tc_fence_after();
-                const long long nn = (len - j * C) < C ? (len - j * C) : C;
-                float yv[32];
-                tmem_ld32(tm + TM_Y + xy + lane_base + col, yv);
-                tmem_wait_ld();
-                if (c < nn) {
-                    bf16 *dst = P.o + ((size_t)(bos + j * C + c) * H + h) * DV + jv * DVT + hf * 32;
-#pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8) {
-                        float o8[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) o8[i] = yv[q8 * 8 + i];
-                        reinterpret_cast<uint4 *>(dst)[q8] = pack8(o8);
-                    }
-                }
-                tc_fence_before();
-            }
         }
         if (ok) store_state(P.S_T, sofs);
     }
@@ -1073,6 +1168,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
                 if (i >= MB_EMPTYB && i < MB_EMPTYB + 3) count = 2;  // MMA commit + e^{Gl} read
                 if (i == MB_UREADY) count = 128;  // epilogue threads of TMEM lanes 64..127
                 if (i == MB_SREADY) count = 256;  // all epilogue threads
+                if (i >= MB_OREADY && i < MB_OREADY + NY) count = 64;  // O epilogue threads
                 mbar_init(&bars[i], count);
             }
             *reinterpret_cast<long long *>(bars + MB_COUNT) = 0;
@@ -1196,6 +1292,9 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
         return cudaErrorInvalidValue;
     P.la = a.log_alpha;
     P.la_scalar = a.la_scalar;
+    P.og_gate = static_cast<const bf16 *>(a.og_gate);
+    P.og_w = a.og_w;
+    P.og_eps = a.og_eps;
     P.q = static_cast<const bf16 *>(a.q);
     P.k = static_cast<const bf16 *>(a.k);
     P.beta = a.beta;

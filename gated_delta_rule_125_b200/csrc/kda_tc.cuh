@@ -253,9 +253,24 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, in
 }
 
 // --------------------------------------------- CTA and GPU-scope sync ----
-// Named barrier `id` (1..15) over `count` threads (a multiple of 32).
+// Named barrier `id` (1..15) over `count` threads (a multiple of 32). The
+// non-aligned form: threads of a warp may arrive separately (a lane that waited
+// alone on a flag, say), which the warp-aligned bar.sync does not allow.
 __device__ __forceinline__ void bar_sync(uint32_t id, uint32_t count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier that also returns the AND of `pred` over its `count` threads.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.and.pred p, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 // Orders this thread's async-proxy global accesses (bulk copies) with its
 // generic-proxy ones (flag releases and acquires).
@@ -268,6 +283,15 @@ __device__ __forceinline__ int ld_acquire_gpu(const int *p) {
 __device__ __forceinline__ int ld_relaxed_gpu(const int *p) {
     int v;
     asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// 8-byte relaxed accesses: single-copy atomic, so a value and its tag travel together.
+__device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 __device__ __forceinline__ void st_release_gpu(int *p, int v) {

@@ -129,6 +129,36 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
                        kda_stream_t stream);
 
 /*
+ * Output step of the KDA layer fused into the store of o ("[Kimi-2] Kimi
+ * Linear" §6 and §6.3): per (token, head), a head-wise RMSNorm over the d_v
+ * channels followed by a sigmoid gate computed from the layer input,
+ *
+ *     o_t <- o_t / sqrt(mean_j(o_tj^2) + eps) * weight * sigmoid(gate_t).
+ *
+ *   gate    [T][H][dv] (prefill) / [N][H][dv] (decode), the dtype of q, k, v:
+ *           the gate's pre-activation; 16-byte aligned
+ *   weight  [dv] fp32, one RMSNorm weight vector shared by the heads; 4-byte aligned
+ *   eps     RMSNorm epsilon (> 0)
+ * The pages give neither eps nor the weight's shape; both are the caller's.
+ */
+typedef struct kda_output_gate {
+    const void *gate;
+    const float *weight;
+    float eps;
+} kda_output_gate;
+
+/*
+ * kda_prefill with the output step fused (out_gate != NULL) or not (NULL, then
+ * identical to kda_prefill). Same arguments and rules as kda_prefill otherwise.
+ */
+kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *S0, const int32_t *cu_seqlens,
+                          int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                          int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                          const kda_output_gate *out_gate, void *o, float *S_T, void *workspace,
+                          size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_prefill without a workspace argument, for callers that cannot allocate
  * device memory where they run the prefill (a runtime that owns all device
  * memory through its own pool and forbids library allocations, a plugin whose
@@ -183,6 +213,12 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v, const fl
                            const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
                            int32_t dv, kda_dtype dtype, uint32_t flags, void *o,
                            kda_stream_t stream);
+
+/* kda_decode_step with the output step fused (out_gate != NULL; see kda_output_gate). */
+kda_status kda_decode_step_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                              const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
+                              int32_t dv, kda_dtype dtype, uint32_t flags,
+                              const kda_output_gate *out_gate, void *o, kda_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -393,3 +393,84 @@ def test_workload_gdn_8k():
     T, H = inp["beta"].shape
     expanded = dict(inp, log_alpha=inp["log_alpha"][:, :, None].expand(T, H, 128).contiguous())
     check(o, S_T, expanded, torch.bfloat16, heads=[3, 30], label="gdn_8k")
+
+
+# ------------------------------------------- fused output step (§6.3) ----
+# kda_prefill_ex / kda_decode_step_ex with a kda_output_gate: o <- RMSNorm(o)
+# * weight * sigmoid(gate) per (token, head). The oracle is its recurrence
+# followed by oracle.output_gate (pinned in test_oracle_pins). RMSNorm rescales
+# every row to unit mean square, so gated outputs are compared relative to
+# their largest magnitude with the workload's tolerance for o.
+
+def _gate_inputs(T, H, dv, dtype, seed):
+    g = torch.Generator(device=DEV)
+    g.manual_seed(1000 + seed)
+    gate = torch.randn((T, H, dv), generator=g, device=DEV).to(dtype)
+    w = 1.0 + 0.1 * torch.randn((dv,), generator=g, device=DEV)
+    return gate, w, 1e-6
+
+
+def _check_gated(o, inp, gate, w, eps, dtype, heads=None, label=""):
+    o_ref, _, ti, hi, _ = ref_prefill(inp, heads)
+    pick = lambda x: host(x.index_select(0, ti.to(x.device)).index_select(1, hi.to(x.device)))
+    y_ref = oracle.output_gate(o_ref, pick(gate), host(w), eps)
+    y = pick(o)
+    atol = TOL[dtype][0] * max(1.0, float(np.abs(y_ref).max()))
+    err = float(np.abs(y - y_ref).max())
+    assert np.isfinite(y).all() and err <= atol, "%s: max|y-y_ref| = %.3e > %.3e" % (label, err, atol)
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64), (torch.float32, 128)])
+def test_output_gate_prefill(dtype, d):
+    inp = make([0, 130, 1, 257, 64], 3, d, d, dtype, seed=41)
+    T = sum(inp["lengths"])
+    gate, w, eps = _gate_inputs(T, 3, d, dtype, 41)
+    o0, S0_ = run(inp)
+    o1, S1 = run(inp, out_gate=(gate, w, eps))
+    assert torch.equal(S0_, S1)  # the output step leaves the state alone
+    _check_gated(o1, inp, gate, w, eps, dtype, label="gated %s d=%d" % (dtype, d))
+
+
+def test_output_gate_many_units_small_ring():
+    """Tensor-core path, 72 units over 32 streams and the smallest ring: the two scan
+    CTAs of a stream exchange their halves' sums of squares chunk after chunk."""
+    lengths = [0, 130, 1, 64, 700, 0, 65, 257]
+    H = 9
+    inp = make(lengths, H, 128, 128, torch.bfloat16, seed=43)
+    gate, w, eps = _gate_inputs(sum(lengths), H, 128, torch.bfloat16, 43)
+    mn = kda.kda_prefill_workspace_min(len(lengths), sum(lengths), max(lengths), H, 128, 128,
+                                       torch.bfloat16)
+    ws = torch.empty(mn, dtype=torch.uint8, device=DEV)
+    o1, _ = run(inp, out_gate=(gate, w, eps), workspace=ws)
+    o2, _ = run(inp, out_gate=(gate, w, eps))
+    assert torch.equal(o1, o2)
+    _check_gated(o1, inp, gate, w, eps, torch.bfloat16, label="gated streams")
+    assert kda.kda_device_error() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_output_gate_decode(dtype):
+    N, H, d, steps = 5, 3, 128, 3
+    w_ = KI.decode_workload(N, H, d, steps, dtype, DEV, seed=45, s0_std=0.1)
+    gate, w, eps = _gate_inputs(steps * N, H, d, dtype, 45)
+    gate = gate.view(steps, N, H, d)
+    S = w_["S0"].clone()
+    S_ref = host(S)
+    atol0 = TOL[dtype][0]
+    for t in range(steps):
+        o = kda.kda_decode_step(w_["q"][t], w_["k"][t], w_["v"][t], w_["log_alpha"][t], w_["beta"][t], S,
+                                out_gate=(gate[t].contiguous(), w, eps))
+        torch.cuda.synchronize()
+        o_ref, S_ref = oracle.decode_step(host(w_["q"][t]), host(w_["k"][t]), host(w_["v"][t]),
+                                          host(w_["log_alpha"][t]), host(w_["beta"][t]), S_ref)
+        y_ref = oracle.output_gate(o_ref, host(gate[t]), host(w), eps)
+        assert float(np.abs(host(o) - y_ref).max()) <= atol0 * max(1.0, float(np.abs(y_ref).max()))
+        assert rel_fro(host(S), S_ref) <= TOL[dtype][1]
+
+
+def test_output_gate_workload_prefill_8k():
+    """prefill_8k with the fused output step; heads {5, 26} checked over all 8192 tokens."""
+    inp = KI.prefill_workload("prefill_8k", DEV)
+    gate, w, eps = _gate_inputs(8192, 32, 128, torch.bfloat16, 47)
+    o, _ = run(inp, out_gate=(gate, w, eps))
+    _check_gated(o, inp, gate, w, eps, torch.bfloat16, heads=[5, 26], label="gated prefill_8k")
