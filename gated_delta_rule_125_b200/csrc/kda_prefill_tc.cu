@@ -221,12 +221,14 @@ constexpr uint32_t SS_BAR = SS_U + 8192;        // 31 mbarriers, the consumed-po
 constexpr uint32_t SS_OGW = SS_BAR + 512;       // output-step weights of this CTA's 64 columns
 constexpr uint32_t SS_BYTES = SS_OGW + 256;
 constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 512;
+constexpr int NY = 4;  // Y buffers in TMEM: the O epilogue may lag NY - 1 chunks
+constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = TM_Y + 64 * NY;  // scan TMEM columns: X x2, Y x NY, Z
+static_assert(TM_Z + 64 <= 512, "scan TMEM columns");
 // scan mbarrier indices
 constexpr int MB_FULLA = 0, MB_FULLB = 2, MB_FULLV = 5, MB_EMPTYA = 9, MB_EMPTYB = 11, MB_EMPTYV = 14,
-              MB_U = 18, MB_S = 19, MB_O = 20, MB_UREADY = 24, MB_SREADY = 25, MB_FIN = 26, MB_OREADY = 27,
-              MB_COUNT = 31;  // MB_O and MB_OREADY: one barrier per Y buffer
-constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = 384;  // scan TMEM columns: X x2, Y x4, Z
-constexpr int NY = 4;                                  // Y buffers: the O epilogue may lag NY - 1 chunks
+              MB_U = 18, MB_S = 19, MB_O = 20,  // MB_O and MB_OREADY: one barrier per Y buffer
+              MB_UREADY = MB_O + NY, MB_SREADY = MB_UREADY + 1, MB_FIN = MB_SREADY + 1, MB_OREADY = MB_FIN + 1,
+              MB_COUNT = MB_OREADY + NY;
 
 // Per-CTA control block after both layouts.
 struct Ctrl {
