@@ -640,7 +640,11 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         // 5. In place, AF (A) becomes X = (I + Diag(beta) A)^{-1}: diagonal 16x16 blocks by
         //    forward substitution, then the 2x2 block recursion with tf32 tensor-core products:
         //    [X11 0; X21 X22] with X21 = -X22 (Diag(beta_2) A21) X11, written over A21 once
-        //    A21 is consumed.
+        //    A21 is consumed. Each block of T = X Diag(beta) (bf16, the A operand of W and the
+        //    slot's T tile) is written as its X block is produced; warps 4..7 zero T's upper blocks.
+        auto t_store = [&](int r, int c, float xv) {
+            *reinterpret_cast<bf16 *>(TT + kmaj_off(r, c, 64)) = __float2bfloat16_rn(xv * sbeta[c]);
+        };
         {
             float x[16];
             const int b = tid >> 4, cc = tid & 15;
@@ -652,6 +656,16 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
 #pragma unroll
                     for (int ii = 0; ii < rr; ++ii) acc += AF[r * ALD + 16 * b + ii] * x[ii];
                     x[rr] = (rr == cc) ? 1.f : (rr > cc ? -sbeta[r] * acc : 0.f);
+                }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) t_store(16 * b + rr, 16 * b + cc, x[rr]);
+            } else if (tid >= 128) {
+                // upper blocks (bi, bj), bj > bi: 6 blocks x 16 rows x 2 chunks of 8 columns
+                for (int i = tid - 128; i < 6 * 16 * 2; i += 128) {
+                    const int blk = i >> 5, rr = (i >> 1) & 15, half = i & 1;
+                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                    *reinterpret_cast<uint4 *>(TT + kmaj_chunk(16 * bi + rr, 2 * bj + half, 64)) = make_uint4(0, 0, 0, 0);
                 }
             }
             sync();  // every diagonal block of A has been read
@@ -673,7 +687,10 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             warp_gemm_16x8<16>(
                 lane, [&](int r, int kk) { return AF[(o + 16 + r) * ALD + o + 16 + kk]; },
                 [&](int kk, int nn) { return Rw[kk * 8 + nn]; },
-                [&](int r, int nn, float v) { AF[(o + 16 + r) * ALD + o + nh + nn] = -v; });
+                [&](int r, int nn, float v) {
+                    AF[(o + 16 + r) * ALD + o + nh + nn] = -v;
+                    t_store(o + 16 + r, o + nh + nn, -v);
+                });
         }
         sync();
         // 32-row level: R2 = (Diag(beta) A)[32..63][0..31] X[0..31][0..31], then X[32..63][0..31] = -X22 R2.
@@ -687,19 +704,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             warp_gemm_16x8<32>(
                 lane, [&](int r, int kk) { return AF[(32 + 16 * mt + r) * ALD + 32 + kk]; },
                 [&](int kk, int nn) { return R2[kk * 32 + 8 * nt + nn]; },
-                [&](int r, int nn, float v) { AF[(32 + 16 * mt + r) * ALD + 8 * nt + nn] = -v; });
-        }
-        sync();
-        // T = X Diag(beta), lower triangle, bf16: A operand of W (smem) and the slot's T tile.
-        for (int e2 = tid; e2 < C * 8; e2 += PT) {
-            const int r = e2 >> 3, cc8 = e2 & 7;
-            float t8[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = cc8 * 8 + i;
-                t8[i] = (c <= r) ? AF[r * ALD + c] * sbeta[c] : 0.f;
-            }
-            *reinterpret_cast<uint4 *>(TT + kmaj_chunk(r, cc8, 64)) = pack8(t8);
+                [&](int r, int nn, float v) { t_store(32 + 16 * mt + r, 8 * nt + nn, -v); });
         }
         fence_async_smem();
         tc_fence_before();
