@@ -88,6 +88,8 @@ __host__ __device__ inline size_t ws_ring(long long NH) { return ru1024(ws_xch(N
 struct FusedParams {
     CUtensorMap tmap_la;  // log_alpha [T][H][128] fp32, box 128 x 1 x 64
     CUtensorMap tmap_v;   // v [T][H][128] bf16, box 64 x 1 x 64, SW128
+    CUtensorMap tmap_q;   // q, k: as v
+    CUtensorMap tmap_k;
     const bf16 *q, *k;
     const float *beta, *S0;
     const float *la;  // log_alpha, read directly when it is one gate per (token, head)
@@ -197,7 +199,7 @@ constexpr uint32_t PS_GA = 32768;              // [Qg ; Kg] K-major 128 x 128 ->
 constexpr uint32_t PS_GB = PS_GA + 32768;      // q of the next item, then K e^-G (K-major 64 x 128)
 constexpr uint32_t PS_KS = PS_GB + 16384;      // k of the next item (K-major 64 x 128)
 constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[2][64] eGl[128] gate[2][64]
-constexpr uint32_t PS_BAR = PS_SMALL + 2048;   // la, mma barriers; 3 item records; flags
+constexpr uint32_t PS_BAR = PS_SMALL + 2048;   // la, mma, q/k barriers; 3 item records; flags
 constexpr uint32_t PS_BYTES = PS_BAR + 128;
 constexpr uint32_t PS_STRIDE = 101376;         // engine 1 starts here (1024-aligned)
 constexpr int ALD = 68;                        // row stride of A / X (floats)
@@ -250,6 +252,7 @@ struct ItemS {
     long long t0, p;  // first token; position in the stream
     int n, h, st, valid;
 };
+static_assert(3 * 8 + 3 * sizeof(ItemS) + 2 * 4 <= PS_BYTES - PS_BAR, "prep barrier block");
 
 // Item g of the global claim order: position-major over the streams still
 // running at that position, longest streams first.
@@ -345,10 +348,10 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     uint8_t *KS = sm + PS_KS;
     float *invq = reinterpret_cast<float *>(sm + PS_SMALL);
     float *invk = invq + 64, *sbeta2 = invk + 64, *eGl = sbeta2 + 128, *sgate2 = eGl + 128;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA, [2] q, k boxes
     // Item records of iterations it (current), it + 1 (claimed during the Gram)
     // and it - 1 (published by the store thread) in entries it % 3, ...
-    ItemS *sitem = reinterpret_cast<ItemS *>(bars + 2);
+    ItemS *sitem = reinterpret_cast<ItemS *>(bars + 3);
     int *sflag = reinterpret_cast<int *>(sitem + 3);  // [0] unsafe range, [1] a wait failed
     Hdr *hd = reinterpret_cast<Hdr *>(P.ws);
     const long long NH = (long long)P.N * H;
@@ -356,7 +359,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     int *freed = ready + kFlagInts;
     char *ring = P.ws + ws_ring(NH);
     auto sync = [&]() { bar_sync(bar_id, PT); };
-    uint32_t la_phase = 0, mma_phase = 0;
+    uint32_t la_phase = 0, mma_phase = 0, qk_phase = 0;
     const int c8 = tid & 15, rb = tid >> 4;  // thread's 16-byte channel chunk and first row
 
     auto slot_index = [&](const ItemS &it) { return it.st * R + (int)(it.p % R); };
@@ -371,6 +374,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     bool slot_ok = false;       // store thread: the current item's slot is known to be free
     bool prev_pending = false;  // store thread: the previous item is not yet published
     bool la_pending = false;    // store thread: a log_alpha box is in flight
+    bool qk_pending = false;    // store thread: q, k boxes are in flight
     auto publish_prev = [&](const ItemS &pv) {
         if (!prev_pending) return;
         bulk_wait_all();
@@ -392,19 +396,20 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         tma_load_3d(G, &P.tmap_la, 0, it.h, (int)it.t0, &bars[0]);
         la_pending = true;
     };
-    // q and k rows rb + 16 m, chunk c8, by cp.async into GB / KS at the chunk's
-    // place in a K-major SW128 64 x 128 tile (the thread reads back exactly what
-    // it copied; K e^-G later overwrites q in place); beta of row `tid` (threads
-    // < 64) into sbeta2[buf], and with a scalar gate log_alpha of row `tid` into
-    // sgate2[buf]. Rows past the sequence are zero-filled.
+    // The item's q and k rows into GB / KS (K-major SW128 64 x 128 tiles) by four
+    // TMA boxes from the store thread (K e^-G later overwrites q in place; rows
+    // past the sequence are cleared after arrival); beta of row `tid` (threads
+    // < 64) by cp.async into sbeta2[buf], and with a scalar gate log_alpha of row
+    // `tid` into sgate2[buf] (zero past the sequence).
     auto fetch_qk = [&](const ItemS &it, int buf) {
+        if (tid == kStoreTid) {
+            mbar_arrive_expect_tx(&bars[2], 32768u);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int r = rb + 16 * m;
-            const size_t off = ((size_t)(it.t0 + (r < it.n ? r : 0)) * H + it.h) * DK + c8 * 8;
-            const uint32_t bytes = r < it.n ? 16u : 0u;
-            cp_async16(GB + kmaj_chunk(r, c8, 64), P.q + off, bytes);
-            cp_async16(KS + kmaj_chunk(r, c8, 64), P.k + off, bytes);
+            for (int half = 0; half < 2; ++half) {
+                tma_load_3d(GB + half * 8192, &P.tmap_q, 64 * half, it.h, (int)it.t0, &bars[2]);
+                tma_load_3d(KS + half * 8192, &P.tmap_k, 64 * half, it.h, (int)it.t0, &bars[2]);
+            }
+            qk_pending = true;
         }
         if (tid < C) {
             const size_t row = (size_t)(it.t0 + (tid < it.n ? tid : 0)) * H + it.h;
@@ -441,7 +446,13 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         // 1. Warps 0..3: G = cumulative sum of log_alpha over the rows, in place, one
         //    thread per channel. Warps 4..7: the row norms of q (threads 128..191) and
         //    k (192..255), one row per thread, from the chunks every thread copied.
-        cp_async_wait_all();  // this thread's q, k chunks and beta
+        cp_async_wait_all();  // this thread's beta (and scalar gate)
+        {
+            const bool qk_in = mbar_wait(&bars[2], qk_phase, kWaitNs);
+            if (!qk_in) sflag[1] = 1;
+            if (tid == kStoreTid && qk_in) qk_pending = false;
+            qk_phase ^= 1;
+        }
         sync();
         if (tid < DK) {
             const float *sgate = sgate2 + (iter & 1) * 64;
@@ -464,7 +475,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             if (-run > kTau) sflag[0] = 1;
         } else {
             const int r = tid & (C - 1);
-            const uint8_t *src = (tid < 192) ? GB : KS;
+            uint8_t *src = (tid < 192) ? GB : KS;
             float ss = 0.f;
 #pragma unroll
             for (int cc = 0; cc < 16; ++cc) {
@@ -472,6 +483,11 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                 unpack8(*reinterpret_cast<const uint4 *>(src + kmaj_chunk(r, cc, 64)), x);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+            }
+            if (r >= n) {  // the box ran into the next sequence (or the zero fill past the end)
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc)
+                    *reinterpret_cast<uint4 *>(src + kmaj_chunk(r, cc, 64)) = make_uint4(0, 0, 0, 0);
             }
             // 1 / max(||x||, eps) = rsqrt(max(||x||^2, eps^2))
             const float inv = (r >= n) ? 0.f : (P.l2norm ? rsqrtf(fmaxf(ss, P.eps * P.eps)) : 1.f);
@@ -552,7 +568,10 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     mma_bf16(tm, kmaj_desc(a, s8, 128), kmaj_desc(b, s8, 64), idg, s8 > 0);
                 mma_commit(&bars[1]);
             }
-            if (tid == kStoreTid) claim(next);
+            if (tid == kStoreTid) {
+                claim(next);
+                if (next.valid && !P.la_scalar) tma_prefetch_3d(&P.tmap_la, 0, next.h, (int)next.t0);
+            }
             if (!mbar_wait(&bars[1], mma_phase, kWaitNs)) sflag[1] = 1;
             mma_phase ^= 1;
             tc_fence_after();
@@ -641,7 +660,8 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         //    forward substitution, then the 2x2 block recursion with tf32 tensor-core products:
         //    [X11 0; X21 X22] with X21 = -X22 (Diag(beta_2) A21) X11, written over A21 once
         //    A21 is consumed. Each block of T = X Diag(beta) (bf16, the A operand of W and the
-        //    slot's T tile) is written as its X block is produced; warps 4..7 zero T's upper blocks.
+        //    slot's T tile) is written as its X block is produced: the diagonal blocks and the
+        //    zero upper blocks by warps 4..7 while warps 0..3 run the 16-row level.
         auto t_store = [&](int r, int c, float xv) {
             *reinterpret_cast<bf16 *>(TT + kmaj_off(r, c, 64)) = __float2bfloat16_rn(xv * sbeta[c]);
         };
@@ -657,8 +677,6 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     for (int ii = 0; ii < rr; ++ii) acc += AF[r * ALD + 16 * b + ii] * x[ii];
                     x[rr] = (rr == cc) ? 1.f : (rr > cc ? -sbeta[r] * acc : 0.f);
                 }
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) t_store(16 * b + rr, 16 * b + cc, x[rr]);
             } else if (tid >= 128) {
                 // upper blocks (bi, bj), bj > bi: 6 blocks x 16 rows x 2 chunks of 8 columns
                 for (int i = tid - 128; i < 6 * 16 * 2; i += 128) {
@@ -676,7 +694,14 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         }
         sync();
         // 16-row level: warps 0, 1 build X[16..31][0..15], warps 2, 3 X[48..63][32..47] (8-column halves).
-        if (warp < 4) {
+        if (warp >= 4) {
+            // T's diagonal blocks: block i >> 5, row (i >> 1) & 15, 8-column half i & 1
+            const int i = tid - 128, bd = i >> 5, r = 16 * bd + ((i >> 1) & 15), c0 = 16 * bd + 8 * (i & 1);
+            float t8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) t8[j] = (c0 + j <= r) ? AF[r * ALD + c0 + j] * sbeta[c0 + j] : 0.f;
+            *reinterpret_cast<uint4 *>(TT + kmaj_chunk(r, c0 >> 3, 64)) = pack8(t8);
+        } else {
             const int o = (warp >> 1) * 32, nh = (warp & 1) * 8;  // block offset, column half
             float *Rw = R2 + warp * 128;                          // 16 x 8 scratch per warp
             warp_gemm_16x8<16>(
@@ -776,6 +801,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         bulk_wait_all();
         if (!failed && !sflag[1]) publish_prev(sitem[(iter + 2) % 3]);  // the last item
         if (la_pending) mbar_wait(&bars[0], la_phase ^ (failed ? 1u : 0u), kWaitNs);
+        if (qk_pending) mbar_wait(&bars[2], qk_phase ^ 1u, kWaitNs);  // only after a failed wait
     }
     sync();
     if (tid == 0 && (failed || sflag[1])) fail_call(P);
@@ -816,7 +842,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
     if (warp == 9) {
         // ---------------- ring-slot copies (one thread) ----------------
         if (lane != 0) return;
-        long long p = 0;
+        long long p = 0, nA = 0, nB = 0;  // positions whose A / B groups were issued
         bool ok = true;
         for (long long kk = 0; kk < K && ok; ++kk) {
             int s, h;
@@ -824,27 +850,33 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             unit_bounds(kk, s, h, bos, eos);
             const long long nch = (eos - bos + C - 1) / C;
             for (long long j = 0; j < nch; ++j, ++p) {
+                // The slot's ready flag first (usually set long before: its gpu-scope read
+                // then overlaps the wait for a free buffer), then the B group (three
+                // buffers: free one position before the A group's two), then A.
                 const int ab = (int)(p & 1), bb = (int)(p % 3);
-                if (p >= 2) ok = mbar_wait(&emptyA[ab], (uint32_t)((p / 2 - 1) & 1), kWaitNs);
-                if (ok && p >= 3) ok = mbar_wait(&emptyB[bb], (uint32_t)((p / 3 - 1) & 1), kWaitNs);
                 const int slot = st * R + (int)(p % R);
-                if (ok) ok = wait_flag_geq(&ready[slot], (int)(p / R) + 1, &hd->abort_flag);
+                ok = wait_flag_geq(&ready[slot], (int)(p / R) + 1, &hd->abort_flag, 32);
+                if (ok && p >= 3) ok = mbar_wait(&emptyB[bb], (uint32_t)((p / 3 - 1) & 1), kWaitNs);
                 if (!ok) break;
                 fence_proxy_async_global();
                 const char *g = ring + (size_t)slot * SL_BYTES;
                 uint8_t *A = sm + SS_A + ab * SA_BYTES, *B = sm + SS_B + bb * SB_BYTES;
-                mbar_arrive_expect_tx(&fullA[ab], COPY_A);
-                bulk_g2s(A + SA_WQ, g + SL_WQ, 32768, &fullA[ab]);
-                bulk_g2s(A + SA_KD, g + SL_KD, 16384, &fullA[ab]);
                 mbar_arrive_expect_tx(&fullB[bb], COPY_B);
                 bulk_g2s(B + SB_T, g + SL_T, 8192, &fullB[bb]);
                 bulk_g2s(B + SB_P, g + SL_P, 8192, &fullB[bb]);
                 bulk_g2s(B + SB_D, g + SL_D, 512, &fullB[bb]);
+                nB = p + 1;
+                if (p >= 2) ok = mbar_wait(&emptyA[ab], (uint32_t)((p / 2 - 1) & 1), kWaitNs);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&fullA[ab], COPY_A);
+                bulk_g2s(A + SA_WQ, g + SL_WQ, 32768, &fullA[ab]);
+                bulk_g2s(A + SA_KD, g + SL_KD, 16384, &fullA[ab]);
+                nA = p + 1;
             }
         }
         // Settle the copies still in flight (consumed ones return at once).
-        for (long long q = (p > 2 ? p - 2 : 0); q < p; ++q) mbar_wait(&fullA[q & 1], (uint32_t)((q / 2) & 1), kWaitNs);
-        for (long long q = (p > 3 ? p - 3 : 0); q < p; ++q) mbar_wait(&fullB[q % 3], (uint32_t)((q / 3) & 1), kWaitNs);
+        for (long long q = (nA > 2 ? nA - 2 : 0); q < nA; ++q) mbar_wait(&fullA[q & 1], (uint32_t)((q / 2) & 1), kWaitNs);
+        for (long long q = (nB > 3 ? nB - 3 : 0); q < nB; ++q) mbar_wait(&fullB[q % 3], (uint32_t)((q / 3) & 1), kWaitNs);
         if (!ok) fail_call(P);
         return;
     }
@@ -950,8 +982,6 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             for (int s8 = 0; s8 < DK / 16; ++s8)
                 mma_bf16(tm + TM_Y + yb, dWQa + kmaj_step(s8, 128), dS + mnmaj_step(s8), id128, s8 > 0);
             mma_commit(bU);
-            // T V of the next position runs while U(p) is formed.
-            if (p + 1 < L && !(ok = issue_x(p + 1))) break;
             ok = mbar_wait(uready, (uint32_t)(p & 1), kWaitNs);  // U(p) in smem
             if (!ok) break;
             tc_fence_after();
@@ -966,6 +996,9 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             mma_commit(&bO[p % NY]);
             mma_commit(&emptyA[ab]);
             mma_commit(&emptyB[bb]);
+            // T V of the next position, while S(p + 1) is formed (after Z: a late
+            // T or V tile never holds up the state chain).
+            if (p + 1 < L && !(ok = issue_x(p + 1))) break;
         }
         mma_commit(bFin);  // every MMA of this CTA completes before TMEM is freed
         if (!mbar_wait(bFin, 0, kWaitNs)) ok = false;
@@ -1184,7 +1217,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
                 uint64_t *bars = reinterpret_cast<uint64_t *>(sm + e * PS_STRIDE + PS_BAR);
                 mbar_init(&bars[0], 1);
                 mbar_init(&bars[1], 1);
-                int *sflag = reinterpret_cast<int *>(reinterpret_cast<ItemS *>(bars + 2) + 3);
+                mbar_init(&bars[2], 1);
+                int *sflag = reinterpret_cast<int *>(reinterpret_cast<ItemS *>(bars + 3) + 3);
                 sflag[0] = 0;
                 sflag[1] = 0;
             }
@@ -1232,8 +1266,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
     return fn;
 }
 
-// v viewed as [T][H][DV] bf16; a box is 64 columns x 1 head x 64 tokens, SW128.
-bool make_v_map(CUtensorMap *m, const void *v, int64_t total, int H) {
+// q, k or v viewed as [T][H][128] bf16; a box is 64 columns x 1 head x 64 tokens, SW128.
+bool make_rows_map(CUtensorMap *m, const void *v, int64_t total, int H) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)DV, (cuuint64_t)H, (cuuint64_t)total};
@@ -1295,7 +1329,8 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
     FusedParams P;
     memset(&P, 0, sizeof(P));
     if (a.total > 0 && ((!a.la_scalar && !make_la_map(&P.tmap_la, a.log_alpha, a.total, a.H)) ||
-                        !make_v_map(&P.tmap_v, a.v, a.total, a.H)))
+                        !make_rows_map(&P.tmap_v, a.v, a.total, a.H) || !make_rows_map(&P.tmap_q, a.q, a.total, a.H) ||
+                        !make_rows_map(&P.tmap_k, a.k, a.total, a.H)))
         return cudaErrorInvalidValue;
     P.la = a.log_alpha;
     P.la_scalar = a.la_scalar;

@@ -252,6 +252,13 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, in
         : "memory");
 }
 
+// Prefetch of a 3-D tensor-map tile into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap), "r"(x), "r"(y),
+                 "r"(z)
+                 : "memory");
+}
+
 // --------------------------------------------- CTA and GPU-scope sync ----
 // Named barrier `id` (1..15) over `count` threads (a multiple of 32). The
 // non-aligned form: threads of a warp may arrive separately (a lane that waited
