@@ -18,6 +18,11 @@ Functions and the passages they follow (pages cited by title and section):
 * :func:`output_gate` -- the layer's output step after the recurrence, §6 and
   §6.3 (and "Kimi Linear — 逐通道的遺忘", 其他零件): head-wise RMSNorm of o_t,
   then a product with a sigmoid gate computed from the input.
+* :func:`short_conv_swish` / :func:`short_conv_step` -- the layer's step before
+  the recurrence, §6 and §6.1 (and "Kimi Delta Attention：把遗忘门做到每个通道",
+  进状态之前 q/k 还要过一道预处理): a causal short convolution over the token
+  axis, then Swish, on the q, k, v projections (the L2 norm of q, k follows, in
+  the recurrence's functions above).
 
 Arrays are ``numpy`` (any real dtype; converted to fp64). Layouts::
 
@@ -164,3 +169,54 @@ def output_gate(o, g, w, eps=1e-6):
     w = np.asarray(w, dtype=np.float64)
     rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
     return o / rms * w / (1.0 + np.exp(-g))
+
+
+def _silu(x):
+    return x / (1.0 + np.exp(-x))
+
+
+def short_conv_swish(x, w, cu_seqlens=None, state0=None):
+    """Causal depthwise short convolution over each sequence's tokens, then Swish.
+
+    x ``[T, C]`` (C channels, e.g. H * d of a q, k or v projection), w ``[C, W]``:
+    the pre-activation of token t, channel c is ``sum_j w[c, j] * x[t - W + 1 + j, c]``
+    (``w[c, W-1]`` weighs the current token), positions before a sequence's start
+    read its initial state ``state0[s]`` ``[W-1, C]`` (oldest first) or zero, and the
+    output is ``z * sigmoid(z)``. The pages give neither the window nor a bias; the
+    window is the caller's and there is no bias (the plainest reading of "a short
+    causal convolution"). Returns ``(y [T, C], state_T [N, W-1, C])``, state_T
+    holding each sequence's last W-1 inputs (oldest first, reaching into state0 when
+    the sequence is shorter). fp64 numpy, a loop over the sequences.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    T, C = x.shape
+    W = w.shape[1]
+    cu = np.array([0, T]) if cu_seqlens is None else np.asarray(cu_seqlens, dtype=np.int64)
+    N = len(cu) - 1
+    y = np.zeros((T, C))
+    state_T = np.zeros((N, W - 1, C))
+    for s in range(N):
+        bos, eos = int(cu[s]), int(cu[s + 1])
+        hist = np.zeros((W - 1, C)) if state0 is None else np.asarray(state0[s], dtype=np.float64)
+        xs = np.concatenate([hist, x[bos:eos]], axis=0)  # [W-1+L, C]
+        L = eos - bos
+        for t in range(L):
+            z = np.zeros(C)
+            for j in range(W):
+                z += w[:, j] * xs[t + j]
+            y[bos + t] = _silu(z)
+        state_T[s] = xs[L:L + W - 1]
+    return y, state_T
+
+
+def short_conv_step(x, w, state):
+    """One decode token of :func:`short_conv_swish` for N sequences: x ``[N, C]``,
+    state ``[N, W-1, C]`` (the previous W-1 inputs, oldest first). Returns
+    ``(y [N, C], new_state [N, W-1, C])``."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    state = np.asarray(state, dtype=np.float64)
+    window = np.concatenate([state, x[:, None, :]], axis=1)  # [N, W, C], newest last
+    z = np.einsum("cj,njc->nc", w, window)
+    return _silu(z), window[:, 1:, :].copy()

@@ -439,3 +439,145 @@ def test_output_gate_pins_catch_planted_mistakes(kind):
         except AssertionError:
             failed += 1
     assert failed > 0, kind
+
+
+# ------------------------------------------ short conv + Swish (§6.1) ----
+# oracle.short_conv_swish / short_conv_step: a causal short convolution over the
+# token axis, then Swish ("[Kimi-2] Kimi Linear" §6 and §6.1; "Kimi Delta
+# Attention：把遗忘门做到每个通道", the pre-processing of q, k). Pinned to a library
+# convolution, closed forms and the properties "causal" and "per sequence" fix;
+# each planted mistake below must fail at least one pin.
+
+def _silu_ref(z):
+    from scipy.special import expit
+    return z * expit(z)
+
+
+def sc_pin_numpy_convolve(f):
+    # one sequence from zero history: per channel, the pre-activation is the
+    # library's full convolution with the taps reversed, cut to the first T outputs
+    rng = np.random.default_rng(11)
+    x, w = rng.normal(size=(23, 5)), rng.normal(size=(5, 4))
+    y, _ = f(x, w)
+    for c in range(5):
+        z = np.convolve(x[:, c], w[c, ::-1])[:23]
+        np.testing.assert_allclose(y[:, c], _silu_ref(z), rtol=1e-12, atol=1e-14)
+
+
+def sc_pin_impulse(f):
+    # a unit impulse at t0 gives silu(w[c, W-1-j]) at t0 + j (j < W), zero elsewhere
+    W, t0 = 4, 5
+    w = np.array([[0.5, -1.0, 2.0, 3.0], [1.5, 0.25, -0.75, 1.0]])
+    x = np.zeros((12, 2))
+    x[t0] = 1.0
+    y, _ = f(x, w)
+    want = np.zeros((12, 2))
+    for j in range(W):
+        want[t0 + j] = _silu_ref(w[:, W - 1 - j])
+    np.testing.assert_allclose(y, want, rtol=1e-14, atol=0.0)
+
+
+def sc_pin_swish_values(f):
+    # W = 1, w = 1: y = silu(x); silu(0) = 0, silu(1) = 1/(1+e^-1), silu(-1) = -1/(1+e)
+    y, st = f(np.array([[0.0], [1.0], [-1.0]]), np.ones((1, 1)))
+    np.testing.assert_allclose(y[:, 0], [0.0, 1.0 / (1.0 + np.exp(-1.0)), -1.0 / (1.0 + np.e)], rtol=1e-15)
+    assert st.shape == (1, 0, 1)
+
+
+def sc_pin_sequences_independent(f):
+    # varlen: equal to each sequence run alone (nothing crosses a boundary)
+    rng = np.random.default_rng(12)
+    lens = [3, 1, 9, 2]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    x, w = rng.normal(size=(cu[-1], 3)), rng.normal(size=(3, 3))
+    s0 = rng.normal(size=(4, 2, 3))
+    y, st = f(x, w, cu, s0)
+    for s in range(4):
+        ys, sts = f(x[cu[s]:cu[s + 1]], w, None, s0[s:s + 1])
+        np.testing.assert_allclose(y[cu[s]:cu[s + 1]], ys, rtol=1e-14, atol=0.0)
+        np.testing.assert_allclose(st[s], sts[0], rtol=0, atol=0)
+
+
+def sc_pin_continuation(f):
+    # a sequence split anywhere, the second part started from the first part's
+    # final state, gives the same outputs and final state (also splits shorter than W-1)
+    rng = np.random.default_rng(13)
+    x, w = rng.normal(size=(17, 4)), rng.normal(size=(4, 4))
+    y, st = f(x, w)
+    for t1 in (1, 2, 7):
+        y1, st1 = f(x[:t1], w)
+        y2, st2 = f(x[t1:], w, None, st1)
+        np.testing.assert_allclose(np.concatenate([y1, y2]), y, rtol=1e-14, atol=0.0)
+        np.testing.assert_allclose(st2, st, rtol=0, atol=0)
+
+
+def sc_pin_state_holds_last_inputs(f):
+    # the final state is the last W-1 raw inputs, oldest first
+    x = np.arange(10, dtype=np.float64).reshape(5, 2)
+    _, st = f(x, np.ones((2, 3)))
+    np.testing.assert_array_equal(st[0], x[3:5])
+
+
+SC_PINS = [sc_pin_numpy_convolve, sc_pin_impulse, sc_pin_swish_values, sc_pin_sequences_independent,
+           sc_pin_continuation, sc_pin_state_holds_last_inputs]
+
+
+@pytest.mark.parametrize("pin", SC_PINS, ids=lambda p: p.__name__)
+def test_short_conv_pin(pin):
+    pin(oracle.short_conv_swish)
+
+
+def test_short_conv_decode_steps_match_prefill():
+    # T single-token steps on a carried state equal the sequence form
+    rng = np.random.default_rng(14)
+    x, w, s0 = rng.normal(size=(3, 11, 6)), rng.normal(size=(6, 4)), rng.normal(size=(3, 3, 6))
+    cu = np.arange(0, 34, 11)
+    y, st = oracle.short_conv_swish(x.reshape(33, 6), w, cu, s0)
+    state = s0.copy()
+    for t in range(11):
+        yt, state = oracle.short_conv_step(x[:, t], w, state)
+        np.testing.assert_allclose(yt, y.reshape(3, 11, 6)[:, t], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(state, st, rtol=0, atol=0)
+
+
+def _sc_mutant(kind):
+    def f(x, w, cu_seqlens=None, state0=None):
+        x, w = np.asarray(x, dtype=np.float64), np.asarray(w, dtype=np.float64)
+        T, C = x.shape
+        W = w.shape[1]
+        cu = np.array([0, T]) if cu_seqlens is None else np.asarray(cu_seqlens)
+        if kind == "leaks_across_sequences":
+            cu = np.array([0, T])
+        N = len(cu) - 1
+        y, st = np.zeros((T, C)), np.zeros((N, W - 1, C))
+        for s in range(N):
+            bos, eos = int(cu[s]), int(cu[s + 1])
+            hist = np.zeros((W - 1, C))
+            if state0 is not None and kind != "ignores_state":
+                hist = np.asarray(state0[s], dtype=np.float64)
+            xs = np.concatenate([hist, x[bos:eos]])
+            L = eos - bos
+            for t in range(L):
+                taps = w[:, ::-1] if kind == "taps_reversed" else w
+                z = sum(taps[:, j] * xs[t + j] for j in range(W))
+                if kind == "off_by_one":
+                    z = sum(taps[:, j] * xs[t + j - 1] for j in range(W)) if t > 0 else z
+                y[bos + t] = z if kind == "no_swish" else z / (1.0 + np.exp(-z))
+            st[s] = xs[L:L + W - 1] if kind != "state_newest_first" else xs[L:L + W - 1][::-1]
+        if kind == "leaks_across_sequences" and cu_seqlens is not None:
+            st = np.repeat(st, len(cu_seqlens) - 1, axis=0)
+        return y, st
+    return f
+
+
+@pytest.mark.parametrize("kind", ["taps_reversed", "no_swish", "off_by_one", "ignores_state",
+                                  "leaks_across_sequences", "state_newest_first"])
+def test_short_conv_pins_catch_planted_mistakes(kind):
+    f = _sc_mutant(kind)
+    failed = 0
+    for pin in SC_PINS:
+        try:
+            pin(f)
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    assert failed > 0, kind
