@@ -10,6 +10,7 @@ Build the library with ``python -m gated_delta_rule_125_b200.build``.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -29,12 +30,19 @@ KDA_FLAG_NO_L2NORM, KDA_FLAG_EXACT, KDA_FLAG_SCALAR_GATE = 0x1, 0x2, 0x4
 EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_size",
                     "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
                     "kda_prefill_ex", "kda_decode_step", "kda_decode_step_ex", "kda_device_error",
-                    "kda_prefill_noalloc")
+                    "kda_prefill_noalloc", "kda_short_conv_swish", "kda_short_conv_launches",
+                    "kda_decode_step_conv")
 
 
 class OutputGate(ctypes.Structure):
     """``kda_output_gate``: the fused output step (RMSNorm over d_v, sigmoid gate)."""
     _fields_ = [("gate", ctypes.c_void_p), ("weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
+class ShortConv(ctypes.Structure):
+    """``kda_short_conv``: causal short convolution + Swish (width, weight, states)."""
+    _fields_ = [("width", ctypes.c_int32), ("weight", ctypes.c_void_p), ("state_in", ctypes.c_void_p),
+                ("state_out", ctypes.c_void_p)]
 
 _lib = None
 
@@ -88,6 +96,14 @@ def load_library():
     lib.kda_prefill_noalloc.restype = ctypes.c_int
     lib.kda_device_error.argtypes = [ctypes.POINTER(i32), i32]
     lib.kda_device_error.restype = ctypes.c_int
+    sc = ctypes.POINTER(ShortConv)
+    lib.kda_short_conv_swish.argtypes = [vp, vp, sc, ip, i32, i64, i32, ctypes.c_int, vp]
+    lib.kda_short_conv_swish.restype = ctypes.c_int
+    lib.kda_short_conv_launches.argtypes = [i32, i32, i64]
+    lib.kda_short_conv_launches.restype = i64
+    lib.kda_decode_step_conv.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
+                                         u32, sc, sc, sc, og, vp, vp]
+    lib.kda_decode_step_conv.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -131,6 +147,14 @@ def _out_gate(out_gate):
         return None
     g, w, eps = out_gate
     return ctypes.byref(OutputGate(_ptr(g), _ptr(w), float(eps)))
+
+
+def _conv(conv):
+    """(weight [C, W] fp32, state_in or None, state_out or None) -> a ``kda_short_conv`` (None -> NULL)."""
+    if conv is None:
+        return None
+    w, sin, sout = conv
+    return ctypes.byref(ShortConv(int(w.shape[-1]), _ptr(w), _ptr(sin), _ptr(sout)))
 
 
 def _stream(stream, device):
@@ -232,21 +256,51 @@ def kda_prefill_noalloc(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, m
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, S, *, l2norm=True, o=None, out_gate=None,
-                    stream=None):
+                    conv=None, stream=None):
     """One KDA decode step (``kda_decode_step`` in ``include/kda.h``), S updated in place.
 
     q, k ``[N,H,dk]``, v ``[N,H,dv]``, log_alpha ``[N,H,dk]`` (or ``[N,H]``, one gate per
     head) fp32, beta ``[N,H]`` fp32,
-    S ``[N,H,dk,dv]`` fp32. Returns o ``[N,H,dv]``.
+    S ``[N,H,dk,dv]`` fp32. Returns o ``[N,H,dv]``. ``conv=(cq, ck, cv)``, each None or
+    ``(weight [H*d, W] fp32, state_in, state_out)`` with states ``[N, W-1, H*d]``: the
+    short convolution + Swish fused into the loads (``kda_decode_step_conv``).
     """
     lib = load_library()
     N, H, dk = q.shape
     dv = v.shape[-1]
     if o is None:
         o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
-    rc = lib.kda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
-                                N, H, dk, dv, _dtype_code(q), _flags(l2norm, False, log_alpha.dim() == 2),
-                                _out_gate(out_gate), _ptr(o), _stream(stream, q.device))
+    if conv is None:
+        rc = lib.kda_decode_step_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
+                                    N, H, dk, dv, _dtype_code(q), _flags(l2norm, False, log_alpha.dim() == 2),
+                                    _out_gate(out_gate), _ptr(o), _stream(stream, q.device))
+    else:
+        cq, ck, cv = conv
+        rc = lib.kda_decode_step_conv(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S),
+                                      N, H, dk, dv, _dtype_code(q), _flags(l2norm, False, log_alpha.dim() == 2),
+                                      _conv(cq), _conv(ck), _conv(cv), _out_gate(out_gate), _ptr(o),
+                                      _stream(stream, q.device))
     if rc != KDA_OK:
         raise KDAError(rc, "kda_decode_step")
     return o
+
+
+def kda_short_conv_swish(x, weight, cu_seqlens=None, *, state_in=None, state_out=None, y=None,
+                         stream=None):
+    """Causal short convolution + Swish (``kda_short_conv_swish`` in ``include/kda.h``).
+
+    x ``[T, C]`` (or ``[T, H, d]``, C = H * d) in bf16 or fp32, weight ``[C, W]`` fp32,
+    states ``[N, W-1, C]`` in x's dtype (state_out may be state_in). Returns y like x.
+    """
+    lib = load_library()
+    T = x.shape[0]
+    C = int(math.prod(x.shape[1:]))
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if y is None:
+        y = torch.empty_like(x)
+    c = ShortConv(int(weight.shape[-1]), _ptr(weight), _ptr(state_in), _ptr(state_out))
+    rc = lib.kda_short_conv_swish(_ptr(x), _ptr(y), ctypes.byref(c), _ptr(cu_seqlens), N, T, C,
+                                  _dtype_code(x), _stream(stream, x.device))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_short_conv_swish")
+    return y

@@ -301,7 +301,81 @@ kda_status kda_decode_step_ex(const void *q, const void *k, const void *v, const
                                      (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0, kEps,
                                      out_gate ? out_gate->gate : nullptr,
                                      out_gate ? out_gate->weight : nullptr, out_gate ? out_gate->eps : 0.f,
-                                     o, reinterpret_cast<cudaStream_t>(stream));
+                                     nullptr, o, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_short_conv_swish(const void *x, void *y, const kda_short_conv *conv, const int32_t *cu_seqlens,
+                                int32_t num_seqs, int64_t total_tokens, int32_t channels, kda_dtype dtype,
+                                kda_stream_t stream) {
+    if (!conv || num_seqs < 1 || total_tokens < 0 || channels < 8 || channels % 8) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (conv->width < 1 || conv->width > KDA_MAX_CONV_WIDTH) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens == nullptr && num_seqs != 1) return KDA_ERR_INVALID_ARG;
+    if (total_tokens > 0 && (!x || !y || !conv->weight)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(conv->state_in) || !aligned16(conv->state_out))
+        return KDA_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(conv->weight) & 3u) return KDA_ERR_MISALIGNED;
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    const uintptr_t xb = reinterpret_cast<uintptr_t>(x), yb = reinterpret_cast<uintptr_t>(y);
+    const uintptr_t bytes = (uintptr_t)total_tokens * (uintptr_t)channels * es;
+    if (total_tokens > 0 && xb < yb + bytes && yb < xb + bytes) return KDA_ERR_INVALID_ARG;  // y overlaps x
+    kda::ShortConvArgs a;
+    a.x = x;
+    a.y = y;
+    a.w = conv->weight;
+    a.state_in = conv->state_in;
+    a.state_out = conv->state_out;
+    a.cu = cu_seqlens;
+    a.N = num_seqs;
+    a.total = total_tokens;
+    a.C = channels;
+    a.W = conv->width;
+    const cudaError_t e = kda::short_conv_swish(a, dtype == KDA_DTYPE_BF16, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int64_t kda_short_conv_launches(int32_t width, int32_t writes_state, int64_t total_tokens) {
+    if (width < 1 || width > KDA_MAX_CONV_WIDTH || total_tokens < 0) return -1;
+    return kda::short_conv_launches(width, writes_state != 0, total_tokens);
+}
+
+kda_status kda_decode_step_conv(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, float *S, int32_t N, int32_t H, int32_t dk, int32_t dv,
+                                kda_dtype dtype, uint32_t flags, const kda_short_conv *conv_q,
+                                const kda_short_conv *conv_k, const kda_short_conv *conv_v,
+                                const kda_output_gate *out_gate, void *o, kda_stream_t stream) {
+    if (N < 1 || H < 1 || dk < 1 || dv < 1 || (int64_t)N * H > INT32_MAX) return KDA_ERR_INVALID_ARG;
+    if (flags & ~kKnownFlags) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_DTYPE_F32 && dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (!dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(beta) & 3u) return KDA_ERR_MISALIGNED;
+    if (!gate_aligned(log_alpha, flags)) return KDA_ERR_MISALIGNED;
+    kda_status rc = check_output_gate(out_gate, true);
+    if (rc != KDA_OK) return rc;
+    kda::DecodeConv cv{};
+    const kda_short_conv *cs[3] = {conv_q, conv_k, conv_v};
+    for (int i = 0; i < 3; ++i) {
+        if (!cs[i]) continue;
+        if (cs[i]->width < 1 || cs[i]->width > KDA_MAX_CONV_WIDTH) return KDA_ERR_UNSUPPORTED;
+        if (!cs[i]->weight) return KDA_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(cs[i]->weight) & 3u) return KDA_ERR_MISALIGNED;
+        if (!aligned16(cs[i]->state_in) || !aligned16(cs[i]->state_out)) return KDA_ERR_MISALIGNED;
+        cv.W[i] = cs[i]->width;
+        cv.w[i] = cs[i]->weight;
+        cv.state_in[i] = cs[i]->state_in;
+        cv.state_out[i] = cs[i]->state_out;
+    }
+    cudaError_t e = kda::decode_step(q, k, v, log_alpha, beta, S, N, H, dk, dv,
+                                     dtype == KDA_DTYPE_BF16, (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1,
+                                     (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0, kEps,
+                                     out_gate ? out_gate->gate : nullptr,
+                                     out_gate ? out_gate->weight : nullptr, out_gate ? out_gate->eps : 0.f,
+                                     &cv, o, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

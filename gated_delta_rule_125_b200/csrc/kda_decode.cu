@@ -14,19 +14,52 @@
 // (read once, evict-first; written once, streaming). The two column sums
 // over d_k (S~^T k and S~^T q) are per-thread partial sums finished through
 // shared memory; nothing else touches HBM.
+//
+// Optionally the layer's causal short convolution + Swish (§6.1) is applied to
+// q, k, v as they are loaded: the step's raw projection and the channel's last
+// W-1 raw inputs (the convolution state, read and then shifted in place by the
+// same thread) give z = sum_j w[c][j] x_{t-W+1+j}, and the input becomes
+// z sigmoid(z) (then q, k are L2-normalised as before).
 #include "kda_internal.cuh"
 
 namespace kda {
 namespace {
 
 constexpr int kDecodeThreads = 256;
+constexpr int kMaxConvW = 8;
+
+// Short convolution + Swish of channel c (of C) of sequence s, input xt; the
+// state's W-1 entries are read first and then written back shifted by one.
+template <typename T>
+__device__ __forceinline__ float conv_swish(float xt, int W, const float *__restrict__ w, const void *sin_,
+                                            void *sout_, int s, int C, int c) {
+    const T *sin = static_cast<const T *>(sin_);
+    T *sout = static_cast<T *>(sout_);
+    float hist[kMaxConvW - 1];
+    float z = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxConvW - 1; ++j) {
+        if (j < W - 1) {
+            hist[j] = sin ? IO<T>::ld(sin + ((size_t)s * (W - 1) + j) * C + c) : 0.f;
+            z = fmaf(w[(size_t)c * W + j], hist[j], z);
+        }
+    }
+    z = fmaf(w[(size_t)c * W + W - 1], xt, z);
+    if (sout) {
+#pragma unroll
+        for (int j = 0; j < kMaxConvW - 1; ++j)
+            if (j < W - 1) IO<T>::st(sout + ((size_t)s * (W - 1) + j) * C + c, j + 1 < W - 1 ? hist[j + 1] : xt);
+    }
+    return z / (1.f + __expf(-z));
+}
 
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
               float *__restrict__ S, T *__restrict__ o, int l2norm, int la_scalar, float eps,
-              const T *__restrict__ og_gate, const float *__restrict__ og_w, float og_eps) {
+              const T *__restrict__ og_gate, const float *__restrict__ og_w, float og_eps, DecodeConv cv,
+              int H) {
     constexpr int CG = DV / 4;                // 16-byte column groups per state row
     constexpr int RPP = kDecodeThreads / CG;  // state rows covered per pass
     constexpr int R = DK / RPP;               // rows held per thread
@@ -51,6 +84,7 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
     // 2. Token inputs while the state is in flight: warp 0 normalises q, k and
     //    forms k.q; warp 1 exponentiates the gate; warp 2 stages v and beta.
     const int warp = tid >> 5, lane = tid & 31;
+    const int seq = unit / H, hc = unit % H;  // for the convolution state
     if (warp == 0) {
         float qq = 0.f, kk = 0.f, qk = 0.f;
         float qv[DK / 32], kv[DK / 32];
@@ -58,6 +92,12 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         for (int m = 0; m < DK / 32; ++m) {
             qv[m] = IO<T>::ld(q + (size_t)unit * DK + lane + 32 * m);
             kv[m] = IO<T>::ld(k + (size_t)unit * DK + lane + 32 * m);
+            if (cv.W[0])
+                qv[m] = conv_swish<T>(qv[m], cv.W[0], cv.w[0], cv.state_in[0], cv.state_out[0], seq, H * DK,
+                                      hc * DK + lane + 32 * m);
+            if (cv.W[1])
+                kv[m] = conv_swish<T>(kv[m], cv.W[1], cv.w[1], cv.state_in[1], cv.state_out[1], seq, H * DK,
+                                      hc * DK + lane + 32 * m);
             qq += qv[m] * qv[m];
             kk += kv[m] * kv[m];
             qk += qv[m] * kv[m];
@@ -83,7 +123,12 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         for (int i = lane; i < DK; i += 32)
             s_a[i] = expf(la_scalar ? log_alpha[unit] : log_alpha[(size_t)unit * DK + i]);
     } else if (warp == 2) {
-        for (int j = lane; j < DV; j += 32) s_v[j] = IO<T>::ld(v + (size_t)unit * DV + j);
+        for (int j = lane; j < DV; j += 32) {
+            const float vj = IO<T>::ld(v + (size_t)unit * DV + j);
+            s_v[j] = cv.W[2] ? conv_swish<T>(vj, cv.W[2], cv.w[2], cv.state_in[2], cv.state_out[2], seq, H * DV,
+                                             hc * DV + j)
+                             : vj;
+        }
         if (lane == 0) s_misc[0] = beta[unit];
     }
     __syncthreads();
@@ -154,23 +199,23 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
 template <int DK, int DV, typename T>
 cudaError_t launch(const void *q, const void *k, const void *v, const float *la, const float *beta,
                    float *S, int N, int H, int l2norm, int la_scalar, float eps, const void *og_gate,
-                   const float *og_w, float og_eps, void *o, cudaStream_t st) {
+                   const float *og_w, float og_eps, const DecodeConv &cv, void *o, cudaStream_t st) {
     const unsigned units = (unsigned)N * (unsigned)H;
     decode_kernel<DK, DV, T><<<units, kDecodeThreads, 0, st>>>(
         (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps,
-        (const T *)og_gate, og_w, og_eps);
+        (const T *)og_gate, og_w, og_eps, cv, H);
     return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t dispatch(const void *q, const void *k, const void *v, const float *la,
                      const float *beta, float *S, int N, int H, int dk, int dv, int l2norm,
-                     int la_scalar, float eps, const void *og, const float *ow, float oe, void *o,
-                     cudaStream_t st) {
-    if (dk == 128 && dv == 128) return launch<128, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
-    if (dk == 128 && dv == 64) return launch<128, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
-    if (dk == 64 && dv == 128) return launch<64, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
-    if (dk == 64 && dv == 64) return launch<64, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, o, st);
+                     int la_scalar, float eps, const void *og, const float *ow, float oe, const DecodeConv &cv,
+                     void *o, cudaStream_t st) {
+    if (dk == 128 && dv == 128) return launch<128, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, cv, o, st);
+    if (dk == 128 && dv == 64) return launch<128, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, cv, o, st);
+    if (dk == 64 && dv == 128) return launch<64, 128, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, cv, o, st);
+    if (dk == 64 && dv == 64) return launch<64, 64, T>(q, k, v, la, beta, S, N, H, l2norm, la_scalar, eps, og, ow, oe, cv, o, st);
     return cudaErrorInvalidValue;
 }
 
@@ -179,11 +224,14 @@ cudaError_t dispatch(const void *q, const void *k, const void *v, const float *l
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
                         int l2norm, int la_scalar, float eps, const void *og_gate, const float *og_w,
-                        float og_eps, void *o, cudaStream_t st) {
+                        float og_eps, const DecodeConv *conv, void *o, cudaStream_t st) {
+    DecodeConv cv{};
+    if (conv) cv = *conv;
     if (bf16)
         return dispatch<__nv_bfloat16>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, og_gate, og_w,
-                                       og_eps, o, st);
-    return dispatch<float>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, og_gate, og_w, og_eps, o, st);
+                                       og_eps, cv, o, st);
+    return dispatch<float>(q, k, v, la, beta, S, N, H, dk, dv, l2norm, la_scalar, eps, og_gate, og_w, og_eps, cv,
+                           o, st);
 }
 
 }  // namespace kda

@@ -75,11 +75,35 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
 // out), or nullptr if it cannot be resolved.
 int *device_error_word();
 
+// Causal short convolution + Swish of one projection x [T][C] (C % 8 == 0).
+struct ShortConvArgs {
+    const void *x;
+    void *y;
+    const float *w;        // [C][W]
+    const void *state_in;  // [N][W-1][C] or nullptr (zeros)
+    void *state_out;       // [N][W-1][C] or nullptr
+    const int32_t *cu;     // [N+1] or nullptr (one sequence)
+    int N;
+    int64_t total;
+    int C, W;
+};
+cudaError_t short_conv_swish(const ShortConvArgs &a, bool bf16, cudaStream_t st);
+int short_conv_launches(int W, bool state_out, int64_t total);
+
+// The same convolution fused into a decode step's loads of q, k, v (index 0, 1, 2):
+// W[i] == 0 leaves that input as it is. States are [N][W-1][H * d].
+struct DecodeConv {
+    int W[3];
+    const float *w[3];
+    const void *state_in[3];
+    void *state_out[3];
+};
+
 // decode step
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,
                         int l2norm, int la_scalar, float eps, const void *og_gate, const float *og_w,
-                        float og_eps, void *o, cudaStream_t st);
+                        float og_eps, const DecodeConv *conv, void *o, cudaStream_t st);
 // fp32 CUDA-core path: the output step applied to o in place after the prefill.
 cudaError_t simt_output_gate(const PrefillArgs &a, bool bf16, cudaStream_t st);
 

@@ -220,6 +220,67 @@ kda_status kda_decode_step_ex(const void *q, const void *k, const void *v, const
                               int32_t dv, kda_dtype dtype, uint32_t flags,
                               const kda_output_gate *out_gate, void *o, kda_stream_t stream);
 
+/*
+ * Causal short convolution followed by Swish, the layer's step before the
+ * recurrence ("[Kimi-2] Kimi Linear：用 KDA 重写长上下文注意力" §6 and §6.1;
+ * "Kimi Delta Attention：把遗忘门做到每个通道", the pre-processing of q and k):
+ * every channel c of a projection x [T][C] is convolved over the tokens of its
+ * own sequence with its own W taps, then passed through Swish,
+ *
+ *     z_t[c] = sum_{j<W} weight[c][j] * x_{t-W+1+j}[c],   y_t[c] = z_t[c] * sigmoid(z_t[c]),
+ *
+ * positions before a sequence's first token reading that sequence's initial
+ * state (or zero). The pages give neither the window nor a bias: the window is
+ * the caller's (1 .. KDA_MAX_CONV_WIDTH) and there is no bias. q and k are
+ * L2-normalised afterwards by kda_prefill / kda_decode_step (flag default).
+ *
+ *   width      W
+ *   weight     [C][W] fp32, device, 4-byte aligned; weight[c][W-1] weighs the
+ *              current token, weight[c][0] the one W-1 tokens earlier
+ *   state_in   [N][W-1][C] in the io dtype, device, 16-byte aligned: each
+ *              sequence's previous W-1 raw inputs, oldest first; NULL = zeros
+ *   state_out  [N][W-1][C], 16-byte aligned: each sequence's last W-1 raw
+ *              inputs after the call (reaching into state_in when a sequence is
+ *              shorter than W-1); NULL = not written. May alias state_in.
+ */
+#define KDA_MAX_CONV_WIDTH 8
+typedef struct kda_short_conv {
+    int32_t width;
+    const float *weight;
+    const void *state_in;
+    void *state_out;
+} kda_short_conv;
+
+/*
+ * The prefill form: y [T][C] from x [T][C] (the io dtype, device, 16-byte
+ * aligned, C a multiple of 8; y must not overlap x). Sequences as in
+ * kda_prefill (cu_seqlens device [N+1], or NULL for one sequence). Enqueued on
+ * `stream` as kda_short_conv_launches() kernels (the outputs, then state_out
+ * when requested). Run it on the q, k and v projections and pass the results
+ * to kda_prefill. Errors as kda_prefill's (KDA_ERR_UNSUPPORTED: a width
+ * outside 1 .. KDA_MAX_CONV_WIDTH).
+ */
+kda_status kda_short_conv_swish(const void *x, void *y, const kda_short_conv *conv,
+                                const int32_t *cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                                int32_t channels, kda_dtype dtype, kda_stream_t stream);
+
+/* Kernels kda_short_conv_swish launches (writes_state: state_out != NULL); -1 for a bad width. */
+int64_t kda_short_conv_launches(int32_t width, int32_t writes_state, int64_t total_tokens);
+
+/*
+ * kda_decode_step_ex with the short convolution + Swish fused into the loads of
+ * q, k and v: here q, k, v are the step's raw projections ([N][H][d]) and
+ * conv_q, conv_k, conv_v (each NULL: that input is used as it is) carry
+ * C = H * d channels with states [N][W-1][H * d] (normally state_in ==
+ * state_out: updated in place, one token per call).
+ */
+kda_status kda_decode_step_conv(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
+                                int32_t dv, kda_dtype dtype, uint32_t flags,
+                                const kda_short_conv *conv_q, const kda_short_conv *conv_k,
+                                const kda_short_conv *conv_v, const kda_output_gate *out_gate, void *o,
+                                kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

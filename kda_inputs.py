@@ -14,7 +14,11 @@ generator on the target device):
 * beta: sigmoid(N(0, 1)), fp32;
 * log_alpha: -softplus(N(mu, 1)) per key channel, fp32 (mu = -3, or -4 for
   the long-memory 1M-token workload);
-* S0: N(0, s0_std^2) fp32, or zeros.
+* S0: N(0, s0_std^2) fp32, or zeros;
+* short-convolution inputs (the layer's q, k, v projections before the
+  convolution): raw projections N(0, 1) in the workload dtype, taps
+  N(0, 1/W) fp32 per channel, initial convolution states N(0, 1) in the
+  workload dtype.
 """
 from __future__ import annotations
 
@@ -23,7 +27,8 @@ import torch.nn.functional as F
 
 _BLOCK = 1 << 16  # tokens drawn per generator call (bounds fp32 temporaries)
 
-_IDS = {"q": 1, "k": 2, "v": 3, "beta": 4, "log_alpha": 5, "S0": 6, "len": 7, "log_alpha_scalar": 8}
+_IDS = {"q": 1, "k": 2, "v": 3, "beta": 4, "log_alpha": 5, "S0": 6, "len": 7, "log_alpha_scalar": 8,
+        "conv_x": 9, "conv_w": 10, "conv_state": 11}
 
 
 def _gen(device, seed, name, block=0):
@@ -138,3 +143,15 @@ def decode_workload(N, H, d, steps, dtype=torch.bfloat16, device="cpu", seed=0, 
     return dict(q=q.view(*shp, d), k=k.view(*shp, d), v=v.view(*shp, d),
                 log_alpha=la.view(*shp, d), beta=beta.view(*shp),
                 S0=initial_state(N, H, d, d, s0_std, device, seed))
+
+
+def conv_inputs(T, C, W, N=1, dtype=torch.bfloat16, device="cpu", seed=0, tensor=0, with_state=True):
+    """Short-convolution inputs for one projection: x [T, C] N(0,1) in ``dtype``,
+    taps [C, W] N(0, 1/W) fp32 and an initial state [N, W-1, C] N(0,1) in ``dtype``
+    (None without state). ``tensor`` separates the q / k / v draws."""
+    x = _normal((T, C), device, seed * 3 + tensor, "conv_x").to(dtype)
+    w = _normal((C, W), device, seed * 3 + tensor, "conv_w") / float(W) ** 0.5
+    st = None
+    if with_state:
+        st = _normal((N, W - 1, C), device, seed * 3 + tensor, "conv_state").to(dtype)
+    return x, w, st

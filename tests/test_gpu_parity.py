@@ -474,3 +474,158 @@ def test_output_gate_workload_prefill_8k():
     gate, w, eps = _gate_inputs(8192, 32, 128, torch.bfloat16, 47)
     o, _ = run(inp, out_gate=(gate, w, eps))
     _check_gated(o, inp, gate, w, eps, torch.bfloat16, heads=[5, 26], label="gated prefill_8k")
+
+
+# ------------------------------------- short convolution + Swish (§6.1) ----
+# The convolution's output is one fp32 dot product of W taps then Swish, stored
+# in the io dtype: it must lie within the io dtype's rounding of the fp64 value
+# (bf16: 2^-8 relative; fp32: 1e-5 relative, fast exponential). States are raw
+# input copies: bit-exact.
+
+def _conv_ref(x, w, cu=None, st=None):
+    return oracle.short_conv_swish(host(x).reshape(x.shape[0], -1), host(w),
+                                   None if cu is None else cu.cpu().numpy(), None if st is None else host(st))
+
+
+def _conv_close(y, y_ref, dtype, label):
+    rel = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-5
+    err = np.abs(host(y).reshape(y_ref.shape) - y_ref)
+    bound = rel * np.abs(y_ref) + 1e-6
+    assert np.isfinite(err).all(), label
+    assert np.all(err <= bound), "%s: worst excess %.3e" % (label, float((err - bound).max()))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 8])
+def test_short_conv_varlen(W, dtype):
+    """Empty, one-token and ragged sequences (tiles of 32 tokens cross their boundaries)."""
+    lengths = [37, 0, 1, 200, 5, 64, 3]
+    T, N, C = sum(lengths), len(lengths), 96
+    x, w, st = KI.conv_inputs(T, C, W, N, dtype, DEV, seed=W)
+    cu = KI.cu_from_lengths(lengths, DEV)
+    st_out = torch.full_like(st, float("nan"))
+    y = kda.kda_short_conv_swish(x, w, cu, state_in=st, state_out=st_out)
+    torch.cuda.synchronize()
+    y_ref, st_ref = _conv_ref(x, w, cu, st)
+    _conv_close(y, y_ref, dtype, "W=%d" % W)
+    np.testing.assert_array_equal(host(st_out), st_ref)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_short_conv_zero_state_and_aliased_state(dtype):
+    T, C, W = 150, 64, 4
+    x, w, st = KI.conv_inputs(T, C, W, 1, dtype, DEV, seed=21)
+    y0 = kda.kda_short_conv_swish(x, w)  # one sequence, no state: zero history
+    y_ref, st_ref0 = _conv_ref(x, w)
+    _conv_close(y0, y_ref, dtype, "zero state")
+    st_keep = st.clone()
+    y1 = kda.kda_short_conv_swish(x, w, state_in=st, state_out=st)  # state updated in place
+    torch.cuda.synchronize()
+    y_ref1, st_ref1 = _conv_ref(x, w, None, st_keep)
+    _conv_close(y1, y_ref1, dtype, "aliased state")
+    np.testing.assert_array_equal(host(st), st_ref1)
+
+
+def test_short_conv_rejects_bad_arguments():
+    x, w, _ = KI.conv_inputs(16, 64, 4, 1, torch.bfloat16, DEV, seed=22, with_state=False)
+    with pytest.raises(kda.KDAError):
+        kda.kda_short_conv_swish(x, torch.zeros((64, 9), device=DEV))  # width 9 > KDA_MAX_CONV_WIDTH
+    with pytest.raises(kda.KDAError):
+        kda.kda_short_conv_swish(x, w, y=x)  # y overlaps x
+    lib = kda.load_library()
+    assert lib.kda_short_conv_launches(4, 1, 16) == 2 and lib.kda_short_conv_launches(1, 1, 16) == 1
+    assert lib.kda_short_conv_launches(4, 0, 0) == 0 and lib.kda_short_conv_launches(0, 0, 16) == -1
+
+
+def test_short_conv_workload_prefill_8k():
+    """The q projection of prefill_8k (T=8192, C=32*128), W=4: every output vs the oracle."""
+    x, w, st = KI.conv_inputs(8192, 4096, 4, 1, torch.bfloat16, DEV, seed=23)
+    st_out = torch.empty_like(st)
+    y = kda.kda_short_conv_swish(x, w, state_in=st, state_out=st_out)
+    torch.cuda.synchronize()
+    y_ref, st_ref = _conv_ref(x, w, None, st)
+    _conv_close(y, y_ref, torch.bfloat16, "prefill_8k q")
+    np.testing.assert_array_equal(host(st_out), st_ref)
+
+
+def test_short_conv_then_prefill():
+    """q, k, v through the convolution, then the prefill (the oracle on the same bits)."""
+    lengths, H, d, W = [100, 64, 1], 2, 128, 4
+    T, N = sum(lengths), len(lengths)
+    cu = KI.cu_from_lengths(lengths, DEV)
+    outs = []
+    for i in range(3):
+        x, w, st = KI.conv_inputs(T, H * d, W, N, torch.bfloat16, DEV, seed=24, tensor=i)
+        outs.append(kda.kda_short_conv_swish(x, w, cu, state_in=st).view(T, H, d))
+    inp = make(lengths, H, d, d, torch.bfloat16, seed=24)
+    inp.update(q=outs[0], k=outs[1], v=outs[2])
+    o, S_T = run(inp)
+    check(o, S_T, inp, torch.bfloat16, label="conv then prefill")
+
+
+@pytest.mark.parametrize("dtype,d,with_v", [(torch.bfloat16, 128, True), (torch.float32, 64, True),
+                                            (torch.bfloat16, 128, False)])
+def test_decode_conv_steps(dtype, d, with_v):
+    """Decode steps with the convolution fused into the q, k (, v) loads; states in place."""
+    N, H, W, steps = 4, 3, 4, 4
+    wl = KI.decode_workload(N, H, d, steps, dtype, DEV, seed=25, s0_std=0.1)
+    convs, refs = [], []
+    for i in range(3):
+        x, w, st = KI.conv_inputs(steps * N, H * d, W, N, dtype, DEV, seed=25, tensor=i)
+        raw = x.view(steps, N, H, d)
+        convs.append((w, st, st, raw))
+        refs.append(host(st))
+    if not with_v:
+        convs[2] = (None, None, None, wl["v"])
+    S = wl["S0"].clone()
+    S_ref = host(S)
+    atol, stol = TOL[dtype]
+    for t in range(steps):
+        cq, ck, cv = [None if c[0] is None else (c[0], c[1], c[2]) for c in convs]
+        o = kda.kda_decode_step(convs[0][3][t], convs[1][3][t], convs[2][3][t], wl["log_alpha"][t],
+                                wl["beta"][t], S, conv=(cq, ck, cv))
+        torch.cuda.synchronize()
+        xs = []
+        for i in range(3):
+            if convs[i][0] is None:
+                xs.append(host(wl["v"][t]))
+                continue
+            y, refs[i] = oracle.short_conv_step(host(convs[i][3][t]).reshape(N, H * d), host(convs[i][0]), refs[i])
+            xs.append(y.reshape(N, H, d))
+        o_ref, S_ref = oracle.decode_step(xs[0], xs[1], xs[2], host(wl["log_alpha"][t]), host(wl["beta"][t]), S_ref)
+        assert float(np.abs(host(o) - o_ref).max()) <= atol, "step %d" % t
+        assert rel_fro(host(S), S_ref) <= stol, "step %d" % t
+        for i in range(3):
+            if convs[i][0] is not None:
+                np.testing.assert_array_equal(host(convs[i][1]), refs[i])
+
+
+def test_decode_conv_continues_prefill_conv():
+    """fp32: conv + prefill over T-3 tokens, then 3 decode steps with the fused convolution
+    continuing from the prefill's conv states == conv + prefill over all T tokens."""
+    T, H, d, W = 67, 2, 128, 4
+    m = T - 3
+    raw, ws = [], []
+    for i in range(3):
+        x, w, _ = KI.conv_inputs(T, H * d, W, 1, torch.float32, DEV, seed=26, tensor=i, with_state=False)
+        raw.append(x)
+        ws.append(w)
+    inp = make([T], H, d, d, torch.float32, seed=26)
+    full = [kda.kda_short_conv_swish(raw[i], ws[i]).view(T, H, d) for i in range(3)]
+    inp_all = dict(inp, q=full[0], k=full[1], v=full[2])
+    o_all, S_all = run(inp_all)
+    states, part = [], []
+    for i in range(3):
+        st = torch.empty((1, W - 1, H * d), device=DEV)
+        part.append(kda.kda_short_conv_swish(raw[i][:m].contiguous(), ws[i], state_out=st).view(m, H, d))
+        states.append(st)
+    inp_m = dict(q=part[0], k=part[1], v=part[2], log_alpha=inp["log_alpha"][:m], beta=inp["beta"][:m],
+                 S0=inp["S0"], cu_seqlens=KI.cu_from_lengths([m], DEV), lengths=[m])
+    _, S = run(inp_m)
+    for t in range(m, T):
+        xs = [raw[i][t:t + 1].view(1, H, d).clone() for i in range(3)]
+        cv = [(ws[i], states[i], states[i]) for i in range(3)]
+        o = kda.kda_decode_step(xs[0], xs[1], xs[2], inp["log_alpha"][t:t + 1].clone(),
+                                inp["beta"][t:t + 1].clone(), S, conv=tuple(cv))
+        torch.testing.assert_close(o[0], o_all[t], atol=2e-5, rtol=0)
+    torch.testing.assert_close(S, S_all, atol=2e-5, rtol=0)
