@@ -47,6 +47,12 @@ PREFILL_STATE_BYTES = 2 * H * D * D * 4
 GDN_BYTES_PER_TOKEN = 3 * H * D * 2 + H * 4 + H * 4 + H * D * 2
 # decode per step: state read + write, q,k,v bf16, log_alpha fp32, beta fp32, o bf16
 DECODE_BYTES = DEC_N * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
+CONV_W = 4  # short-convolution window of the conv lines (the pages leave it open)
+# one short convolution over a [T8K, H*D] bf16 projection: x read, y written, taps,
+# the state read and written
+CONV_BYTES = 2 * T8K * H * D * 2 + H * D * CONV_W * 4 + 2 * (CONV_W - 1) * H * D * 2
+# decode with the convolution fused into the q, k, v loads: + three states read and written, taps
+DECODE_CONV_BYTES = DECODE_BYTES + 3 * (2 * DEC_N * (CONV_W - 1) * H * D * 2 + H * D * CONV_W * 4)
 
 
 def peaks():
@@ -290,6 +296,56 @@ def run_kda(args, world, rank, local):
     og_gbs = og_bytes / (ev0.elapsed_time(ev1) / args.steps * 1e-3) / 1e9
     del og
 
+    # ---- the layer's step before the recurrence: short convolution + Swish on the
+    #      q, k, v projections (W = 4, states written for a following decode), alone
+    #      and followed by the prefill
+    conv_in = [KI.conv_inputs(T8K, H * D, CONV_W, 1, torch.bfloat16, dev, seed=rank, tensor=i) for i in range(3)]
+    conv_out = [torch.empty_like(c[0]) for c in conv_in]
+    conv_st = [torch.empty_like(c[2]) for c in conv_in]
+    conv_launches = kda.load_library().kda_short_conv_launches(CONV_W, 1, T8K)
+
+    def convs():
+        for (x, w, st), y, so in zip(conv_in, conv_out, conv_st):
+            kda.kda_short_conv_swish(x, w, state_in=st, state_out=so, y=y)
+
+    def conv_prefill():
+        convs()
+        kda.kda_prefill(conv_out[0].view(T8K, H, D), conv_out[1].view(T8K, H, D), conv_out[2].view(T8K, H, D),
+                        la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
+
+    # Three short convolutions (two launches each, ~30 us of GPU time): the host issues them
+    # more slowly than the GPU runs them,
+    # so the convolution line replays them from a CUDA graph (captured once).
+    conv_graph = None
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            convs()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        conv_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(conv_graph):
+            convs()
+        torch.cuda.synchronize()
+    except RuntimeError:
+        conv_graph = None
+    conv_ms = {}
+    for name, fn in (("conv", conv_graph.replay if conv_graph is not None else convs), ("conv_prefill", conv_prefill)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        conv_ms[name] = (ev0.elapsed_time(ev1) / args.steps, max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev))
+    conv_gbs = 3 * CONV_BYTES / (conv_ms["conv"][0] * 1e-3) / 1e9
+    conv_graph_used = conv_graph is not None
+    del conv_graph, conv_in, conv_out, conv_st
+
     # ---- end to end through the C ABI: pinned host inputs -> device -> host
     h_in = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v", "log_alpha", "beta", "S0")}
     h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -342,6 +398,30 @@ def run_kda(args, world, rank, local):
     dec_us_max = max_over_ranks(dec_us, world, dev)
     dec_gbs = DECODE_BYTES / (dec_us * 1e-6) / 1e9
 
+    # ---- decode with the short convolution fused into the q, k, v loads (states in place)
+    dconv = []
+    for i in range(3):
+        _, w_, st_ = KI.conv_inputs(1, H * D, CONV_W, DEC_N, torch.bfloat16, dev, seed=rank, tensor=i)
+        dconv.append((w_, st_, st_))
+
+    def decode_conv(t):
+        i = t % DEC_STEPS_POOL
+        kda.kda_decode_step(dec["q"][i], dec["k"][i], dec["v"][i], dec["log_alpha"][i],
+                            dec["beta"][i], S, o=od, conv=tuple(dconv))
+
+    for t in range(max(3, args.warmup)):
+        decode_conv(t)
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for t in range(dsteps):
+        decode_conv(t)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    dconv_us = ev0.elapsed_time(ev1) * 1e3 / dsteps
+    dconv_us_max = max_over_ranks(dconv_us, world, dev)
+    dconv_gbs = DECODE_CONV_BYTES / (dconv_us * 1e-6) / 1e9
+
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
@@ -359,7 +439,8 @@ def run_kda(args, world, rank, local):
                      "algorithmic_bytes": bytes_pass, "peak_source": peak_src},
         "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 3 * args.steps * launches_prefill + dsteps,
+        "gpu_launches": (3 * args.steps * launches_prefill + dsteps + args.steps * 3 * conv_launches
+                         + args.steps * (3 * conv_launches + launches_prefill) + dsteps),
         "clocks": clk.summary(),
         "gdn": {"value": world * T8K / (gdn_ms * 1e-3), "unit": "tokens/s", "ms_per_step": gdn_ms,
                 "workload": "gdn_8k: prefill_8k with one forget gate per (token, head) "
@@ -384,6 +465,24 @@ def run_kda(args, world, rank, local):
                                 "traffic": profiled_traffic("decode_kernel_decode_256.md", DECODE_SOURCES),
                                 "kernel": "decode_kernel<128,128,bf16>",
                                 "algorithmic_bytes": DECODE_BYTES, "peak_source": peak_src}},
+        "short_conv": {"value": world * T8K / (conv_ms["conv"][1] * 1e-3), "unit": "tokens/s",
+                       "ms_per_step": conv_ms["conv"][1], "cuda_graph": conv_graph_used,
+                       "workload": "short convolution (W=%d) + Swish of the q, k, v projections of prefill_8k "
+                                   "([8192, 32*128] bf16 each, states written; page section 6.1)" % CONV_W,
+                       "conv_then_prefill": {"value": world * T8K / (conv_ms["conv_prefill"][1] * 1e-3),
+                                             "unit": "tokens/s", "ms_per_step": conv_ms["conv_prefill"][1]},
+                       "roofline": {"bound": "hbm", "achieved": conv_gbs, "peak": hbm, "unit": "GB/s",
+                                    "frac": conv_gbs / hbm, "traffic": None,
+                                    "kernel": "conv_kernel<4,bf16> + conv_state_kernel (x3)",
+                                    "algorithmic_bytes": 3 * CONV_BYTES, "peak_source": peak_src}},
+        "decode_conv": {"value": DECODE_CONV_BYTES / (dconv_us_max * 1e-6) / 1e9, "unit": "GB/s",
+                        "us_per_step": dconv_us_max, "steps": dsteps,
+                        "workload": "decode_256 with the short convolution (W=%d) + Swish fused into the q, k, v "
+                                    "loads, bf16 states [256, %d, 4096] x3 in place" % (CONV_W, CONV_W - 1),
+                        "roofline": {"bound": "hbm", "achieved": dconv_gbs, "peak": hbm, "unit": "GB/s",
+                                     "frac": dconv_gbs / hbm, "traffic": None,
+                                     "kernel": "decode_kernel<128,128,bf16> with the convolution",
+                                     "algorithmic_bytes": DECODE_CONV_BYTES, "peak_source": peak_src}},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v_cpu, cores, desc = oracle_sample(seconds_target=args.cpu_seconds)

@@ -361,7 +361,7 @@ kda_status kda_decode_step_conv(const void *q, const void *k, const void *v, con
     const kda_short_conv *cs[3] = {conv_q, conv_k, conv_v};
     for (int i = 0; i < 3; ++i) {
         if (!cs[i]) continue;
-        if (cs[i]->width < 1 || cs[i]->width > KDA_MAX_CONV_WIDTH) return KDA_ERR_UNSUPPORTED;
+        if (cs[i]->width < 1 || cs[i]->width > kda::kDecodeMaxConvWidth) return KDA_ERR_UNSUPPORTED;
         if (!cs[i]->weight) return KDA_ERR_INVALID_ARG;
         if (reinterpret_cast<uintptr_t>(cs[i]->weight) & 3u) return KDA_ERR_MISALIGNED;
         if (!aligned16(cs[i]->state_in) || !aligned16(cs[i]->state_out)) return KDA_ERR_MISALIGNED;

@@ -26,34 +26,55 @@ namespace kda {
 namespace {
 
 constexpr int kDecodeThreads = 256;
-constexpr int kMaxConvW = 8;
+constexpr int kMaxConvW = kDecodeMaxConvWidth;
 
-// Short convolution + Swish of channel c (of C) of sequence s, input xt; the
-// state's W-1 entries are read first and then written back shifted by one.
-template <typename T>
-__device__ __forceinline__ float conv_swish(float xt, int W, const float *__restrict__ w, const void *sin_,
-                                            void *sout_, int s, int C, int c) {
+// Short convolution + Swish of a lane's NM channels cbase + lane + 32 m of
+// sequence s (C channels per state row): every load is issued first (the
+// step's input, the W-1 state entries, the W taps), then z and Swish, then the
+// state is written back shifted by one (the same thread read it: in place is safe).
+template <typename T, int NM>
+__device__ __forceinline__ void conv_swish_lane(const T *__restrict__ xrow, int W, const float *__restrict__ w,
+                                                const void *sin_, void *sout_, int s, int C, int cbase,
+                                                int lane, float (&out)[NM]) {
     const T *sin = static_cast<const T *>(sin_);
     T *sout = static_cast<T *>(sout_);
-    float hist[kMaxConvW - 1];
-    float z = 0.f;
+    float xv[NM], h[NM][kMaxConvW - 1], wv[NM][kMaxConvW];
 #pragma unroll
-    for (int j = 0; j < kMaxConvW - 1; ++j) {
-        if (j < W - 1) {
-            hist[j] = sin ? IO<T>::ld(sin + ((size_t)s * (W - 1) + j) * C + c) : 0.f;
-            z = fmaf(w[(size_t)c * W + j], hist[j], z);
-        }
-    }
-    z = fmaf(w[(size_t)c * W + W - 1], xt, z);
-    if (sout) {
+    for (int m = 0; m < NM; ++m) {
+        const int c = cbase + lane + 32 * m;
+        xv[m] = IO<T>::ld(xrow + lane + 32 * m);
 #pragma unroll
         for (int j = 0; j < kMaxConvW - 1; ++j)
-            if (j < W - 1) IO<T>::st(sout + ((size_t)s * (W - 1) + j) * C + c, j + 1 < W - 1 ? hist[j + 1] : xt);
+            h[m][j] = (j < W - 1 && sin) ? IO<T>::ld(sin + ((size_t)s * (W - 1) + j) * C + c) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxConvW; ++j) wv[m][j] = j < W ? w[(size_t)c * W + j] : 0.f;
     }
-    return z / (1.f + __expf(-z));
+#pragma unroll
+    for (int m = 0; m < NM; ++m) {
+        float z = 0.f;
+#pragma unroll
+        for (int j = 0; j < kMaxConvW; ++j) {
+            if (j < W - 1) z = fmaf(wv[m][j], h[m][j < kMaxConvW - 1 ? j : 0], z);
+            else if (j == W - 1) z = fmaf(wv[m][j], xv[m], z);
+        }
+        out[m] = __fdividef(z, 1.f + __expf(-z));
+    }
+    if (sout) {
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+            const int c = cbase + lane + 32 * m;
+#pragma unroll
+            for (int j = 0; j < kMaxConvW - 1; ++j) {
+                if (j < W - 1) {
+                    const float nv = (j + 1 < W - 1) ? h[m][j + 1 < kMaxConvW - 1 ? j + 1 : 0] : xv[m];
+                    IO<T>::st(sout + ((size_t)s * (W - 1) + j) * C + c, nv);
+                }
+            }
+        }
+    }
 }
 
-template <int DK, int DV, typename T>
+template <int DK, int DV, typename T, bool CONV>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -85,19 +106,77 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
     //    forms k.q; warp 1 exponentiates the gate; warp 2 stages v and beta.
     const int warp = tid >> 5, lane = tid & 31;
     const int seq = unit / H, hc = unit % H;  // for the convolution state
-    if (warp == 0) {
+    if constexpr (CONV) {
+        // 2'. With the short convolution: warp 0 q, warp 3 k, warp 2 v and beta (each
+        //     convolved or as is), warp 1 the gate; then warp 0 normalises q, k.
+        if (warp == 0 || warp == 3) {
+            const bool isq = warp == 0;
+            const T *x = isq ? q : k;
+            const int Wc = isq ? cv.W[0] : cv.W[1];
+            float xs[DK / 32];
+            if (Wc) {
+                conv_swish_lane<T, DK / 32>(x + (size_t)unit * DK, Wc, isq ? cv.w[0] : cv.w[1],
+                                            isq ? cv.state_in[0] : cv.state_in[1],
+                                            isq ? cv.state_out[0] : cv.state_out[1], seq, H * DK, hc * DK, lane, xs);
+            } else {
+#pragma unroll
+                for (int m = 0; m < DK / 32; ++m) xs[m] = IO<T>::ld(x + (size_t)unit * DK + lane + 32 * m);
+            }
+            float *dst = warp == 0 ? s_q : s_k;
+#pragma unroll
+            for (int m = 0; m < DK / 32; ++m) dst[lane + 32 * m] = xs[m];
+        } else if (warp == 1) {
+            for (int i = lane; i < DK; i += 32)
+                s_a[i] = expf(la_scalar ? log_alpha[unit] : log_alpha[(size_t)unit * DK + i]);
+        } else if (warp == 2) {
+            float vs[DV / 32];
+            if (cv.W[2]) {
+                conv_swish_lane<T, DV / 32>(v + (size_t)unit * DV, cv.W[2], cv.w[2], cv.state_in[2], cv.state_out[2],
+                                            seq, H * DV, hc * DV, lane, vs);
+            } else {
+#pragma unroll
+                for (int m = 0; m < DV / 32; ++m) vs[m] = IO<T>::ld(v + (size_t)unit * DV + lane + 32 * m);
+            }
+#pragma unroll
+            for (int m = 0; m < DV / 32; ++m) s_v[lane + 32 * m] = vs[m];
+            if (lane == 0) s_misc[0] = beta[unit];
+        }
+        __syncthreads();
+        if (warp == 0) {
+            float qq = 0.f, kk = 0.f, qk = 0.f;
+#pragma unroll
+            for (int m = 0; m < DK / 32; ++m) {
+                const float a = s_q[lane + 32 * m], b = s_k[lane + 32 * m];
+                qq += a * a;
+                kk += b * b;
+                qk += a * b;
+            }
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                qq += __shfl_xor_sync(0xffffffffu, qq, off);
+                kk += __shfl_xor_sync(0xffffffffu, kk, off);
+                qk += __shfl_xor_sync(0xffffffffu, qk, off);
+            }
+            float iq = 1.f, ik = 1.f;
+            if (l2norm) {
+                iq = 1.f / fmaxf(sqrtf(qq), eps);
+                ik = 1.f / fmaxf(sqrtf(kk), eps);
+            }
+#pragma unroll
+            for (int m = 0; m < DK / 32; ++m) {
+                s_q[lane + 32 * m] *= iq;
+                s_k[lane + 32 * m] *= ik;
+            }
+            if (lane == 0) s_misc[1] = qk * iq * ik;
+        }
+    } else {
+      if (warp == 0) {
         float qq = 0.f, kk = 0.f, qk = 0.f;
         float qv[DK / 32], kv[DK / 32];
 #pragma unroll
         for (int m = 0; m < DK / 32; ++m) {
             qv[m] = IO<T>::ld(q + (size_t)unit * DK + lane + 32 * m);
             kv[m] = IO<T>::ld(k + (size_t)unit * DK + lane + 32 * m);
-            if (cv.W[0])
-                qv[m] = conv_swish<T>(qv[m], cv.W[0], cv.w[0], cv.state_in[0], cv.state_out[0], seq, H * DK,
-                                      hc * DK + lane + 32 * m);
-            if (cv.W[1])
-                kv[m] = conv_swish<T>(kv[m], cv.W[1], cv.w[1], cv.state_in[1], cv.state_out[1], seq, H * DK,
-                                      hc * DK + lane + 32 * m);
             qq += qv[m] * qv[m];
             kk += kv[m] * kv[m];
             qk += qv[m] * kv[m];
@@ -119,17 +198,13 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
             s_k[lane + 32 * m] = kv[m] * ik;
         }
         if (lane == 0) s_misc[1] = qk * iq * ik;
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         for (int i = lane; i < DK; i += 32)
             s_a[i] = expf(la_scalar ? log_alpha[unit] : log_alpha[(size_t)unit * DK + i]);
-    } else if (warp == 2) {
-        for (int j = lane; j < DV; j += 32) {
-            const float vj = IO<T>::ld(v + (size_t)unit * DV + j);
-            s_v[j] = cv.W[2] ? conv_swish<T>(vj, cv.W[2], cv.w[2], cv.state_in[2], cv.state_out[2], seq, H * DV,
-                                             hc * DV + j)
-                             : vj;
-        }
+      } else if (warp == 2) {
+        for (int j = lane; j < DV; j += 32) s_v[j] = IO<T>::ld(v + (size_t)unit * DV + j);
         if (lane == 0) s_misc[0] = beta[unit];
+      }
     }
     __syncthreads();
 
@@ -201,9 +276,14 @@ cudaError_t launch(const void *q, const void *k, const void *v, const float *la,
                    float *S, int N, int H, int l2norm, int la_scalar, float eps, const void *og_gate,
                    const float *og_w, float og_eps, const DecodeConv &cv, void *o, cudaStream_t st) {
     const unsigned units = (unsigned)N * (unsigned)H;
-    decode_kernel<DK, DV, T><<<units, kDecodeThreads, 0, st>>>(
-        (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps,
-        (const T *)og_gate, og_w, og_eps, cv, H);
+    if (cv.W[0] | cv.W[1] | cv.W[2])
+        decode_kernel<DK, DV, T, true><<<units, kDecodeThreads, 0, st>>>(
+            (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps,
+            (const T *)og_gate, og_w, og_eps, cv, H);
+    else
+        decode_kernel<DK, DV, T, false><<<units, kDecodeThreads, 0, st>>>(
+            (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps,
+            (const T *)og_gate, og_w, og_eps, cv, H);
     return cudaGetLastError();
 }
 

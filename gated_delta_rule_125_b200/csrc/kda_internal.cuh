@@ -90,6 +90,7 @@ struct ShortConvArgs {
 cudaError_t short_conv_swish(const ShortConvArgs &a, bool bf16, cudaStream_t st);
 int short_conv_launches(int W, bool state_out, int64_t total);
 
+constexpr int kDecodeMaxConvWidth = 4;  // widest window the decode step fuses
 // The same convolution fused into a decode step's loads of q, k, v (index 0, 1, 2):
 // W[i] == 0 leaves that input as it is. States are [N][W-1][H * d].
 struct DecodeConv {

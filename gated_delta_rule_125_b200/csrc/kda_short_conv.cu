@@ -8,10 +8,13 @@
 // inputs, oldest first) or zero.
 //
 // HBM-bound streaming: a thread owns 8 consecutive channels (one 16-byte bf16
-// vector) of kTile consecutive tokens and slides a W-deep register window down
-// them, so each input is read from HBM once (the W-1 halo rows of a tile are
-// the previous tile's last rows, L2 hits). Consecutive threads take consecutive
-// channel vectors of the same tokens: every warp access is a coalesced sweep.
+// vector) of kTile consecutive tokens. A tile inside one sequence issues all
+// its kTile + W - 1 row loads before the first use (kept as loaded, unpacked
+// into a sliding W-deep window as they are used); each input is read from HBM
+// once (the W-1 halo rows are the previous tile's last rows, L2 hits). A tile
+// that meets a sequence boundary takes the token-by-token path. Consecutive
+// threads take consecutive channel vectors of the same tokens: every warp
+// access is a coalesced sweep.
 // A second launch writes each sequence's last W-1 inputs (the state a decode
 // step continues from); one thread per (sequence, channel vector) reads all it
 // needs before it writes, so the output state may alias the input state.
@@ -21,10 +24,20 @@ namespace kda {
 namespace {
 
 constexpr int kConvThreads = 256;
-constexpr int kTile = 32;  // tokens per thread
+constexpr int kTile = 8;  // tokens per thread
 
 template <typename T> struct Vec8;
 template <> struct Vec8<__nv_bfloat16> {
+    using Raw = uint4;  // 8 channels as loaded
+    static __device__ __forceinline__ Raw ldraw(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint4 *>(p); }
+    static __device__ __forceinline__ void unpack(const Raw &u, float (&x)[8]) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
     static __device__ __forceinline__ void ld(const __nv_bfloat16 *p, float (&x)[8]) {
         const uint4 u = *reinterpret_cast<const uint4 *>(p);
         const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -45,6 +58,16 @@ template <> struct Vec8<__nv_bfloat16> {
     }
 };
 template <> struct Vec8<float> {
+    struct Raw {
+        float4 a, b;
+    };
+    static __device__ __forceinline__ Raw ldraw(const float *p) {
+        return Raw{reinterpret_cast<const float4 *>(p)[0], reinterpret_cast<const float4 *>(p)[1]};
+    }
+    static __device__ __forceinline__ void unpack(const Raw &r, float (&x)[8]) {
+        x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
+        x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
+    }
     static __device__ __forceinline__ void ld(const float *p, float (&x)[8]) {
         const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
@@ -101,6 +124,33 @@ conv_kernel(const T *__restrict__ x, T *__restrict__ y, const float *__restrict_
 
     int s = cu ? seq_of(cu, N, t0) : 0;
     int64_t bos = cu ? cu[s] : 0, eos = cu ? cu[s + 1] : total;
+    if (t0 - bos >= W - 1 && t0 + kTile <= eos) {
+        // the whole window of the tile lies in one sequence: every row load first
+        typename Vec8<T>::Raw raw[kTile + W - 1];
+#pragma unroll
+        for (int r = 0; r < kTile + W - 1; ++r) raw[r] = Vec8<T>::ldraw(x + (size_t)(t0 - (W - 1) + r) * C + c0);
+        float win[W][8];
+#pragma unroll
+        for (int j = 0; j < W - 1; ++j) Vec8<T>::unpack(raw[j], win[j]);
+#pragma unroll
+        for (int r = 0; r < kTile; ++r) {
+            Vec8<T>::unpack(raw[r + W - 1], win[W - 1]);
+            float out[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                float z = 0.f;
+#pragma unroll
+                for (int j = 0; j < W; ++j) z = fmaf(wt[i][j], win[j][i], z);
+                out[i] = __fdividef(z, 1.f + __expf(-z));
+            }
+            Vec8<T>::st(y + (size_t)(t0 + r) * C + c0, out);
+#pragma unroll
+            for (int j = 0; j < W - 1; ++j)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) win[j][i] = win[j + 1][i];
+        }
+        return;
+    }
     float win[W][8];  // win[W-1] is the current token, win[0] the oldest
     auto fill = [&](int64_t t) {  // window positions t-W+1 .. t-1 of t's sequence
 #pragma unroll
@@ -123,7 +173,7 @@ conv_kernel(const T *__restrict__ x, T *__restrict__ y, const float *__restrict_
             float z = 0.f;
 #pragma unroll
             for (int j = 0; j < W; ++j) z = fmaf(wt[i][j], win[j][i], z);
-            out[i] = z / (1.f + __expf(-z));
+            out[i] = __fdividef(z, 1.f + __expf(-z));
         }
         Vec8<T>::st(y + (size_t)t * C + c0, out);
 #pragma unroll

@@ -272,8 +272,11 @@ int64_t kda_short_conv_launches(int32_t width, int32_t writes_state, int64_t tot
  * q, k and v: here q, k, v are the step's raw projections ([N][H][d]) and
  * conv_q, conv_k, conv_v (each NULL: that input is used as it is) carry
  * C = H * d channels with states [N][W-1][H * d] (normally state_in ==
- * state_out: updated in place, one token per call).
+ * state_out: updated in place, one token per call). Windows up to
+ * KDA_DECODE_MAX_CONV_WIDTH (KDA_ERR_UNSUPPORTED beyond: run
+ * kda_short_conv_swish on the step's tokens and kda_decode_step_ex instead).
  */
+#define KDA_DECODE_MAX_CONV_WIDTH 4
 kda_status kda_decode_step_conv(const void *q, const void *k, const void *v, const float *log_alpha,
                                 const float *beta, float *S, int32_t N, int32_t H, int32_t dk,
                                 int32_t dv, kda_dtype dtype, uint32_t flags,

@@ -532,6 +532,11 @@ def test_short_conv_rejects_bad_arguments():
         kda.kda_short_conv_swish(x, torch.zeros((64, 9), device=DEV))  # width 9 > KDA_MAX_CONV_WIDTH
     with pytest.raises(kda.KDAError):
         kda.kda_short_conv_swish(x, w, y=x)  # y overlaps x
+    wl = KI.decode_workload(2, 1, 128, 1, torch.bfloat16, DEV, seed=22, s0_std=0.1)
+    w5 = torch.zeros((128, 5), device=DEV)  # the fused decode step takes windows up to 4
+    with pytest.raises(kda.KDAError):
+        kda.kda_decode_step(wl["q"][0], wl["k"][0], wl["v"][0], wl["log_alpha"][0], wl["beta"][0],
+                            wl["S0"].clone(), conv=((w5, None, None), None, None))
     lib = kda.load_library()
     assert lib.kda_short_conv_launches(4, 1, 16) == 2 and lib.kda_short_conv_launches(1, 1, 16) == 1
     assert lib.kda_short_conv_launches(4, 0, 0) == 0 and lib.kda_short_conv_launches(0, 0, 16) == -1
