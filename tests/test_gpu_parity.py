@@ -479,8 +479,9 @@ def test_output_gate_workload_prefill_8k():
 # ------------------------------------- short convolution + Swish (§6.1) ----
 # The convolution's output is one fp32 dot product of W taps then Swish, stored
 # in the io dtype: it must lie within the io dtype's rounding of the fp64 value
-# (bf16: 2^-8 relative; fp32: 1e-5 relative, fast exponential). States are raw
-# input copies: bit-exact.
+# (bf16 round-to-nearest: 2^-8 relative, the unit roundoff of an 8-bit
+# significand, plus 1 % of it for the fp32 arithmetic before the rounding; fp32:
+# 1e-5 relative, fast exponential). States are raw input copies: bit-exact.
 
 def _conv_ref(x, w, cu=None, st=None):
     return oracle.short_conv_swish(host(x).reshape(x.shape[0], -1), host(w),
@@ -488,7 +489,7 @@ def _conv_ref(x, w, cu=None, st=None):
 
 
 def _conv_close(y, y_ref, dtype, label):
-    rel = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-5
+    rel = 1.01 * 2.0 ** -8 if dtype == torch.bfloat16 else 1e-5
     err = np.abs(host(y).reshape(y_ref.shape) - y_ref)
     bound = rel * np.abs(y_ref) + 1e-6
     assert np.isfinite(err).all(), label
