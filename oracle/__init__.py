@@ -18,6 +18,11 @@ Functions and the passages they follow (pages cited by title and section):
 * :func:`output_gate` -- the layer's output step after the recurrence, §6 and
   §6.3 (and "Kimi Linear — 逐通道的遺忘", 其他零件): head-wise RMSNorm of o_t,
   then a product with a sigmoid gate computed from the input.
+* :func:`backward` -- gradients of the recurrence's outputs (o and the final
+  state) with respect to every input, derived here by reverse-mode
+  differentiation of the §3 three-step form token by token (the pages mention
+  training but give no backward); pinned to central finite differences of
+  :func:`recurrent` and to torch autograd.
 * :func:`short_conv_swish` / :func:`short_conv_step` -- the layer's step before
   the recurrence, §6 and §6.1 (and "Kimi Delta Attention：把遗忘门做到每个通道",
   进状态之前 q/k 还要过一道预处理): a causal short convolution over the token
@@ -220,3 +225,85 @@ def short_conv_step(x, w, state):
     window = np.concatenate([state, x[:, None, :]], axis=1)  # [N, W, C], newest last
     z = np.einsum("cj,njc->nc", w, window)
     return _silu(z), window[:, 1:, :].copy()
+
+
+def _l2_back(x, dxh, eps):
+    """Gradient through xh = x / max(||x||, eps), per row of x [..., d]."""
+    n = np.linalg.norm(x, axis=-1, keepdims=True)
+    big = n > eps
+    xh = x / np.where(big, n, 1.0)
+    proj = np.sum(xh * dxh, axis=-1, keepdims=True)
+    return np.where(big, (dxh - xh * proj) / np.where(big, n, 1.0), dxh / eps)
+
+
+def backward(q, k, v, log_alpha, beta, do, dS_T=None, S0=None, cu_seqlens=None, l2norm=True,
+             eps=1e-6):
+    """Gradients of a loss L through the recurrence of :func:`recurrent`, given
+    ``do = dL/do [T,H,dv]`` and ``dS_T = dL/dS_T [N,H,dk,dv]`` (None: zero).
+
+    Per token, with q, k normalised (q^, k^) and a = exp(log_alpha_t):
+    forward ``S~ = Diag(a) S_{t-1}``, ``u = beta (v - S~^T k^)``, ``S_t = S~ + k^ u^T``,
+    ``o_t = S_t^T q^``; backward, from t = T down to 1 with G = dL/dS_t:
+    ``G += q^ do_t^T``, ``dq^ = S_t do_t``, ``du = G^T k^``, ``dk^ = G u - beta S~ du``,
+    ``dv = beta du``, ``dbeta = du . (v - S~^T k^)``, ``dS~ = G - beta k^ du^T``,
+    ``dlog_alpha = a * rowsum(dS~ * S_{t-1})``, ``G <- Diag(a) dS~`` (dL/dS_{t-1});
+    then through the normalisation. log_alpha [T,H] (one gate per head) gets the
+    sum over the key channels. Returns ``(dq, dk, dv, dlog_alpha, dbeta, dS0)``.
+    fp64 numpy, loops over sequences, heads and tokens (small cases).
+    """
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    la = np.asarray(log_alpha, dtype=np.float64)
+    b = np.asarray(beta, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    scalar = la.ndim == 2
+    cu = np.array([0, T]) if cu_seqlens is None else np.asarray(cu_seqlens, dtype=np.int64)
+    N = len(cu) - 1
+    S0 = np.zeros((N, H, dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float64)
+    dST = np.zeros((N, H, dk, dv)) if dS_T is None else np.asarray(dS_T, dtype=np.float64)
+    if l2norm:
+        nq = np.maximum(np.linalg.norm(q, axis=-1, keepdims=True), eps)
+        nk = np.maximum(np.linalg.norm(k, axis=-1, keepdims=True), eps)
+        qh, kh = q / nq, k / nk
+    else:
+        qh, kh = q, k
+    dqh, dkh = np.zeros_like(q), np.zeros_like(k)
+    gv, gla, gb = np.zeros_like(v), np.zeros_like(la), np.zeros_like(b)
+    dS0 = np.zeros((N, H, dk, dv))
+    for s in range(N):
+        bos, eos = int(cu[s]), int(cu[s + 1])
+        for h in range(H):
+            alpha = lambda t: np.exp(np.full(dk, la[t, h]) if scalar else la[t, h])
+            states = [S0[s, h].copy()]  # S_{t-1} of every token, then the last S_t
+            for t in range(bos, eos):
+                St = alpha(t)[:, None] * states[-1]
+                u = b[t, h] * (v[t, h] - St.T @ kh[t, h])
+                states.append(St + np.outer(kh[t, h], u))
+            G = dST[s, h].copy()
+            for i in range(eos - bos - 1, -1, -1):
+                t = bos + i
+                a = alpha(t)
+                Sp, Sn = states[i], states[i + 1]
+                St = a[:, None] * Sp
+                r = v[t, h] - St.T @ kh[t, h]
+                u = b[t, h] * r
+                G += np.outer(qh[t, h], do[t, h])
+                dqh[t, h] = Sn @ do[t, h]
+                du = G.T @ kh[t, h]
+                dkh[t, h] = G @ u - b[t, h] * (St @ du)
+                gv[t, h] = b[t, h] * du
+                gb[t, h] = du @ r
+                dSt = G - b[t, h] * np.outer(kh[t, h], du)
+                g = a * np.sum(dSt * Sp, axis=1)
+                if scalar:
+                    gla[t, h] = g.sum()
+                else:
+                    gla[t, h] = g
+                G = a[:, None] * dSt
+            dS0[s, h] = G
+    if l2norm:
+        gq, gk = _l2_back(q, dqh, eps), _l2_back(k, dkh, eps)
+    else:
+        gq, gk = dqh, dkh
+    return gq, gk, gv, gla, gb, dS0

@@ -581,3 +581,126 @@ def test_short_conv_pins_catch_planted_mistakes(kind):
         except (AssertionError, ValueError, IndexError):
             failed += 1
     assert failed > 0, kind
+
+
+# ------------------------------------------- backward (training, §5) ----
+# oracle.backward: gradients of L = <do, o> + <dS_T, S_T> through the recurrence,
+# derived by hand (the pages give no backward). Pinned to central finite
+# differences of oracle.recurrent (itself pinned above) and to torch autograd of
+# a separately written forward; each planted mistake below must fail the
+# finite-difference pin.
+
+def _bw_case(seed, scalar_gate=False):
+    rng = np.random.default_rng(seed)
+    T, H, dk, dv = 7, 2, 3, 2
+    cu = np.array([0, 4, 4, 7])  # an empty sequence in the middle
+    q, k = rng.normal(size=(T, H, dk)), rng.normal(size=(T, H, dk))
+    v = rng.normal(size=(T, H, dv))
+    la = -np.abs(rng.normal(size=(T, H) if scalar_gate else (T, H, dk))) * 0.4
+    b = 1.0 / (1.0 + np.exp(-rng.normal(size=(T, H))))
+    S0 = rng.normal(size=(3, H, dk, dv))
+    Wo, WS = rng.normal(size=(T, H, dv)), rng.normal(size=(3, H, dk, dv))
+    return dict(q=q, k=k, v=v, la=la, b=b, S0=S0, cu=cu, Wo=Wo, WS=WS)
+
+
+def _bw_fd(c, l2norm=True):
+    """Central finite differences of L through oracle.recurrent, for every input."""
+    names = ["q", "k", "v", "la", "b", "S0"]
+
+    def loss(vals):
+        la = vals["la"]
+        if la.ndim == 2:  # one gate per (token, head): the same gate on every key channel
+            la = np.repeat(la[..., None], c["q"].shape[2], axis=-1)
+        o, ST = oracle.recurrent(vals["q"], vals["k"], vals["v"], la, vals["b"], vals["S0"],
+                                 c["cu"], l2norm=l2norm, threads=1)
+        return float((o * c["Wo"]).sum() + (ST * c["WS"]).sum())
+
+    out = []
+    h = 1e-6
+    for n in names:
+        x = c[n]
+        g = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            vals = {m: c[m] for m in names}
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            vals[n] = xp
+            lp = loss(vals)
+            vals[n] = xm
+            g[idx] = (lp - loss(vals)) / (2 * h)
+        out.append(g)
+    return out
+
+
+def _bw_run(f, c, l2norm=True):
+    return f(c["q"], c["k"], c["v"], c["la"], c["b"], c["Wo"], c["WS"], c["S0"], c["cu"], l2norm=l2norm)
+
+
+@pytest.mark.parametrize("scalar_gate,l2norm", [(False, True), (True, True), (False, False)])
+def test_backward_matches_finite_differences(scalar_gate, l2norm):
+    c = _bw_case(31 + scalar_gate, scalar_gate)
+    fd = _bw_fd(c, l2norm)
+    for name, g, want in zip(["q", "k", "v", "log_alpha", "beta", "S0"], _bw_run(oracle.backward, c, l2norm), fd):
+        np.testing.assert_allclose(g, want, rtol=0, atol=2e-7 * max(1.0, np.abs(want).max()), err_msg=name)
+
+
+def test_backward_matches_torch_autograd():
+    c = _bw_case(35)
+    t = {n: torch.tensor(c[n], dtype=torch.float64, requires_grad=True) for n in ["q", "k", "v", "la", "b", "S0"]}
+    loss = torch.zeros((), dtype=torch.float64)
+    for s in range(len(c["cu"]) - 1):
+        for h in range(c["q"].shape[1]):
+            S = t["S0"][s, h]
+            for i in range(int(c["cu"][s]), int(c["cu"][s + 1])):
+                qh = t["q"][i, h] / t["q"][i, h].norm()
+                kh = t["k"][i, h] / t["k"][i, h].norm()
+                Sd = torch.exp(t["la"][i, h])[:, None] * S
+                u = t["b"][i, h] * (t["v"][i, h] - Sd.T @ kh)
+                S = Sd + torch.outer(kh, u)
+                loss = loss + (S.T @ qh) @ torch.tensor(c["Wo"][i, h])
+            loss = loss + (S * torch.tensor(c["WS"][s, h])).sum()
+    loss.backward()
+    for name, g in zip(["q", "k", "v", "la", "b", "S0"], _bw_run(oracle.backward, c)):
+        np.testing.assert_allclose(g, t[name].grad.numpy(), rtol=1e-11, atol=1e-12, err_msg=name)
+
+
+def test_backward_beta_zero_closed_form():
+    # beta = 0: no write, so dL/dv = 0 and, without a normalisation, dL/dq_t = S_t do_t
+    # with S_t = Diag(exp(sum of log_alpha)) S0 (the pure decay closed form)
+    c = _bw_case(36)
+    c["b"] = np.zeros_like(c["b"])
+    gq, gk, gv, gla, gb, gS0 = _bw_run(oracle.backward, c, l2norm=False)
+    assert np.all(gv == 0.0)
+    s, h, t = 2, 1, 5  # token 5 of sequence 2 (tokens 4..6)
+    St = np.exp(c["la"][4:t + 1, h].sum(axis=0))[:, None] * c["S0"][s, h]
+    np.testing.assert_allclose(gq[t, h], St @ c["Wo"][t, h], rtol=1e-13)
+
+
+_BW_MUTANTS = {
+    "decay_not_propagated": ("G = a[:, None] * dSt", "G = dSt"),
+    "write_sign": ("dSt = G - b[t, h] * np.outer(kh[t, h], du)", "dSt = G + b[t, h] * np.outer(kh[t, h], du)"),
+    "dk_read_term_dropped": ("dkh[t, h] = G @ u - b[t, h] * (St @ du)", "dkh[t, h] = G @ u"),
+    "gate_uses_new_state": ("g = a * np.sum(dSt * Sp, axis=1)", "g = a * np.sum(dSt * Sn, axis=1)"),
+    "dbeta_wrong_factor": ("gb[t, h] = du @ r", "gb[t, h] = du @ u"),
+    "readout_before_update": ("dqh[t, h] = Sn @ do[t, h]", "dqh[t, h] = Sp @ do[t, h]"),
+    "no_norm_backward": ("gq, gk = _l2_back(q, dqh, eps), _l2_back(k, dkh, eps)", "gq, gk = dqh / nq, dkh / nk"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(_BW_MUTANTS))
+def test_backward_pins_catch_planted_mistakes(name):
+    import inspect
+    import textwrap
+    src = textwrap.dedent(inspect.getsource(oracle.backward))
+    old, new = _BW_MUTANTS[name]
+    assert src.count(old) == 1, name
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    c = _bw_case(37)
+    fd = _bw_fd(c)
+    bad = False
+    for g, want in zip(_bw_run(ns["backward"], c), fd):
+        if not np.allclose(g, want, rtol=0, atol=2e-7 * max(1.0, np.abs(want).max())):
+            bad = True
+    assert bad, "planted mistake %r passed the finite-difference pin" % name
