@@ -23,6 +23,9 @@ Functions and the passages they follow (pages cited by title and section):
   differentiation of the §3 three-step form token by token (the pages mention
   training but give no backward); pinned to central finite differences of
   :func:`recurrent` and to torch autograd.
+* :func:`chunkwise_backward` -- the same gradients through the chunkwise form
+  of §5 (a second CPU form: the algebra a chunked GPU backward implements),
+  pinned to :func:`backward`.
 * :func:`short_conv_swish` / :func:`short_conv_step` -- the layer's step before
   the recurrence, §6 and §6.1 (and "Kimi Delta Attention：把遗忘门做到每个通道",
   进状态之前 q/k 还要过一道预处理): a causal short convolution over the token
@@ -302,6 +305,111 @@ def backward(q, k, v, log_alpha, beta, do, dS_T=None, S0=None, cu_seqlens=None, 
                     gla[t, h] = g
                 G = a[:, None] * dSt
             dS0[s, h] = G
+    if l2norm:
+        gq, gk = _l2_back(q, dqh, eps), _l2_back(k, dkh, eps)
+    else:
+        gq, gk = dqh, dkh
+    return gq, gk, gv, gla, gb, dS0
+
+
+def chunkwise_backward(q, k, v, log_alpha, beta, do, dS_T=None, S0=None, cu_seqlens=None, chunk=64,
+                       l2norm=True, eps=1e-6):
+    """:func:`backward` through the chunkwise form. Per chunk (rows r, entry state S,
+    G the inclusive cumsum of log_alpha, g its last row; Qg = Q e^G, Kg = K e^G,
+    Kn = K e^-G, Kd = K e^(g-G); A = strict_lower(Kg Kn^T), P = lower(Qg Kn^T);
+    X = (I + Diag(beta) A)^-1, T = X Diag(beta), W = T Kg, U = T V - W S;
+    O = Qg S + P U, S' = Diag(e^g) S + Kd^T U), the reverse sweep over chunks,
+    given dO and dS':
+
+        dS  = Diag(e^g) dS' + Qg^T dO - W^T dU,   dU = Kd dS' + P^T dO
+        dKd = U dS'^T,  dP = lower(dO U^T),  dQg = dO S^T,  dW = -dU S^T
+        dT  = dU V^T + dW Kg^T,  dV = T^T dU,  dKg = T^T dW
+        dX  = dT Diag(beta),  dM = -X^T dX X^T,  dA = strict_lower(Diag(beta) dM)
+        dbeta_i = sum_r dT_ri X_ri + sum_i' dM_ii' A_ii'
+        A, P: dKg += dA Kn,  dKn = dA^T Kg + dP^T Qg,  dQg += dP Kn
+        exponents: dG = dQg Qg + dKg Kg - dKn Kn - dKd Kd (element-wise),
+                   dg = colsum(dKd Kd) + e^g rowsum(dS' S)
+        dlog_alpha_r = sum_{r' >= r} dG_r' + dg
+
+    then through the normalisation of q, k. Entry states come from a forward pass
+    over the chunks. Returns what :func:`backward` returns (KDA gates only).
+    """
+    q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    la = np.asarray(log_alpha, dtype=np.float64)
+    b = np.asarray(beta, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.array([0, T]) if cu_seqlens is None else np.asarray(cu_seqlens, dtype=np.int64)
+    N = len(cu) - 1
+    S0 = np.zeros((N, H, dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float64)
+    dST = np.zeros((N, H, dk, dv)) if dS_T is None else np.asarray(dS_T, dtype=np.float64)
+    if l2norm:
+        nq = np.maximum(np.linalg.norm(q, axis=-1, keepdims=True), eps)
+        nk = np.maximum(np.linalg.norm(k, axis=-1, keepdims=True), eps)
+        qh, kh = q / nq, k / nk
+    else:
+        qh, kh = q, k
+    dqh, dkh = np.zeros_like(q), np.zeros_like(k)
+    gv, gla, gb = np.zeros_like(v), np.zeros_like(la), np.zeros_like(b)
+    dS0 = np.zeros((N, H, dk, dv))
+
+    def chunk_terms(rows, h):
+        Q, K, V = qh[rows, h], kh[rows, h], v[rows, h]
+        G = np.cumsum(la[rows, h], axis=0)
+        g = G[-1]
+        Qg, Kg, Kn, Kd = Q * np.exp(G), K * np.exp(G), K * np.exp(-G), K * np.exp(g - G)
+        n = len(rows)
+        A = np.tril(Kg @ Kn.T, -1)
+        P = np.tril(Qg @ Kn.T)
+        bt = b[rows, h]
+        X = np.linalg.inv(np.eye(n) + bt[:, None] * A)
+        Tm = X * bt[None, :]
+        return dict(V=V, G=G, g=g, Qg=Qg, Kg=Kg, Kn=Kn, Kd=Kd, A=A, P=P, bt=bt, X=X, T=Tm, W=Tm @ Kg)
+
+    for s in range(N):
+        bos, eos = int(cu[s]), int(cu[s + 1])
+        starts = list(range(bos, eos, chunk))
+        for h in range(H):
+            entry = [S0[s, h].copy()]
+            for c0 in starts:
+                rows = np.arange(c0, min(c0 + chunk, eos))
+                m = chunk_terms(rows, h)
+                S = entry[-1]
+                U = m["T"] @ m["V"] - m["W"] @ S
+                entry.append(np.exp(m["g"])[:, None] * S + m["Kd"].T @ U)
+            dSn = dST[s, h].copy()  # dL/dS' of the current chunk
+            for ci in range(len(starts) - 1, -1, -1):
+                c0 = starts[ci]
+                rows = np.arange(c0, min(c0 + chunk, eos))
+                m = chunk_terms(rows, h)
+                S = entry[ci]
+                U = m["T"] @ m["V"] - m["W"] @ S
+                dO = do[rows, h]
+                eg = np.exp(m["g"])
+                dU = m["Kd"] @ dSn + m["P"].T @ dO
+                dKd = U @ dSn.T
+                dP = np.tril(dO @ U.T)
+                dQg = dO @ S.T
+                dW = -dU @ S.T
+                dS = eg[:, None] * dSn + m["Qg"].T @ dO - m["W"].T @ dU
+                dT = np.tril(dU @ m["V"].T + dW @ m["Kg"].T)
+                gv[rows, h] = m["T"].T @ dU
+                dKg = m["T"].T @ dW
+                dX = dT * m["bt"][None, :]
+                dM = -m["X"].T @ dX @ m["X"].T
+                dA = np.tril(m["bt"][:, None] * dM, -1)
+                gb[rows, h] = np.sum(dT * m["X"], axis=0) + np.sum(dM * m["A"], axis=1)
+                dKg = dKg + dA @ m["Kn"]
+                dKn = dA.T @ m["Kg"] + dP.T @ m["Qg"]
+                dQg = dQg + dP @ m["Kn"]
+                dG = dQg * m["Qg"] + dKg * m["Kg"] - dKn * m["Kn"] - dKd * m["Kd"]
+                dg = np.sum(dKd * m["Kd"], axis=0) + eg * np.sum(dSn * S, axis=1)
+                gla[rows, h] = np.cumsum(dG[::-1], axis=0)[::-1] + dg[None, :]
+                dqh[rows, h] = dQg * np.exp(m["G"])
+                dkh[rows, h] = dKg * np.exp(m["G"]) + dKn * np.exp(-m["G"]) + dKd * np.exp(m["g"] - m["G"])
+                dSn = dS
+            dS0[s, h] = dSn
     if l2norm:
         gq, gk = _l2_back(q, dqh, eps), _l2_back(k, dkh, eps)
     else:

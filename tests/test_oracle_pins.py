@@ -704,3 +704,22 @@ def test_backward_pins_catch_planted_mistakes(name):
         if not np.allclose(g, want, rtol=0, atol=2e-7 * max(1.0, np.abs(want).max())):
             bad = True
     assert bad, "planted mistake %r passed the finite-difference pin" % name
+
+
+@pytest.mark.parametrize("chunk", [1, 16, 64])
+def test_chunkwise_backward_equals_token_backward(chunk):
+    # the chunked algebra (partial last chunks, an empty sequence) gives the token
+    # form's gradients to rounding
+    rng = np.random.default_rng(38)
+    T, H, dk, dv = 150, 2, 8, 6
+    cu = np.array([0, 70, 70, 150])
+    q, k = rng.normal(size=(T, H, dk)), rng.normal(size=(T, H, dk))
+    v = rng.normal(size=(T, H, dv))
+    la = -np.log1p(np.exp(rng.normal(-3.0, 1.0, size=(T, H, dk))))
+    b = 1.0 / (1.0 + np.exp(-rng.normal(size=(T, H))))
+    S0, dST = rng.normal(size=(3, H, dk, dv)), rng.normal(size=(3, H, dk, dv))
+    do = rng.normal(size=(T, H, dv))
+    want = oracle.backward(q, k, v, la, b, do, dST, S0, cu)
+    got = oracle.chunkwise_backward(q, k, v, la, b, do, dST, S0, cu, chunk=chunk)
+    for name, g, w in zip(["q", "k", "v", "log_alpha", "beta", "S0"], got, want):
+        np.testing.assert_allclose(g, w, rtol=0, atol=1e-12 * max(1.0, np.abs(w).max()), err_msg=name)
