@@ -48,6 +48,9 @@ GDN_BYTES_PER_TOKEN = 3 * H * D * 2 + H * 4 + H * 4 + H * D * 2
 # decode per step: state read + write, q,k,v bf16, log_alpha fp32, beta fp32, o bf16
 DECODE_BYTES = DEC_N * H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2)
 CONV_W = 4  # short-convolution window of the conv lines (the pages leave it open)
+# backward of prefill_8k: q, k, v, do (bf16), log_alpha, beta read; dq, dk, dv, dlog_alpha,
+# dbeta (fp32) written; S0 and dS_T read, dS0 written
+BACKWARD_BYTES = T8K * H * (4 * D * 2 + D * 4 + 4 + 4 * D * 4 + 4) + 3 * H * D * D * 4
 # one short convolution over a [T8K, H*D] bf16 projection: x read, y written, taps,
 # the state read and written
 CONV_BYTES = 2 * T8K * H * D * 2 + H * D * CONV_W * 4 + 2 * (CONV_W - 1) * H * D * 2
@@ -421,6 +424,34 @@ def run_kda(args, world, rank, local):
     dconv_us = ev0.elapsed_time(ev1) * 1e3 / dsteps
     dconv_us_max = max_over_ranks(dconv_us, world, dev)
     dconv_gbs = DECODE_CONV_BYTES / (dconv_us * 1e-6) / 1e9
+    del dec, dconv
+
+    # ---- backward of the prefill (training): gradients of prefill_8k given dL/do, dL/dS_T
+    bw = {}
+    bw_steps = 3
+    g_bw = torch.Generator(device=dev)
+    g_bw.manual_seed(2000 + rank)
+    d_o = torch.randn((T8K, H, D), generator=g_bw, device=dev).to(torch.bfloat16)
+    d_ST = torch.randn((1, H, D, D), generator=g_bw, device=dev)
+    bw_wsb = kda.load_library().kda_backward_workspace_size(1, T8K, T8K, H, D, D, 1, 64, 0)
+    bw_ws = torch.empty(bw_wsb, dtype=torch.uint8, device=dev)
+
+    def backward():
+        kda.kda_backward(q, k, v, la, beta, d_o, d_ST, S0, cu, max_seqlen=T8K, workspace=bw_ws)
+
+    for _ in range(max(3, args.warmup)):
+        backward()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record(stream)
+    for _ in range(bw_steps):
+        backward()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    bw_ms = ev0.elapsed_time(ev1) / bw_steps
+    bw["ms"] = max_over_ranks(bw_ms, world, dev)
+    bw["gbs"] = BACKWARD_BYTES / (bw_ms * 1e-3) / 1e9
+    del bw_ws, d_o, d_ST
 
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
@@ -440,7 +471,7 @@ def run_kda(args, world, rank, local):
         "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": (3 * args.steps * launches_prefill + dsteps + args.steps * 3 * conv_launches
-                         + args.steps * (3 * conv_launches + launches_prefill) + dsteps),
+                         + args.steps * (3 * conv_launches + launches_prefill) + dsteps + 5 * bw_steps),
         "clocks": clk.summary(),
         "gdn": {"value": world * T8K / (gdn_ms * 1e-3), "unit": "tokens/s", "ms_per_step": gdn_ms,
                 "workload": "gdn_8k: prefill_8k with one forget gate per (token, head) "
@@ -475,6 +506,14 @@ def run_kda(args, world, rank, local):
                                     "frac": conv_gbs / hbm, "traffic": None,
                                     "kernel": "conv_kernel<4,bf16> + conv_state_kernel (x3)",
                                     "algorithmic_bytes": 3 * CONV_BYTES, "peak_source": peak_src}},
+        "backward": {"value": world * T8K / (bw["ms"] * 1e-3), "unit": "tokens/s", "ms_per_step": bw["ms"],
+                     "steps": bw_steps,
+                     "workload": "gradients of prefill_8k w.r.t. q, k, v, log_alpha, beta, S0 given dL/do "
+                                 "(bf16) and dL/dS_T (fp32); fp32 CUDA-core reference-grade kernels",
+                     "roofline": {"bound": "hbm", "achieved": bw["gbs"], "peak": hbm, "unit": "GB/s",
+                                  "frac": bw["gbs"] / hbm, "traffic": None,
+                                  "kernel": "bw_prep + bw_fwd + bw_bwd + bw_grads + bw_norm",
+                                  "algorithmic_bytes": BACKWARD_BYTES, "peak_source": peak_src}},
         "decode_conv": {"value": DECODE_CONV_BYTES / (dconv_us_max * 1e-6) / 1e9, "unit": "GB/s",
                         "us_per_step": dconv_us_max, "steps": dsteps,
                         "workload": "decode_256 with the short convolution (W=%d) + Swish fused into the q, k, v "

@@ -16,7 +16,7 @@ import os
 import torch
 
 __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size", "kda_prefill_launches",
-           "kda_device_error", "kda_prefill_noalloc",
+           "kda_device_error", "kda_prefill_noalloc", "kda_short_conv_swish", "kda_backward",
            "kda_prefill_workspace_min", "kda_status_string", "kda_version", "KDAError",
            "library_path", "load_library", "KDA_OK", "KDA_ERR_INVALID_ARG",
            "KDA_ERR_UNSUPPORTED", "KDA_ERR_MISALIGNED", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA",
@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_s
                     "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
                     "kda_prefill_ex", "kda_decode_step", "kda_decode_step_ex", "kda_device_error",
                     "kda_prefill_noalloc", "kda_short_conv_swish", "kda_short_conv_launches",
-                    "kda_decode_step_conv")
+                    "kda_decode_step_conv", "kda_backward_workspace_size", "kda_backward")
 
 
 class OutputGate(ctypes.Structure):
@@ -104,6 +104,11 @@ def load_library():
     lib.kda_decode_step_conv.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
                                          u32, sc, sc, sc, og, vp, vp]
     lib.kda_decode_step_conv.restype = ctypes.c_int
+    lib.kda_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, ctypes.c_int, i32, u32]
+    lib.kda_backward_workspace_size.restype = sz
+    lib.kda_backward.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32, i32, ctypes.c_int, i32, u32,
+                                 vp, fp, fp, fp, fp, fp, fp, fp, vp, sz, vp]
+    lib.kda_backward.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -304,3 +309,36 @@ def kda_short_conv_swish(x, weight, cu_seqlens=None, *, state_in=None, state_out
     if rc != KDA_OK:
         raise KDAError(rc, "kda_short_conv_swish")
     return y
+
+
+def kda_backward(q, k, v, log_alpha, beta, do, dS_T=None, S0=None, cu_seqlens=None, *, max_seqlen=None,
+                 l2norm=True, workspace=None, want_dS0=True, stream=None):
+    """Backward of the prefill (``kda_backward`` in ``include/kda.h``): the gradients of a
+    loss through ``o`` and ``S_T`` given ``do = dL/do`` ``[T,H,dv]`` (io dtype) and
+    ``dS_T = dL/dS_T`` ``[N,H,dk,dv]`` fp32 (None: zero). Returns fp32
+    ``(dq, dk, dv, dlog_alpha, dbeta, dS0)`` (dS0 None unless ``want_dS0``)."""
+    lib = load_library()
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if max_seqlen is None:
+        max_seqlen = T if cu_seqlens is None else int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item())
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq, dkk = torch.empty((T, H, dk), **f32), torch.empty((T, H, dk), **f32)
+    dvv, dla = torch.empty((T, H, dv), **f32), torch.empty((T, H, dk), **f32)
+    db = torch.empty((T, H), **f32)
+    dS0 = torch.empty((N, H, dk, dv), **f32) if want_dS0 else None
+    flags = _flags(l2norm, False, log_alpha.dim() == 2)
+    code = _dtype_code(q)
+    if workspace is None:
+        nbytes = lib.kda_backward_workspace_size(N, T, max_seqlen, H, dk, dv, code, 64, flags)
+        if nbytes == 0:
+            raise KDAError(KDA_ERR_UNSUPPORTED if log_alpha.dim() == 2 else 1, "kda_backward_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    rc = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                          N, T, max_seqlen, H, dk, dv, code, 64, flags, _ptr(do), _ptr(dS_T),
+                          _ptr(dq), _ptr(dkk), _ptr(dvv), _ptr(dla), _ptr(db), _ptr(dS0),
+                          _ptr(workspace), workspace.numel(), _stream(stream, q.device))
+    if rc != KDA_OK:
+        raise KDAError(rc, "kda_backward")
+    return dq, dkk, dvv, dla, db, dS0

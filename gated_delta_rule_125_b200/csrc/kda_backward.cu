@@ -1,0 +1,469 @@
+// kda_backward.cu -- gradients of the chunkwise prefill (training backward).
+//
+// The pages mention training ("[Kimi-2] Kimi Linear：用 KDA 重写长上下文注意力"
+// §5) but give no backward; this follows the chunked reverse-mode algebra
+// derived for the fp64 oracle's chunkwise backward. Per chunk (rows r, entry
+// state S, G the inclusive cumsum of log_alpha, g its last row; Qg = Q e^G,
+// Kg = K e^G, Kn = K e^-G, Kd = K e^(g-G); A = strict_lower(Kg Kn^T),
+// P = lower(Qg Kn^T); X = (I + Diag(beta) A)^-1, T = X Diag(beta), W = T Kg,
+// U = T V - W S; O = Qg S + P U, S' = Diag(e^g) S + Kd^T U) and given dO, dS':
+//
+//   dS  = Diag(e^g) dS' + Qg^T dO - W^T dU,   dU = Kd dS' + P^T dO
+//   dKd = U dS'^T,  dP = lower(dO U^T),  dQg = dO S^T,  dW = -dU S^T
+//   dT  = lower(dU V^T + dW Kg^T),  dV = T^T dU,  dKg = T^T dW
+//   dX  = dT Diag(beta),  dM = -X^T dX X^T,  dA = strict_lower(Diag(beta) dM)
+//   dbeta_i = sum_r dT_ri X_ri + sum_m dM_im A_im
+//   dKg += dA Kn,  dKn = dA^T Kg + dP^T Qg,  dQg += dP Kn
+//   dG  = dQg Qg + dKg Kg - dKn Kn - dKd Kd,  dg = colsum(dKd Kd) + e^g rowsum(dS' S)
+//   dlog_alpha_r = sum_{r' >= r} dG_r' + dg
+//
+// then through q/max(|q|, eps), k/max(|k|, eps).
+//
+// A reference-grade CUDA-core implementation in fp32, five launches:
+//   1. bw_prep   (one CTA per chunk): normalised q, k; G, Qg, Kg, Kn, Kd, A, P,
+//                the unit-lower-triangular inverse X by column forward
+//                substitution, T, W, T V;
+//   2. bw_fwd    (one CTA per (sequence, head)): the chunks' entry states and U;
+//   3. bw_bwd    (one CTA per (sequence, head)): dU and the state gradient
+//                entering each chunk, in reverse chunk order; dS0;
+//   4. bw_grads  (one CTA per chunk): every per-chunk gradient above;
+//   5. bw_norm   (one warp per (token, head)): through the L2 normalisation.
+// Everything lives in the caller's workspace (fp32); each product is a plain
+// loop over its output elements. The factorised exponents need e^-G finite:
+// a chunk whose decay range exceeds 60 nats sets device error code 2.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int C = kChunk;  // 64
+constexpr int kBwThreads = 256;
+constexpr float kBwRange = 60.f;
+
+// Per-chunk scratch (floats), in this order.
+struct Slot {
+    int dk, dv;
+    __host__ __device__ size_t cd() const { return (size_t)C * dk; }
+    __host__ __device__ size_t cv() const { return (size_t)C * dv; }
+    __host__ __device__ size_t kv() const { return (size_t)dk * dv; }
+    __host__ __device__ size_t floats() const { return 11 * cd() + 9 * (size_t)C * C + 3 * cv() + 2 * kv(); }
+};
+struct SlotPtr {
+    float *G, *Qg, *Kg, *Kn, *Kd, *W;          // C x dk
+    float *dKd, *dQg, *dW, *dKg, *dKn;         // C x dk
+    float *A, *P, *X, *T, *dP, *dT, *dM, *Y, *dA;  // C x C
+    float *TV, *U, *dU;                        // C x dv
+    float *S, *dSn;                            // dk x dv
+    __device__ SlotPtr(float *base, const Slot &s) {
+        float *p = base;
+        G = p; p += s.cd(); Qg = p; p += s.cd(); Kg = p; p += s.cd(); Kn = p; p += s.cd();
+        Kd = p; p += s.cd(); W = p; p += s.cd();
+        dKd = p; p += s.cd(); dQg = p; p += s.cd(); dW = p; p += s.cd(); dKg = p; p += s.cd();
+        dKn = p; p += s.cd();
+        A = p; p += C * C; P = p; p += C * C; X = p; p += C * C; T = p; p += C * C;
+        dP = p; p += C * C; dT = p; p += C * C; dM = p; p += C * C; Y = p; p += C * C; dA = p; p += C * C;
+        TV = p; p += s.cv(); U = p; p += s.cv(); dU = p; p += s.cv();
+        S = p; p += s.kv(); dSn = p;
+    }
+};
+
+struct BwArgs {
+    const void *q, *k, *v, *dout;
+    const float *la, *beta, *S0, *dST;
+    const int32_t *cu;
+    int64_t total;
+    int N, H, dk, dv, NC;  // NC: chunk slots per (sequence, head)
+    int l2norm;
+    float eps;
+    float *dq, *dkk, *dvv, *dla, *dbeta, *dS0;
+    float *slots;          // N * H * NC slots
+    float *qh, *kh, *dqh, *dkh, *nq, *nk;  // per (token, head)
+    int *err;
+};
+
+__device__ __forceinline__ void chunk_rows(const BwArgs &a, int s, int j, int64_t &t0, int &n) {
+    int64_t bos, eos;
+    seq_bounds(a.cu, s, a.total, bos, eos);
+    t0 = bos + (int64_t)j * C;
+    const int64_t rem = eos - t0;
+    n = rem <= 0 ? 0 : (rem < C ? (int)rem : C);
+}
+
+// 1. Per chunk: normalised q, k; G, Qg, Kg, Kn, Kd; A, P; X, T; W = T Kg; T V.
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads) bw_prep(BwArgs a) {
+    const int slot = blockIdx.x, unit = slot / a.NC, j = slot % a.NC;
+    const int s = unit / a.H, h = unit % a.H;
+    int64_t t0;
+    int n;
+    chunk_rows(a, s, j, t0, n);
+    if (n == 0) return;
+    const int dk = a.dk, dv = a.dv, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const Slot sl{dk, dv};
+    SlotPtr m(a.slots + (size_t)slot * sl.floats(), sl);
+    const T *q = static_cast<const T *>(a.q), *k = static_cast<const T *>(a.k), *v = static_cast<const T *>(a.v);
+    // normalised rows (a warp per row)
+    for (int r = warp; r < n; r += kBwThreads / 32) {
+        const size_t row = (size_t)(t0 + r) * a.H + h;
+        float sq = 0.f, sk = 0.f;
+        for (int c = lane; c < dk; c += 32) {
+            const float x = IO<T>::ld(q + row * dk + c), y = IO<T>::ld(k + row * dk + c);
+            sq += x * x;
+            sk += y * y;
+        }
+        for (int off = 16; off; off >>= 1) {
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        }
+        const float nq = a.l2norm ? fmaxf(sqrtf(sq), a.eps) : 1.f, nk = a.l2norm ? fmaxf(sqrtf(sk), a.eps) : 1.f;
+        for (int c = lane; c < dk; c += 32) {
+            a.qh[row * dk + c] = IO<T>::ld(q + row * dk + c) / nq;
+            a.kh[row * dk + c] = IO<T>::ld(k + row * dk + c) / nk;
+        }
+        if (lane == 0) {
+            a.nq[row] = a.l2norm ? sqrtf(sq) : 1.f;
+            a.nk[row] = a.l2norm ? sqrtf(sk) : 1.f;
+        }
+    }
+    __syncthreads();
+    // G (cumsum over the rows), exponent factors
+    for (int c = tid; c < dk; c += kBwThreads) {
+        float run = 0.f;
+        for (int r = 0; r < n; ++r) {
+            run += a.la[(size_t)(t0 + r) * a.H * dk + (size_t)h * dk + c];
+            m.G[r * dk + c] = run;
+        }
+        if (-run > kBwRange && a.err) atomicCAS(a.err, 0, 2);
+    }
+    __syncthreads();
+    for (int e = tid; e < n * dk; e += kBwThreads) {
+        const int r = e / dk, c = e % dk;
+        const size_t row = (size_t)(t0 + r) * a.H + h;
+        const float G = m.G[e], g = m.G[(n - 1) * dk + c];
+        const float qv = a.qh[row * dk + c], kv = a.kh[row * dk + c];
+        m.Qg[e] = qv * expf(G);
+        m.Kg[e] = kv * expf(G);
+        m.Kn[e] = kv * expf(-G);
+        m.Kd[e] = kv * expf(g - G);
+    }
+    __syncthreads();
+    // A = strict_lower(Kg Kn^T), P = lower(Qg Kn^T)
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        const int r = e / C, i = e % C;
+        float sa = 0.f, sp = 0.f;
+        if (r < n && i <= r) {
+            for (int c = 0; c < dk; ++c) {
+                sa += m.Kg[r * dk + c] * m.Kn[i * dk + c];
+                sp += m.Qg[r * dk + c] * m.Kn[i * dk + c];
+            }
+        }
+        m.A[e] = (r < n && i < r) ? sa : 0.f;
+        m.P[e] = (r < n && i <= r) ? sp : 0.f;
+    }
+    __syncthreads();
+    // X = (I + Diag(beta) A)^-1: column i by forward substitution (rows >= i)
+    const float *bt = a.beta;
+    for (int i = tid; i < C; i += kBwThreads) {
+        for (int r = 0; r < C; ++r) {
+            float x = 0.f;
+            if (r < n && i < n && r >= i) {
+                if (r == i) {
+                    x = 1.f;
+                } else {
+                    float acc = 0.f;
+                    for (int mm = i; mm < r; ++mm) acc += m.A[r * C + mm] * m.X[mm * C + i];
+                    x = -bt[(size_t)(t0 + r) * a.H + h] * acc;
+                }
+            }
+            m.X[r * C + i] = x;
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        const int i = e % C;
+        m.T[e] = i < n ? m.X[e] * bt[(size_t)(t0 + i) * a.H + h] : 0.f;
+    }
+    __syncthreads();
+    // W = T Kg, TV = T V
+    for (int e = tid; e < n * dk; e += kBwThreads) {
+        const int r = e / dk, c = e % dk;
+        float acc = 0.f;
+        for (int i = 0; i <= r; ++i) acc += m.T[r * C + i] * m.Kg[i * dk + c];
+        m.W[e] = acc;
+    }
+    for (int e = tid; e < n * dv; e += kBwThreads) {
+        const int r = e / dv, c = e % dv;
+        float acc = 0.f;
+        for (int i = 0; i <= r; ++i) acc += m.T[r * C + i] * IO<T>::ld(v + ((size_t)(t0 + i) * a.H + h) * dv + c);
+        m.TV[e] = acc;
+    }
+}
+
+// 2. Entry states and U, chunk by chunk (the state in shared memory).
+__global__ void __launch_bounds__(kBwThreads) bw_fwd(BwArgs a) {
+    extern __shared__ float sS[];
+    const int unit = blockIdx.x, s = unit / a.H, tid = threadIdx.x;
+    const int dk = a.dk, dv = a.dv;
+    const Slot sl{dk, dv};
+    for (int e = tid; e < dk * dv; e += kBwThreads) sS[e] = a.S0 ? a.S0[(size_t)unit * dk * dv + e] : 0.f;
+    __syncthreads();
+    for (int j = 0; j < a.NC; ++j) {
+        int64_t t0;
+        int n;
+        chunk_rows(a, s, j, t0, n);
+        if (n == 0) break;
+        SlotPtr m(a.slots + ((size_t)unit * a.NC + j) * sl.floats(), sl);
+        for (int e = tid; e < dk * dv; e += kBwThreads) m.S[e] = sS[e];
+        for (int e = tid; e < n * dv; e += kBwThreads) {
+            const int r = e / dv, c = e % dv;
+            float acc = m.TV[e];
+            for (int i = 0; i < dk; ++i) acc -= m.W[r * dk + i] * sS[i * dv + c];
+            m.U[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < dk * dv; e += kBwThreads) {
+            const int i = e / dv, c = e % dv;
+            float acc = expf(m.G[(n - 1) * dk + i]) * sS[e];
+            for (int r = 0; r < n; ++r) acc += m.Kd[r * dk + i] * m.U[r * dv + c];
+            sS[e] = acc;
+        }
+        __syncthreads();
+    }
+}
+
+// 3. State gradient entering each chunk (reverse order), dU; dS0.
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads) bw_bwd(BwArgs a) {
+    extern __shared__ float sG[];
+    const int unit = blockIdx.x, s = unit / a.H, h = unit % a.H, tid = threadIdx.x;
+    const int dk = a.dk, dv = a.dv;
+    const Slot sl{dk, dv};
+    const T *dout = static_cast<const T *>(a.dout);
+    for (int e = tid; e < dk * dv; e += kBwThreads) sG[e] = a.dST ? a.dST[(size_t)unit * dk * dv + e] : 0.f;
+    __syncthreads();
+    for (int j = a.NC - 1; j >= 0; --j) {
+        int64_t t0;
+        int n;
+        chunk_rows(a, s, j, t0, n);
+        if (n == 0) continue;
+        SlotPtr m(a.slots + ((size_t)unit * a.NC + j) * sl.floats(), sl);
+        for (int e = tid; e < dk * dv; e += kBwThreads) m.dSn[e] = sG[e];
+        // dU = Kd dS' + P^T dO
+        for (int e = tid; e < n * dv; e += kBwThreads) {
+            const int r = e / dv, c = e % dv;
+            float acc = 0.f;
+            for (int i = 0; i < dk; ++i) acc += m.Kd[r * dk + i] * sG[i * dv + c];
+            for (int rr = r; rr < n; ++rr) acc += m.P[rr * C + r] * IO<T>::ld(dout + ((size_t)(t0 + rr) * a.H + h) * dv + c);
+            m.dU[e] = acc;
+        }
+        __syncthreads();
+        // dS = Diag(e^g) dS' + Qg^T dO - W^T dU
+        for (int e = tid; e < dk * dv; e += kBwThreads) {
+            const int i = e / dv, c = e % dv;
+            float acc = expf(m.G[(n - 1) * dk + i]) * sG[e];
+            for (int r = 0; r < n; ++r)
+                acc += m.Qg[r * dk + i] * IO<T>::ld(dout + ((size_t)(t0 + r) * a.H + h) * dv + c) -
+                       m.W[r * dk + i] * m.dU[r * dv + c];
+            sG[e] = acc;
+        }
+        __syncthreads();
+    }
+    if (a.dS0)
+        for (int e = tid; e < dk * dv; e += kBwThreads) a.dS0[(size_t)unit * dk * dv + e] = sG[e];
+}
+
+// 4. Every per-chunk gradient.
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
+    const int slot = blockIdx.x, unit = slot / a.NC, j = slot % a.NC;
+    const int s = unit / a.H, h = unit % a.H;
+    int64_t t0;
+    int n;
+    chunk_rows(a, s, j, t0, n);
+    if (n == 0) return;
+    const int dk = a.dk, dv = a.dv, tid = threadIdx.x;
+    const Slot sl{dk, dv};
+    SlotPtr m(a.slots + (size_t)slot * sl.floats(), sl);
+    const T *dout = static_cast<const T *>(a.dout), *v = static_cast<const T *>(a.v);
+    auto dO = [&](int r, int c) { return IO<T>::ld(dout + ((size_t)(t0 + r) * a.H + h) * dv + c); };
+    auto V = [&](int r, int c) { return IO<T>::ld(v + ((size_t)(t0 + r) * a.H + h) * dv + c); };
+    auto beta = [&](int r) { return a.beta[(size_t)(t0 + r) * a.H + h]; };
+    // (1) dKd = U dS'^T, dQg = dO S^T, dW = -dU S^T (n x dk); dP = lower(dO U^T)
+    for (int e = tid; e < n * dk; e += kBwThreads) {
+        const int r = e / dk, i = e % dk;
+        float kd = 0.f, qg = 0.f, w = 0.f;
+        for (int c = 0; c < dv; ++c) {
+            kd += m.U[r * dv + c] * m.dSn[i * dv + c];
+            qg += dO(r, c) * m.S[i * dv + c];
+            w -= m.dU[r * dv + c] * m.S[i * dv + c];
+        }
+        m.dKd[e] = kd;
+        m.dQg[e] = qg;
+        m.dW[e] = w;
+    }
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        const int r = e / C, i = e % C;
+        float acc = 0.f;
+        if (r < n && i <= r)
+            for (int c = 0; c < dv; ++c) acc += dO(r, c) * m.U[i * dv + c];
+        m.dP[e] = acc;
+    }
+    __syncthreads();
+    // (2) dT = lower(dU V^T + dW Kg^T); dV = T^T dU
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        const int r = e / C, i = e % C;
+        float acc = 0.f;
+        if (r < n && i <= r) {
+            for (int c = 0; c < dv; ++c) acc += m.dU[r * dv + c] * V(i, c);
+            for (int c = 0; c < dk; ++c) acc += m.dW[r * dk + c] * m.Kg[i * dk + c];
+        }
+        m.dT[e] = acc;
+    }
+    for (int e = tid; e < n * dv; e += kBwThreads) {
+        const int r = e / dv, c = e % dv;
+        float acc = 0.f;
+        for (int rr = r; rr < n; ++rr) acc += m.T[rr * C + r] * m.dU[rr * dv + c];
+        a.dvv[((size_t)(t0 + r) * a.H + h) * dv + c] = acc;
+    }
+    __syncthreads();
+    // (3) dKg = T^T dW; Y = X^T dX with dX = dT Diag(beta)
+    for (int e = tid; e < n * dk; e += kBwThreads) {
+        const int r = e / dk, c = e % dk;
+        float acc = 0.f;
+        for (int rr = r; rr < n; ++rr) acc += m.T[rr * C + r] * m.dW[rr * dk + c];
+        m.dKg[e] = acc;
+    }
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        const int r = e / C, i = e % C;
+        float acc = 0.f;
+        if (r < n && i < n)
+            for (int mm = 0; mm < n; ++mm) acc += m.X[mm * C + r] * m.dT[mm * C + i] * beta(i);
+        m.Y[e] = acc;
+    }
+    __syncthreads();
+    // (4) dM = -Y X^T
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        const int r = e / C, i = e % C;
+        float acc = 0.f;
+        if (r < n && i < n)
+            for (int mm = 0; mm < n; ++mm) acc -= m.Y[r * C + mm] * m.X[i * C + mm];
+        m.dM[e] = acc;
+    }
+    __syncthreads();
+    // (5) dA = strict_lower(Diag(beta) dM); dbeta
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        const int r = e / C, i = e % C;
+        m.dA[e] = (r < n && i < r) ? beta(r) * m.dM[e] : 0.f;
+    }
+    for (int i = tid; i < n; i += kBwThreads) {
+        float acc = 0.f;
+        for (int r = 0; r < n; ++r) acc += m.dT[r * C + i] * m.X[r * C + i];
+        for (int mm = 0; mm < i; ++mm) acc += m.dM[i * C + mm] * m.A[i * C + mm];
+        a.dbeta[(size_t)(t0 + i) * a.H + h] = acc;
+    }
+    __syncthreads();
+    // (6) dKg += dA Kn; dKn = dA^T Kg + dP^T Qg; dQg += dP Kn
+    for (int e = tid; e < n * dk; e += kBwThreads) {
+        const int r = e / dk, c = e % dk;
+        float kg = 0.f, kn = 0.f, qg = 0.f;
+        for (int i = 0; i < n; ++i) {
+            kg += m.dA[r * C + i] * m.Kn[i * dk + c];
+            kn += m.dA[i * C + r] * m.Kg[i * dk + c] + m.dP[i * C + r] * m.Qg[i * dk + c];
+            qg += m.dP[r * C + i] * m.Kn[i * dk + c];
+        }
+        m.dKg[e] += kg;
+        m.dKn[e] = kn;
+        m.dQg[e] += qg;
+    }
+    __syncthreads();
+    // (7)(8) dG, dg, dlog_alpha (reverse cumsum); d q^, d k^ through the exponents
+    for (int c = tid; c < dk; c += kBwThreads) {
+        const float g = m.G[(n - 1) * dk + c];
+        float dg = 0.f;
+        for (int r = 0; r < n; ++r) dg += m.dKd[r * dk + c] * m.Kd[r * dk + c];
+        float ss = 0.f;
+        for (int cc = 0; cc < dv; ++cc) ss += m.dSn[c * dv + cc] * m.S[c * dv + cc];
+        dg += expf(g) * ss;
+        float run = 0.f;
+        for (int r = n - 1; r >= 0; --r) {
+            const int e = r * dk + c;
+            run += m.dQg[e] * m.Qg[e] + m.dKg[e] * m.Kg[e] - m.dKn[e] * m.Kn[e] - m.dKd[e] * m.Kd[e];
+            const size_t row = (size_t)(t0 + r) * a.H + h;
+            a.dla[row * dk + c] = run + dg;
+            const float G = m.G[e];
+            a.dqh[row * dk + c] = m.dQg[e] * expf(G);
+            a.dkh[row * dk + c] = m.dKg[e] * expf(G) + m.dKn[e] * expf(-G) + m.dKd[e] * expf(g - G);
+        }
+    }
+}
+
+// 5. Through x / max(|x|, eps): a warp per (token, head).
+__global__ void __launch_bounds__(kBwThreads) bw_norm(BwArgs a) {
+    const int64_t w = ((int64_t)blockIdx.x * kBwThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31, dk = a.dk;
+    if (w >= a.total * a.H) return;
+    for (int which = 0; which < 2; ++which) {
+        const float *xh = which ? a.kh : a.qh, *dxh = which ? a.dkh : a.dqh;
+        const float nrm = (which ? a.nk : a.nq)[w];
+        float *dx = which ? a.dkk : a.dq;
+        float dot = 0.f;
+        for (int c = lane; c < dk; c += 32) dot += xh[w * dk + c] * dxh[w * dk + c];
+        for (int off = 16; off; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        for (int c = lane; c < dk; c += 32) {
+            const float g = dxh[w * dk + c];
+            float out = g;
+            if (a.l2norm) out = nrm > a.eps ? (g - xh[w * dk + c] * dot) / nrm : g / a.eps;
+            dx[w * dk + c] = out;
+        }
+    }
+}
+
+template <typename T>
+cudaError_t run(const BwArgs &a, cudaStream_t st) {
+    const unsigned units = (unsigned)a.N * (unsigned)a.H;
+    const size_t state_smem = (size_t)a.dk * a.dv * sizeof(float);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(bw_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)state_smem)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(bw_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)state_smem)) !=
+        cudaSuccess)
+        return e;
+    bw_prep<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
+    bw_fwd<<<units, kBwThreads, state_smem, st>>>(a);
+    bw_bwd<T><<<units, kBwThreads, state_smem, st>>>(a);
+    bw_grads<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
+    const int64_t warps = a.total * a.H;
+    if (warps > 0) bw_norm<<<(unsigned)((warps * 32 + kBwThreads - 1) / kBwThreads), kBwThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int N, int H, int64_t total, int dk, int dv, int NC) {
+    const Slot sl{dk, dv};
+    return ((size_t)N * H * NC * sl.floats() + (size_t)total * H * (4 * (size_t)dk + 2)) * sizeof(float);
+}
+
+cudaError_t backward(const BackwardArgs &b, bool bf16, cudaStream_t st) {
+    BwArgs a;
+    a.q = b.q; a.k = b.k; a.v = b.v; a.dout = b.dout;
+    a.la = b.log_alpha; a.beta = b.beta; a.S0 = b.S0; a.dST = b.dS_T; a.cu = b.cu;
+    a.total = b.total; a.N = b.N; a.H = b.H; a.dk = b.dk; a.dv = b.dv; a.NC = b.NC;
+    a.l2norm = b.l2norm; a.eps = b.eps;
+    a.dq = b.dq; a.dkk = b.dk_out; a.dvv = b.dv_out; a.dla = b.dlog_alpha; a.dbeta = b.dbeta; a.dS0 = b.dS0;
+    const Slot sl{b.dk, b.dv};
+    float *p = static_cast<float *>(b.ws);
+    a.slots = p;
+    p += (size_t)b.N * b.H * b.NC * sl.floats();
+    const size_t th = (size_t)b.total * b.H;
+    a.qh = p; p += th * b.dk;
+    a.kh = p; p += th * b.dk;
+    a.dqh = p; p += th * b.dk;
+    a.dkh = p; p += th * b.dk;
+    a.nq = p; p += th;
+    a.nk = p;
+    a.err = b.err;
+    return bf16 ? run<__nv_bfloat16>(a, st) : run<float>(a, st);
+}
+
+}  // namespace kda

@@ -100,6 +100,22 @@ struct DecodeConv {
     void *state_out[3];
 };
 
+// Backward of the chunkwise prefill (fp32 CUDA cores; gradients fp32).
+struct BackwardArgs {
+    const void *q, *k, *v, *dout;  // io dtype
+    const float *log_alpha, *beta, *S0, *dS_T;
+    const int32_t *cu;
+    int64_t total;
+    int N, H, dk, dv, NC;  // NC: chunks of the longest sequence
+    int l2norm;
+    float eps;
+    float *dq, *dk_out, *dv_out, *dlog_alpha, *dbeta, *dS0;
+    void *ws;
+    int *err;
+};
+size_t backward_workspace_bytes(int N, int H, int64_t total, int dk, int dv, int NC);
+cudaError_t backward(const BackwardArgs &b, bool bf16, cudaStream_t st);
+
 // decode step
 cudaError_t decode_step(const void *q, const void *k, const void *v, const float *la,
                         const float *beta, float *S, int N, int H, int dk, int dv, bool bf16,

@@ -284,6 +284,37 @@ kda_status kda_decode_step_conv(const void *q, const void *k, const void *v, con
                                 const kda_short_conv *conv_v, const kda_output_gate *out_gate, void *o,
                                 kda_stream_t stream);
 
+/*
+ * Backward of the prefill (training): the gradients of a loss L with respect
+ * to q, k, v, log_alpha, beta and S0, given dL/do and dL/dS_T. The pages
+ * mention training but give no backward; the chunked reverse-mode algebra
+ * implemented here is stated in csrc/kda_backward.cu. The same inputs and
+ * rules as kda_prefill (chunk 64; KDA_FLAG_NO_L2NORM honoured; one gate per
+ * (token, head) is not supported: KDA_ERR_UNSUPPORTED), plus:
+ *
+ *   dout         [T][H][dv] in the io dtype: dL/do
+ *   dS_T         [N][H][dk][dv] fp32: dL/dS_T, or NULL (zero)
+ *   grad_q, grad_k        [T][H][dk] fp32 out;  grad_v [T][H][dv] fp32 out
+ *   grad_log_alpha        [T][H][dk] fp32 out;  grad_beta [T][H] fp32 out
+ *   grad_S0               [N][H][dk][dv] fp32 out, or NULL (not written)
+ *   workspace    kda_backward_workspace_size() bytes, 16-byte aligned
+ *
+ * fp32 CUDA-core arithmetic (a reference-grade implementation; five
+ * launches). It factors e^{G_r - G_i} = e^{G_r} e^{-G_i} inside each chunk:
+ * a chunk whose decay range (minus the sum of log_alpha over it) exceeds 60
+ * sets device error code 2 (kda_device_error) and its gradients are not valid.
+ */
+size_t kda_backward_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen,
+                                   int32_t H, int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk,
+                                   uint32_t flags);
+kda_status kda_backward(const void *q, const void *k, const void *v, const float *log_alpha,
+                        const float *beta, const float *S0, const int32_t *cu_seqlens,
+                        int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                        int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                        const void *dout, const float *dS_T, float *grad_q, float *grad_k,
+                        float *grad_v, float *grad_log_alpha, float *grad_beta, float *grad_S0, void *workspace,
+                        size_t workspace_bytes, kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -635,3 +635,56 @@ def test_decode_conv_continues_prefill_conv():
                                 inp["beta"][t:t + 1].clone(), S, conv=tuple(cv))
         torch.testing.assert_close(o[0], o_all[t], atol=2e-5, rtol=0)
     torch.testing.assert_close(S, S_all, atol=2e-5, rtol=0)
+
+
+# ------------------------------------------------ backward (training) ----
+# The CUDA backward (fp32 CUDA cores) against the fp64 oracle's token backward on
+# the same input bits: gradients agree to fp32 accumulation error, checked as
+# max|g - g_ref| <= 1e-3 * max(1, max|g_ref|) per gradient tensor.
+
+def _bw_inputs(lengths, H, d, dtype, seed):
+    inp = make(lengths, H, d, d, dtype, seed=seed)
+    T, N = sum(lengths), len(lengths)
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(9000 + seed)
+    do = torch.randn((T, H, d), generator=gen, device=DEV).to(dtype)
+    dST = torch.randn((N, H, d, d), generator=gen, device=DEV)
+    return inp, do, dST
+
+
+def _bw_check(got, inp, do, dST, l2norm=True, label=""):
+    ref = oracle.backward(host(inp["q"]), host(inp["k"]), host(inp["v"]), host(inp["log_alpha"]),
+                          host(inp["beta"]), host(do), None if dST is None else host(dST), host(inp["S0"]),
+                          inp["cu_seqlens"].cpu().numpy(), l2norm=l2norm)
+    for name, g, w in zip(["dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"], got, ref):
+        if g is None:
+            continue
+        gh = host(g)
+        assert np.isfinite(gh).all(), (label, name)
+        err = float(np.abs(gh - w).max()) if w.size else 0.0
+        assert err <= 1e-3 * max(1.0, float(np.abs(w).max()) if w.size else 0.0), "%s %s: %.3e" % (label, name, err)
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 128), (torch.float32, 128)])
+def test_backward_matches_oracle(dtype, d):
+    """Partial chunks, an empty and a one-token sequence, S0 and dS_T given."""
+    inp, do, dST = _bw_inputs([70, 0, 130, 1], 2, d, dtype, seed=51)
+    got = kda.kda_backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], do, dST, inp["S0"],
+                           inp["cu_seqlens"], max_seqlen=130)
+    torch.cuda.synchronize()
+    _bw_check(got, inp, do, dST, label="backward %s d=%d" % (dtype, d))
+
+
+def test_backward_no_l2norm_no_state_gradient():
+    inp, do, _ = _bw_inputs([100, 37], 1, 64, torch.float32, seed=52)
+    got = kda.kda_backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], do, None, inp["S0"],
+                           inp["cu_seqlens"], max_seqlen=100, l2norm=False)
+    torch.cuda.synchronize()
+    _bw_check(got, inp, do, None, l2norm=False, label="no l2norm")
+
+
+def test_backward_rejects_scalar_gate():
+    inp, do, dST = _bw_inputs([16], 1, 64, torch.float32, seed=53)
+    la = inp["log_alpha"][..., 0].contiguous()
+    with pytest.raises(kda.KDAError):
+        kda.kda_backward(inp["q"], inp["k"], inp["v"], la, inp["beta"], do, dST, inp["S0"], inp["cu_seqlens"])
