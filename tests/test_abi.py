@@ -156,3 +156,93 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setenv("KDA_LIBRARY", "/nonexistent/libkda.so")
     with pytest.raises(OSError):
         kda.load_library()
+
+
+# ------------------------------------------------ the next rows' entry points ----
+
+def test_short_conv_launch_counts(lib):
+    f = lib.kda_short_conv_launches
+    assert f(4, 1, 16) == 2 and f(4, 0, 16) == 1 and f(1, 1, 16) == 1
+    assert f(4, 1, 0) == 1 and f(4, 0, 0) == 0
+    assert f(0, 0, 16) == -1 and f(9, 0, 16) == -1 and f(4, 0, -1) == -1
+
+
+def short_conv(lib, width=4, weight=A, sin=None, sout=None, **over):
+    a = dict(x=A, y=A + (1 << 24), cu=None, N=1, T=64, C=256, dt=1, stream=None)
+    a.update(over)
+    c = kda.ShortConv(width, weight, sin, sout)
+    return lib.kda_short_conv_swish(a["x"], a["y"], ctypes.byref(c), a["cu"], a["N"], a["T"], a["C"],
+                                    a["dt"], a["stream"])
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(width=0), kda.KDA_ERR_UNSUPPORTED),
+    (dict(width=9), kda.KDA_ERR_UNSUPPORTED),
+    (dict(C=12), kda.KDA_ERR_INVALID_ARG),
+    (dict(C=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=2), kda.KDA_ERR_INVALID_ARG),            # several sequences need cu_seqlens
+    (dict(T=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dt=3), kda.KDA_ERR_INVALID_ARG),
+    (dict(weight=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(x=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(x=A + 8), kda.KDA_ERR_MISALIGNED),
+    (dict(sin=A + 4), kda.KDA_ERR_MISALIGNED),
+    (dict(sout=A + 2), kda.KDA_ERR_MISALIGNED),
+    (dict(weight=A + 2), kda.KDA_ERR_MISALIGNED),
+    (dict(y=A + 512), kda.KDA_ERR_INVALID_ARG),     # y overlaps x (64 x 256 bf16 = 32 KiB)
+])
+def test_short_conv_rejects(lib, over, code):
+    assert short_conv(lib, **over) == code
+
+
+@no_gpu
+def test_decode_conv_rejects(lib):
+    ok = kda.ShortConv(4, A, A, A)
+    wide = kda.ShortConv(5, A, A, A)  # the fused decode takes windows up to 4
+    odd = kda.ShortConv(4, A, A + 8, A)
+    call = lambda cq: lib.kda_decode_step_conv(A, A, A, A, A, A, 4, 2, 128, 128, 1, 0, cq, None, None,
+                                               None, A, None)
+    assert call(ctypes.byref(wide)) == kda.KDA_ERR_UNSUPPORTED
+    assert call(ctypes.byref(odd)) == kda.KDA_ERR_MISALIGNED
+    assert lib.kda_decode_step_conv(None, A, A, A, A, A, 4, 2, 128, 128, 1, 0, ctypes.byref(ok), None, None,
+                                    None, A, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_backward_workspace_queries(lib):
+    f = lib.kda_backward_workspace_size
+    a = f(1, 8192, 8192, 32, 128, 128, 1, 64, 0)
+    assert a > 0
+    assert f(1, 1024, 1024, 32, 128, 128, 1, 64, 0) < a  # per-chunk scratch grows with the chunks
+    assert f(2, 8192, 4096, 32, 128, 128, 1, 64, 0) > 0
+    assert f(1, 10, 10, 1, 128, 128, 1, 64, kda.KDA_FLAG_SCALAR_GATE) == 0  # one gate per head: not yet
+    assert f(1, 10, 10, 1, 96, 128, 1, 64, 0) == 0
+    assert f(0, 10, 10, 1, 128, 128, 1, 64, 0) == 0
+
+
+def backward(lib, **over):
+    a = dict(q=A, k=A, v=A, la=A, beta=A, S0=None, cu=None, N=1, T=128, L=128, H=2, dk=64, dv=64, dt=1,
+             chunk=64, flags=0, do=A, dST=None, dq=A, dk_=A, dv_=A, dla=A, db=A, dS0=None, ws=A,
+             wsb=1 << 30, stream=None)
+    a.update(over)
+    return lib.kda_backward(a["q"], a["k"], a["v"], a["la"], a["beta"], a["S0"], a["cu"], a["N"], a["T"],
+                            a["L"], a["H"], a["dk"], a["dv"], a["dt"], a["chunk"], a["flags"], a["do"],
+                            a["dST"], a["dq"], a["dk_"], a["dv_"], a["dla"], a["db"], a["dS0"], a["ws"],
+                            a["wsb"], a["stream"])
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(do=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(db=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=3), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(flags=kda.KDA_FLAG_SCALAR_GATE), kda.KDA_ERR_UNSUPPORTED),
+    (dict(ws=None), kda.KDA_ERR_WORKSPACE),
+    (dict(wsb=4096), kda.KDA_ERR_WORKSPACE),
+    (dict(ws=A + 4), kda.KDA_ERR_MISALIGNED),
+])
+def test_backward_rejects(lib, over, code):
+    assert backward(lib, **over) == code
