@@ -67,6 +67,22 @@ def peaks():
         return 6650.0, "fallback"
 
 
+def bf16_peak():
+    """Dense bf16 tensor peak in TFLOP/s: the measured burst figure, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+# Prefill FLOPs per token at H heads: the pages' count (6 d^2 + 3 C d + C^2 per head-token)
+# and this path's own count (6 d^2 + 10 C d per head-token: every Gram, solve-application
+# and scan product at 2 flop per multiply-add).
+FLOPS_PAGES_PER_TOKEN = H * (6 * D * D + 3 * 64 * D + 64 * 64)
+FLOPS_OWN_PER_TOKEN = H * (6 * D * D + 10 * 64 * D)
+
+
 class Clocks:
     """Sample SM clocks and throttle reasons while the timed region runs."""
 
@@ -472,6 +488,12 @@ def run_kda(args, world, rank, local):
                      "traffic": profiled_traffic("fused_kernel_prefill_8k.md", PREFILL_SOURCES),
                      "kernel": "kda_prefill = plan_kernel + persistent fused_kernel (timed together)",
                      "algorithmic_bytes": bytes_pass, "peak_source": peak_src},
+        "tensor": {"bound_note": "HBM binds (intensity below the ridge); reported for the flop view",
+                   "tflops_pages_count": FLOPS_PAGES_PER_TOKEN * T8K / (ms * 1e-3) / 1e12,
+                   "tflops_own_count": FLOPS_OWN_PER_TOKEN * T8K / (ms * 1e-3) / 1e12,
+                   "peak_tflops": bf16_peak()[0], "peak_source": bf16_peak()[1],
+                   "frac_pages_count": FLOPS_PAGES_PER_TOKEN * T8K / (ms * 1e-3) / 1e12 / bf16_peak()[0],
+                   "frac_own_count": FLOPS_OWN_PER_TOKEN * T8K / (ms * 1e-3) / 1e12 / bf16_peak()[0]},
         "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": (3 * args.steps * launches_prefill + dsteps + args.steps * 3 * conv_launches
