@@ -2,10 +2,18 @@
 
 One timed "step" is one chunkwise prefill of the single-sequence workload
 (B=1, H=32, T=8192, d_k=d_v=128, bf16 q/k/v, fp32 gates and state; inputs
-~404 MB > L2, so no flush is needed). The decode step of the batched workload
-(256 sequences x 32 heads, 512 MiB fp32 state in place, > L2) is timed as a
-second region and reported in ``decode``. Everything runs in libkda's CUDA
-kernels; inputs are seeded synthetic tensors (``kda_inputs``).
+~404 MB > L2, so no flush is needed). Further lines on the same JSON record:
+  * varlen_16 (16 packed sequences, lengths U[512, 8192]), prefill_1m
+    (T = 1,048,576) and tiny_f32 (H=2, T=256, d=64, fp32; L2 flushed before
+    each timed call), each with tokens/s and its HBM roofline;
+  * gdn (one gate per token and head), output_gate (RMSNorm + sigmoid gate
+    fused), short_conv (the convolution before the recurrence), backward;
+  * decode: 256 sequences x 32 heads, 512 MiB fp32 state in place (> L2),
+    1000 consecutive steps on 1000 pregenerated inputs, as plain launches and
+    replayed from a CUDA graph; decode_conv: the same with the convolution
+    fused into the loads.
+Everything runs in libkda's CUDA kernels; inputs are seeded synthetic tensors
+(``kda_inputs``).
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
 Multi-GPU: launched with torchrun, one rank per GPU; every rank runs its own
@@ -37,7 +45,8 @@ import kda_inputs as KI  # noqa: E402
 METRIC = "KDA prefill tokens/s at H=32,d=128; decode-step HBM GB/s vs B200 peak"
 PREFILL = "prefill_8k"
 T8K, H, D = 8192, 32, 128
-DEC_N, DEC_STEPS_POOL = 256, 64
+DEC_N = 256
+BACKWARD_LAUNCHES = 5  # bw_prep, bw_fwd, bw_bwd, bw_grads, bw_norm
 # Algorithmic HBM bytes (inputs read once, outputs written once):
 #   prefill per token (all 32 heads): q,k,v bf16 3*32*128*2 + log_alpha 32*128*4 + beta 32*4
 #   + o 32*128*2 = 49,280 B; plus S0 read and S_T written (2 MiB each at H=32).
@@ -232,12 +241,80 @@ def profiled_traffic(profile, sources):
     return int(m.group(1))
 
 
+def timed(fn, steps, warmup, world, dev, stream):
+    """CUDA-event time per call of ``fn`` over ``steps`` calls after ``warmup`` untimed ones,
+    bracketed by a barrier and a device synchronisation. Returns (this rank's ms, max over ranks)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        fn()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1) / steps
+    return ms, max_over_ranks(ms, world, dev)
+
+
+def timed_flushed(fn, steps, warmup, world, dev, stream):
+    """As ``timed`` for inputs that fit in L2: each call is timed alone, after a write of a
+    buffer larger than L2 (the flush is outside the events). Returns (ms, max over ranks)."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = sum(e0.elapsed_time(e1) for e0, e1 in evs) / steps
+    del flush
+    return ms, max_over_ranks(ms, world, dev)
+
+
+def prefill_bytes(tokens, n_seqs, heads, d, io_bytes, gate_per_channel=True, reads_s0=True):
+    """Algorithmic HBM bytes of one prefill: q, k, v read and o written in the io dtype,
+    log_alpha and beta read (fp32), S_T written and S0 read (when given), fp32."""
+    per_token = heads * (3 * d * io_bytes + (d if gate_per_channel else 1) * 4 + 4 + d * io_bytes)
+    state = n_seqs * heads * d * d * 4
+    return tokens * per_token + state * (2 if reads_s0 else 1)
+
+
+def prefill_entry(tokens, ms_local, ms_max, world, nbytes, hbm, peak_src, workload, kernel,
+                  traffic=None, flops=True, extra=None):
+    """One prefill line: tokens/s over all ranks, the HBM roofline of one pass and the flop view."""
+    achieved = nbytes / (ms_local * 1e-3) / 1e9
+    e = {"value": world * tokens / (ms_max * 1e-3), "unit": "tokens/s", "ms_per_step": ms_max,
+         "workload": workload,
+         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                      "frac": achieved / hbm, "traffic": traffic, "kernel": kernel,
+                      "algorithmic_bytes": nbytes, "peak_source": peak_src}}
+    if flops:
+        pk, pk_src = bf16_peak()
+        tp = FLOPS_PAGES_PER_TOKEN * tokens / (ms_local * 1e-3) / 1e12
+        to = FLOPS_OWN_PER_TOKEN * tokens / (ms_local * 1e-3) / 1e12
+        e["tensor"] = {"tflops_pages_count": tp, "tflops_own_count": to, "peak_tflops": pk,
+                       "peak_source": pk_src, "frac_pages_count": tp / pk, "frac_own_count": to / pk}
+    if extra:
+        e.update(extra)
+    return e
+
+
 def run_kda(args, world, rank, local):
     import gated_delta_rule_125_b200 as kda
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
     hbm, peak_src = peaks()
+    launches = 0  # this library's kernel launches inside timed regions
 
     # ---- prefill workload, resident in HBM
     inp = KI.prefill_workload(PREFILL, dev, seed=rank)
@@ -251,21 +328,9 @@ def run_kda(args, world, rank, local):
     def prefill():
         kda.kda_prefill(q, k, v, la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
 
-    for _ in range(args.warmup):
-        prefill()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with Clocks(local) as clk:
-        torch.cuda.synchronize()
-        ev0.record(stream)
-        for _ in range(args.steps):
-            prefill()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = ev0.elapsed_time(ev1) / args.steps
-    ms_max = max_over_ranks(ms, world, dev)
+        ms, ms_max = timed(prefill, args.steps, args.warmup, world, dev, stream)
+    launches += args.steps * launches_prefill
     tokens_per_s = world * T8K / (ms_max * 1e-3)
     bytes_pass = T8K * PREFILL_BYTES_PER_TOKEN + PREFILL_STATE_BYTES
     achieved = bytes_pass / (ms * 1e-3) / 1e9
@@ -277,18 +342,9 @@ def run_kda(args, world, rank, local):
         kda.kda_prefill(gdn["q"], gdn["k"], gdn["v"], gdn["log_alpha"], gdn["beta"], gdn["S0"], cu,
                         max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
 
-    for _ in range(args.warmup):
-        prefill_gdn()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        prefill_gdn()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    gdn_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    gdn_ms, gdn_ms_max = timed(prefill_gdn, args.steps, args.warmup, world, dev, stream)
+    launches += args.steps * launches_prefill
     gdn_bytes = T8K * GDN_BYTES_PER_TOKEN + PREFILL_STATE_BYTES
-    gdn_gbs = gdn_bytes / (ev0.elapsed_time(ev1) / args.steps * 1e-3) / 1e9
     del gdn
 
     # ---- the same workload with the layer's output step fused (RMSNorm + sigmoid gate)
@@ -301,18 +357,9 @@ def run_kda(args, world, rank, local):
         kda.kda_prefill(q, k, v, la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws,
                         out_gate=og)
 
-    for _ in range(args.warmup):
-        prefill_gated()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        prefill_gated()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    og_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
+    og_ms, og_ms_max = timed(prefill_gated, args.steps, args.warmup, world, dev, stream)
+    launches += args.steps * launches_prefill
     og_bytes = T8K * (PREFILL_BYTES_PER_TOKEN + H * D * 2) + PREFILL_STATE_BYTES
-    og_gbs = og_bytes / (ev0.elapsed_time(ev1) / args.steps * 1e-3) / 1e9
     del og
 
     # ---- the layer's step before the recurrence: short convolution + Swish on the
@@ -333,8 +380,8 @@ def run_kda(args, world, rank, local):
                         la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
 
     # Three short convolutions (two launches each, ~30 us of GPU time): the host issues them
-    # more slowly than the GPU runs them,
-    # so the convolution line replays them from a CUDA graph (captured once).
+    # more slowly than the GPU runs them, so the convolution line replays them from a CUDA
+    # graph (captured once).
     conv_graph = None
     try:
         side = torch.cuda.Stream(dev)
@@ -351,16 +398,8 @@ def run_kda(args, world, rank, local):
         conv_graph = None
     conv_ms = {}
     for name, fn in (("conv", conv_graph.replay if conv_graph is not None else convs), ("conv_prefill", conv_prefill)):
-        for _ in range(args.warmup):
-            fn()
-        torch.cuda.synchronize()
-        barrier(world)
-        ev0.record(stream)
-        for _ in range(args.steps):
-            fn()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        conv_ms[name] = (ev0.elapsed_time(ev1) / args.steps, max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev))
+        conv_ms[name] = timed(fn, args.steps, args.warmup, world, dev, stream)
+    launches += args.steps * (3 * conv_launches) + args.steps * (3 * conv_launches + launches_prefill)
     conv_gbs = 3 * CONV_BYTES / (conv_ms["conv"][0] * 1e-3) / 1e9
     conv_graph_used = conv_graph is not None
     del conv_graph, conv_in, conv_out, conv_st
@@ -381,72 +420,98 @@ def run_kda(args, world, rank, local):
         h_o.copy_(o, non_blocking=True)
         h_S.copy_(S_T, non_blocking=True)
 
-    for _ in range(args.warmup):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, world, dev)
-    del d_in, h_in
+    _, e2e_ms = timed(e2e_step, args.steps, args.warmup, world, dev, stream)
+    launches += args.steps * launches_prefill
+    del d_in, h_in, inp, q, k, v, la, beta, S0, o, S_T
 
-    # ---- decode: 256 x 32 heads, state 512 MiB in place
-    dec = KI.decode_workload(DEC_N, H, D, DEC_STEPS_POOL, torch.bfloat16, dev, seed=rank)
-    S = dec["S0"].clone()
-    od = torch.empty((DEC_N, H, D), dtype=torch.bfloat16, device=dev)
+    # ---- the other prefill workloads: packed variable length, 1M tokens, tiny fp32
+    others = {}
+    for name, steps in (("varlen_16", args.steps), ("prefill_1m", 3), ("tiny_f32", args.steps)):
+        w = KI.WORKLOADS[name]
+        lens = KI.workload_lengths(name, 0)  # the same sizes on every rank, own data
+        wi = KI.prefill_workload(name, dev, seed=rank, lengths=lens)
+        Tn, Nn, dn = sum(lens), len(lens), w["d"]
+        dt = KI.torch_dtype(w["dtype"])
+        s0 = wi["S0"] if w["s0_std"] else None  # S0 = 0: not passed (nothing to read)
+        wo = torch.empty_like(wi["v"])
+        wS = torch.empty((Nn, w["H"], dn, dn), dtype=torch.float32, device=dev)
+        nb = kda.kda_prefill_workspace_size(Nn, Tn, max(lens), w["H"], dn, dn, dt)
+        wws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        wl = kda.kda_prefill_launches(Nn, Tn, max(lens), w["H"], dn, dn, dt, nb)
 
-    def decode(t):
-        i = t % DEC_STEPS_POOL
-        kda.kda_decode_step(dec["q"][i], dec["k"][i], dec["v"][i], dec["log_alpha"][i],
-                            dec["beta"][i], S, o=od)
+        def fn(wi=wi, s0=s0, wo=wo, wS=wS, wws=wws, lens=lens):
+            kda.kda_prefill(wi["q"], wi["k"], wi["v"], wi["log_alpha"], wi["beta"], s0, wi["cu_seqlens"],
+                            max_seqlen=max(lens), o=wo, S_T=wS, workspace=wws)
 
+        io = 2 if dt == torch.bfloat16 else 4
+        nbytes = prefill_bytes(Tn, Nn, w["H"], dn, io, reads_s0=s0 is not None)
+        in_l2 = nbytes < (64 << 20)
+        t_local, t_max = (timed_flushed if in_l2 else timed)(fn, steps, args.warmup, world, dev, stream)
+        launches += steps * wl
+        others[name] = prefill_entry(
+            Tn, t_local, t_max, world, nbytes, hbm, peak_src,
+            "%s: %d sequence(s), %d tokens, H=%d, d_k=d_v=%d, %s q/k/v, fp32 gates/state, chunk 64%s" % (
+                name, Nn, Tn, w["H"], dn, w["dtype"], ", S0=0" if s0 is None else ""),
+            "kda_prefill (%s path, %d launches)" % ("tensor-core" if wl == 2 else "fp32 CUDA-core", wl),
+            flops=(dt == torch.bfloat16),
+            extra={"steps": steps, "l2": ("%d KB of inputs: L2 flushed before each timed call" % (nbytes >> 10))
+                   if in_l2 else "inputs %.1f GB > L2 (no flush)" % (nbytes / 1e9)})
+        del wi, wo, wS, wws, fn
+
+    # ---- decode: 256 x 32 heads, state 512 MiB in place, 1000 consecutive steps on
+    #      1000 pregenerated inputs; plain launches and the 1000 launches replayed from a
+    #      CUDA graph
     dsteps = args.decode_steps
-    for t in range(max(3, args.warmup)):
-        decode(t)
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record(stream)
-    for t in range(dsteps):
-        decode(t)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    dec_us = ev0.elapsed_time(ev1) * 1e3 / dsteps
-    dec_us_max = max_over_ranks(dec_us, world, dev)
+    dec = KI.decode_workload(DEC_N, H, D, dsteps, torch.bfloat16, dev, seed=rank)
+    S = dec["S0"].clone()
+    od = torch.empty((dsteps, DEC_N, H, D), dtype=torch.bfloat16, device=dev)
+
+    def decode_all(conv=None):
+        for t in range(dsteps):
+            kda.kda_decode_step(dec["q"][t], dec["k"][t], dec["v"][t], dec["log_alpha"][t],
+                                dec["beta"][t], S, o=od[t], conv=conv)
+
+    dec_ms, dec_ms_max = timed(decode_all, 1, 1, world, dev, stream)
+    launches += dsteps
+    dec_us, dec_us_max = 1e3 * dec_ms / dsteps, 1e3 * dec_ms_max / dsteps
     dec_gbs = DECODE_BYTES / (dec_us * 1e-6) / 1e9
+    dec_graph = {}
+    try:
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            decode_all()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            decode_all()
+        gms, gms_max = timed(g.replay, 1, 1, world, dev, stream)
+        launches += dsteps
+        dec_graph = {"us_per_step": 1e3 * gms_max / dsteps,
+                     "value": DECODE_BYTES / (1e-3 * gms_max / dsteps) / 1e9,
+                     "frac": DECODE_BYTES / (1e-3 * gms / dsteps) / 1e9 / hbm}
+        del g
+    except RuntimeError as exc:
+        dec_graph = {"error": str(exc)[:200]}
 
     # ---- decode with the short convolution fused into the q, k, v loads (states in place)
     dconv = []
     for i in range(3):
         _, w_, st_ = KI.conv_inputs(1, H * D, CONV_W, DEC_N, torch.bfloat16, dev, seed=rank, tensor=i)
         dconv.append((w_, st_, st_))
-
-    def decode_conv(t):
-        i = t % DEC_STEPS_POOL
-        kda.kda_decode_step(dec["q"][i], dec["k"][i], dec["v"][i], dec["log_alpha"][i],
-                            dec["beta"][i], S, o=od, conv=tuple(dconv))
-
-    for t in range(max(3, args.warmup)):
-        decode_conv(t)
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record(stream)
-    for t in range(dsteps):
-        decode_conv(t)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    dconv_us = ev0.elapsed_time(ev1) * 1e3 / dsteps
-    dconv_us_max = max_over_ranks(dconv_us, world, dev)
+    dc_ms, dc_ms_max = timed(lambda: decode_all(tuple(dconv)), 1, 1, world, dev, stream)
+    launches += dsteps
+    dconv_us, dconv_us_max = 1e3 * dc_ms / dsteps, 1e3 * dc_ms_max / dsteps
     dconv_gbs = DECODE_CONV_BYTES / (dconv_us * 1e-6) / 1e9
-    del dec, dconv
+    del dec, dconv, od, S
 
     # ---- backward of the prefill (training): gradients of prefill_8k given dL/do, dL/dS_T
     #      (an error of this line is reported in it, not fatal to the others)
     bw = {}
     bw_steps = 3
     try:
+        inp = KI.prefill_workload(PREFILL, dev, seed=rank)
         g_bw = torch.Generator(device=dev)
         g_bw.manual_seed(2000 + rank)
         d_o = torch.randn((T8K, H, D), generator=g_bw, device=dev).to(torch.bfloat16)
@@ -455,21 +520,13 @@ def run_kda(args, world, rank, local):
         bw_ws = torch.empty(bw_wsb, dtype=torch.uint8, device=dev)
 
         def backward():
-            kda.kda_backward(q, k, v, la, beta, d_o, d_ST, S0, cu, max_seqlen=T8K, workspace=bw_ws)
+            kda.kda_backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], d_o, d_ST,
+                             inp["S0"], inp["cu_seqlens"], max_seqlen=T8K, workspace=bw_ws)
 
-        for _ in range(max(3, args.warmup)):
-            backward()
-        torch.cuda.synchronize()
-        barrier(world)
-        ev0.record(stream)
-        for _ in range(bw_steps):
-            backward()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        bw_ms = ev0.elapsed_time(ev1) / bw_steps
-        bw["ms"] = max_over_ranks(bw_ms, world, dev)
+        bw_ms, bw["ms"] = timed(backward, bw_steps, args.warmup, world, dev, stream)
+        launches += bw_steps * BACKWARD_LAUNCHES
         bw["gbs"] = BACKWARD_BYTES / (bw_ms * 1e-3) / 1e9
-        del bw_ws, d_o, d_ST
+        del bw_ws, d_o, d_ST, inp
     except RuntimeError as exc:  # KDAError included
         bw = {"error": str(exc)[:200]}
 
@@ -496,33 +553,30 @@ def run_kda(args, world, rank, local):
                    "frac_own_count": FLOPS_OWN_PER_TOKEN * T8K / (ms * 1e-3) / 1e12 / bf16_peak()[0]},
         "e2e": {"value": world * T8K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": (3 * args.steps * launches_prefill + dsteps + args.steps * 3 * conv_launches
-                         + args.steps * (3 * conv_launches + launches_prefill) + dsteps
-                         + (5 * bw_steps if "ms" in bw else 0)),
+        "gpu_launches": launches,
         "clocks": clk.summary(),
-        "gdn": {"value": world * T8K / (gdn_ms * 1e-3), "unit": "tokens/s", "ms_per_step": gdn_ms,
-                "workload": "gdn_8k: prefill_8k with one forget gate per (token, head) "
-                            "(log_alpha [T][H], the Gated DeltaNet form)",
-                "roofline": {"bound": "hbm", "achieved": gdn_gbs, "peak": hbm, "unit": "GB/s",
-                             "frac": gdn_gbs / hbm, "traffic": None,
-                             "kernel": "kda_prefill with KDA_FLAG_SCALAR_GATE (timed like the main line)",
-                             "algorithmic_bytes": gdn_bytes, "peak_source": peak_src}},
-        "output_gate": {"value": world * T8K / (og_ms * 1e-3), "unit": "tokens/s", "ms_per_step": og_ms,
-                        "workload": "prefill_8k with the output step fused: RMSNorm over d_v and "
-                                    "a sigmoid gate [T][H][d_v] bf16 (page section 6.3)",
-                        "roofline": {"bound": "hbm", "achieved": og_gbs, "peak": hbm, "unit": "GB/s",
-                                     "frac": og_gbs / hbm, "traffic": None,
-                                     "kernel": "kda_prefill_ex with a kda_output_gate",
-                                     "algorithmic_bytes": og_bytes, "peak_source": peak_src}},
+        "varlen_16": others["varlen_16"],
+        "prefill_1m": others["prefill_1m"],
+        "tiny_f32": others["tiny_f32"],
+        "gdn": prefill_entry(T8K, gdn_ms, gdn_ms_max, world, gdn_bytes, hbm, peak_src,
+                             "gdn_8k: prefill_8k with one forget gate per (token, head) "
+                             "(log_alpha [T][H], the Gated DeltaNet form)",
+                             "kda_prefill with KDA_FLAG_SCALAR_GATE (timed like the main line)", flops=False),
+        "output_gate": prefill_entry(T8K, og_ms, og_ms_max, world, og_bytes, hbm, peak_src,
+                                     "prefill_8k with the output step fused: RMSNorm over d_v and "
+                                     "a sigmoid gate [T][H][d_v] bf16 (page section 6.3)",
+                                     "kda_prefill_ex with a kda_output_gate", flops=False),
         "decode": {"value": DECODE_BYTES / (dec_us_max * 1e-6) / 1e9, "unit": "GB/s",
                    "us_per_step": dec_us_max, "steps": dsteps,
                    "workload": "decode_256: 256 seqs x 32 heads, d=128, bf16 q/k/v, fp32 state "
-                               "512 MiB in place (> L2)",
+                               "512 MiB in place (> L2); %d consecutive steps on %d pregenerated "
+                               "inputs" % (dsteps, dsteps),
                    "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
                                 "frac": dec_gbs / hbm,
                                 "traffic": profiled_traffic("decode_kernel_decode_256.md", DECODE_SOURCES),
                                 "kernel": "decode_kernel<128,128,bf16>",
-                                "algorithmic_bytes": DECODE_BYTES, "peak_source": peak_src}},
+                                "algorithmic_bytes": DECODE_BYTES, "peak_source": peak_src},
+                   "cuda_graph": dec_graph},
         "short_conv": {"value": world * T8K / (conv_ms["conv"][1] * 1e-3), "unit": "tokens/s",
                        "ms_per_step": conv_ms["conv"][1], "cuda_graph": conv_graph_used,
                        "workload": "short convolution (W=%d) + Swish of the q, k, v projections of prefill_8k "
@@ -565,7 +619,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
-    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

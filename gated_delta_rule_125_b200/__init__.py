@@ -17,7 +17,7 @@ import torch
 
 __all__ = ["kda_prefill", "kda_decode_step", "kda_prefill_workspace_size", "kda_prefill_launches",
            "kda_device_error", "kda_prefill_noalloc", "kda_short_conv_swish", "kda_backward",
-           "kda_prefill_workspace_min", "kda_status_string", "kda_version", "KDAError",
+           "kda_prefill_workspace_min", "kda_set_wait_limit_ns", "kda_status_string", "kda_version", "KDAError",
            "library_path", "load_library", "KDA_OK", "KDA_ERR_INVALID_ARG",
            "KDA_ERR_UNSUPPORTED", "KDA_ERR_MISALIGNED", "KDA_ERR_WORKSPACE", "KDA_ERR_CUDA",
            "KDA_ERR_TIMEOUT", "KDA_FLAG_NO_L2NORM", "KDA_FLAG_EXACT", "KDA_FLAG_SCALAR_GATE"]
@@ -31,7 +31,8 @@ EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_s
                     "kda_prefill_workspace_min", "kda_prefill_launches", "kda_prefill",
                     "kda_prefill_ex", "kda_decode_step", "kda_decode_step_ex", "kda_device_error",
                     "kda_prefill_noalloc", "kda_short_conv_swish", "kda_short_conv_launches",
-                    "kda_decode_step_conv", "kda_backward_workspace_size", "kda_backward")
+                    "kda_decode_step_conv", "kda_backward_workspace_size", "kda_backward",
+                    "kda_set_wait_limit_ns")
 
 
 class OutputGate(ctypes.Structure):
@@ -109,6 +110,8 @@ def load_library():
     lib.kda_backward.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32, i32, ctypes.c_int, i32, u32,
                                  vp, fp, fp, fp, fp, fp, fp, fp, vp, sz, vp]
     lib.kda_backward.restype = ctypes.c_int
+    lib.kda_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.kda_set_wait_limit_ns.restype = ctypes.c_uint64
     _lib = lib
     return lib
 
@@ -126,6 +129,12 @@ def kda_device_error(reset: bool = True) -> int:
     code = ctypes.c_int32(0)
     load_library().kda_device_error(ctypes.byref(code), int(bool(reset)))
     return int(code.value)
+
+
+def kda_set_wait_limit_ns(ns: int) -> int:
+    """Bound (ns) of the prefill's waits between CTAs for later calls; 0 = default (2 s).
+    Returns the previous bound (``kda_set_wait_limit_ns`` in ``include/kda.h``)."""
+    return int(load_library().kda_set_wait_limit_ns(int(ns)))
 
 
 def _dtype_code(t: torch.Tensor) -> int:

@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "kda_internal.cuh"
 
@@ -123,17 +124,49 @@ namespace kda {
 
 __device__ int g_device_error;  // set by kernels whose bounded waits ran out
 
-int *device_error_word() {
-    // One word per device; its address is resolved for the current device.
-    static int *addr[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
+namespace {
+// cuCtxGetCurrent / cuCtxGetId through the runtime's driver entry points (no
+// libcuda link): the identity of the current context, unique for the life of
+// the process, so a cached device address is re-resolved after the device's
+// context was destroyed and recreated (cudaDeviceReset).
+typedef int (*PfnCtxGetCurrent)(void **);
+typedef int (*PfnCtxGetId)(void *, unsigned long long *);
+bool context_id(unsigned long long *id) {
+    static PfnCtxGetCurrent get_current = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-        addr[dev] = static_cast<int *>(p);
-    }
-    return addr[dev];
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PfnCtxGetCurrent>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PfnCtxGetId>(p);
+    });
+    void *ctx = nullptr;
+    return get_current && get_id && get_current(&ctx) == 0 && ctx && get_id(ctx, id) == 0;
+}
+}  // namespace
+
+void *symbol_address(const void *symbol, SymbolCache &cache) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= SymbolCache::kMaxDevices) return nullptr;
+    unsigned long long ctx = 0;
+    std::lock_guard<std::mutex> lock(cache.mu);
+    if (context_id(&ctx) && cache.addr[dev] && cache.ctx[dev] == ctx) return cache.addr[dev];
+    // (the runtime makes the device's primary context current here if it is not yet)
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess || !p) return nullptr;
+    cache.addr[dev] = p;
+    cache.ctx[dev] = context_id(&ctx) ? ctx : 0;  // 0: never matches, resolved on every call
+    return p;
+}
+
+int *device_error_word() {
+    static SymbolCache cache;
+    return static_cast<int *>(symbol_address(reinterpret_cast<const void *>(&g_device_error), cache));
 }
 
 }  // namespace kda
@@ -271,6 +304,8 @@ kda_status kda_device_error(int32_t *code, int32_t reset) {
     *code = v;
     return v == 0 ? KDA_OK : KDA_ERR_TIMEOUT;
 }
+
+uint64_t kda_set_wait_limit_ns(uint64_t ns) { return kda::tc_set_wait_limit(ns); }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                            const float *beta, float *S, int32_t N, int32_t H, int32_t dk,

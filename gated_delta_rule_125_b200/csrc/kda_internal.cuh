@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "kda.h"
 
 namespace kda {
@@ -70,6 +72,21 @@ size_t tc_workspace_bytes(long long NH, int ns, int R);   // NH = N * H units
 int tc_ring_slots(long long NH, int ns, size_t bytes);   // R for a workspace (capped)
 int tc_max_ring();
 cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, int *err, cudaStream_t st);
+// Bound of the tensor-core prefill's waits between CTAs (ns), for calls enqueued from now on.
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+uint64_t tc_set_wait_limit(uint64_t ns);
+
+// Device address of a __device__ variable in the current device's context,
+// resolved with cudaGetSymbolAddress on the first use in that context (with the
+// device current) and cached per device; a new context on the device (after
+// cudaDeviceReset) resolves it again. nullptr if it cannot be resolved.
+struct SymbolCache {
+    static constexpr int kMaxDevices = 64;
+    std::mutex mu;
+    unsigned long long ctx[kMaxDevices] = {};
+    void *addr[kMaxDevices] = {};
+};
+void *symbol_address(const void *symbol, SymbolCache &cache);
 
 // Address of this device's error word (set by kernels whose bounded waits ran
 // out), or nullptr if it cannot be resolved.

@@ -17,8 +17,6 @@
 // prefill's own planning kernel clears at the start of every call. Calls that overlap
 // on the GPU (different streams, or several host threads) race on the array
 // and give wrong results; the caller must order them.
-#include <mutex>
-
 #include "kda_internal.cuh"
 
 namespace {
@@ -27,22 +25,13 @@ constexpr size_t kNoAllocScratchBytes = size_t(KDA_NOALLOC_SCRATCH_BYTES);
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void *g_noalloc_addr[kMaxDevices] = {};
+kda::SymbolCache g_noalloc_cache;
 
-// Device address of the scratch array on the current device. Resolved once per
-// device, with that device current, on the first call made on it.
+// Device address of the scratch array on the current device: resolved with
+// cudaGetSymbolAddress, with that device current, on the first call made in
+// the device's context, then cached (resolved again for a new context).
 void *noalloc_scratch() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return nullptr;
-        g_noalloc_addr[dev] = p;
-    }
-    return g_noalloc_addr[dev];
+    return kda::symbol_address(reinterpret_cast<const void *>(&g_noalloc_scratch), g_noalloc_cache);
 }
 
 }  // namespace

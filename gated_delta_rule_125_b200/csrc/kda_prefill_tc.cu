@@ -32,6 +32,7 @@
 #include <cudaTypedefs.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "kda_internal.cuh"
@@ -48,7 +49,7 @@ constexpr int DK = 128;
 constexpr int DV = 128;
 constexpr int DVT = 64;                      // state columns per scan CTA
 constexpr float kTau = 60.f;                 // largest per-chunk decay range for the factorised Gram
-constexpr uint64_t kWaitNs = 2000000000ull;  // bound of every device-side wait (2 s)
+constexpr uint64_t kWaitNs = kDefaultWaitNs;  // bound of a CTA's waits for its own copies and products (2 s)
 constexpr int kThreads = 512;                // per CTA: two prep engines, or one scan CTA
 constexpr int kMaxRing = 16;                 // ring slots per stream, upper bound (~34 MB at 32 streams)
 
@@ -102,6 +103,7 @@ struct FusedParams {
     char *ws;
     int *err;
     long long total;  // tokens
+    unsigned long long xwait_ns;  // bound of the waits between CTAs (ring flags, row-sum exchange)
     int N, H, ns, R, l2norm, la_scalar;
     float eps;
 };
@@ -115,16 +117,29 @@ __device__ __forceinline__ void fail_call(const FusedParams &P) {
     atomicExch(&hd->abort_flag, 1);
     flag_error(P.err, 1);
 }
-// Wait until *flag >= target (gpu-scope acquire); false on abort or after kWaitNs.
-// Polls every `sleep_ns` (0: back to back, for waits expected to be short).
+// Wait until *flag >= target (gpu-scope acquire), a flag another CTA sets; false on
+// abort or after `limit_ns`. Polls every `sleep_ns` (0: back to back, for waits
+// expected to be short).
 __device__ __forceinline__ bool wait_flag_geq(const int *flag, int target, const int *abort_flag,
-                                              unsigned sleep_ns = 100) {
+                                              uint64_t limit_ns, unsigned sleep_ns = 100) {
     if (ld_acquire_gpu(flag) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (sleep_ns) __nanosleep(sleep_ns);
         if (ld_acquire_gpu(flag) >= target) return true;
-        if (ld_relaxed_gpu(abort_flag) || globaltimer_ns() - t0 > kWaitNs) return false;
+        if (ld_relaxed_gpu(abort_flag) || globaltimer_ns() - t0 > limit_ns) return false;
+    }
+}
+// mbarrier wait of a scan thread on another thread of its CTA: like mbar_wait
+// (bound kWaitNs), and it also gives up once the call's abort flag is set, so a
+// failed call ends within microseconds. Not for a CTA's own copies and products
+// in flight: those are always waited for (bounded) before the CTA exits.
+__device__ __forceinline__ bool mbar_wait_call(uint64_t *bar, uint32_t parity, const int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((n & 31) == 0 && (ld_relaxed_gpu(abort_flag) || globaltimer_ns() - t0 > kWaitNs)) return false;
     }
 }
 
@@ -438,7 +453,8 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             // have released its previous generation.
             if (!slot_ok) {
                 publish_prev(prev);
-                if (!wait_flag_geq(&freed[slot_index(cur)], 2 * (int)(cur.p / R), &hd->abort_flag)) sflag[1] = 1;
+                if (!wait_flag_geq(&freed[slot_index(cur)], 2 * (int)(cur.p / R), &hd->abort_flag, P.xwait_ns))
+                    sflag[1] = 1;
             }
             slot_ok = false;
         }
@@ -855,8 +871,8 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 // buffers: free one position before the A group's two), then A.
                 const int ab = (int)(p & 1), bb = (int)(p % 3);
                 const int slot = st * R + (int)(p % R);
-                ok = wait_flag_geq(&ready[slot], (int)(p / R) + 1, &hd->abort_flag, 32);
-                if (ok && p >= 3) ok = mbar_wait(&emptyB[bb], (uint32_t)((p / 3 - 1) & 1), kWaitNs);
+                ok = wait_flag_geq(&ready[slot], (int)(p / R) + 1, &hd->abort_flag, P.xwait_ns, 32);
+                if (ok && p >= 3) ok = mbar_wait_call(&emptyB[bb], (uint32_t)((p / 3 - 1) & 1), &hd->abort_flag);
                 if (!ok) break;
                 fence_proxy_async_global();
                 const char *g = ring + (size_t)slot * SL_BYTES;
@@ -866,7 +882,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 bulk_g2s(B + SB_P, g + SL_P, 8192, &fullB[bb]);
                 bulk_g2s(B + SB_D, g + SL_D, 512, &fullB[bb]);
                 nB = p + 1;
-                if (p >= 2) ok = mbar_wait(&emptyA[ab], (uint32_t)((p / 2 - 1) & 1), kWaitNs);
+                if (p >= 2) ok = mbar_wait_call(&emptyA[ab], (uint32_t)((p / 2 - 1) & 1), &hd->abort_flag);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&fullA[ab], COPY_A);
                 bulk_g2s(A + SA_WQ, g + SL_WQ, 32768, &fullA[ab]);
@@ -921,7 +937,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             const long long nch = (eos - bos + C - 1) / C;
             for (long long j = 0; j < nch; ++j, ++p) {
                 const int vb = (int)(p & 3);
-                if (p >= 4) ok = mbar_wait(&emptyV[vb], (uint32_t)((p / 4 - 1) & 1), kWaitNs);
+                if (p >= 4) ok = mbar_wait_call(&emptyV[vb], (uint32_t)((p / 4 - 1) & 1), &hd->abort_flag);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&fullV[vb], SV_BYTES);
                 tma_load_3d(sm + SS_V + vb * SV_BYTES, &P.tmap_v, jv * DVT, h, (int)(bos + j * C), &fullV[vb]);
@@ -947,8 +963,8 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         // X[q & 1] = [filler ; T] V of position q, once its T and V tiles are in.
         auto issue_x = [&](long long q) {
             const int bb = (int)(q % 3), vb = (int)(q & 3);
-            if (!(mbar_wait(&fullB[bb], (uint32_t)((q / 3) & 1), kWaitNs) &&
-                  mbar_wait(&fullV[vb], (uint32_t)((q >> 2) & 1), kWaitNs)))
+            if (!(mbar_wait_call(&fullB[bb], (uint32_t)((q / 3) & 1), &hd->abort_flag) &&
+                  mbar_wait_call(&fullV[vb], (uint32_t)((q >> 2) & 1), &hd->abort_flag)))
                 return false;
             tc_fence_after();
 #pragma unroll
@@ -963,7 +979,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         for (long long p = 0; p < L && ok; ++p) {
             const int ab = (int)(p & 1), bb = (int)(p % 3);
             const uint32_t yb = (uint32_t)(p % NY) * 64;
-            ok = mbar_wait(&fullA[ab], (uint32_t)((p >> 1) & 1), kWaitNs);
+            ok = mbar_wait_call(&fullA[ab], (uint32_t)((p >> 1) & 1), &hd->abort_flag);
             if (!ok) break;
             // Both tile groups of position p are in shared memory (B was waited for
             // with X(p)): its ring slot can be released.
@@ -971,8 +987,8 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             *consumed = p + 1;
             // S(p) in smem, and O(p - NY) read out of Y[p % NY] (one barrier per Y buffer: it
             // completes for positions p % NY, p % NY + NY, ... and so never runs two ahead)
-            ok = mbar_wait(sready, (uint32_t)(p & 1), kWaitNs) &&
-                 (p < NY || mbar_wait(&oready[p % NY], (uint32_t)((p / NY + 1) & 1), kWaitNs));
+            ok = mbar_wait_call(sready, (uint32_t)(p & 1), &hd->abort_flag) &&
+                 (p < NY || mbar_wait_call(&oready[p % NY], (uint32_t)((p / NY + 1) & 1), &hd->abort_flag));
             if (!ok) break;
             if (p >= 1) mbar_arrive(&emptyB[(p - 1) % 3]);  // e^{Gl} of p-1 has been read
             tc_fence_after();
@@ -982,7 +998,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             for (int s8 = 0; s8 < DK / 16; ++s8)
                 mma_bf16(tm + TM_Y + yb, dWQa + kmaj_step(s8, 128), dS + mnmaj_step(s8), id128, s8 > 0);
             mma_commit(bU);
-            ok = mbar_wait(uready, (uint32_t)(p & 1), kWaitNs);  // U(p) in smem
+            ok = mbar_wait_call(uready, (uint32_t)(p & 1), &hd->abort_flag);  // U(p) in smem
             if (!ok) break;
             tc_fence_after();
             // Z = Kd^T U first (the state chain), then O: Y += [P ; filler] U
@@ -1032,7 +1048,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 const uint32_t ybuf = tm + TM_Y + (uint32_t)(p % NY) * 64 + lane_base;
                 // one bO barrier per Y buffer: it completes for positions p % NY, p % NY + NY, ...
                 // (the MMA thread may run up to NY - 1 positions ahead of these warps)
-                ok = __all_sync(0xffffffffu, mbar_wait(&bO[p % NY], (uint32_t)((p / NY) & 1), kWaitNs));
+                ok = __all_sync(0xffffffffu, mbar_wait_call(&bO[p % NY], (uint32_t)((p / NY) & 1), &hd->abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 const long long nn = (len - j * C) < C ? (len - j * C) : C;
@@ -1061,7 +1077,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                     if ((got >> 32) != (tag >> 32)) {
                         const uint64_t t0 = globaltimer_ns();
                         while (((got = ld_relaxed_gpu_u64(pw)) >> 32) != (tag >> 32))
-                            if (globaltimer_ns() - t0 > kWaitNs || ld_relaxed_gpu(&hd->abort_flag)) break;
+                            if (globaltimer_ns() - t0 > P.xwait_ns || ld_relaxed_gpu(&hd->abort_flag)) break;
                     }
                     ok = __all_sync(0xffffffffu, (got >> 32) == (tag >> 32));
                     if (!ok) break;
@@ -1155,7 +1171,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             const uint32_t par = (uint32_t)(p & 1);
             if (q4 >= 2) {
                 // U = T V - W S for rows r = c - 64 (TMEM lanes 64..127)
-                ok = __all_sync(0xffffffffu, mbar_wait(bU, par, kWaitNs));
+                ok = __all_sync(0xffffffffu, mbar_wait_call(bU, par, &hd->abort_flag));
                 if (!ok) break;
                 tc_fence_after();
                 float xv[32], yv[32];
@@ -1174,8 +1190,8 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 mbar_arrive(uready);
             }
             // S' = Diag(e^{G_last}) S + Z  (row c)
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(bS, par, kWaitNs) && mbar_wait(&fullB[p % 3], (uint32_t)((p / 3) & 1), kWaitNs));
+            ok = __all_sync(0xffffffffu, mbar_wait_call(bS, par, &hd->abort_flag) &&
+                                             mbar_wait_call(&fullB[p % 3], (uint32_t)((p / 3) & 1), &hd->abort_flag));
             if (!ok) break;
             tc_fence_after();
             const float dc = reinterpret_cast<const float *>(sm + SS_B + (p % 3) * SB_BYTES + SB_D)[c];
@@ -1307,6 +1323,11 @@ int tc_ring_slots(long long NH, int ns, size_t bytes) {
 
 int tc_max_ring() { return kMaxRing; }
 
+namespace {
+std::atomic<unsigned long long> g_xwait_ns{kDefaultWaitNs};
+}
+uint64_t tc_set_wait_limit(uint64_t ns) { return g_xwait_ns.exchange(ns ? ns : kDefaultWaitNs); }
+
 cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, int *err, cudaStream_t st) {
     cudaError_t e;
     // Per device (context): cheap enough to set on every call.
@@ -1347,6 +1368,7 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
     P.ws = ws;
     P.err = err;
     P.total = a.total;
+    P.xwait_ns = g_xwait_ns.load();
     P.N = a.N;
     P.H = a.H;
     P.ns = ns;

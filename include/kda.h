@@ -199,6 +199,22 @@ kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v, cons
 kda_status kda_device_error(int32_t *code, int32_t reset);
 
 /*
+ * Bound, in nanoseconds, of the waits between the CTAs of a tensor-core
+ * prefill, for every call enqueued after it (any host thread): a scan CTA
+ * waiting for a prepared chunk, a preparing CTA waiting for a free ring slot,
+ * and the two scan CTAs of a stream exchanging the fused output step's row
+ * sums. When one runs out the call abandons its work within microseconds (the
+ * kernel returns; its outputs are not valid) and kda_device_error() reports
+ * code 1 (KDA_ERR_TIMEOUT). A watchdog setting: the default, 2 s, is far above
+ * any normal wait; a bound shorter than the time a prefill takes to prepare
+ * its first chunk (tens of microseconds) makes every call fail. The waits for
+ * a CTA's own copies and tensor-core products keep the 2 s bound. ns = 0
+ * restores the default. Returns the previous bound. Not a per-stream setting:
+ * calls already enqueued keep the bound they were enqueued with.
+ */
+uint64_t kda_set_wait_limit_ns(uint64_t ns);
+
+/*
  * One decode step for N independent sequences, state updated in place
  * ("[Kimi-2] Kimi Linear" §5: S_(t-1) + current token -> S_t + output).
  *
@@ -297,7 +313,12 @@ kda_status kda_decode_step_conv(const void *q, const void *k, const void *v, con
  *   grad_q, grad_k        [T][H][dk] fp32 out;  grad_v [T][H][dv] fp32 out
  *   grad_log_alpha        [T][H][dk] fp32 out;  grad_beta [T][H] fp32 out
  *   grad_S0               [N][H][dk][dv] fp32 out, or NULL (not written)
- *   workspace    kda_backward_workspace_size() bytes, 16-byte aligned
+ *   workspace    kda_backward_workspace_size() bytes, 16-byte aligned: fp32 scratch of
+ *                about (11 C dk + 9 C^2 + 3 C dv + 2 dk dv) * 4 bytes (C = 64; 737 KB
+ *                at dk = dv = 128) for each of N * H * ceil(L / 64) chunk slots,
+ *                L = max_seqlen (total_tokens when max_seqlen <= 0), plus about
+ *                (4 dk + 2) * 4 bytes per (token, head): 3.0 GB + 0.5 GB for one sequence of
+ *                8192 tokens and 32 heads (3.6 GB). Pass max_seqlen for varlen batches.
  *
  * fp32 CUDA-core arithmetic (a reference-grade implementation; five
  * launches). It factors e^{G_r - G_i} = e^{G_r} e^{-G_i} inside each chunk:

@@ -653,6 +653,7 @@ def _bw_inputs(lengths, H, d, dtype, seed):
 
 
 def _bw_check(got, inp, do, dST, l2norm=True, label=""):
+    assert kda.kda_device_error(reset=True) == 0, label  # no chunk flagged, no wait ran out
     ref = oracle.backward(host(inp["q"]), host(inp["k"]), host(inp["v"]), host(inp["log_alpha"]),
                           host(inp["beta"]), host(do), None if dST is None else host(dST), host(inp["S0"]),
                           inp["cu_seqlens"].cpu().numpy(), l2norm=l2norm)
@@ -688,3 +689,16 @@ def test_backward_rejects_scalar_gate():
     la = inp["log_alpha"][..., 0].contiguous()
     with pytest.raises(kda.KDAError):
         kda.kda_backward(inp["q"], inp["k"], inp["v"], la, inp["beta"], do, dST, inp["S0"], inp["cu_seqlens"])
+
+
+def test_backward_flags_strong_decay():
+    """A chunk whose decay range exceeds 60 nats (log_alpha about -1.5 per token, 64 rows)
+    is not computed by the factorised backward: it sets device error code 2."""
+    inp, do, dST = _bw_inputs([100], 1, 64, torch.float32, seed=54)
+    inp["log_alpha"] = torch.full_like(inp["log_alpha"], -1.5)
+    assert kda.kda_device_error(reset=True) == 0
+    kda.kda_backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], do, dST, inp["S0"],
+                     inp["cu_seqlens"], max_seqlen=100)
+    torch.cuda.synchronize()
+    assert kda.kda_device_error(reset=True) == 2
+    assert kda.kda_device_error(reset=True) == 0
