@@ -215,12 +215,13 @@ constexpr uint32_t PS_GB = PS_GA + 32768;      // q of the next item, then K e^-
 constexpr uint32_t PS_KS = PS_GB + 16384;      // k of the next item (K-major 64 x 128)
 constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[2][64] eGl[128] gate[2][64]
 constexpr uint32_t PS_BAR = PS_SMALL + 2048;   // la, mma, q/k barriers; 3 item records; flags
-constexpr uint32_t PS_BYTES = PS_BAR + 128;
+constexpr uint32_t PS_BYTES = PS_BAR + 256;
 constexpr uint32_t PS_STRIDE = 101376;         // engine 1 starts here (1024-aligned)
 constexpr int ALD = 68;                        // row stride of A / X (floats)
 constexpr uint32_t PS_AF = PS_LA;              // A, then X in place: 64 x 68 fp32
-constexpr uint32_t PS_R2 = PS_LA + 17408;      // solve scratch, 4 KB
-constexpr uint32_t PS_T = PS_LA + 21504;       // T, 64 x 64 bf16 K-major (1024-aligned)
+constexpr uint32_t PS_T = PS_LA + 17408;       // T, 64 x 64 bf16 K-major (1024-aligned)
+constexpr uint32_t PS_R2 = PS_LA + 25600;      // solve scratch: 32 x R2LD fp32
+constexpr int R2LD = 36;
 static_assert(PS_BYTES <= PS_STRIDE, "prep engine layout");
 
 // Scan CTA: the tiles of a chunk from its ring slot: A (WQ, KD) double-buffered,
@@ -237,7 +238,7 @@ constexpr uint32_t SS_U = SS_S + 16384;         // [64 (r)][64 (j)] MN-major bf1
 constexpr uint32_t SS_BAR = SS_U + 8192;        // 31 mbarriers, the consumed-position counter, a flag
 constexpr uint32_t SS_OGW = SS_BAR + 512;       // output-step weights of this CTA's 64 columns
 constexpr uint32_t SS_BYTES = SS_OGW + 256;
-constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 512;
+constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 1024;
 constexpr int NY = 4;  // Y buffers in TMEM: the O epilogue may lag NY - 1 chunks
 constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = TM_Y + 64 * NY;  // scan TMEM columns: X x2, Y x NY, Z
 static_assert(TM_Z + 64 <= 512, "scan TMEM columns");
@@ -251,12 +252,17 @@ constexpr int MB_FULLA = 0, MB_FULLB = 2, MB_FULLV = 5, MB_EMPTYA = 9, MB_EMPTYB
 struct Ctrl {
     uint32_t tbase;
     int uniform;
+    int ucache, ccache;  // the unit starts / the sequence bounds are cached in shared memory
     long long total, maxlen;
     long long L[kTcMaxStreams];
     int order[kTcMaxStreams];
 };
 constexpr uint32_t CTRL_OFF = SS_BYTES > 2 * PS_STRIDE ? SS_BYTES : 2 * PS_STRIDE;
-constexpr uint32_t SMEM_ALLOC = CTRL_OFF + 512 + 1024;  // + alignment slack
+// Prep CTAs cache each unit's first position in its stream and the sequence bounds
+// (when they fit), so that mapping a claimed item to its chunk costs no global loads.
+constexpr int kUnitCache = 2048, kSeqCache = 1025;
+constexpr uint32_t CACHE_OFF = CTRL_OFF + 512;
+constexpr uint32_t SMEM_ALLOC = CACHE_OFF + 4 * (kUnitCache + kSeqCache) + 1024;  // + alignment slack
 static_assert(2 * PS_STRIDE <= CTRL_OFF, "prep engines overlap the control block");
 static_assert(MB_O + NY == MB_UREADY && MB_OREADY + NY == MB_COUNT, "scan barrier indices");
 static_assert(MB_COUNT * 8 + 16 <= SS_OGW - SS_BAR, "scan barrier area");
@@ -266,8 +272,9 @@ static_assert(sizeof(Ctrl) <= 512, "control block");
 struct ItemS {
     long long t0, p;  // first token; position in the stream
     int n, h, st, valid;
+    int slot, gen;
 };
-static_assert(3 * 8 + 3 * sizeof(ItemS) + 2 * 4 <= PS_BYTES - PS_BAR, "prep barrier block");
+
 
 // Item g of the global claim order: position-major over the streams still
 // running at that position, longest streams first.
@@ -276,9 +283,9 @@ __device__ bool map_item(unsigned long long g, const FusedParams &P, const Ctrl 
     const int ns = P.ns;
     long long p;
     int i;
-    if (ctl->uniform) {
-        p = (long long)(g / (unsigned long long)ns);
-        i = (int)(g % (unsigned long long)ns);
+    if (ctl->uniform) {  // item indices, positions and units fit in 32 bits (checked on the host)
+        p = (long long)((unsigned)g / (unsigned)ns);
+        i = (int)((unsigned)g % (unsigned)ns);
     } else {
         // largest p with sum_st min(L_st, p) <= g
         long long lo = 0, hi = ctl->maxlen - 1;
@@ -297,29 +304,38 @@ __device__ bool map_item(unsigned long long g, const FusedParams &P, const Ctrl 
     const int st = ctl->order[i];
     const long long NH = (long long)P.N * P.H;
     const long long *ustart = reinterpret_cast<const long long *>(P.ws + WS_USTART);
-    long long lo = 0, hi = (NH - st + ns - 1) / ns - 1;  // last unit of the stream starting at or before p
+    const int *uc = reinterpret_cast<const int *>(reinterpret_cast<const uint8_t *>(ctl) + 512);
+    long long lo = 0, hi = (long long)(((unsigned)(NH - st) + (unsigned)ns - 1u) / (unsigned)ns) - 1;  // last unit of the stream starting at or before p
     while (lo < hi) {
         const long long mid = (lo + hi + 1) >> 1;
-        if (ustart[st + mid * ns] <= p) lo = mid;
+        const long long us = ctl->ucache ? (long long)uc[st + mid * ns] : ustart[st + mid * ns];
+        if (us <= p) lo = mid;
         else hi = mid - 1;
     }
     const long long u = st + lo * ns;
-    const long long j = p - ustart[u];
+    const long long j = p - (ctl->ucache ? (long long)uc[u] : ustart[u]);
     int64_t bos, eos;
-    seq_bounds(P.cu, (int)(u / P.H), P.total, bos, eos);
+    const int s = (int)((unsigned)u / (unsigned)P.H);
+    if (ctl->ccache) {
+        bos = uc[kUnitCache + s];
+        eos = uc[kUnitCache + s + 1];
+    } else {
+        seq_bounds(P.cu, s, P.total, bos, eos);
+    }
     it.t0 = bos + j * C;
     it.n = (int)((eos - it.t0) < C ? (eos - it.t0) : C);
-    it.h = (int)(u % P.H);
+    it.h = (int)((unsigned)u % (unsigned)P.H);
     it.st = st;
     it.p = p;
+    it.slot = st * P.R + (int)((unsigned)p % (unsigned)P.R);
+    it.gen = (int)((unsigned)p / (unsigned)P.R);
     return true;
 }
 
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+// An fp32 value rounded to tf32 (10 stored significand bits), to nearest with ties away
+// from zero, done on the bit pattern (finite inputs): the operand format of the tf32
+// mma.sync below.
+__device__ __forceinline__ uint32_t tf32_bits(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
 // D (16x8) += A (16x8, row-major) x B (8x8) with tf32 operands, fp32 accumulation.
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
     asm volatile(
@@ -327,23 +343,26 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// One warp: C[16 x 8] = A[16 x K] B[K x 8] for A(r, k), B(k, n) given as functors;
-// the result is handed back through `out(r, n, value)`.
-template <int K, typename FA, typename FB, typename FO>
-__device__ __forceinline__ void warp_gemm_16x8(int lane, FA A, FB B, FO out) {
+// One warp: C[16 x 8] = A[16 x K] B[K x 8] for A(r, k), B(k, n) given as functors (every
+// operand is read first, then the K / 8 products run back to back). The result stays in
+// the accumulator layout: acc = C(g, 2t), C(g, 2t+1), C(g+8, 2t), C(g+8, 2t+1) for lane
+// 4g + t.
+template <int K, typename FA, typename FB>
+__device__ __forceinline__ void warp_gemm_16x8(int lane, FA A, FB B, float (&acc)[4]) {
     const int g = lane >> 2, t = lane & 3;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t a[K / 8][4], b[K / 8][2];
 #pragma unroll
     for (int ks = 0; ks < K / 8; ++ks) {
-        const uint32_t a[4] = {to_tf32(A(g, 8 * ks + t)), to_tf32(A(g + 8, 8 * ks + t)),
-                               to_tf32(A(g, 8 * ks + t + 4)), to_tf32(A(g + 8, 8 * ks + t + 4))};
-        const uint32_t b[2] = {to_tf32(B(8 * ks + t, g)), to_tf32(B(8 * ks + t + 4, g))};
-        mma_tf32(acc, a, b);
+        a[ks][0] = tf32_bits(A(g, 8 * ks + t));
+        a[ks][1] = tf32_bits(A(g + 8, 8 * ks + t));
+        a[ks][2] = tf32_bits(A(g, 8 * ks + t + 4));
+        a[ks][3] = tf32_bits(A(g + 8, 8 * ks + t + 4));
+        b[ks][0] = tf32_bits(B(8 * ks + t, g));
+        b[ks][1] = tf32_bits(B(8 * ks + t + 4, g));
     }
-    out(g, 2 * t, acc[0]);
-    out(g, 2 * t + 1, acc[1]);
-    out(g + 8, 2 * t, acc[2]);
-    out(g + 8, 2 * t + 1, acc[3]);
+    acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < K / 8; ++ks) mma_tf32(acc, a[ks], b[ks]);
 }
 
 // Prep engine e (threads 256 e .. 256 e + 255) with its shared memory `sm` and
@@ -377,7 +396,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     uint32_t la_phase = 0, mma_phase = 0, qk_phase = 0;
     const int c8 = tid & 15, rb = tid >> 4;  // thread's 16-byte channel chunk and first row
 
-    auto slot_index = [&](const ItemS &it) { return it.st * R + (int)(it.p % R); };
+
     // Thread 128 claims items, issues the slot's bulk stores (bulk groups belong
     // to the issuing thread) and the log_alpha boxes, and publishes each item:
     // after the item's generic slot stores (ordered before it by the engine's
@@ -394,11 +413,11 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         if (!prev_pending) return;
         bulk_wait_all();
         fence_proxy_async_global();
-        st_release_gpu(&ready[slot_index(pv)], (int)(pv.p / R) + 1);
+        st_release_gpu(&ready[pv.slot], pv.gen + 1);
         prev_pending = false;
     };
     auto slot_free = [&](const ItemS &it) {
-        return ld_acquire_gpu(&freed[slot_index(it)]) >= 2 * (int)(it.p / R);
+        return ld_acquire_gpu(&freed[it.slot]) >= 2 * it.gen;
     };
     auto claim = [&](ItemS &it) {
         it.valid = 0;
@@ -445,7 +464,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         ItemS &next = sitem[(iter + 1) % 3];
         const ItemS &prev = sitem[(iter + 2) % 3];
         const int n = cur.n;
-        char *gslot = ring + (size_t)slot_index(cur) * SL_BYTES;
+        char *gslot = ring + (size_t)cur.slot * SL_BYTES;
         const float *sbeta = sbeta2 + (iter & 1) * 64;
         if (tid == kStoreTid) {
             bulk_wait_read();  // the previous item's bulk stores no longer read GA
@@ -453,7 +472,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             // have released its previous generation.
             if (!slot_ok) {
                 publish_prev(prev);
-                if (!wait_flag_geq(&freed[slot_index(cur)], 2 * (int)(cur.p / R), &hd->abort_flag, P.xwait_ns))
+                if (!wait_flag_geq(&freed[cur.slot], 2 * cur.gen, &hd->abort_flag, P.xwait_ns))
                     sflag[1] = 1;
             }
             slot_ok = false;
@@ -542,7 +561,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     pq[w] = pack_bf16(q0 * ep0, q1 * ep1);
                     pk[w] = pack_bf16(k0 * ep0, k1 * ep1);
                     pn[w] = pack_bf16(n0, n1);
-                    pd[w] = pack_bf16(n0 * d.x, n1 * d.y);
+                    pd[w] = pn[w];  // the slot carries K e^-G; the scan scales by DZ
                 }
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -568,7 +587,10 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                 *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = pack8(kd);
             }
         }
-        if (tid < DK) reinterpret_cast<float *>(gslot + SL_D)[tid] = eGl[tid];
+        if (tid < DK) {
+            reinterpret_cast<float *>(gslot + SL_D)[tid] = eGl[tid];
+            reinterpret_cast<float *>(gslot + SL_D)[DK + tid] = safe ? eGl[tid] : 1.f;
+        }
         fence_async_smem();
         tc_fence_before();
         sync();
@@ -584,7 +606,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     mma_bf16(tm, kmaj_desc(a, s8, 128), kmaj_desc(b, s8, 64), idg, s8 > 0);
                 mma_commit(&bars[1]);
             }
-            if (tid == kStoreTid) {
+            if (tid == kStoreTid + 32) {  // another warp than the store thread's
                 claim(next);
                 if (next.valid && !P.la_scalar) tma_prefetch_3d(&P.tmap_la, 0, next.h, (int)next.t0);
             }
@@ -627,7 +649,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(rr, c8, 128)) = pack8(x);
             }
             fence_async_smem();
-            if (tid == kStoreTid) claim(next);
+            if (tid == kStoreTid + 32) claim(next);
             sync();  // G is overwritten by A below
         }
         if (tid == 0) sflag[0] = 0;
@@ -672,44 +694,43 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             if (next.valid) slot_ok = slot_free(next);
         }
 
-        // 5. In place, AF (A) becomes X = (I + Diag(beta) A)^{-1}: diagonal 16x16 blocks by
-        //    forward substitution, then the 2x2 block recursion with tf32 tensor-core products:
-        //    [X11 0; X21 X22] with X21 = -X22 (Diag(beta_2) A21) X11, written over A21 once
-        //    A21 is consumed. Each block of T = X Diag(beta) (bf16, the A operand of W and the
-        //    slot's T tile) is written as its X block is produced: the diagonal blocks and the
-        //    zero upper blocks by warps 4..7 while warps 0..3 run the 16-row level.
-        auto t_store = [&](int r, int c, float xv) {
-            *reinterpret_cast<bf16 *>(TT + kmaj_off(r, c, 64)) = __float2bfloat16_rn(xv * sbeta[c]);
-        };
-        {
-            float x[16];
-            const int b = tid >> 4, cc = tid & 15;
-            if (tid < C) {
+        // 5. X = (I + Diag(beta) A)^{-1}, in place over A (fp32), and T = X Diag(beta) (bf16,
+        //    the A operand of W and the slot's T tile), by 16 x 16 blocks.
+        //    Level 0, warps 0..3: diagonal block b = warp by a right-looking forward
+        //    substitution in registers, one column per lane (lanes 16..31 repeat 0..15):
+        //    after x_i is known, its term is added to every later row's sum at once, so the
+        //    dependent chain is one multiply-add per row. Warps 4..7: T's zero upper blocks.
+        if (warp < 4) {
+            const int r0 = 16 * warp, cc = lane & 15;
+            float x[16], acc[16];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int r = 16 * b + rr;
-                    float acc = 0.f;
+            for (int r = 0; r < 16; ++r) acc[r] = 0.f;
 #pragma unroll
-                    for (int ii = 0; ii < rr; ++ii) acc += AF[r * ALD + 16 * b + ii] * x[ii];
-                    x[rr] = (rr == cc) ? 1.f : (rr > cc ? -sbeta[r] * acc : 0.f);
-                }
-            } else if (tid >= 128) {
-                // upper blocks (bi, bj), bj > bi: 6 blocks x 16 rows x 2 chunks of 8 columns
-                for (int i = tid - 128; i < 6 * 16 * 2; i += 128) {
-                    const int blk = i >> 5, rr = (i >> 1) & 15, half = i & 1;
-                    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                    *reinterpret_cast<uint4 *>(TT + kmaj_chunk(16 * bi + rr, 2 * bj + half, 64)) = make_uint4(0, 0, 0, 0);
-                }
+            for (int i = 0; i < 16; ++i) {
+                x[i] = (i == cc) ? 1.f : (i > cc ? -sbeta[r0 + i] * acc[i] : 0.f);
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) acc[r] = fmaf(AF[(r0 + r) * ALD + r0 + i], x[i], acc[r]);
             }
-            sync();  // every diagonal block of A has been read
-            if (tid < C) {
+            __syncwarp();  // every lane has read the block
+            if (lane < 16) {
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) AF[(16 * b + rr) * ALD + 16 * b + cc] = x[rr];
+                for (int r = 0; r < 16; ++r) AF[(r0 + r) * ALD + r0 + cc] = x[r];
+            }
+        } else {
+            // upper blocks (bi, bj), bj > bi: 6 blocks x 16 rows x 2 chunks of 8 columns
+            for (int i = tid - 128; i < 6 * 16 * 2; i += 128) {
+                const int blk = i >> 5, rr = (i >> 1) & 15, half = i & 1;
+                const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+                const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                *reinterpret_cast<uint4 *>(TT + kmaj_chunk(16 * bi + rr, 2 * bj + half, 64)) = make_uint4(0, 0, 0, 0);
             }
         }
         sync();
-        // 16-row level: warps 0, 1 build X[16..31][0..15], warps 2, 3 X[48..63][32..47] (8-column halves).
+        // T's element pair (r, c), (r, c + 1) from X's, scaled by beta of the columns.
+        auto t_store2 = [&](int r, int c, float x0, float x1) {
+            *reinterpret_cast<uint32_t *>(TT + kmaj_off(r, c, 64)) = pack_bf16(x0 * sbeta[c], x1 * sbeta[c + 1]);
+        };
+        const int fg = lane >> 2, ft = lane & 3;  // accumulator layout of the tf32 products
         if (warp >= 4) {
             // T's diagonal blocks: block i >> 5, row (i >> 1) & 15, 8-column half i & 1
             const int i = tid - 128, bd = i >> 5, r = 16 * bd + ((i >> 1) & 15), c0 = 16 * bd + 8 * (i & 1);
@@ -718,34 +739,47 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             for (int j = 0; j < 8; ++j) t8[j] = (c0 + j <= r) ? AF[r * ALD + c0 + j] * sbeta[c0 + j] : 0.f;
             *reinterpret_cast<uint4 *>(TT + kmaj_chunk(r, c0 >> 3, 64)) = pack8(t8);
         } else {
-            const int o = (warp >> 1) * 32, nh = (warp & 1) * 8;  // block offset, column half
-            float *Rw = R2 + warp * 128;                          // 16 x 8 scratch per warp
+            // Level 1, warps 0..3: X21 = -X22 (Diag(beta) A21) X11 for the 32-row blocks at 0
+            // (warps 0, 1) and 32 (warps 2, 3), 8 of the 16 columns per warp; R = N21 X11
+            // passes through a per-warp scratch to become the second product's B operand.
+            const int o = (warp >> 1) * 32, nh = (warp & 1) * 8;
+            float *Rw = R2 + warp * 128;  // 16 x 8
+            float acc[4];
             warp_gemm_16x8<16>(
                 lane, [&](int r, int kk) { return sbeta[o + 16 + r] * AF[(o + 16 + r) * ALD + o + kk]; },
-                [&](int kk, int nn) { return AF[(o + kk) * ALD + o + nh + nn]; },
-                [&](int r, int nn, float v) { Rw[r * 8 + nn] = v; });
-            bar_sync(3 + 2 * e + (warp >> 1), 64);  // both column halves have read A21
+                [&](int kk, int nn) { return AF[(o + kk) * ALD + o + nh + nn]; }, acc);
+            *reinterpret_cast<float2 *>(Rw + fg * 8 + 2 * ft) = make_float2(acc[0], acc[1]);
+            *reinterpret_cast<float2 *>(Rw + (fg + 8) * 8 + 2 * ft) = make_float2(acc[2], acc[3]);
+            bar_sync(3 + 2 * e + (warp >> 1), 64);  // both column halves have read A21; R is in
             warp_gemm_16x8<16>(
                 lane, [&](int r, int kk) { return AF[(o + 16 + r) * ALD + o + 16 + kk]; },
-                [&](int kk, int nn) { return Rw[kk * 8 + nn]; },
-                [&](int r, int nn, float v) {
-                    AF[(o + 16 + r) * ALD + o + nh + nn] = -v;
-                    t_store(o + 16 + r, o + nh + nn, -v);
-                });
+                [&](int kk, int nn) { return Rw[kk * 8 + nn]; }, acc);
+            const int r = o + 16 + fg, c = o + nh + 2 * ft;
+            *reinterpret_cast<float2 *>(AF + r * ALD + c) = make_float2(-acc[0], -acc[1]);
+            *reinterpret_cast<float2 *>(AF + (r + 8) * ALD + c) = make_float2(-acc[2], -acc[3]);
+            t_store2(r, c, -acc[0], -acc[1]);
+            t_store2(r + 8, c, -acc[2], -acc[3]);
         }
         sync();
-        // 32-row level: R2 = (Diag(beta) A)[32..63][0..31] X[0..31][0..31], then X[32..63][0..31] = -X22 R2.
+        // Level 2, all warps: R2 = (Diag(beta) A)[32..63][0..31] X[0..31][0..31] (kept transposed,
+        // row stride R2LD), then X[32..63][0..31] = -X[32..63][32..63] R2, of which only T is kept.
         {
             const int mt = warp >> 2, nt = warp & 3;  // 16-row tile, 8-column tile
+            float acc[4];
             warp_gemm_16x8<32>(
                 lane, [&](int r, int kk) { return sbeta[32 + 16 * mt + r] * AF[(32 + 16 * mt + r) * ALD + kk]; },
-                [&](int kk, int nn) { return AF[kk * ALD + 8 * nt + nn]; },
-                [&](int r, int nn, float v) { R2[(16 * mt + r) * 32 + 8 * nt + nn] = v; });
+                [&](int kk, int nn) { return AF[kk * ALD + 8 * nt + nn]; }, acc);
+            const int rr = 16 * mt + fg, cc = 8 * nt + 2 * ft;
+            R2[cc * R2LD + rr] = acc[0];
+            R2[(cc + 1) * R2LD + rr] = acc[1];
+            R2[cc * R2LD + rr + 8] = acc[2];
+            R2[(cc + 1) * R2LD + rr + 8] = acc[3];
             sync();
             warp_gemm_16x8<32>(
                 lane, [&](int r, int kk) { return AF[(32 + 16 * mt + r) * ALD + 32 + kk]; },
-                [&](int kk, int nn) { return R2[kk * 32 + 8 * nt + nn]; },
-                [&](int r, int nn, float v) { t_store(32 + 16 * mt + r, 8 * nt + nn, -v); });
+                [&](int kk, int nn) { return R2[(8 * nt + nn) * R2LD + kk]; }, acc);
+            t_store2(32 + rr, cc, -acc[0], -acc[1]);
+            t_store2(32 + rr + 8, cc, -acc[2], -acc[3]);
         }
         fence_async_smem();
         tc_fence_before();
@@ -859,6 +893,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         // ---------------- ring-slot copies (one thread) ----------------
         if (lane != 0) return;
         long long p = 0, nA = 0, nB = 0;  // positions whose A / B groups were issued
+        int rpos = 0, rgen = 0;           // p % R and p / R
         bool ok = true;
         for (long long kk = 0; kk < K && ok; ++kk) {
             int s, h;
@@ -870,8 +905,12 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 // then overlaps the wait for a free buffer), then the B group (three
                 // buffers: free one position before the A group's two), then A.
                 const int ab = (int)(p & 1), bb = (int)(p % 3);
-                const int slot = st * R + (int)(p % R);
-                ok = wait_flag_geq(&ready[slot], (int)(p / R) + 1, &hd->abort_flag, P.xwait_ns, 32);
+                const int slot = st * R + rpos;
+                ok = wait_flag_geq(&ready[slot], rgen + 1, &hd->abort_flag, P.xwait_ns, 32);
+                if (++rpos == R) {
+                    rpos = 0;
+                    ++rgen;
+                }
                 if (ok && p >= 3) ok = mbar_wait_call(&emptyB[bb], (uint32_t)((p / 3 - 1) & 1), &hd->abort_flag);
                 if (!ok) break;
                 fence_proxy_async_global();
@@ -880,7 +919,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                 mbar_arrive_expect_tx(&fullB[bb], COPY_B);
                 bulk_g2s(B + SB_T, g + SL_T, 8192, &fullB[bb]);
                 bulk_g2s(B + SB_P, g + SL_P, 8192, &fullB[bb]);
-                bulk_g2s(B + SB_D, g + SL_D, 512, &fullB[bb]);
+                bulk_g2s(B + SB_D, g + SL_D, 1024, &fullB[bb]);
                 nB = p + 1;
                 if (p >= 2) ok = mbar_wait_call(&emptyA[ab], (uint32_t)((p / 2 - 1) & 1), &hd->abort_flag);
                 if (!ok) break;
@@ -1194,13 +1233,14 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
                                              mbar_wait_call(&fullB[p % 3], (uint32_t)((p / 3) & 1), &hd->abort_flag));
             if (!ok) break;
             tc_fence_after();
-            const float dc = reinterpret_cast<const float *>(sm + SS_B + (p % 3) * SB_BYTES + SB_D)[c];
+            const float *dd = reinterpret_cast<const float *>(sm + SS_B + (p % 3) * SB_BYTES + SB_D);
+            const float dc = dd[c], dz = dd[DK + c];
             {
                 float zv[32];
                 tmem_ld32(tm + TM_Z + lane_base + col, zv);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) Sr[i] = dc * Sr[i] + zv[i];
+                for (int i = 0; i < 32; ++i) Sr[i] = fmaf(dc, Sr[i], dz * zv[i]);
             }
             if (j + 1 < nch) state_to_smem();
         }
@@ -1252,6 +1292,17 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
             ctl->maxlen = hd->maxlen;
             ctl->uniform = hd->uniform;
         }
+        const long long NH = (long long)P.N * P.H;
+        int *uc = reinterpret_cast<int *>(sm + CACHE_OFF);
+        const bool ucache = NH <= kUnitCache, ccache = P.cu != nullptr && P.N + 1 <= kSeqCache;
+        if (tid == 96) {
+            ctl->ucache = ucache;
+            ctl->ccache = ccache;
+        }
+        if (ucache)  // positions in a stream fit in 32 bits
+            for (int u = tid; u < (int)NH; u += kThreads) uc[u] = (int)reinterpret_cast<const long long *>(P.ws + WS_USTART)[u];
+        if (ccache)
+            for (int s = tid; s <= P.N; s += kThreads) uc[kUnitCache + s] = P.cu[s];
     }
     if (warp == 0) {
         tmem_alloc(&ctl->tbase, 512);

@@ -279,6 +279,19 @@ __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool pred) 
         : "memory");
     return r != 0;
 }
+// Named barrier that also returns the OR of `pred` over its `count` threads.
+__device__ __forceinline__ bool bar_or(uint32_t id, uint32_t count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.red.or.pred p, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
 // Orders this thread's async-proxy global accesses (bulk copies) with its
 // generic-proxy ones (flag releases and acquires).
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
@@ -322,6 +335,47 @@ __device__ __forceinline__ void cp_async4(void *smem_dst, const void *gsrc, uint
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// ------------------------------------------------- packed fp32 pairs ----
+// Two fp32 values in one 64-bit register pair, for the sm_100 f32x2 arithmetic
+// (one instruction does both lanes, each rounded as its scalar form would be).
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t f2(float lo, float hi) {
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float f2lo(f2_t a) { return __uint_as_float((uint32_t)a); }
+__device__ __forceinline__ float f2hi(f2_t a) { return __uint_as_float((uint32_t)(a >> 32)); }
+__device__ __forceinline__ f2_t f2mul(f2_t a, f2_t b) {
+    f2_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2_t f2add(f2_t a, f2_t b) {
+    f2_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f2_t f2fma(f2_t a, f2_t b, f2_t c) {
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// 2^x by the hardware approximation (PTX ex2.approx.ftz), for exponents kept in base 2.
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// A pair of fp32 values -> a bf16 pair (round to nearest even), low value in the low half.
+__device__ __forceinline__ uint32_t pack2(f2_t a) {
+    uint32_t r;
+    asm("{\n\t.reg .f32 lo, hi;\n\tmov.b64 {lo, hi}, %1;\n\tcvt.rn.bf16x2.f32 %0, hi, lo;\n\t}" : "=r"(r) : "l"(a));
+    return r;
+}
+// A bf16 pair (low value in the low half) -> a pair of fp32 values.
+__device__ __forceinline__ f2_t unpack2(uint32_t w) { return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u)); }
 
 // bf16 pair packing / unpacking
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
