@@ -74,27 +74,32 @@ __device__ __forceinline__ void conv_swish_lane(const T *__restrict__ xrow, int 
     }
 }
 
-template <int DK, int DV, typename T, bool CONV>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+template <int DK, int DV, typename T, bool CONV, int SPLIT = 1>
+__global__ void __launch_bounds__(kDecodeThreads, 2 * SPLIT)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
               float *__restrict__ S, T *__restrict__ o, int l2norm, int la_scalar, float eps,
               const T *__restrict__ og_gate, const float *__restrict__ og_w, float og_eps, DecodeConv cv,
               int H) {
-    constexpr int CG = DV / 4;                // 16-byte column groups per state row
+    // SPLIT > 1: the unit's state columns are divided among SPLIT CTAs (columns are
+    // independent: each needs only its own column sums, and k . q, which every CTA forms).
+    constexpr int DVC = DV / SPLIT;           // state columns of this CTA
+    constexpr int CG = DVC / 4;               // 16-byte column groups per state row
     constexpr int RPP = kDecodeThreads / CG;  // state rows covered per pass
     constexpr int R = DK / RPP;               // rows held per thread
-    static_assert(R * RPP == DK && CG * 4 == DV, "shape");
+    static_assert(R * RPP == DK && CG * 4 == DVC, "shape");
+    static_assert(SPLIT == 1 || !CONV, "the fused convolution runs unsplit");
 
     __shared__ float s_q[DK], s_k[DK], s_a[DK], s_v[DV], s_u[DV];
     __shared__ float s_red[RPP][CG][8];
     __shared__ float s_misc[2];  // beta, k.q
     __shared__ float s_o[DV], s_gss[DV / 32];  // fused output step: o, per-warp sums of o^2
 
-    const int unit = blockIdx.x;  // sequence * H + head
+    const int unit = blockIdx.x / SPLIT;  // sequence * H + head
+    const int c0 = (blockIdx.x % SPLIT) * DVC;  // first state column of this CTA
     const int tid = threadIdx.x;
     const int cg = tid % CG, r0 = tid / CG;
-    float *Su = S + (size_t)unit * DK * DV;
+    float *Su = S + (size_t)unit * DK * DV + c0;
 
     // 1. Issue the whole state tile load first (R independent 16-byte loads).
     float4 s[R];
@@ -202,7 +207,7 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
         for (int i = lane; i < DK; i += 32)
             s_a[i] = expf(la_scalar ? log_alpha[unit] : log_alpha[(size_t)unit * DK + i]);
       } else if (warp == 2) {
-        for (int j = lane; j < DV; j += 32) s_v[j] = IO<T>::ld(v + (size_t)unit * DV + j);
+        for (int j = lane; j < DVC; j += 32) s_v[j] = IO<T>::ld(v + (size_t)unit * DV + c0 + j);
         if (lane == 0) s_misc[0] = beta[unit];
       }
     }
@@ -222,7 +227,7 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
     __syncthreads();
 
     // 4. Finish the sums per column: u = beta (v - S~^T k), o = S~^T q + (k.q) u.
-    if (tid < DV) {
+    if (tid < DVC) {
         const int j = tid, g = j >> 2, c = j & 3;
         float yy = 0.f, zz = 0.f;
 #pragma unroll
@@ -241,7 +246,7 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
             for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
             if ((j & 31) == 0) s_gss[j >> 5] = ss;
         } else {
-            IO<T>::st(o + (size_t)unit * DV + j, oj);
+            IO<T>::st(o + (size_t)unit * DV + c0 + j, oj);
         }
     }
     __syncthreads();
@@ -278,6 +283,10 @@ cudaError_t launch(const void *q, const void *k, const void *v, const float *la,
     const unsigned units = (unsigned)N * (unsigned)H;
     if (cv.W[0] | cv.W[1] | cv.W[2])
         decode_kernel<DK, DV, T, true><<<units, kDecodeThreads, 0, st>>>(
+            (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps,
+            (const T *)og_gate, og_w, og_eps, cv, H);
+    else if (og_gate == nullptr && DV == 128)
+        decode_kernel<DK, DV, T, false, 2><<<2 * units, kDecodeThreads, 0, st>>>(
             (const T *)q, (const T *)k, (const T *)v, la, beta, S, (T *)o, l2norm, la_scalar, eps,
             (const T *)og_gate, og_w, og_eps, cv, H);
     else

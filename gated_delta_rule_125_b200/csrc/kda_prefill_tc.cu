@@ -49,6 +49,7 @@ constexpr int DK = 128;
 constexpr int DV = 128;
 constexpr int DVT = 64;                      // state columns per scan CTA
 constexpr float kTau = 60.f;                 // largest per-chunk decay range for the factorised Gram
+constexpr float kLog2e = 1.4426950408889634f;  // G is kept in base 2: e^{+-G} = 2^{+-G log2 e}
 constexpr uint64_t kWaitNs = kDefaultWaitNs;  // bound of a CTA's waits for its own copies and products (2 s)
 constexpr int kThreads = 512;                // per CTA: two prep engines, or one scan CTA
 constexpr int kMaxRing = 16;                 // ring slots per stream, upper bound (~34 MB at 32 streams)
@@ -246,7 +247,8 @@ static_assert(TM_Z + 64 <= 512, "scan TMEM columns");
 constexpr int MB_FULLA = 0, MB_FULLB = 2, MB_FULLV = 5, MB_EMPTYA = 9, MB_EMPTYB = 11, MB_EMPTYV = 14,
               MB_U = 18, MB_S = 19, MB_O = 20,  // MB_O and MB_OREADY: one barrier per Y buffer
               MB_UREADY = MB_O + NY, MB_SREADY = MB_UREADY + 1, MB_FIN = MB_SREADY + 1, MB_OREADY = MB_FIN + 1,
-              MB_COUNT = MB_OREADY + NY;
+              MB_X = MB_OREADY + NY,  // one per X buffer: T V of a position complete
+              MB_FIN2 = MB_X + 2, MB_COUNT = MB_FIN2 + 1;
 
 // Per-CTA control block after both layouts.
 struct Ctrl {
@@ -264,7 +266,7 @@ constexpr int kUnitCache = 2048, kSeqCache = 1025;
 constexpr uint32_t CACHE_OFF = CTRL_OFF + 512;
 constexpr uint32_t SMEM_ALLOC = CACHE_OFF + 4 * (kUnitCache + kSeqCache) + 1024;  // + alignment slack
 static_assert(2 * PS_STRIDE <= CTRL_OFF, "prep engines overlap the control block");
-static_assert(MB_O + NY == MB_UREADY && MB_OREADY + NY == MB_COUNT, "scan barrier indices");
+static_assert(MB_O + NY == MB_UREADY && MB_OREADY + NY == MB_X, "scan barrier indices");
 static_assert(MB_COUNT * 8 + 16 <= SS_OGW - SS_BAR, "scan barrier area");
 static_assert(sizeof(Ctrl) <= 512, "control block");
 
@@ -272,8 +274,9 @@ static_assert(sizeof(Ctrl) <= 512, "control block");
 struct ItemS {
     long long t0, p;  // first token; position in the stream
     int n, h, st, valid;
-    int slot, gen;
+    int slot, gen;    // ring slot (stream st, position p % R) and its generation p / R
 };
+static_assert(3 * 8 + 3 * sizeof(ItemS) + 3 * 4 <= PS_BYTES - PS_BAR, "prep barrier block: mbarriers, item records, flags");
 
 
 // Item g of the global claim order: position-major over the streams still
@@ -372,7 +375,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                                             uint32_t tm) {
     const int tid = (int)threadIdx.x - PT * e, warp = tid >> 5, lane = tid & 31;
     const uint32_t bar_id = 1 + e;
-    const int H = P.H, R = P.R;
+    const int H = P.H;
     float *G = reinterpret_cast<float *>(sm + PS_LA);
     float *AF = reinterpret_cast<float *>(sm + PS_AF);
     float *R2 = reinterpret_cast<float *>(sm + PS_R2);
@@ -386,7 +389,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     // Item records of iterations it (current), it + 1 (claimed during the Gram)
     // and it - 1 (published by the store thread) in entries it % 3, ...
     ItemS *sitem = reinterpret_cast<ItemS *>(bars + 3);
-    int *sflag = reinterpret_cast<int *>(sitem + 3);  // [0] unsafe range, [1] a wait failed
+    int *sflag = reinterpret_cast<int *>(sitem + 3);  // [0] unsafe range, [1] a wait failed, [2] next slot known free
     Hdr *hd = reinterpret_cast<Hdr *>(P.ws);
     const long long NH = (long long)P.N * H;
     int *ready = reinterpret_cast<int *>(P.ws + ws_flags(NH));
@@ -405,7 +408,6 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     // (warps 4..7 are idle there), or at once if the current item has to wait
     // for its slot (that wait may depend on the previous item).
     constexpr int kStoreTid = 128;
-    bool slot_ok = false;       // store thread: the current item's slot is known to be free
     bool prev_pending = false;  // store thread: the previous item is not yet published
     bool la_pending = false;    // store thread: a log_alpha box is in flight
     bool qk_pending = false;    // store thread: q, k boxes are in flight
@@ -467,15 +469,14 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         char *gslot = ring + (size_t)cur.slot * SL_BYTES;
         const float *sbeta = sbeta2 + (iter & 1) * 64;
         if (tid == kStoreTid) {
-            bulk_wait_read();  // the previous item's bulk stores no longer read GA
             // This item's slot is written below: both scan CTAs of the stream must
             // have released its previous generation.
-            if (!slot_ok) {
+            if (!sflag[2]) {
                 publish_prev(prev);
                 if (!wait_flag_geq(&freed[cur.slot], 2 * cur.gen, &hd->abort_flag, P.xwait_ns))
                     sflag[1] = 1;
             }
-            slot_ok = false;
+            sflag[2] = 0;
         }
 
         // 1. Warps 0..3: G = cumulative sum of log_alpha over the rows, in place, one
@@ -502,12 +503,12 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                     v[i] = (r0 + i < n) ? (P.la_scalar ? sgate[r0 + i] : G[(r0 + i) * DK + c]) : 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    run += v[i];
+                    run = fmaf(v[i], kLog2e, run);
                     G[(r0 + i) * DK + c] = run;
                 }
             }
-            eGl[c] = expf(run);
-            if (-run > kTau) sflag[0] = 1;
+            eGl[c] = ex2f(run);
+            if (-run > kTau * kLog2e) sflag[0] = 1;
         } else {
             const int r = tid & (C - 1);
             uint8_t *src = (tid < 192) ? GB : KS;
@@ -529,6 +530,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             ((tid < 192) ? invq : invk)[r] = inv;
         }
         if (!P.la_scalar) la_phase ^= 1;
+        if (tid == kStoreTid) bulk_wait_read();  // the previous item's bulk stores no longer read GA
         sync();
         if (sflag[1]) {
             failed = true;
@@ -549,24 +551,22 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                 const uint4 kv = *reinterpret_cast<const uint4 *>(KS + kmaj_chunk(r, c8, 64));
                 const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
                 const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
-                uint32_t pq[4], pk[4], pn[4], pd[4];
+                uint32_t pq[4], pk[4], pn[4];
+                const f2_t iq2 = f2(iq, iq), ik2 = f2(ik, ik);
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const float2 g = *reinterpret_cast<const float2 *>(G + r * DK + c8 * 8 + 2 * w);
-                    const float2 d = *reinterpret_cast<const float2 *>(eGl + c8 * 8 + 2 * w);
-                    const float k0 = __uint_as_float(kw[w] << 16) * ik, k1 = __uint_as_float(kw[w] & 0xFFFF0000u) * ik;
-                    const float q0 = __uint_as_float(qw[w] << 16) * iq, q1 = __uint_as_float(qw[w] & 0xFFFF0000u) * iq;
-                    const float ep0 = __expf(g.x), ep1 = __expf(g.y);
-                    const float n0 = k0 * __expf(-g.x), n1 = k1 * __expf(-g.y);
-                    pq[w] = pack_bf16(q0 * ep0, q1 * ep1);
-                    pk[w] = pack_bf16(k0 * ep0, k1 * ep1);
-                    pn[w] = pack_bf16(n0, n1);
-                    pd[w] = pn[w];  // the slot carries K e^-G; the scan scales by DZ
+                for (int w = 0; w < 4; ++w) {  // channel pairs, in fp32 pairs
+                    const f2_t g = *reinterpret_cast<const f2_t *>(G + r * DK + c8 * 8 + 2 * w);
+                    const float gx = f2lo(g), gy = f2hi(g);
+                    const f2_t ep = f2(ex2f(gx), ex2f(gy)), en = f2(ex2f(-gx), ex2f(-gy));
+                    const f2_t qn = f2mul(unpack2(qw[w]), iq2), kn = f2mul(unpack2(kw[w]), ik2);
+                    pq[w] = pack2(f2mul(qn, ep));
+                    pk[w] = pack2(f2mul(kn, ep));
+                    pn[w] = pack2(f2mul(kn, en));
                 }
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = make_uint4(pq[0], pq[1], pq[2], pq[3]);
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 *reinterpret_cast<uint4 *>(GB + kmaj_chunk(r, c8, 64)) = make_uint4(pn[0], pn[1], pn[2], pn[3]);
-                *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = make_uint4(pd[0], pd[1], pd[2], pd[3]);
+                *reinterpret_cast<uint4 *>(gslot + SL_KD + mnmaj_chunk(r, c8, 64)) = make_uint4(pn[0], pn[1], pn[2], pn[3]);  // the slot carries K e^-G
             }
         } else {
 #pragma unroll
@@ -580,7 +580,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                 for (int i = 0; i < 8; ++i) {
                     kf[i] *= ik;
                     qf[i] *= iq;
-                    kd[i] = kf[i] * __expf(G[(C - 1) * DK + c8 * 8 + i] - G[r * DK + c8 * 8 + i]);
+                    kd[i] = kf[i] * ex2f(G[(C - 1) * DK + c8 * 8 + i] - G[r * DK + c8 * 8 + i]);
                 }
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(r, c8, 128)) = pack8(qf);
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(64 + r, c8, 128)) = pack8(kf);
@@ -629,7 +629,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                         const int ii = i0 + i;
                         const float ki = __bfloat162float(*reinterpret_cast<const bf16 *>(GA + kmaj_off(64 + ii, c, 128)));
                         const bool keep = isq ? (ii <= r) : (ii < r);
-                        acc[i] += keep ? xr * ki * __expf(gr - G[ii * DK + c]) : 0.f;
+                        acc[i] += keep ? xr * ki * ex2f(gr - G[ii * DK + c]) : 0.f;
                     }
                 }
                 tmem_st16(tm + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)i0, acc);
@@ -645,7 +645,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
                 float x[8];
                 unpack8(*reinterpret_cast<const uint4 *>(GA + kmaj_chunk(rr, c8, 128)), x);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) x[i] *= __expf(G[r2 * DK + c8 * 8 + i]);
+                for (int i = 0; i < 8; ++i) x[i] *= ex2f(G[r2 * DK + c8 * 8 + i]);
                 *reinterpret_cast<uint4 *>(GA + kmaj_chunk(rr, c8, 128)) = pack8(x);
             }
             fence_async_smem();
@@ -691,8 +691,8 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
         if (next.valid) fetch_qk(next, (iter + 1) & 1);
         if (tid == kStoreTid) {  // warp 4 is idle in the diagonal-block solve below
             publish_prev(prev);
-            if (next.valid) slot_ok = slot_free(next);
         }
+        if (tid == kStoreTid + 96 && next.valid) sflag[2] = slot_free(next);  // beside the publish
 
         // 5. X = (I + Diag(beta) A)^{-1}, in place over A (fp32), and T = X Diag(beta) (bf16,
         //    the A operand of W and the slot's T tile), by 16 x 16 blocks.
@@ -859,8 +859,10 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
 // ---------------------------------------------------------------- scan ----
 // Scan CTA for stream st, state columns [64 jv, 64 jv + 64). Warps 0..7:
 // TMEM-lane epilogues (warp w: lanes 32 (w % 4) .., columns 32 (w / 4) ..);
-// warp 8: MMA issue; warp 9: ring-slot copies; warp 10: V copies; warp 11: slot
-// release; warps 12, 13: O rows to HBM (with the fused output step: RMSNorm over
+// warp 8: the state chain's MMAs (Y, Z); warp 14: the other MMAs (O, the next
+// position's T V), from its own thread so that their issue (tens of cycles per
+// instruction) never delays the chain; warp 9: ring-slot copies; warp 10: V copies;
+// warp 11: slot release; warps 12, 13: O rows to HBM (with the fused output step: RMSNorm over
 // the row's 128 columns, the two scan CTAs of a stream exchanging their halves'
 // sums of squares, and the sigmoid gate). TMEM lanes 0..63 hold O = Q e^G S + P U,
 // 64..127 hold W S and T V (their difference is U); Z = Kd^T U fills all 128.
@@ -881,7 +883,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
     uint64_t *fullA = bars + MB_FULLA, *fullB = bars + MB_FULLB, *fullV = bars + MB_FULLV, *emptyA = bars + MB_EMPTYA,
              *emptyB = bars + MB_EMPTYB, *emptyV = bars + MB_EMPTYV, *bU = bars + MB_U, *bS = bars + MB_S,
              *bO = bars + MB_O, *uready = bars + MB_UREADY, *sready = bars + MB_SREADY, *bFin = bars + MB_FIN,
-             *oready = bars + MB_OREADY;
+             *oready = bars + MB_OREADY, *bX = bars + MB_X, *bFin2 = bars + MB_FIN2;
     auto unit_bounds = [&](long long kk, int &s, int &h, int64_t &bos, int64_t &eos) {
         const long long u = st + kk * ns;
         s = (int)(u / H);
@@ -987,41 +989,23 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         return;
     }
     if (warp == 8) {
-        // ---------------- MMA issue (one thread) ----------------
+        // ---------------- the state chain's MMAs (one thread) ----------------
         if (lane != 0) return;
         const uint32_t id128 = idesc_bf16(128, DVT, false, true);  // K-major A, MN-major B
         const uint32_t idKd = idesc_bf16(128, DVT, true, true);    // MN-major A (Kd^T)
         // Descriptors of buffer 0; buffer i is i strides further (16-byte units).
         const uint64_t dWQ = sdesc(smem_u32(sm + SS_A + SA_WQ), 16, 1024);
         const uint64_t dKD = sdesc(smem_u32(sm + SS_A + SA_KD), C * 128, 1024);
-        const uint64_t dTf = sdesc(smem_u32(sm + SS_B + SB_T) - 8192, 16, 1024);  // filler, then T
-        const uint64_t dP = sdesc(smem_u32(sm + SS_B + SB_P), 16, 1024);          // P, then filler
-        const uint64_t dV = sdesc(smem_u32(sm + SS_V), C * 128, 1024);
         const uint64_t dS = sdesc(smem_u32(sS), DK * 128, 1024), dU = sdesc(smem_u32(sU), C * 128, 1024);
-        constexpr uint64_t kA = SA_BYTES >> 4, kB = SB_BYTES >> 4, kV = SV_BYTES >> 4;
-        // X[q & 1] = [filler ; T] V of position q, once its T and V tiles are in.
-        auto issue_x = [&](long long q) {
-            const int bb = (int)(q % 3), vb = (int)(q & 3);
-            if (!(mbar_wait_call(&fullB[bb], (uint32_t)((q / 3) & 1), &hd->abort_flag) &&
-                  mbar_wait_call(&fullV[vb], (uint32_t)((q >> 2) & 1), &hd->abort_flag)))
-                return false;
-            tc_fence_after();
-#pragma unroll
-            for (int s4 = 0; s4 < C / 16; ++s4)
-                mma_bf16(tm + TM_X + (uint32_t)(q & 1) * 64, dTf + bb * kB + kmaj_step(s4, 128), dV + vb * kV + mnmaj_step(s4),
-                         id128, s4 > 0);
-            mma_commit(&emptyV[vb]);
-            return true;
-        };
+        constexpr uint64_t kA = SA_BYTES >> 4;
         bool ok = true;
-        if (L > 0) ok = issue_x(0);
         for (long long p = 0; p < L && ok; ++p) {
-            const int ab = (int)(p & 1), bb = (int)(p % 3);
+            const int ab = (int)(p & 1);
             const uint32_t yb = (uint32_t)(p % NY) * 64;
-            ok = mbar_wait_call(&fullA[ab], (uint32_t)((p >> 1) & 1), &hd->abort_flag);
+            ok = mbar_wait_call(&fullA[ab], (uint32_t)((p >> 1) & 1), &hd->abort_flag) &&
+                 mbar_wait_call(&fullB[p % 3], (uint32_t)((p / 3) & 1), &hd->abort_flag);
             if (!ok) break;
-            // Both tile groups of position p are in shared memory (B was waited for
-            // with X(p)): its ring slot can be released.
+            // Both tile groups of position p are in shared memory: its ring slot can be released.
             __threadfence_block();
             *consumed = p + 1;
             // S(p) in smem, and O(p - NY) read out of Y[p % NY] (one barrier per Y buffer: it
@@ -1032,7 +1016,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             if (p >= 1) mbar_arrive(&emptyB[(p - 1) % 3]);  // e^{Gl} of p-1 has been read
             tc_fence_after();
             // Y = [Q e^G ; W] S
-            const uint64_t dWQa = dWQ + ab * kA, dKDa = dKD + ab * kA, dPb = dP + bb * kB;
+            const uint64_t dWQa = dWQ + ab * kA, dKDa = dKD + ab * kA;
 #pragma unroll
             for (int s8 = 0; s8 < DK / 16; ++s8)
                 mma_bf16(tm + TM_Y + yb, dWQa + kmaj_step(s8, 128), dS + mnmaj_step(s8), id128, s8 > 0);
@@ -1040,20 +1024,12 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             ok = mbar_wait_call(uready, (uint32_t)(p & 1), &hd->abort_flag);  // U(p) in smem
             if (!ok) break;
             tc_fence_after();
-            // Z = Kd^T U first (the state chain), then O: Y += [P ; filler] U
+            // Z = Kd^T U (the state chain)
 #pragma unroll
             for (int s4 = 0; s4 < C / 16; ++s4)
                 mma_bf16(tm + TM_Z, dKDa + mnmaj_step(s4), dU + mnmaj_step(s4), idKd, s4 > 0);
             mma_commit(bS);
-#pragma unroll
-            for (int s4 = 0; s4 < C / 16; ++s4)
-                mma_bf16(tm + TM_Y + yb, dPb + kmaj_step(s4, 128), dU + mnmaj_step(s4), id128, 1);
-            mma_commit(&bO[p % NY]);
             mma_commit(&emptyA[ab]);
-            mma_commit(&emptyB[bb]);
-            // T V of the next position, while S(p + 1) is formed (after Z: a late
-            // T or V tile never holds up the state chain).
-            if (p + 1 < L && !(ok = issue_x(p + 1))) break;
         }
         mma_commit(bFin);  // every MMA of this CTA completes before TMEM is freed
         if (!mbar_wait(bFin, 0, kWaitNs)) ok = false;
@@ -1156,7 +1132,56 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         if (!ok) fail_call(P);
         return;
     }
-    if (warp >= 8) return;  // warps 14, 15 idle
+    if (warp == 14) {
+        // ---------------- the other MMAs (one thread) ----------------
+        // After U(p) is in shared memory: O(p) into Y[p % NY] (Y(p) has completed: the U
+        // epilogue read it) and T V of the next position into its X buffer (read by the
+        // U epilogue of position p - 1, which has finished).
+        if (lane != 0) return;
+        const uint32_t id128 = idesc_bf16(128, DVT, false, true);  // K-major A, MN-major B
+        const uint64_t dTf = sdesc(smem_u32(sm + SS_B + SB_T) - 8192, 16, 1024);  // filler, then T
+        const uint64_t dP = sdesc(smem_u32(sm + SS_B + SB_P), 16, 1024);          // P, then filler
+        const uint64_t dV = sdesc(smem_u32(sm + SS_V), C * 128, 1024);
+        const uint64_t dU = sdesc(smem_u32(sU), C * 128, 1024);
+        constexpr uint64_t kB = SB_BYTES >> 4, kV = SV_BYTES >> 4;
+        // X[q & 1] = [filler ; T] V of position q, once its T and V tiles are in.
+        auto issue_x = [&](long long q) {
+            const int bb = (int)(q % 3), vb = (int)(q & 3);
+            if (!(mbar_wait_call(&fullB[bb], (uint32_t)((q / 3) & 1), &hd->abort_flag) &&
+                  mbar_wait_call(&fullV[vb], (uint32_t)((q >> 2) & 1), &hd->abort_flag)))
+                return false;
+            tc_fence_after();
+#pragma unroll
+            for (int s4 = 0; s4 < C / 16; ++s4)
+                mma_bf16(tm + TM_X + (uint32_t)(q & 1) * 64, dTf + bb * kB + kmaj_step(s4, 128), dV + vb * kV + mnmaj_step(s4),
+                         id128, s4 > 0);
+            mma_commit(&emptyV[vb]);
+            mma_commit(&bX[q & 1]);
+            return true;
+        };
+        bool ok = true;
+        if (L > 0) ok = issue_x(0);
+        for (long long p = 0; p < L && ok; ++p) {
+            const int bb = (int)(p % 3);
+            const uint32_t yb = (uint32_t)(p % NY) * 64;
+            // Z(p) complete (so U(p) is in smem and Y(p) complete): the chain's product runs first
+            ok = mbar_wait_call(bS, (uint32_t)(p & 1), &hd->abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            // O: Y += [P ; filler] U
+#pragma unroll
+            for (int s4 = 0; s4 < C / 16; ++s4)
+                mma_bf16(tm + TM_Y + yb, dP + bb * kB + kmaj_step(s4, 128), dU + mnmaj_step(s4), id128, 1);
+            mma_commit(&bO[p % NY]);
+            mma_commit(&emptyB[bb]);
+            if (p + 1 < L && !(ok = issue_x(p + 1))) break;
+        }
+        mma_commit(bFin2);  // every MMA of this thread completes before TMEM is freed
+        if (!mbar_wait(bFin2, 0, kWaitNs)) ok = false;
+        if (!ok) fail_call(P);
+        return;
+    }
+    if (warp >= 8) return;  // warp 15 idle
 
     // ---------------- epilogues (TMEM lane = state row c) ----------------
     const int q4 = warp & 3, hf = warp >> 2;
@@ -1209,8 +1234,12 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
             const uint32_t xb = (uint32_t)(p & 1) * 64, yb = (uint32_t)(p % NY) * 64;
             const uint32_t par = (uint32_t)(p & 1);
             if (q4 >= 2) {
-                // U = T V - W S for rows r = c - 64 (TMEM lanes 64..127)
-                ok = __all_sync(0xffffffffu, mbar_wait_call(bU, par, &hd->abort_flag));
+                // U = T V - W S for rows r = c - 64 (TMEM lanes 64..127), once Y(p) and X(p) have
+                // completed and O(p - 1) has read the previous U
+                ok = __all_sync(0xffffffffu, mbar_wait_call(bU, par, &hd->abort_flag) &&
+                                                 mbar_wait_call(&bX[p & 1], (uint32_t)((p >> 1) & 1), &hd->abort_flag) &&
+                                                 (p == 0 || mbar_wait_call(&bO[(p - 1) % NY], (uint32_t)(((p - 1) / NY) & 1),
+                                                                           &hd->abort_flag)));
                 if (!ok) break;
                 tc_fence_after();
                 float xv[32], yv[32];
@@ -1277,6 +1306,7 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
                 int *sflag = reinterpret_cast<int *>(reinterpret_cast<ItemS *>(bars + 3) + 3);
                 sflag[0] = 0;
                 sflag[1] = 0;
+                sflag[2] = 0;
             }
         }
         fence_barrier_init();

@@ -14,6 +14,7 @@ import torch
 import gated_delta_rule_125_b200 as kda
 import kda_inputs as KI
 import oracle
+from bf16_round import bf16_neighbours
 
 pytestmark = pytest.mark.gpu
 
@@ -477,11 +478,16 @@ def test_output_gate_workload_prefill_8k():
 
 
 # ------------------------------------- short convolution + Swish (§6.1) ----
-# The convolution's output is one fp32 dot product of W taps then Swish, stored
-# in the io dtype: it must lie within the io dtype's rounding of the fp64 value
-# (bf16 round-to-nearest: 2^-8 relative, the unit roundoff of an 8-bit
-# significand, plus 1 % of it for the fp32 arithmetic before the rounding; fp32:
-# 1e-5 relative, fast exponential). States are raw input copies: bit-exact.
+# The convolution's output is one fp32 dot product of W taps then Swish, stored in
+# the io dtype. The fp32 value z lies within CONV_FP32 = (relative, absolute) of
+# the fp64 reference (absolute: the dot product's cancellation near zero). For
+# bf16 the check separates that error from the rounding: rounding to nearest
+# (ties to even) is monotone, so every output must lie between the roundings of
+# y_ref - delta and y_ref + delta, delta = 4e-6 |y_ref| + 1e-6; the test reports
+# how many outputs are not the rounding of y_ref itself. fp32 outputs: within
+# 1e-5 relative + 1e-6 (fast exponential). States are raw input copies: bit-exact.
+CONV_FP32 = (4e-6, 1e-6)
+
 
 def _conv_ref(x, w, cu=None, st=None):
     return oracle.short_conv_swish(host(x).reshape(x.shape[0], -1), host(w),
@@ -489,11 +495,19 @@ def _conv_ref(x, w, cu=None, st=None):
 
 
 def _conv_close(y, y_ref, dtype, label):
-    rel = 1.01 * 2.0 ** -8 if dtype == torch.bfloat16 else 1e-5
-    err = np.abs(host(y).reshape(y_ref.shape) - y_ref)
-    bound = rel * np.abs(y_ref) + 1e-6
-    assert np.isfinite(err).all(), label
-    assert np.all(err <= bound), "%s: worst excess %.3e" % (label, float((err - bound).max()))
+    got = host(y).reshape(y_ref.shape)
+    assert np.isfinite(got).all(), label
+    if dtype != torch.bfloat16:
+        err = np.abs(got - y_ref)
+        assert np.all(err <= 1e-5 * np.abs(y_ref) + 1e-6), "%s: worst excess %.3e" % (
+            label, float((err - 1e-5 * np.abs(y_ref) - 1e-6).max()))
+        return 0
+    delta = CONV_FP32[0] * np.abs(y_ref) + CONV_FP32[1]
+    lo, hi = bf16_neighbours(y_ref - delta)[0], bf16_neighbours(y_ref + delta)[0]
+    ok = (got >= lo) & (got <= hi)
+    assert ok.all(), "%s: %d outputs are not a bf16 rounding of a value within the fp32 error (worst |y - y_ref| = %.3e)" % (
+        label, int((~ok).sum()), float(np.abs(got - y_ref)[~ok].max()))
+    return int((got != bf16_neighbours(y_ref)[0]).sum())  # not the rounding of y_ref itself
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
