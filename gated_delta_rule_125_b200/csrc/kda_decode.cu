@@ -8,12 +8,16 @@
 //
 // The step is HBM-bound: per (sequence, head) it reads and writes the fp32
 // d_k x d_v state (64 KiB each way at d = 128) and touches < 1.5 KiB of
-// token inputs. One CTA of 256 threads owns one (sequence, head) state:
-// thread (row group, column group) keeps R rows x 4 contiguous columns of S
-// in registers, so every warp access is a coalesced 16-byte-per-lane sweep
-// (read once, evict-first; written once, streaming). The two column sums
-// over d_k (S~^T k and S~^T q) are per-thread partial sums finished through
-// shared memory; nothing else touches HBM.
+// token inputs. CTAs of 256 threads own the state columns of one (sequence,
+// head): all d_v of them, or (the plain step at d_v = 128) half of them, since
+// the columns are independent (each needs its own column sums and k . q,
+// which every CTA forms). Two CTAs per state halve the registers a thread
+// needs, so twice as many CTAs (and bytes in flight) fit on an SM. Thread (row
+// group, column group) keeps R rows x 4 contiguous columns of S in registers,
+// so every warp access is a coalesced 16-byte-per-lane sweep (read once,
+// evict-first; written once, streaming). The two column sums over d_k (S~^T k
+// and S~^T q) are per-thread partial sums finished through shared memory;
+// nothing else touches HBM.
 //
 // Optionally the layer's causal short convolution + Swish (§6.1) is applied to
 // q, k, v as they are loaded: the step's raw projection and the channel's last

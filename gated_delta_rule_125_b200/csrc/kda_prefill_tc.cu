@@ -57,10 +57,12 @@ constexpr int kMaxRing = 16;                 // ring slots per stream, upper bou
 // ---------------------------------------------------------------- slot ----
 // One ring slot per item, bytes (every tile 1024-byte aligned):
 //   WQ [Q e^G ; W]   128 x 128 bf16, K-major SW128      (A operand of [Qg;W] S)
-//   KD K e^{Gl-G}    64 (r) x 128 (c) bf16, MN-major     (A operand of Kd^T U)
+//   KD K e^-G        64 (r) x 128 (c) bf16, MN-major     (A operand of Kd^T U)
 //   T                64 x 64 bf16, K-major               (A operand of T V)
 //   P                64 x 64 bf16, K-major               (A operand of P U)
-//   D  e^{G_last}    128 fp32
+//   D  e^{G_last}, DZ  2 x 128 fp32: the scan forms S' = Diag(D) S + Diag(DZ) Kd^T U,
+//                    so DZ = e^{G_last} with KD = K e^-G; a chunk past kTau ships
+//                    KD = K e^{G_last - G} (element-wise exponents) with DZ = 1
 constexpr uint32_t SL_WQ = 0, SL_KD = 32768, SL_T = 49152, SL_P = 57344, SL_D = 65536;
 constexpr uint32_t SL_BYTES = 66560;
 
