@@ -379,6 +379,13 @@ def run_kda(args, world, rank, local):
         kda.kda_prefill(conv_out[0].view(T8K, H, D), conv_out[1].view(T8K, H, D), conv_out[2].view(T8K, H, D),
                         la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws)
 
+    # the same, with the convolution inside the prefill's loads (kda_prefill_conv)
+    fused_conv = tuple((w, st, so) for (x, w, st), so in zip(conv_in, conv_st))
+
+    def prefill_conv():
+        kda.kda_prefill(conv_in[0][0].view(T8K, H, D), conv_in[1][0].view(T8K, H, D), conv_in[2][0].view(T8K, H, D),
+                        la, beta, S0, cu, max_seqlen=T8K, o=o, S_T=S_T, workspace=ws, conv=fused_conv)
+
     # Three short convolutions (two launches each, ~30 us of GPU time): the host issues them
     # more slowly than the GPU runs them, so the convolution line replays them from a CUDA
     # graph (captured once).
@@ -397,9 +404,11 @@ def run_kda(args, world, rank, local):
     except RuntimeError:
         conv_graph = None
     conv_ms = {}
-    for name, fn in (("conv", conv_graph.replay if conv_graph is not None else convs), ("conv_prefill", conv_prefill)):
+    for name, fn in (("conv", conv_graph.replay if conv_graph is not None else convs), ("conv_prefill", conv_prefill),
+                     ("prefill_conv", prefill_conv)):
         conv_ms[name] = timed(fn, args.steps, args.warmup, world, dev, stream)
     launches += args.steps * (3 * conv_launches) + args.steps * (3 * conv_launches + launches_prefill)
+    launches += args.steps * (launches_prefill + 3)  # the fused form: prefill launches + three conv-state kernels
     conv_gbs = 3 * CONV_BYTES / (conv_ms["conv"][0] * 1e-3) / 1e9
     conv_graph_used = conv_graph is not None
     del conv_graph, conv_in, conv_out, conv_st
@@ -583,6 +592,10 @@ def run_kda(args, world, rank, local):
                                    "([8192, 32*128] bf16 each, states written; page section 6.1)" % CONV_W,
                        "conv_then_prefill": {"value": world * T8K / (conv_ms["conv_prefill"][1] * 1e-3),
                                              "unit": "tokens/s", "ms_per_step": conv_ms["conv_prefill"][1]},
+                       "prefill_conv": {"value": world * T8K / (conv_ms["prefill_conv"][1] * 1e-3),
+                                        "unit": "tokens/s", "ms_per_step": conv_ms["prefill_conv"][1],
+                                        "kernel": "kda_prefill_conv: the convolution of q, k in the prep engines' "
+                                                  "loads and of v on the scan CTAs, then the three conv states"},
                        "roofline": {"bound": "hbm", "achieved": conv_gbs, "peak": hbm, "unit": "GB/s",
                                     "frac": conv_gbs / hbm, "traffic": None,
                                     "kernel": "conv_kernel<4,bf16> + conv_state_kernel (x3)",

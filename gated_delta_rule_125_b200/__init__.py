@@ -32,7 +32,7 @@ EXPORTED_SYMBOLS = ("kda_status_string", "kda_version", "kda_prefill_workspace_s
                     "kda_prefill_ex", "kda_decode_step", "kda_decode_step_ex", "kda_device_error",
                     "kda_prefill_noalloc", "kda_short_conv_swish", "kda_short_conv_launches",
                     "kda_decode_step_conv", "kda_backward_workspace_size", "kda_backward",
-                    "kda_set_wait_limit_ns")
+                    "kda_set_wait_limit_ns", "kda_prefill_conv")
 
 
 class OutputGate(ctypes.Structure):
@@ -105,6 +105,9 @@ def load_library():
     lib.kda_decode_step_conv.argtypes = [vp, vp, vp, fp, fp, fp, i32, i32, i32, i32, ctypes.c_int,
                                          u32, sc, sc, sc, og, vp, vp]
     lib.kda_decode_step_conv.restype = ctypes.c_int
+    lib.kda_prefill_conv.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32, i32,
+                                     ctypes.c_int, i32, u32, sc, sc, sc, og, vp, fp, vp, sz, vp]
+    lib.kda_prefill_conv.restype = ctypes.c_int
     lib.kda_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, ctypes.c_int, i32, u32]
     lib.kda_backward_workspace_size.restype = sz
     lib.kda_backward.argtypes = [vp, vp, vp, fp, fp, fp, ip, i32, i64, i32, i32, i32, i32, ctypes.c_int, i32, u32,
@@ -208,7 +211,7 @@ def kda_prefill_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, w
 
 def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqlen=None,
                 chunk=64, l2norm=True, exact=False, o=None, S_T=None, workspace=None,
-                out_gate=None, stream=None):
+                out_gate=None, conv=None, stream=None):
     """Chunkwise KDA prefill (``kda_prefill`` in ``include/kda.h``).
 
     q, k ``[T,H,dk]``, v ``[T,H,dv]`` (bf16 or fp32), log_alpha ``[T,H,dk]`` fp32
@@ -217,7 +220,10 @@ def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqle
     the workspace are allocated with torch when not given. ``max_seqlen`` (host
     int) avoids a device-to-host read of ``cu_seqlens``. ``out_gate = (gate
     [T,H,dv] (dtype of q), weight [dv] fp32, eps)`` fuses the layer's output step
-    (``kda_prefill_ex``): o <- RMSNorm(o) * weight * sigmoid(gate).
+    (``kda_prefill_ex``): o <- RMSNorm(o) * weight * sigmoid(gate). ``conv=(cq, ck, cv)``,
+    each None or ``(weight [H*d, W] fp32, state_in, state_out)`` with states
+    ``[N, W-1, H*d]`` (None: zeros / not written): q, k, v are the raw projections and the
+    short convolution + Swish runs inside the prefill's loads (``kda_prefill_conv``).
     """
     lib = load_library()
     T, H, dk = q.shape
@@ -241,10 +247,17 @@ def kda_prefill(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, max_seqle
         if nbytes == 0:
             nbytes = 256
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    rc = lib.kda_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
-                            _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, code, chunk, flags,
-                            _out_gate(out_gate), _ptr(o), _ptr(S_T), _ptr(workspace),
-                            workspace.numel(), _stream(stream, dev))
+    if conv is None:
+        rc = lib.kda_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, code, chunk, flags,
+                                _out_gate(out_gate), _ptr(o), _ptr(S_T), _ptr(workspace),
+                                workspace.numel(), _stream(stream, dev))
+    else:
+        cq, ck, cv = conv
+        rc = lib.kda_prefill_conv(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                                  _ptr(cu_seqlens), N, T, int(max_seqlen), H, dk, dv, code, chunk, flags,
+                                  _conv(cq), _conv(ck), _conv(cv), _out_gate(out_gate), _ptr(o), _ptr(S_T),
+                                  _ptr(workspace), workspace.numel(), _stream(stream, dev))
     if rc != KDA_OK:
         raise KDAError(rc, "kda_prefill")
     return o, S_T

@@ -232,12 +232,17 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
                           workspace_bytes, stream);
 }
 
-kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const float *log_alpha,
-                          const float *beta, const float *S0, const int32_t *cu_seqlens,
-                          int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
-                          int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
-                          const kda_output_gate *out_gate, void *o, float *S_T, void *workspace,
-                          size_t workspace_bytes, kda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// kda_prefill_ex and kda_prefill_conv: `conv` holds the three inputs' short
+// convolutions (nullptr entries, or a nullptr array: none).
+kda_status prefill_impl(const void *q, const void *k, const void *v, const float *log_alpha,
+                        const float *beta, const float *S0, const int32_t *cu_seqlens, int32_t num_seqs,
+                        int64_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
+                        kda_dtype dtype, int32_t chunk, uint32_t flags, const kda_short_conv *const *conv,
+                        const kda_output_gate *out_gate, void *o, float *S_T, void *workspace,
+                        size_t workspace_bytes, kda_stream_t stream) {
     kda_status rc = check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags);
     if (rc != KDA_OK) return rc;
     if ((rc = check_output_gate(out_gate, total_tokens > 0)) != KDA_OK) return rc;
@@ -251,6 +256,16 @@ kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const flo
     if (!gate_aligned(log_alpha, flags)) return KDA_ERR_MISALIGNED;
 
     Plan p = make_plan(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, flags);
+    bool any_conv = false;
+    for (int i = 0; conv && i < 3; ++i) {
+        const kda_short_conv *c = conv[i];
+        if (!c) continue;
+        if (!p.tc || c->width < 1 || c->width > kda::kPrefillMaxConvWidth) return KDA_ERR_UNSUPPORTED;
+        if (!c->weight) return KDA_ERR_INVALID_ARG;
+        if (reinterpret_cast<uintptr_t>(c->weight) & 3u) return KDA_ERR_MISALIGNED;
+        if (!aligned16(c->state_in) || !aligned16(c->state_out)) return KDA_ERR_MISALIGNED;
+        any_conv = true;
+    }
     if (workspace_bytes < min_bytes(p)) return KDA_ERR_WORKSPACE;
 
     kda::PrefillArgs a;
@@ -265,6 +280,12 @@ kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const flo
     a.og_eps = out_gate ? out_gate->eps : 0.f;
     a.o = o; a.S_T = S_T;
     a.slot_bytes = p.slot_bytes;
+    for (int i = 0; i < 3; ++i) {
+        const kda_short_conv *c = conv ? conv[i] : nullptr;
+        a.conv_W[i] = c ? c->width : 0;
+        a.conv_w[i] = c ? c->weight : nullptr;
+        a.conv_state[i] = c ? c->state_in : nullptr;
+    }
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     char *ws = static_cast<char *>(workspace);
@@ -274,7 +295,25 @@ kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const flo
         if (!err) return KDA_ERR_CUDA;
         a.state = nullptr;
         a.slots = nullptr;
-        return kda::tc_prefill(a, ws, workspace_bytes, p.streams, err, st) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+        if (kda::tc_prefill(a, ws, workspace_bytes, p.streams, err, st) != cudaSuccess) return KDA_ERR_CUDA;
+        // each sequence's last W-1 raw inputs, after the prefill has read the initial states
+        for (int i = 0; any_conv && i < 3; ++i) {
+            const kda_short_conv *c = conv[i];
+            if (!c || !c->state_out || c->width < 2) continue;
+            kda::ShortConvArgs sa;
+            sa.x = i == 0 ? q : i == 1 ? k : v;
+            sa.y = nullptr;
+            sa.w = c->weight;
+            sa.state_in = c->state_in;
+            sa.state_out = c->state_out;
+            sa.cu = cu_seqlens;
+            sa.N = num_seqs;
+            sa.total = total_tokens;
+            sa.C = H * (i == 2 ? dv : dk);
+            sa.W = c->width;
+            if (kda::short_conv_state(sa, true, st) != cudaSuccess) return KDA_ERR_CUDA;
+        }
+        return KDA_OK;
     }
     const int64_t nw = waves_chunks(p, workspace_bytes);
     const bool multi = nw < p.max_chunks;
@@ -289,6 +328,31 @@ kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const flo
     }
     if (a.og_gate && total_tokens > 0 && kda::simt_output_gate(a, bf16, st) != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+kda_status kda_prefill_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *S0, const int32_t *cu_seqlens,
+                          int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                          int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                          const kda_output_gate *out_gate, void *o, float *S_T, void *workspace,
+                          size_t workspace_bytes, kda_stream_t stream) {
+    return prefill_impl(q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                        dtype, chunk, flags, nullptr, out_gate, o, S_T, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_prefill_conv(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, const float *S0, const int32_t *cu_seqlens,
+                            int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                            int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                            const kda_short_conv *conv_q, const kda_short_conv *conv_k,
+                            const kda_short_conv *conv_v, const kda_output_gate *out_gate, void *o,
+                            float *S_T, void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    const kda_short_conv *conv[3] = {conv_q, conv_k, conv_v};
+    return prefill_impl(q, k, v, log_alpha, beta, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                        dtype, chunk, flags, conv, out_gate, o, S_T, workspace, workspace_bytes, stream);
 }
 
 kda_status kda_device_error(int32_t *code, int32_t reset) {

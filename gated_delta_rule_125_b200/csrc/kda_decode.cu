@@ -61,7 +61,7 @@ __device__ __forceinline__ void conv_swish_lane(const T *__restrict__ xrow, int 
             if (j < W - 1) z = fmaf(wv[m][j], h[m][j < kMaxConvW - 1 ? j : 0], z);
             else if (j == W - 1) z = fmaf(wv[m][j], xv[m], z);
         }
-        out[m] = __fdividef(z, 1.f + __expf(-z));
+        out[m] = swish(z);
     }
     if (sout) {
 #pragma unroll

@@ -13,6 +13,19 @@ namespace kda {
 
 constexpr int kChunk = 64;  // chunk length C of the chunkwise prefill
 
+// Swish of the short convolution ("[Kimi-2] Kimi Linear" §6.1): z sigmoid(z) =
+// z / (1 + 2^(-z log2 e)) with the hardware's approximate 2^x and reciprocal (PTX
+// ex2.approx / rcp.approx, relative errors about 2^-22 and 2^-23) and every other
+// operation an explicit round-to-nearest one, so that each convolution kernel (and the
+// pair form in kda_tc.cuh) gets the same bits. A large negative z gives e = inf and -0.
+constexpr float kSwishNegLog2e = -1.4426950408889634f;
+__device__ __forceinline__ float swish(float z) {
+    float e, r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(__fmul_rn(z, kSwishNegLog2e)));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(__fadd_rn(1.f, e)));
+    return __fmul_rn(z, r);
+}
+
 // Element I/O for the two input/output dtypes; arithmetic is always fp32.
 template <typename T> struct IO;
 template <> struct IO<float> {
@@ -53,6 +66,12 @@ struct PrefillArgs {
     float og_eps;
     void *o;
     float *S_T;
+    // causal short convolution + Swish fused into the loads of q, k, v (index 0, 1, 2;
+    // tensor-core path): window (0: the input is used as it is), taps [H * d][W] fp32,
+    // initial states [N][W - 1][H * d] in the io dtype (nullptr: zeros)
+    int conv_W[3];
+    const float *conv_w[3];
+    const void *conv_state[3];
     // workspace
     float *state;      // running state between waves ([N][H][dk][dv]) or nullptr
     char *slots;       // per-chunk slots of this wave
@@ -105,6 +124,9 @@ struct ShortConvArgs {
     int C, W;
 };
 cudaError_t short_conv_swish(const ShortConvArgs &a, bool bf16, cudaStream_t st);
+// Only the final states (state_out from x and state_in; a.y unused).
+cudaError_t short_conv_state(const ShortConvArgs &a, bool bf16, cudaStream_t st);
+constexpr int kPrefillMaxConvWidth = 4;  // KDA_PREFILL_MAX_CONV_WIDTH
 int short_conv_launches(int W, bool state_out, int64_t total);
 
 constexpr int kDecodeMaxConvWidth = 4;  // widest window the decode step fuses

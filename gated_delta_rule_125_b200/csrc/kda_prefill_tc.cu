@@ -70,8 +70,8 @@ constexpr uint32_t SL_BYTES = 66560;
 // [header 256 B][L: int64 per stream][order: int32 per stream] (1 KiB)
 // [ustart: int64 per unit][nch: int32 per unit] (1 KiB aligned)
 // [ready: int32 x kMaxStreams*kMaxRing][freed: same]
-// [output-step exchange: per scan CTA, 2 x 64 words (row sum of squares, position tag)]
 // [ring: NS*R slots]
+// [output-step exchange: per scan CTA, 4 x 64 words (row sum of squares, position tag)]
 struct Hdr {
     unsigned long long claim;  // next item to claim
     long long total;           // items over all streams
@@ -85,16 +85,20 @@ constexpr size_t kFlagInts = (size_t)kTcMaxStreams * kMaxRing;
 __host__ __device__ inline size_t ru1024(size_t x) { return (x + 1023) & ~size_t(1023); }
 __host__ __device__ inline size_t ws_nch(long long NH) { return WS_USTART + 8 * (size_t)NH; }
 __host__ __device__ inline size_t ws_flags(long long NH) { return ru1024(ws_nch(NH) + 4 * (size_t)NH); }
-__host__ __device__ inline size_t ws_xch(long long NH) { return ws_flags(NH) + 2 * kFlagInts * sizeof(int); }
-constexpr size_t kXchWords = (size_t)kTcMaxStreams * 2 * 2 * 64;
-__host__ __device__ inline size_t ws_ring(long long NH) { return ru1024(ws_xch(NH) + kXchWords * 8); }
+__host__ __device__ inline size_t ws_ring(long long NH) { return ru1024(ws_flags(NH) + 2 * kFlagInts * sizeof(int)); }
+constexpr size_t kXchWords = (size_t)kTcMaxStreams * 2 * 4 * 64;
+__host__ __device__ inline size_t ws_xch(long long NH, int ns, int R) { return ws_ring(NH) + (size_t)ns * R * SL_BYTES; }
 
 struct FusedParams {
     CUtensorMap tmap_la;  // log_alpha [T][H][128] fp32, box 128 x 1 x 64
     CUtensorMap tmap_v;   // v [T][H][128] bf16, box 64 x 1 x 64, SW128
     CUtensorMap tmap_q;   // q, k: as v
     CUtensorMap tmap_k;
-    const bf16 *q, *k;
+    const bf16 *q, *k, *v;
+    // causal short convolution + Swish fused into the loads of q, k, v (index 0, 1, 2)
+    int cw[3];           // window (0: the input as it is), at most 4
+    const float *cwt[3];  // taps [H * 128][W]
+    const bf16 *cst[3];   // initial states [N][W - 1][H * 128] (nullptr: zeros)
     const float *beta, *S0;
     const float *la;  // log_alpha, read directly when it is one gate per (token, head)
     const int32_t *cu;
@@ -152,7 +156,7 @@ __device__ __forceinline__ bool mbar_wait_call(uint64_t *bar, uint32_t parity, c
 // decreasing length, and zeroed counters and ring flags.
 constexpr int PLAN_T = 1024;
 __global__ void __launch_bounds__(PLAN_T)
-plan_kernel(const int32_t *__restrict__ cu, long long total, int N, int H, int ns, char *__restrict__ ws) {
+plan_kernel(const int32_t *__restrict__ cu, long long total, int N, int H, int ns, int R, char *__restrict__ ws) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long NH = (long long)N * H;
     Hdr *hd = reinterpret_cast<Hdr *>(ws);
@@ -167,7 +171,7 @@ plan_kernel(const int32_t *__restrict__ cu, long long total, int N, int H, int n
         nch[u] = (int)((eos - bos + C - 1) / C);
     }
     for (size_t i = tid; i < 2 * kFlagInts; i += PLAN_T) flags[i] = 0;
-    for (size_t i = tid; i < kXchWords; i += PLAN_T) reinterpret_cast<unsigned long long *>(ws + ws_xch(NH))[i] = 0;
+    for (size_t i = tid; i < kXchWords; i += PLAN_T) reinterpret_cast<unsigned long long *>(ws + ws_xch(NH, ns, R))[i] = 0;
     __syncthreads();
     // one warp per stream: lanes own contiguous runs of the stream's units
     for (int st = warp; st < ns; st += PLAN_T / 32) {
@@ -218,8 +222,9 @@ constexpr uint32_t PS_GB = PS_GA + 32768;      // q of the next item, then K e^-
 constexpr uint32_t PS_KS = PS_GB + 16384;      // k of the next item (K-major 64 x 128)
 constexpr uint32_t PS_SMALL = PS_KS + 16384;   // invq[64] invk[64] beta[2][64] eGl[128] gate[2][64]
 constexpr uint32_t PS_BAR = PS_SMALL + 2048;   // la, mma, q/k barriers; 3 item records; flags
-constexpr uint32_t PS_BYTES = PS_BAR + 256;
-constexpr uint32_t PS_STRIDE = 101376;         // engine 1 starts here (1024-aligned)
+constexpr uint32_t PS_HALO = PS_BAR + 256;     // fused convolution: 3 raw rows before the item, q and k
+constexpr uint32_t PS_BYTES = PS_HALO + 1536;
+constexpr uint32_t PS_STRIDE = 102400;         // engine 1 starts here (1024-aligned)
 constexpr int ALD = 68;                        // row stride of A / X (floats)
 constexpr uint32_t PS_AF = PS_LA;              // A, then X in place: 64 x 68 fp32
 constexpr uint32_t PS_T = PS_LA + 17408;       // T, 64 x 64 bf16 K-major (1024-aligned)
@@ -240,7 +245,8 @@ constexpr uint32_t SS_S = SS_V + 4 * SV_BYTES;  // [128 (c)][64 (j)] MN-major bf
 constexpr uint32_t SS_U = SS_S + 16384;         // [64 (r)][64 (j)] MN-major bf16 pseudo-values
 constexpr uint32_t SS_BAR = SS_U + 8192;        // 31 mbarriers, the consumed-position counter, a flag
 constexpr uint32_t SS_OGW = SS_BAR + 512;       // output-step weights of this CTA's 64 columns
-constexpr uint32_t SS_BYTES = SS_OGW + 256;
+constexpr uint32_t SS_VPREV = SS_OGW + 256;     // fused convolution of v: raw rows 61..63 of the last tile
+constexpr uint32_t SS_BYTES = SS_VPREV + 384;
 constexpr uint32_t COPY_A = 32768 + 16384, COPY_B = 8192 + 8192 + 1024;
 constexpr int NY = 4;  // Y buffers in TMEM: the O epilogue may lag NY - 1 chunks
 constexpr uint32_t TM_X = 0, TM_Y = 128, TM_Z = TM_Y + 64 * NY;  // scan TMEM columns: X x2, Y x NY, Z
@@ -250,7 +256,9 @@ constexpr int MB_FULLA = 0, MB_FULLB = 2, MB_FULLV = 5, MB_EMPTYA = 9, MB_EMPTYB
               MB_U = 18, MB_S = 19, MB_O = 20,  // MB_O and MB_OREADY: one barrier per Y buffer
               MB_UREADY = MB_O + NY, MB_SREADY = MB_UREADY + 1, MB_FIN = MB_SREADY + 1, MB_OREADY = MB_FIN + 1,
               MB_X = MB_OREADY + NY,  // one per X buffer: T V of a position complete
-              MB_FIN2 = MB_X + 2, MB_COUNT = MB_FIN2 + 1;
+              MB_FIN2 = MB_X + 2,
+              MB_CV = MB_FIN2 + 1,  // four, one per V buffer: the fused convolution of the tile is done
+              MB_COUNT = MB_CV + 4;
 
 // Per-CTA control block after both layouts.
 struct Ctrl {
@@ -276,9 +284,10 @@ static_assert(sizeof(Ctrl) <= 512, "control block");
 struct ItemS {
     long long t0, p;  // first token; position in the stream
     int n, h, st, valid;
+    int s, first;     // sequence; the item is its first chunk
     int slot, gen;    // ring slot (stream st, position p % R) and its generation p / R
 };
-static_assert(3 * 8 + 3 * sizeof(ItemS) + 3 * 4 <= PS_BYTES - PS_BAR, "prep barrier block: mbarriers, item records, flags");
+static_assert(3 * 8 + 3 * sizeof(ItemS) + 3 * 4 <= PS_HALO - PS_BAR, "prep barrier block: mbarriers, item records, flags");
 
 
 // Item g of the global claim order: position-major over the streams still
@@ -329,6 +338,8 @@ __device__ bool map_item(unsigned long long g, const FusedParams &P, const Ctrl 
     }
     it.t0 = bos + j * C;
     it.n = (int)((eos - it.t0) < C ? (eos - it.t0) : C);
+    it.s = s;
+    it.first = j == 0;
     it.h = (int)((unsigned)u % (unsigned)P.H);
     it.st = st;
     it.p = p;
@@ -373,6 +384,7 @@ __device__ __forceinline__ void warp_gemm_16x8(int lane, FA A, FB B, float (&acc
 // Prep engine e (threads 256 e .. 256 e + 255) with its shared memory `sm` and
 // TMEM columns [tm, tm + 256). Named barriers 1 + e (the engine) and 3 + 2e,
 // 4 + 2e (warp pairs of the solve).
+template <bool CV>
 __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ctl, int e, uint8_t *sm,
                                             uint32_t tm) {
     const int tid = (int)threadIdx.x - PT * e, warp = tid >> 5, lane = tid & 31;
@@ -385,6 +397,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
     uint8_t *GA = sm + PS_GA;
     uint8_t *GB = sm + PS_GB;
     uint8_t *KS = sm + PS_KS;
+    uint8_t *HALO = sm + PS_HALO;
     float *invq = reinterpret_cast<float *>(sm + PS_SMALL);
     float *invk = invq + 64, *sbeta2 = invk + 64, *eGl = sbeta2 + 128, *sgate2 = eGl + 128;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PS_BAR);  // [0] log_alpha box, [1] MMA, [2] q, k boxes
@@ -453,8 +466,85 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             const size_t row = (size_t)(it.t0 + (tid < it.n ? tid : 0)) * H + it.h;
             cp_async4(sbeta2 + buf * 64 + tid, P.beta + row, tid < it.n ? 4u : 0u);
             if (P.la_scalar) cp_async4(sgate2 + buf * 64 + tid, P.la + row, tid < it.n ? 4u : 0u);
+        } else if (CV && tid < C + 96) {  // fused convolution: raw rows t0 - 3 .. t0 - 1 of q and k
+            const int hid = tid - C, tsel = hid / 48, jh = (hid % 48) >> 4, cc = hid & 15;
+            const int W = P.cw[tsel];
+            if (W > 0) {
+                const bf16 *x = tsel ? P.k : P.q;
+                const bf16 *srcp = x;
+                uint32_t bytes = 0;
+                if (!it.first) {  // inside the sequence
+                    srcp = x + ((size_t)(it.t0 - 3 + jh) * H + it.h) * DK + cc * 8;
+                    bytes = 16;
+                } else if (P.cst[tsel] != nullptr && jh + W - 4 >= 0) {  // before it: the initial state
+                    srcp = P.cst[tsel] + ((size_t)it.s * (W - 1) + (jh + W - 4)) * ((size_t)H * DK) + (size_t)it.h * DK + cc * 8;
+                    bytes = 16;
+                }
+                cp_async16(HALO + ((tsel * 3 + jh) * 16 + cc) * 16, srcp, bytes);
+            }
         }
         cp_async_commit();
+    };
+
+    // Fused short convolution + Swish of q (threads 0..127) and k (128..255), in place on
+    // the item's GB / KS tiles (before the row norms): warp (tensor, row segment seg) takes
+    // rows 16 seg .. 16 seg + 15, lane c4 channels 4 c4 .. 4 c4 + 3, with the three raw
+    // rows before them from the halo (seg 0) or from the tile before any row is rewritten.
+    // The same arithmetic as the standalone convolution kernel: taps oldest first, one fma
+    // each, then z / (1 + e^-z), rounded to bf16.
+    auto conv_qk = [&](const ItemS &it) {
+        const int tsel = tid >> 7, seg = (tid >> 5) & 3, c4 = tid & 31;
+        const int W = P.cw[tsel];
+        uint8_t *tile = tsel ? KS : GB;
+        const uint32_t cofs = (uint32_t)(c4 & 1) * 8;  // within the 16-byte chunk c4 / 2
+        f2_t wp[2][4], win[3][2];
+        if (W > 0) {
+            const float *wt = P.cwt[tsel] + ((size_t)it.h * DK + c4 * 4) * W;
+#pragma unroll
+            for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int jj = j - (4 - W);  // taps padded in front to four
+                    wp[pr][j] = jj >= 0 ? f2(__ldg(wt + (2 * pr) * W + jj), __ldg(wt + (2 * pr + 1) * W + jj)) : f2(0.f, 0.f);
+                }
+#pragma unroll
+            for (int jh = 0; jh < 3; ++jh) {
+                const uint2 u = seg == 0 ? *reinterpret_cast<const uint2 *>(HALO + ((tsel * 3 + jh) * 16 + (c4 >> 1)) * 16 + cofs)
+                                         : *reinterpret_cast<const uint2 *>(tile + kmaj_chunk(16 * seg - 3 + jh, c4 >> 1, 64) + cofs);
+                win[jh][0] = unpack2(u.x);
+                win[jh][1] = unpack2(u.y);
+            }
+        }
+        sync();  // every window is read before a row is rewritten
+        if (W > 0) {
+            uint8_t *base = tile + kmaj_chunk(16 * seg, c4 >> 1, 64) + cofs;
+#pragma unroll
+            for (int r8 = 0; r8 < 16; r8 += 8) {  // eight rows at a time, loads first
+                uint2 u[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    u[i] = *reinterpret_cast<const uint2 *>(base + (r8 + i) * 128 + ((((c4 >> 1) ^ (r8 + i)) & 7) - ((c4 >> 1) & 7)) * 16);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const f2_t x[2] = {unpack2(u[i].x), unpack2(u[i].y)};
+                    uint32_t ow[2];
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        f2_t z = f2fma(wp[pr][0], win[0][pr], f2(0.f, 0.f));
+                        z = f2fma(wp[pr][1], win[1][pr], z);
+                        z = f2fma(wp[pr][2], win[2][pr], z);
+                        z = f2fma(wp[pr][3], x[pr], z);
+                        ow[pr] = pack2(swish2(z));
+                        win[0][pr] = win[1][pr];
+                        win[1][pr] = win[2][pr];
+                        win[2][pr] = x[pr];
+                    }
+                    *reinterpret_cast<uint2 *>(base + (r8 + i) * 128 + ((((c4 >> 1) ^ (r8 + i)) & 7) - ((c4 >> 1) & 7)) * 16) =
+                        make_uint2(ow[0], ow[1]);
+                }
+            }
+        }
+        sync();
     };
 
     if (tid == kStoreTid) claim(sitem[0]);
@@ -492,6 +582,9 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
             qk_phase ^= 1;
         }
         sync();
+        if constexpr (CV) {
+            if (!sflag[1]) conv_qk(cur);
+        }
         if (tid < DK) {
             const float *sgate = sgate2 + (iter & 1) * 64;
             if (!P.la_scalar && !mbar_wait(&bars[0], la_phase, kWaitNs)) sflag[1] = 1;
@@ -870,6 +963,7 @@ __device__ __forceinline__ void prep_engine(const FusedParams &P, const Ctrl *ct
 // 64..127 hold W S and T V (their difference is U); Z = Kd^T U fills all 128.
 // The 128-row A operands of T V and P U take the 64 rows next to T (before) and
 // P (after) as filler whose output rows are never read.
+template <bool OG, bool CV>
 __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uint32_t tm, int st, int jv) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ns = P.ns, R = P.R, H = P.H;
@@ -885,7 +979,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
     uint64_t *fullA = bars + MB_FULLA, *fullB = bars + MB_FULLB, *fullV = bars + MB_FULLV, *emptyA = bars + MB_EMPTYA,
              *emptyB = bars + MB_EMPTYB, *emptyV = bars + MB_EMPTYV, *bU = bars + MB_U, *bS = bars + MB_S,
              *bO = bars + MB_O, *uready = bars + MB_UREADY, *sready = bars + MB_SREADY, *bFin = bars + MB_FIN,
-             *oready = bars + MB_OREADY, *bX = bars + MB_X, *bFin2 = bars + MB_FIN2;
+             *oready = bars + MB_OREADY, *bX = bars + MB_X, *bFin2 = bars + MB_FIN2, *convV = bars + MB_CV;
     auto unit_bounds = [&](long long kk, int &s, int &h, int64_t &bos, int64_t &eos) {
         const long long u = st + kk * ns;
         s = (int)(u / H);
@@ -1040,95 +1134,231 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
     }
     if (warp == 12 || warp == 13) {
         // ---------------- O rows (warps 12, 13: TMEM lanes 0..63) ----------------
-        // With the fused output step, a row's RMSNorm needs the partner CTA's 64
-        // columns: each thread publishes its row's sum of squares with the position
-        // as tag in one 8-byte word and polls the partner's word for the same row
-        // (two words per row alternate by position parity; a word is rewritten two
-        // positions later, after its reader has moved past it).
         const int c = (warp & 3) * 32 + lane;  // chunk row
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const bool gated = P.og_gate != nullptr;
+        constexpr bool gated = OG;
         float *sw = reinterpret_cast<float *>(sm + SS_OGW);
-        unsigned long long *xw = reinterpret_cast<unsigned long long *>(P.ws + ws_xch(NH));
+        unsigned long long *xw = reinterpret_cast<unsigned long long *>(P.ws + ws_xch(NH, P.ns, P.R));
         if (gated) {
-            sw[c] = P.og_w[jv * DVT + c];
+            sw[c] = 0.5f * P.og_w[jv * DVT + c];
             bar_sync(7, 64);
         }
+        // Row c of position q (Y buffer q % NY) to o: as it is, or with the output step
+        // y * scale * w * sigmoid(g) = a + a tanh(g / 2), a = y scale (w / 2), in fp32 pairs.
+        auto store_row = [&](long long q, int64_t t, int h, long long nn, float scale, const uint4 (&graw)[8]) {
+            const uint32_t ybuf = tm + TM_Y + (uint32_t)(q % NY) * 64 + lane_base;
+            bf16 *dst = P.o + ((size_t)t * H + h) * DV + jv * DVT;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float y[32];
+                tmem_ld32(ybuf + half * 32, y);
+                tmem_wait_ld();
+                if (c < nn) {
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8) {
+                        uint32_t ow[4];
+                        if (gated) {
+                            const uint4 gr = graw[half * 4 + q8];
+                            const uint32_t gw[4] = {gr.x, gr.y, gr.z, gr.w};
+                            const f2_t s2 = f2(scale, scale), h2 = f2(0.5f, 0.5f);
+#pragma unroll
+                            for (int w = 0; w < 4; ++w) {
+                                const f2_t g2 = f2mul(unpack2(gw[w]), h2);
+                                float tl, th;
+                                asm("tanh.approx.f32 %0, %1;" : "=f"(tl) : "f"(f2lo(g2)));
+                                asm("tanh.approx.f32 %0, %1;" : "=f"(th) : "f"(f2hi(g2)));
+                                const f2_t wv = *reinterpret_cast<const f2_t *>(sw + half * 32 + q8 * 8 + 2 * w);
+                                const f2_t a = f2mul(f2mul(f2(y[q8 * 8 + 2 * w], y[q8 * 8 + 2 * w + 1]), s2), wv);
+                                ow[w] = pack2(f2fma(a, f2(tl, th), a));
+                            }
+                        } else {
+#pragma unroll
+                            for (int w = 0; w < 4; ++w) ow[w] = pack2(f2(y[q8 * 8 + 2 * w], y[q8 * 8 + 2 * w + 1]));
+                        }
+                        reinterpret_cast<uint4 *>(dst)[half * 4 + q8] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&oready[q % NY]);  // Y[q % NY] may be overwritten (by Y(q + NY))
+        };
+        auto wait_o = [&](long long q) {  // O(q) complete
+            const bool r = __all_sync(0xffffffffu, mbar_wait_call(&bO[q % NY], (uint32_t)((q / NY) & 1), &hd->abort_flag));
+            tc_fence_after();
+            return r;
+        };
         bool ok = true;
         long long p = 0;
-        for (long long kk = 0; kk < K && ok; ++kk) {
-            int s, h;
-            int64_t bos, eos;
-            unit_bounds(kk, s, h, bos, eos);
-            const long long len = eos - bos, nch = (len + C - 1) / C;
-            for (long long j = 0; j < nch; ++j, ++p) {
-                const uint32_t ybuf = tm + TM_Y + (uint32_t)(p % NY) * 64 + lane_base;
-                // one bO barrier per Y buffer: it completes for positions p % NY, p % NY + NY, ...
-                // (the MMA thread may run up to NY - 1 positions ahead of these warps)
-                ok = __all_sync(0xffffffffu, mbar_wait_call(&bO[p % NY], (uint32_t)((p / NY) & 1), &hd->abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-                const long long nn = (len - j * C) < C ? (len - j * C) : C;
-                const int64_t t = bos + j * C + c;
-                const bf16 *grow = gated ? P.og_gate + ((size_t)t * H + h) * DV + jv * DVT : nullptr;
-                // this row's 64 gate pre-activations, loaded while the exchange runs
-                uint4 graw[8];
+        if (!gated) {
+            const uint4 none[8] = {};
+            // With the fused convolution of v (and no output step) these two warps also
+            // convolve the V tiles, two positions ahead of the O rows they store: lane l
+            // takes channels 2 l, 2 l + 1 of this CTA's 64, warp 12 rows 0..31 and warp 13
+            // rows 32..63 of the tile. Every raw row either warp needs is read before
+            // either rewrites one; warp 13 leaves raw rows 61..63 in VPREV for warp 12's
+            // window at the next chunk (a unit's first chunk reads the initial state).
+            const bool vconv = CV && P.cw[2] != 0;
+            const int hv = warp & 1, ch = jv * DVT + 2 * lane;  // first channel within the head
+            const int Wv = P.cw[2];
+            uint32_t *vprev = reinterpret_cast<uint32_t *>(sm + SS_VPREV);  // [3][32] raw pairs
+            long long vk = -1, vj = 0, vn = 0;  // the convolution's unit and chunk cursor
+            f2_t vw[4] = {0ull, 0ull, 0ull, 0ull};
+            f2_t vstate[3] = {0ull, 0ull, 0ull};  // warp 12: the unit's initial window
+            auto conv_v = [&](long long q) {  // the V tile of position q (positions in order)
+                bool unit_start = false;
+                while (vj >= vn) {  // the next unit with chunks: its taps and initial state
+                    int s, h;
+                    int64_t bos, eos;
+                    unit_bounds(++vk, s, h, bos, eos);
+                    vn = (eos - bos + C - 1) / C;
+                    vj = 0;
+                    unit_start = true;
+                    const float *wt = P.cwt[2] + ((size_t)h * DV + ch) * Wv;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        vw[j] = j - (4 - Wv) >= 0 ? f2(__ldg(wt + j - (4 - Wv)), __ldg(wt + Wv + j - (4 - Wv))) : f2(0.f, 0.f);
+#pragma unroll
+                    for (int jh = 0; jh < 3; ++jh) {
+                        const int js = jh + Wv - 4;
+                        vstate[jh] = (P.cst[2] != nullptr && js >= 0)
+                                         ? unpack2(*reinterpret_cast<const uint32_t *>(
+                                               P.cst[2] + ((size_t)s * (Wv - 1) + js) * ((size_t)H * DV) + (size_t)h * DV + ch))
+                                         : f2(0.f, 0.f);
+                    }
+                }
+                const int vb = (int)(q & 3);
+                if (!__all_sync(0xffffffffu, mbar_wait_call(&fullV[vb], (uint32_t)((q >> 2) & 1), &hd->abort_flag)))
+                    return false;
+                uint8_t *tile = sm + SS_V + vb * SV_BYTES;
+                auto word = [&](int r) {  // this lane's pair of row r (SW128 rows of 128 bytes)
+                    return reinterpret_cast<uint32_t *>(tile + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4);
+                };
+                const int r0 = hv * 32;
+                f2_t win[3];  // the three raw rows before the next one to convolve
+                if (hv == 0) {
+#pragma unroll
+                    for (int jh = 0; jh < 3; ++jh) win[jh] = unit_start ? vstate[jh] : unpack2(vprev[jh * 32 + lane]);
+                } else {
+#pragma unroll
+                    for (int jh = 0; jh < 3; ++jh) win[jh] = unpack2(*word(r0 - 3 + jh));
+                }
+                bar_sync(7, 64);  // the rows each warp needs from the other's half are in registers
+                for (int r8 = 0; r8 < 32; r8 += 8) {  // eight rows at a time, loads first
+                    f2_t x[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) x[i] = unpack2(*word(r0 + r8 + i));
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        f2_t z = f2fma(vw[0], win[0], f2(0.f, 0.f));
+                        z = f2fma(vw[1], win[1], z);
+                        z = f2fma(vw[2], win[2], z);
+                        z = f2fma(vw[3], x[i], z);
+                        *word(r0 + r8 + i) = pack2(swish2(z));
+                        win[0] = win[1];
+                        win[1] = win[2];
+                        win[2] = x[i];
+                    }
+                }
+                if (hv == 1) {
+#pragma unroll
+                    for (int jh = 0; jh < 3; ++jh) vprev[jh * 32 + lane] = pack2(win[jh]);
+                }
+                ++vj;
+                fence_async_smem();  // the rewritten tile is read by the tensor cores
+                bar_sync(7, 64);
+                if (warp == 12 && lane == 0) mbar_arrive(&convV[vb]);
+                return true;
+            };
+            if (vconv)
+                for (long long q = 0; q < 2 && q < L && ok; ++q) ok = conv_v(q);
+            for (long long kk = 0; kk < K && ok; ++kk) {
+                int s, h;
+                int64_t bos, eos;
+                unit_bounds(kk, s, h, bos, eos);
+                const long long len = eos - bos, nch = (len + C - 1) / C;
+                for (long long j = 0; j < nch; ++j, ++p) {
+                    if (!(ok = wait_o(p))) break;
+                    const long long nn = (len - j * C) < C ? (len - j * C) : C;
+                    store_row(p, bos + j * C + c, h, nn, 1.f, none);
+                    if (vconv && p + 2 < L && !(ok = conv_v(p + 2))) break;
+                }
+            }
+        } else {
+            // With the output step a row's RMSNorm needs the partner CTA's 64 columns:
+            // each thread publishes its row's sum of squares, tagged with the position,
+            // in one 8-byte word (four per row, by position modulo 4) and reads the
+            // partner's word one position later: position p - 1 is stored after the sum
+            // of p is published, so the round trip is hidden behind O(p). A word is
+            // rewritten four positions later; the partner has read it by then (it
+            // published p - 2, which this CTA needed for p - 2, only after finishing
+            // p - 4's read).
+            auto publish = [&](long long q, float ss) {
+                const unsigned long long tag = (unsigned long long)(q + 1) << 32;
+                st_relaxed_gpu_u64(&xw[((st * 2 + jv) * 4 + (q & 3)) * 64 + c], tag | __float_as_uint(ss));
+            };
+            auto partner = [&](long long q, float &v) {
+                const unsigned long long tag = (unsigned long long)(q + 1) << 32;
+                const unsigned long long *pw = &xw[((st * 2 + (jv ^ 1)) * 4 + (q & 3)) * 64 + c];
+                unsigned long long got = ld_relaxed_gpu_u64(pw);
+                if ((got >> 32) != (tag >> 32)) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (((got = ld_relaxed_gpu_u64(pw)) >> 32) != (tag >> 32))
+                        if (globaltimer_ns() - t0 > P.xwait_ns || ld_relaxed_gpu(&hd->abort_flag)) break;
+                }
+                v = __uint_as_float((uint32_t)got);
+                return __all_sync(0xffffffffu, (got >> 32) == (tag >> 32));
+            };
+            auto load_gate = [&](int64_t t, int h, long long nn, uint4 (&graw)[8]) {
+                const bf16 *grow = P.og_gate + ((size_t)t * H + h) * DV + jv * DVT;
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
-                    graw[i] = (gated && c < nn) ? __ldg(reinterpret_cast<const uint4 *>(grow) + i) : make_uint4(0, 0, 0, 0);
-                float scale = 1.f;
-                if (gated) {
+                    graw[i] = c < nn ? __ldg(reinterpret_cast<const uint4 *>(grow) + i) : make_uint4(0, 0, 0, 0);
+            };
+            bool havep = false;  // position p - 1 is still to be stored
+            int64_t tp = 0;
+            int hp = 0;
+            long long nnp = 0;
+            float ssp = 0.f;
+            for (long long kk = 0; kk < K && ok; ++kk) {
+                int s, h;
+                int64_t bos, eos;
+                unit_bounds(kk, s, h, bos, eos);
+                const long long len = eos - bos, nch = (len + C - 1) / C;
+                for (long long j = 0; j < nch; ++j, ++p) {
+                    uint4 graw[8];
+                    if (havep) load_gate(tp, hp, nnp, graw);  // in flight during the wait and the sum
+                    if (!(ok = wait_o(p))) break;
                     float ss = 0.f;
+                    const uint32_t ybuf = tm + TM_Y + (uint32_t)(p % NY) * 64 + lane_base;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         float y[32];
                         tmem_ld32(ybuf + half * 32, y);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) ss += y[i] * y[i];
+                        for (int i = 0; i < 32; ++i) ss = fmaf(y[i], y[i], ss);
                     }
-                    const unsigned long long tag = (unsigned long long)(p + 1) << 32;
-                    st_relaxed_gpu_u64(&xw[((st * 2 + jv) * 2 + (p & 1)) * 64 + c], tag | __float_as_uint(ss));
-                    const unsigned long long *pw = &xw[((st * 2 + (jv ^ 1)) * 2 + (p & 1)) * 64 + c];
-                    unsigned long long got = ld_relaxed_gpu_u64(pw);
-                    if ((got >> 32) != (tag >> 32)) {
-                        const uint64_t t0 = globaltimer_ns();
-                        while (((got = ld_relaxed_gpu_u64(pw)) >> 32) != (tag >> 32))
-                            if (globaltimer_ns() - t0 > P.xwait_ns || ld_relaxed_gpu(&hd->abort_flag)) break;
+                    publish(p, ss);
+                    if (havep) {
+                        float other;
+                        if (!(ok = partner(p - 1, other))) break;
+                        store_row(p - 1, tp, hp, nnp, rsqrtf((ssp + other) * (1.f / DV) + P.og_eps), graw);
                     }
-                    ok = __all_sync(0xffffffffu, (got >> 32) == (tag >> 32));
-                    if (!ok) break;
-                    scale = rsqrtf((ss + __uint_as_float((uint32_t)got)) * (1.f / DV) + P.og_eps);
+                    havep = true;
+                    tp = bos + j * C + c;
+                    hp = h;
+                    nnp = (len - j * C) < C ? (len - j * C) : C;
+                    ssp = ss;
+                    if (c < nnp)  // this row's gate, read in the next iteration: into L2 now
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(P.og_gate + ((size_t)tp * H + hp) * DV + jv * DVT));
                 }
-                bf16 *dst = P.o + ((size_t)t * H + h) * DV + jv * DVT;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float y[32];
-                    tmem_ld32(ybuf + half * 32, y);
-                    tmem_wait_ld();
-                    if (c < nn) {
-#pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
-                            float o8[8];
-                            if (gated) {
-                                float g8[8];
-                                unpack8(graw[half * 4 + q8], g8);
-                                const float4 w0 = *reinterpret_cast<const float4 *>(sw + half * 32 + q8 * 8);
-                                const float4 w1 = *reinterpret_cast<const float4 *>(sw + half * 32 + q8 * 8 + 4);
-                                const float w8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                                for (int i = 0; i < 8; ++i)  // y * scale * w * sigmoid(g)
-                                    o8[i] = __fdividef(y[q8 * 8 + i] * scale * w8[i], 1.f + __expf(-g8[i]));
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) o8[i] = y[q8 * 8 + i];
-                            }
-                            reinterpret_cast<uint4 *>(dst)[half * 4 + q8] = pack8(o8);
-                        }
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&oready[p % NY]);  // Y[p % NY] may be overwritten (by Y(p + NY))
+            }
+            if (ok && havep) {
+                uint4 graw[8];
+                load_gate(tp, hp, nnp, graw);
+                float other;
+                if ((ok = partner(p - 1, other)))
+                    store_row(p - 1, tp, hp, nnp, rsqrtf((ssp + other) * (1.f / DV) + P.og_eps), graw);
             }
         }
         if (!ok) fail_call(P);
@@ -1150,7 +1380,7 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         auto issue_x = [&](long long q) {
             const int bb = (int)(q % 3), vb = (int)(q & 3);
             if (!(mbar_wait_call(&fullB[bb], (uint32_t)((q / 3) & 1), &hd->abort_flag) &&
-                  mbar_wait_call(&fullV[vb], (uint32_t)((q >> 2) & 1), &hd->abort_flag)))
+                  mbar_wait_call(CV && P.cw[2] ? &convV[vb] : &fullV[vb], (uint32_t)((q >> 2) & 1), &hd->abort_flag)))
                 return false;
             tc_fence_after();
 #pragma unroll
@@ -1183,7 +1413,77 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
         if (!ok) fail_call(P);
         return;
     }
-    if (warp >= 8) return;  // warp 15 idle
+    if (warp == 15) {
+        // ---------------- fused short convolution of the V tiles ----------------
+        // Lane l takes channels 2 l, 2 l + 1 of this CTA's 64 (SW128 rows of 128 bytes),
+        // row by row in place, keeping the last three raw rows in registers: from the
+        // initial state (or zeros) at a unit's first chunk, then from the previous tile.
+        // The same arithmetic as the standalone convolution kernel.
+        if (!CV || !OG || P.cw[2] == 0) return;  // without the output step warps 12, 13 do it
+        const int W = P.cw[2];
+        const int ch = jv * DVT + 2 * lane;  // channel within the head
+        bool ok = true;
+        long long p = 0;
+        for (long long kk = 0; kk < K && ok; ++kk) {
+            int s, h;
+            int64_t bos, eos;
+            unit_bounds(kk, s, h, bos, eos);
+            const long long nch = (eos - bos + C - 1) / C;
+            if (nch == 0) continue;
+            const float *wt = P.cwt[2] + ((size_t)h * DV + ch) * W;
+            f2_t wp[4], win[3];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int jj = j - (4 - W);
+                wp[j] = jj >= 0 ? f2(__ldg(wt + jj), __ldg(wt + W + jj)) : f2(0.f, 0.f);
+            }
+#pragma unroll
+            for (int jh = 0; jh < 3; ++jh) {
+                const int js = jh + W - 4;
+                win[jh] = (P.cst[2] != nullptr && js >= 0)
+                              ? unpack2(*reinterpret_cast<const uint32_t *>(
+                                    P.cst[2] + ((size_t)s * (W - 1) + js) * ((size_t)H * DV) + (size_t)h * DV + ch))
+                              : f2(0.f, 0.f);
+            }
+            for (long long j = 0; j < nch; ++j, ++p) {
+                const int vb = (int)(p & 3);
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait_call(&fullV[vb], (uint32_t)((p >> 2) & 1), &hd->abort_flag))))
+                    break;
+                uint8_t *tile = sm + SS_V + vb * SV_BYTES;
+                for (int r0 = 0; r0 < C; r0 += 16) {  // 16 rows at a time, all loads first
+                    f2_t ext[19];                       // raw rows r0 - 3 .. r0 + 15
+                    ext[0] = win[0];
+                    ext[1] = win[1];
+                    ext[2] = win[2];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int r = r0 + i;
+                        ext[3 + i] = unpack2(*reinterpret_cast<const uint32_t *>(
+                            tile + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int r = r0 + i;
+                        f2_t z = f2fma(wp[0], ext[i], f2(0.f, 0.f));
+                        z = f2fma(wp[1], ext[i + 1], z);
+                        z = f2fma(wp[2], ext[i + 2], z);
+                        z = f2fma(wp[3], ext[i + 3], z);
+                        *reinterpret_cast<uint32_t *>(tile + r * 128 + (((lane >> 2) ^ (r & 7)) << 4) + (lane & 3) * 4) =
+                            pack2(swish2(z));
+                    }
+                    win[0] = ext[16];
+                    win[1] = ext[17];
+                    win[2] = ext[18];
+                }
+                fence_async_smem();  // the rewritten tile is read by the tensor cores
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&convV[vb]);
+            }
+        }
+        if (!ok) fail_call(P);
+        return;
+    }
+    if (warp >= 8) return;
 
     // ---------------- epilogues (TMEM lane = state row c) ----------------
     const int q4 = warp & 3, hf = warp >> 2;
@@ -1281,6 +1581,9 @@ __device__ __forceinline__ void scan_role(const FusedParams &P, uint8_t *sm, uin
 }
 
 // ----------------------------------------------------------- the kernel ----
+// OG: with the fused output step; CV: with the fused short convolution (each its own
+// instantiation, so that the plain prefill carries neither's code).
+template <bool OG, bool CV>
 __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constant__ FusedParams P) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1344,8 +1647,8 @@ __global__ void __launch_bounds__(kThreads, 1) fused_kernel(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = ctl->tbase;
-    if (scan) scan_role(P, sm, tm, blockIdx.x >> 1, blockIdx.x & 1);
-    else prep_engine(P, ctl, tid >> 8, sm + (tid >> 8) * PS_STRIDE, tm + 256u * (uint32_t)(tid >> 8));
+    if (scan) scan_role<OG, CV>(P, sm, tm, blockIdx.x >> 1, blockIdx.x & 1);
+    else prep_engine<CV>(P, ctl, tid >> 8, sm + (tid >> 8) * PS_STRIDE, tm + 256u * (uint32_t)(tid >> 8));
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tm, 512);
@@ -1394,11 +1697,11 @@ bool make_la_map(CUtensorMap *m, const void *base, int64_t total, int H) {
 }  // namespace
 
 size_t tc_workspace_bytes(long long NH, int ns, int R) {
-    return ws_ring(NH) + (size_t)ns * (size_t)R * SL_BYTES;
+    return ws_xch(NH, ns, R) + kXchWords * 8;
 }
 
 int tc_ring_slots(long long NH, int ns, size_t bytes) {
-    const size_t base = ws_ring(NH);
+    const size_t base = ws_ring(NH) + kXchWords * 8;  // the ring, then the exchange words
     if (ns < 1 || bytes < base) return 0;
     const size_t r = (bytes - base) / ((size_t)ns * SL_BYTES);
     return (int)(r < (size_t)kMaxRing ? r : (size_t)kMaxRing);
@@ -1413,14 +1716,17 @@ uint64_t tc_set_wait_limit(uint64_t ns) { return g_xwait_ns.exchange(ns ? ns : k
 
 cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, int *err, cudaStream_t st) {
     cudaError_t e;
+    const bool og = a.og_gate != nullptr, cv = (a.conv_W[0] | a.conv_W[1] | a.conv_W[2]) != 0;
+    void (*kern)(FusedParams) = og ? (cv ? fused_kernel<true, true> : fused_kernel<true, false>)
+                                   : (cv ? fused_kernel<false, true> : fused_kernel<false, false>);
     // Per device (context): cheap enough to set on every call.
-    if ((e = cudaFuncSetAttribute(fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC)) !=
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC)) !=
         cudaSuccess)
         return e;
     int dev = 0, sms = 0, per_sm = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused_kernel, kThreads, SMEM_ALLOC)) != cudaSuccess)
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, SMEM_ALLOC)) != cudaSuccess)
         return e;
     const int grid = per_sm * sms;
     // At least two prep CTAs beside the scan CTAs.
@@ -1443,6 +1749,12 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
     P.og_eps = a.og_eps;
     P.q = static_cast<const bf16 *>(a.q);
     P.k = static_cast<const bf16 *>(a.k);
+    P.v = static_cast<const bf16 *>(a.v);
+    for (int i = 0; i < 3; ++i) {
+        P.cw[i] = a.conv_W[i];
+        P.cwt[i] = a.conv_w[i];
+        P.cst[i] = static_cast<const bf16 *>(a.conv_state[i]);
+    }
     P.beta = a.beta;
     P.S0 = a.S0;
     P.cu = a.cu;
@@ -1459,7 +1771,7 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
     P.l2norm = a.l2norm;
     P.eps = a.eps;
 
-    plan_kernel<<<1, PLAN_T, 0, st>>>(a.cu, a.total, a.N, a.H, ns, ws);
+    plan_kernel<<<1, PLAN_T, 0, st>>>(a.cu, a.total, a.N, a.H, ns, R, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     cudaLaunchConfig_t cfg;
@@ -1473,7 +1785,7 @@ cudaError_t tc_prefill(const PrefillArgs &a, char *ws, size_t ws_bytes, int ns, 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fused_kernel, P);
+    return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
 }  // namespace kda

@@ -141,7 +141,7 @@ conv_kernel(const T *__restrict__ x, T *__restrict__ y, const float *__restrict_
                 float z = 0.f;
 #pragma unroll
                 for (int j = 0; j < W; ++j) z = fmaf(wt[i][j], win[j][i], z);
-                out[i] = __fdividef(z, 1.f + __expf(-z));
+                out[i] = swish(z);
             }
             Vec8<T>::st(y + (size_t)(t0 + r) * C + c0, out);
 #pragma unroll
@@ -173,7 +173,7 @@ conv_kernel(const T *__restrict__ x, T *__restrict__ y, const float *__restrict_
             float z = 0.f;
 #pragma unroll
             for (int j = 0; j < W; ++j) z = fmaf(wt[i][j], win[j][i], z);
-            out[i] = __fdividef(z, 1.f + __expf(-z));
+            out[i] = swish(z);
         }
         Vec8<T>::st(y + (size_t)t * C + c0, out);
 #pragma unroll
@@ -200,6 +200,18 @@ conv_state_kernel(const T *__restrict__ x, const T *state_in, T *state_out, cons
 #pragma unroll
         for (int j = 0; j < W - 1; ++j) Vec8<T>::st(state_out + ((size_t)s * (W - 1) + j) * C + c0, v[j]);
     }
+}
+
+template <int W, typename T>
+cudaError_t launch_state(const ShortConvArgs &a, cudaStream_t st) {
+    if (W > 1 && a.state_out) {
+        const int64_t threads = (int64_t)a.N * (a.C / 8);
+        conv_state_kernel<W, T><<<(unsigned)((threads + kConvThreads - 1) / kConvThreads), kConvThreads, 0, st>>>(
+            static_cast<const T *>(a.x), static_cast<const T *>(a.state_in), static_cast<T *>(a.state_out), a.cu,
+            a.N, a.total, a.C);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
 }
 
 template <int W, typename T>
@@ -237,10 +249,29 @@ cudaError_t launch_t(const ShortConvArgs &a, cudaStream_t st) {
     }
 }
 
+template <typename T>
+cudaError_t launch_state_t(const ShortConvArgs &a, cudaStream_t st) {
+    switch (a.W) {
+    case 1: return launch_state<1, T>(a, st);
+    case 2: return launch_state<2, T>(a, st);
+    case 3: return launch_state<3, T>(a, st);
+    case 4: return launch_state<4, T>(a, st);
+    case 5: return launch_state<5, T>(a, st);
+    case 6: return launch_state<6, T>(a, st);
+    case 7: return launch_state<7, T>(a, st);
+    case 8: return launch_state<8, T>(a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 }  // namespace
 
 cudaError_t short_conv_swish(const ShortConvArgs &a, bool bf16, cudaStream_t st) {
     return bf16 ? launch_t<__nv_bfloat16>(a, st) : launch_t<float>(a, st);
+}
+
+cudaError_t short_conv_state(const ShortConvArgs &a, bool bf16, cudaStream_t st) {
+    return bf16 ? launch_state_t<__nv_bfloat16>(a, st) : launch_state_t<float>(a, st);
 }
 
 int short_conv_launches(int W, bool state_out, int64_t total) {

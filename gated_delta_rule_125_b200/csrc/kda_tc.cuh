@@ -368,6 +368,17 @@ __device__ __forceinline__ float ex2f(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// swish() of a pair: the same operations lane by lane, the multiplies and the add in pairs.
+__device__ __forceinline__ f2_t swish2(f2_t z) {
+    const f2_t a = f2mul(z, f2(kSwishNegLog2e, kSwishNegLog2e));
+    float el, eh, rl, rh;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(el) : "f"(f2lo(a)));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(eh) : "f"(f2hi(a)));
+    const f2_t d = f2add(f2(1.f, 1.f), f2(el, eh));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rl) : "f"(f2lo(d)));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rh) : "f"(f2hi(d)));
+    return f2mul(z, f2(rl, rh));
+}
 // A pair of fp32 values -> a bf16 pair (round to nearest even), low value in the low half.
 __device__ __forceinline__ uint32_t pack2(f2_t a) {
     uint32_t r;

@@ -11,7 +11,9 @@ Names: the prefill workloads of ``kda_inputs.WORKLOADS`` (``tiny_f32``,
 heads, one step per call), ``decode_256_conv`` (the same with the short
 convolution fused into the loads), ``short_conv_8k`` (the convolution of one
 [8192, 32 * 128] projection), ``backward_1k`` (the backward of one 1024-token
-sequence, 32 heads).
+sequence, 32 heads), ``prefill_8k_conv`` (prefill_8k from raw projections with the
+width-4 short convolution of q, k, v inside the prefill), ``prefill_8k_gate`` (prefill_8k
+with the fused output step).
 """
 from __future__ import annotations
 
@@ -43,6 +45,26 @@ def main():
         for _ in range(args.calls):
             kda.kda_prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
                             inp["cu_seqlens"], max_seqlen=L)
+    elif n in ("prefill_8k_conv", "prefill_8k_gate"):
+        inp = KI.prefill_workload("prefill_8k", dev)
+        T, H, D = inp["v"].shape
+        kw = {}
+        if n.endswith("_conv"):
+            conv, raw = [], []
+            for i in range(3):
+                x, w, st = KI.conv_inputs(T, H * D, 4, 1, torch.bfloat16, dev, tensor=i)
+                raw.append(x.view(T, H, D))
+                conv.append((w, st, torch.empty_like(st)))
+            inp["q"], inp["k"], inp["v"] = raw
+            kw["conv"] = tuple(conv)
+        else:
+            g = torch.Generator(device=dev)
+            g.manual_seed(1000)
+            kw["out_gate"] = (torch.randn((T, H, D), generator=g, device=dev).to(torch.bfloat16),
+                              1.0 + 0.1 * torch.randn((D,), generator=g, device=dev), 1e-6)
+        for _ in range(args.calls):
+            kda.kda_prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["S0"],
+                            inp["cu_seqlens"], max_seqlen=T, **kw)
     elif n in ("decode_256", "decode_256_conv"):
         steps, H, D, N = args.calls, 32, 128, 256
         d = KI.decode_workload(N, H, D, steps, torch.bfloat16, dev)

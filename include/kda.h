@@ -301,6 +301,32 @@ kda_status kda_decode_step_conv(const void *q, const void *k, const void *v, con
                                 kda_stream_t stream);
 
 /*
+ * kda_prefill_ex with the short convolution + Swish fused into the loads of q,
+ * k and v ("[Kimi-2] Kimi Linear" §6 and §6.1): here q, k, v are the raw
+ * projections ([T][H][d], as for kda_prefill) and conv_q, conv_k, conv_v (each
+ * NULL: that input is used as it is) carry C = H * d channels, weight [C][W],
+ * state_in [N][W-1][C] read for each sequence's first W-1 positions (NULL:
+ * zeros) and state_out [N][W-1][C] written with each sequence's last W-1 raw
+ * inputs after the prefill has read state_in (NULL: not written; may alias
+ * state_in). o and S_T equal, bit for bit, those of kda_short_conv_swish on
+ * each input followed by kda_prefill_ex on the results; no convolved copy of
+ * q, k or v is written to device memory. The tensor-core path only (bf16,
+ * d_k = d_v = 128, without KDA_FLAG_EXACT) and windows 1 ..
+ * KDA_PREFILL_MAX_CONV_WIDTH: KDA_ERR_UNSUPPORTED otherwise (run
+ * kda_short_conv_swish and kda_prefill_ex instead). Workspace as for
+ * kda_prefill (kda_prefill_workspace_size). Enqueued as kda_prefill_launches()
+ * kernels, then one kernel per written state_out of a width above 1.
+ */
+#define KDA_PREFILL_MAX_CONV_WIDTH 4
+kda_status kda_prefill_conv(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, const float *S0, const int32_t *cu_seqlens,
+                            int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
+                            int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags,
+                            const kda_short_conv *conv_q, const kda_short_conv *conv_k,
+                            const kda_short_conv *conv_v, const kda_output_gate *out_gate, void *o,
+                            float *S_T, void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * Backward of the prefill (training): the gradients of a loss L with respect
  * to q, k, v, log_alpha, beta and S0, given dL/do and dL/dS_T. The pages
  * mention training but give no backward; the chunked reverse-mode algebra

@@ -620,6 +620,47 @@ def test_decode_conv_steps(dtype, d, with_v):
                 np.testing.assert_array_equal(host(convs[i][1]), refs[i])
 
 
+@pytest.mark.parametrize("W,which,dk", [(2, (False, True, True), 128), (3, (True, False, False), 128),
+                                        (4, (True, True, True), 64)])
+def test_decode_conv_windows_separate_states(W, which, dk):
+    """Decode with the convolution on a subset of q, k, v, windows 2..4 and d_k 64 or 128
+    (d_v = 128: the state split over a two-CTA cluster), reading the conv states from one
+    buffer and writing them to another (the input states stay untouched)."""
+    N, H, dv, steps = 5, 3, 128, 3
+    g = torch.Generator(device=DEV)
+    g.manual_seed(31)
+    dims = (dk, dk, dv)
+    raw = [torch.randn(steps, N, H, dims[i], generator=g, device=DEV).to(torch.bfloat16) for i in range(3)]
+    la = -torch.nn.functional.softplus(torch.randn(steps, N, H, dk, generator=g, device=DEV) - 3.0)
+    beta = torch.sigmoid(torch.randn(steps, N, H, generator=g, device=DEV))
+    S = 0.1 * torch.randn(N, H, dk, dv, generator=g, device=DEV)
+    S_ref = host(S)
+    w = [torch.randn(H * dims[i], W, generator=g, device=DEV) / W ** 0.5 for i in range(3)]
+    st = [torch.randn(N, W - 1, H * dims[i], generator=g, device=DEV).to(torch.bfloat16) for i in range(3)]
+    refs = [host(x) for x in st]
+    for t in range(steps):
+        outs = [torch.empty_like(x) for x in st]
+        cv = tuple((w[i], st[i], outs[i]) if which[i] else None for i in range(3))
+        keep = [x.clone() for x in st]
+        o = kda.kda_decode_step(raw[0][t], raw[1][t], raw[2][t], la[t], beta[t], S, conv=cv)
+        torch.cuda.synchronize()
+        xs = []
+        for i in range(3):
+            if not which[i]:
+                xs.append(host(raw[i][t]))
+                continue
+            y, refs[i] = oracle.short_conv_step(host(raw[i][t]).reshape(N, H * dims[i]), host(w[i]), refs[i])
+            xs.append(y.reshape(N, H, dims[i]))
+        o_ref, S_ref = oracle.decode_step(xs[0], xs[1], xs[2], host(la[t]), host(beta[t]), S_ref)
+        assert float(np.abs(host(o) - o_ref).max()) <= 2e-2, "step %d" % t
+        assert rel_fro(host(S), S_ref) <= 1e-2, "step %d" % t
+        for i in range(3):
+            assert torch.equal(st[i], keep[i]), "input conv state %d written" % i
+            if which[i]:
+                np.testing.assert_array_equal(host(outs[i]), refs[i])
+                st[i] = outs[i]
+
+
 def test_decode_conv_continues_prefill_conv():
     """fp32: conv + prefill over T-3 tokens, then 3 decode steps with the fused convolution
     continuing from the prefill's conv states == conv + prefill over all T tokens."""
@@ -649,6 +690,140 @@ def test_decode_conv_continues_prefill_conv():
                                 inp["beta"][t:t + 1].clone(), S, conv=tuple(cv))
         torch.testing.assert_close(o[0], o_all[t], atol=2e-5, rtol=0)
     torch.testing.assert_close(S, S_all, atol=2e-5, rtol=0)
+
+
+# ------------------------------- short convolution fused into the prefill ----
+
+def _conv_case(lengths, H, W, which, seed, with_state=True):
+    """Raw q, k, v projections with conv taps and initial states for the inputs in `which`."""
+    inp = make(lengths, H, 128, 128, torch.bfloat16, seed=seed)
+    N = len(lengths)
+    convs = []
+    for i, name in enumerate(("q", "k", "v")):
+        if not which[i]:
+            convs.append(None)
+            continue
+        x, w, st = KI.conv_inputs(sum(lengths), H * 128, W, N, torch.bfloat16, DEV, seed=seed, tensor=i,
+                                  with_state=with_state)
+        inp[name] = x.view(-1, H, 128)
+        convs.append((w, st))
+    return inp, convs
+
+
+def _two_step(inp, convs, out_gate=None):
+    """kda_short_conv_swish on each convolved input, then kda_prefill_ex; the states written."""
+    x = dict(inp)
+    states = []
+    for i, name in enumerate(("q", "k", "v")):
+        if convs[i] is None:
+            states.append(None)
+            continue
+        w, st = convs[i]
+        so = torch.empty((len(inp["lengths"]), w.shape[1] - 1, w.shape[0]), dtype=torch.bfloat16, device=DEV)
+        y = kda.kda_short_conv_swish(inp[name].reshape(-1, w.shape[0]), w, inp["cu_seqlens"], state_in=st,
+                                     state_out=so)
+        x[name] = y.view(inp[name].shape)
+        states.append(so)
+    o, S_T = run(x, out_gate=out_gate)
+    return o, S_T, states, x
+
+
+def _fused(inp, convs, out_gate=None, in_place=False):
+    states, conv = [], []
+    for c in convs:
+        if c is None:
+            states.append(None)
+            conv.append(None)
+            continue
+        w, st = c
+        if in_place:
+            so = st.clone() if st is not None else torch.zeros((len(inp["lengths"]), w.shape[1] - 1, w.shape[0]),
+                                                               dtype=torch.bfloat16, device=DEV)
+            conv.append((w, so if st is not None else None, so))
+        else:
+            so = torch.empty((len(inp["lengths"]), w.shape[1] - 1, w.shape[0]), dtype=torch.bfloat16, device=DEV)
+            conv.append((w, st, so))
+        states.append(so)
+    o, S_T = run(inp, conv=tuple(conv), out_gate=out_gate)
+    return o, S_T, states
+
+
+@pytest.mark.parametrize("lengths,H,W,which", [
+    ([300], 4, 4, (True, True, True)),
+    ([1, 2, 3, 64, 65, 130, 0, 200], 3, 4, (True, True, True)),
+    ([129, 70], 2, 3, (True, False, True)),
+    ([64, 5, 190], 2, 2, (False, True, False)),
+    ([2048, 700], 4, 1, (True, True, True)),
+])
+def test_prefill_conv_equals_conv_then_prefill(lengths, H, W, which):
+    """kda_prefill_conv (convolution inside the prefill's loads) gives o, S_T and the conv
+    states bit for bit equal to kda_short_conv_swish on each input followed by kda_prefill."""
+    inp, convs = _conv_case(lengths, H, W, which, seed=40 + W)
+    o2, S2, st2, _ = _two_step(inp, convs)
+    o1, S1, st1 = _fused(inp, convs)
+    assert torch.equal(o1, o2)
+    assert torch.equal(S1, S2)
+    for a, b in zip(st1, st2):
+        if a is not None and W > 1:
+            assert torch.equal(a, b)
+    assert kda.kda_device_error(reset=True) == 0
+
+
+def test_prefill_conv_in_place_states_and_no_initial_state():
+    """States updated in place (state_in == state_out), and no initial state (zeros)."""
+    lengths, H, W = [77, 2, 260], 2, 4
+    inp, convs = _conv_case(lengths, H, W, (True, True, True), seed=47)
+    o2, S2, st2, _ = _two_step(inp, convs)
+    o1, S1, st1 = _fused(inp, convs, in_place=True)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    for a, b in zip(st1, st2):
+        assert torch.equal(a, b)
+    inp0, convs0 = _conv_case(lengths, H, W, (True, True, True), seed=48, with_state=False)
+    o2, S2, _, _ = _two_step(inp0, convs0)
+    o1, S1, _ = _fused(inp0, convs0)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_prefill_conv_matches_oracle():
+    """Against the oracle: short_conv_swish on each raw input (fp64), then the recurrence."""
+    lengths, H, W = [190, 3, 64], 2, 4
+    inp, convs = _conv_case(lengths, H, W, (True, True, True), seed=49)
+    o, S_T, _ = _fused(inp, convs)
+    cu = inp["cu_seqlens"].cpu().numpy().astype(np.int64)
+    ref = dict(inp)
+    for i, name in enumerate(("q", "k", "v")):
+        w, st = convs[i]
+        y, _ = oracle.short_conv_swish(host(inp[name]).reshape(-1, H * 128), host(w), cu, host(st))
+        ref[name] = torch.from_numpy(y.reshape(-1, H, 128)).to(DEV)
+    ref["q"], ref["k"], ref["v"] = (ref[n].to(torch.float64) for n in ("q", "k", "v"))
+    check(o, S_T, ref, torch.bfloat16, label="conv in the prefill vs oracle")
+
+
+def test_prefill_conv_with_output_step():
+    """The fused convolution and the fused output step together."""
+    lengths, H, W = [150, 40], 3, 4
+    inp, convs = _conv_case(lengths, H, W, (True, True, True), seed=50)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(51)
+    og = (torch.randn((sum(lengths), H, 128), generator=g, device=DEV).to(torch.bfloat16),
+          1.0 + 0.1 * torch.randn((128,), generator=g, device=DEV), 1e-6)
+    o2, S2, _, _ = _two_step(inp, convs, out_gate=og)
+    o1, S1, _ = _fused(inp, convs, out_gate=og)
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_prefill_conv_unsupported():
+    """fp32 inputs (the CUDA-core path) and windows above 4 are refused, not approximated."""
+    inp = make([70], 2, 128, 128, torch.float32, seed=52)
+    w = torch.randn(256, 4, device=DEV)
+    with pytest.raises(kda.KDAError) as e:
+        run(inp, conv=((w, None, None), None, None))
+    assert e.value.status == kda.KDA_ERR_UNSUPPORTED
+    inp = make([70], 2, 128, 128, torch.bfloat16, seed=52)
+    w5 = torch.randn(256, 5, device=DEV)
+    with pytest.raises(kda.KDAError) as e:
+        run(inp, conv=((w5, None, None), None, None))
+    assert e.value.status == kda.KDA_ERR_UNSUPPORTED
 
 
 # ------------------------------------------------ backward (training) ----
