@@ -23,9 +23,10 @@
 //   1. bw_prep   (one CTA per chunk): normalised q, k; G, Qg, Kg, Kn, Kd, A, P,
 //                the unit-lower-triangular inverse X by column forward
 //                substitution, T, W, T V;
-//   2. bw_fwd    (one CTA per (sequence, head)): the chunks' entry states and U;
-//   3. bw_bwd    (one CTA per (sequence, head)): dU and the state gradient
-//                entering each chunk, in reverse chunk order; dS0;
+//   2. bw_fwd    (one CTA per 16 state columns of a (sequence, head)): the
+//                chunks' entry states and U, W and Kd staged in shared memory;
+//   3. bw_bwd    (likewise): dU and the state gradient entering each chunk, in
+//                reverse chunk order; dS0;
 //   4. bw_grads  (one CTA per chunk): every per-chunk gradient above;
 //   5. bw_norm   (one warp per (token, head)): through the L2 normalisation.
 // Everything lives in the caller's workspace (fp32); each product is a plain
@@ -199,77 +200,149 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep(BwArgs a) {
     }
 }
 
-// 2. Entry states and U, chunk by chunk (the state in shared memory).
-__global__ void __launch_bounds__(kBwThreads) bw_fwd(BwArgs a) {
-    extern __shared__ float sS[];
-    const int unit = blockIdx.x, s = unit / a.H, tid = threadIdx.x;
+// 2. Entry states and U, chunk by chunk. The recurrence acts on each state column
+//    on its own (S' = Diag(e^g) S + Kd^T (TV - W S), column by column), so a CTA takes
+//    kCols columns of one (sequence, head): the columns in shared memory, and per chunk
+//    W and Kd staged there from the slot.
+constexpr int kCols = 16;
+__host__ __device__ inline size_t fwd_smem_floats(int dk) { return (size_t)dk * kCols + 2 * (size_t)C * dk + C * kCols; }
+__global__ void __launch_bounds__(kBwThreads, 2) bw_fwd(BwArgs a) {
+    extern __shared__ float4 smem4[];
+    const int groups = a.dv / kCols;
+    const int unit = blockIdx.x / groups, c0 = (blockIdx.x % groups) * kCols, s = unit / a.H, tid = threadIdx.x;
     const int dk = a.dk, dv = a.dv;
     const Slot sl{dk, dv};
-    for (int e = tid; e < dk * dv; e += kBwThreads) sS[e] = a.S0 ? a.S0[(size_t)unit * dk * dv + e] : 0.f;
-    __syncthreads();
+    float *sS = reinterpret_cast<float *>(smem4), *sW = sS + dk * kCols, *sKd = sW + C * dk, *sU = sKd + C * dk;
+    for (int e = tid; e < dk * kCols; e += kBwThreads)
+        sS[e] = a.S0 ? a.S0[(size_t)unit * dk * dv + (size_t)(e / kCols) * dv + c0 + e % kCols] : 0.f;
     for (int j = 0; j < a.NC; ++j) {
         int64_t t0;
         int n;
         chunk_rows(a, s, j, t0, n);
         if (n == 0) break;
         SlotPtr m(a.slots + ((size_t)unit * a.NC + j) * sl.floats(), sl);
-        for (int e = tid; e < dk * dv; e += kBwThreads) m.S[e] = sS[e];
-        for (int e = tid; e < n * dv; e += kBwThreads) {
-            const int r = e / dv, c = e % dv;
-            float acc = m.TV[e];
-            for (int i = 0; i < dk; ++i) acc -= m.W[r * dk + i] * sS[i * dv + c];
-            m.U[e] = acc;
+        for (int e = tid; e < n * dk / 4; e += kBwThreads) {
+            reinterpret_cast<float4 *>(sW)[e] = reinterpret_cast<const float4 *>(m.W)[e];
+            reinterpret_cast<float4 *>(sKd)[e] = reinterpret_cast<const float4 *>(m.Kd)[e];
+        }
+        __syncthreads();  // the staged rows; the state columns of the previous chunk
+        for (int e = tid; e < dk * kCols; e += kBwThreads) m.S[(size_t)(e / kCols) * dv + c0 + e % kCols] = sS[e];
+        // U = TV - W S: thread (row r, four columns)
+        if (tid < n * 4) {
+            const int r = tid >> 2, cq = (tid & 3) * 4;
+            float4 acc = *reinterpret_cast<const float4 *>(m.TV + (size_t)r * dv + c0 + cq);
+            for (int i = 0; i < dk; ++i) {
+                const float w = sW[r * dk + i];
+                const float4 x = *reinterpret_cast<const float4 *>(sS + i * kCols + cq);
+                acc.x -= w * x.x;
+                acc.y -= w * x.y;
+                acc.z -= w * x.z;
+                acc.w -= w * x.w;
+            }
+            *reinterpret_cast<float4 *>(sU + r * kCols + cq) = acc;
+            *reinterpret_cast<float4 *>(m.U + (size_t)r * dv + c0 + cq) = acc;
         }
         __syncthreads();
-        for (int e = tid; e < dk * dv; e += kBwThreads) {
-            const int i = e / dv, c = e % dv;
-            float acc = expf(m.G[(n - 1) * dk + i]) * sS[e];
-            for (int r = 0; r < n; ++r) acc += m.Kd[r * dk + i] * m.U[r * dv + c];
-            sS[e] = acc;
+        // S' = Diag(e^g) S + Kd^T U: thread (state row i, eight columns), in place
+        if (tid < 2 * dk) {
+            const int i = tid >> 1, ch = (tid & 1) * 8;
+            const float eg = expf(m.G[(n - 1) * dk + i]);
+            float acc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = eg * sS[i * kCols + ch + q];
+            for (int r = 0; r < n; ++r) {
+                const float kd = sKd[r * dk + i];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] += kd * sU[r * kCols + ch + q];
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) sS[i * kCols + ch + q] = acc[q];
         }
         __syncthreads();
     }
 }
 
-// 3. State gradient entering each chunk (reverse order), dU; dS0.
+// 3. State gradient entering each chunk (reverse order), dU; dS0. Column by column like
+//    bw_fwd: dU = Kd dS' + P^T dO and dS = Diag(e^g) dS' + Qg^T dO - W^T dU act on each
+//    column of dS' and dO on its own.
+__host__ __device__ inline size_t bwd_smem_floats(int dk) {
+    return (size_t)dk * kCols + 2 * (size_t)C * dk + (size_t)C * C + 2 * C * kCols;
+}
 template <typename T>
-__global__ void __launch_bounds__(kBwThreads) bw_bwd(BwArgs a) {
-    extern __shared__ float sG[];
-    const int unit = blockIdx.x, s = unit / a.H, h = unit % a.H, tid = threadIdx.x;
-    const int dk = a.dk, dv = a.dv;
+__global__ void __launch_bounds__(kBwThreads, 2) bw_bwd(BwArgs a) {
+    extern __shared__ float4 smem4[];
+    const int groups = a.dv / kCols;
+    const int unit = blockIdx.x / groups, c0 = (blockIdx.x % groups) * kCols, s = unit / a.H, h = unit % a.H;
+    const int tid = threadIdx.x, dk = a.dk, dv = a.dv;
     const Slot sl{dk, dv};
     const T *dout = static_cast<const T *>(a.dout);
-    for (int e = tid; e < dk * dv; e += kBwThreads) sG[e] = a.dST ? a.dST[(size_t)unit * dk * dv + e] : 0.f;
-    __syncthreads();
+    float *sG = reinterpret_cast<float *>(smem4), *sA = sG + dk * kCols, *sB = sA + C * dk, *sP = sB + C * dk,
+          *sdO = sP + C * C, *sdU = sdO + C * kCols;
+    for (int e = tid; e < dk * kCols; e += kBwThreads)
+        sG[e] = a.dST ? a.dST[(size_t)unit * dk * dv + (size_t)(e / kCols) * dv + c0 + e % kCols] : 0.f;
     for (int j = a.NC - 1; j >= 0; --j) {
         int64_t t0;
         int n;
         chunk_rows(a, s, j, t0, n);
         if (n == 0) continue;
         SlotPtr m(a.slots + ((size_t)unit * a.NC + j) * sl.floats(), sl);
-        for (int e = tid; e < dk * dv; e += kBwThreads) m.dSn[e] = sG[e];
-        // dU = Kd dS' + P^T dO
-        for (int e = tid; e < n * dv; e += kBwThreads) {
-            const int r = e / dv, c = e % dv;
-            float acc = 0.f;
-            for (int i = 0; i < dk; ++i) acc += m.Kd[r * dk + i] * sG[i * dv + c];
-            for (int rr = r; rr < n; ++rr) acc += m.P[rr * C + r] * IO<T>::ld(dout + ((size_t)(t0 + rr) * a.H + h) * dv + c);
-            m.dU[e] = acc;
+        for (int e = tid; e < n * dk / 4; e += kBwThreads) {
+            reinterpret_cast<float4 *>(sA)[e] = reinterpret_cast<const float4 *>(m.Kd)[e];
+            reinterpret_cast<float4 *>(sB)[e] = reinterpret_cast<const float4 *>(m.W)[e];
         }
+        for (int e = tid; e < C * C / 4; e += kBwThreads)
+            reinterpret_cast<float4 *>(sP)[e] = reinterpret_cast<const float4 *>(m.P)[e];
+        for (int e = tid; e < n * kCols; e += kBwThreads)
+            sdO[e] = IO<T>::ld(dout + ((size_t)(t0 + e / kCols) * a.H + h) * dv + c0 + e % kCols);
         __syncthreads();
-        // dS = Diag(e^g) dS' + Qg^T dO - W^T dU
-        for (int e = tid; e < dk * dv; e += kBwThreads) {
-            const int i = e / dv, c = e % dv;
-            float acc = expf(m.G[(n - 1) * dk + i]) * sG[e];
-            for (int r = 0; r < n; ++r)
-                acc += m.Qg[r * dk + i] * IO<T>::ld(dout + ((size_t)(t0 + r) * a.H + h) * dv + c) -
-                       m.W[r * dk + i] * m.dU[r * dv + c];
-            sG[e] = acc;
+        for (int e = tid; e < dk * kCols; e += kBwThreads) m.dSn[(size_t)(e / kCols) * dv + c0 + e % kCols] = sG[e];
+        // dU = Kd dS' + P^T dO: thread (row r, four columns)
+        if (tid < n * 4) {
+            const int r = tid >> 2, cq = (tid & 3) * 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i = 0; i < dk; ++i) {
+                const float w = sA[r * dk + i];
+                const float4 x = *reinterpret_cast<const float4 *>(sG + i * kCols + cq);
+                acc.x += w * x.x;
+                acc.y += w * x.y;
+                acc.z += w * x.z;
+                acc.w += w * x.w;
+            }
+            for (int rr = r; rr < n; ++rr) {
+                const float pv = sP[rr * C + r];
+                const float4 x = *reinterpret_cast<const float4 *>(sdO + rr * kCols + cq);
+                acc.x += pv * x.x;
+                acc.y += pv * x.y;
+                acc.z += pv * x.z;
+                acc.w += pv * x.w;
+            }
+            *reinterpret_cast<float4 *>(sdU + r * kCols + cq) = acc;
+            *reinterpret_cast<float4 *>(m.dU + (size_t)r * dv + c0 + cq) = acc;
+        }
+        __syncthreads();  // Kd is no longer read: Qg takes its place
+        for (int e = tid; e < n * dk / 4; e += kBwThreads)
+            reinterpret_cast<float4 *>(sA)[e] = reinterpret_cast<const float4 *>(m.Qg)[e];
+        __syncthreads();
+        // dS = Diag(e^g) dS' + Qg^T dO - W^T dU: thread (state row i, eight columns), in place
+        if (tid < 2 * dk) {
+            const int i = tid >> 1, ch = (tid & 1) * 8;
+            const float eg = expf(m.G[(n - 1) * dk + i]);
+            float acc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = eg * sG[i * kCols + ch + q];
+            for (int r = 0; r < n; ++r) {
+                const float qg = sA[r * dk + i], w = sB[r * dk + i];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] += qg * sdO[r * kCols + ch + q] - w * sdU[r * kCols + ch + q];
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) sG[i * kCols + ch + q] = acc[q];
         }
         __syncthreads();
     }
     if (a.dS0)
-        for (int e = tid; e < dk * dv; e += kBwThreads) a.dS0[(size_t)unit * dk * dv + e] = sG[e];
+        for (int e = tid; e < dk * kCols; e += kBwThreads)
+            a.dS0[(size_t)unit * dk * dv + (size_t)(e / kCols) * dv + c0 + e % kCols] = sG[e];
 }
 
 // 4. Every per-chunk gradient.
@@ -420,17 +493,17 @@ __global__ void __launch_bounds__(kBwThreads) bw_norm(BwArgs a) {
 
 template <typename T>
 cudaError_t run(const BwArgs &a, cudaStream_t st) {
-    const unsigned units = (unsigned)a.N * (unsigned)a.H;
-    const size_t state_smem = (size_t)a.dk * a.dv * sizeof(float);
+    const unsigned units = (unsigned)a.N * (unsigned)a.H, groups = (unsigned)(a.dv / kCols);
+    const size_t fwd_smem = fwd_smem_floats(a.dk) * sizeof(float), bwd_smem = bwd_smem_floats(a.dk) * sizeof(float);
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(bw_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)state_smem)) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(bw_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fwd_smem)) != cudaSuccess)
         return e;
-    if ((e = cudaFuncSetAttribute(bw_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)state_smem)) !=
+    if ((e = cudaFuncSetAttribute(bw_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_smem)) !=
         cudaSuccess)
         return e;
     bw_prep<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
-    bw_fwd<<<units, kBwThreads, state_smem, st>>>(a);
-    bw_bwd<T><<<units, kBwThreads, state_smem, st>>>(a);
+    bw_fwd<<<units * groups, kBwThreads, fwd_smem, st>>>(a);
+    bw_bwd<T><<<units * groups, kBwThreads, bwd_smem, st>>>(a);
     bw_grads<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
     const int64_t warps = a.total * a.H;
     if (warps > 0) bw_norm<<<(unsigned)((warps * 32 + kBwThreads - 1) / kBwThreads), kBwThreads, 0, st>>>(a);
