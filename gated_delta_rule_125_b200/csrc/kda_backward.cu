@@ -19,7 +19,7 @@
 //
 // then through q/max(|q|, eps), k/max(|k|, eps).
 //
-// A reference-grade CUDA-core implementation in fp32, five launches:
+// A CUDA-core implementation in fp32, six launches:
 //   1. bw_prep   (one CTA per chunk): normalised q, k; G, Qg, Kg, Kn, Kd, A, P,
 //                the unit-lower-triangular inverse X by column forward
 //                substitution, T, W, T V;
@@ -27,7 +27,9 @@
 //                chunks' entry states and U, W and Kd staged in shared memory;
 //   3. bw_bwd    (likewise): dU and the state gradient entering each chunk, in
 //                reverse chunk order; dS0;
-//   4. bw_grads  (one CTA per chunk): every per-chunk gradient above;
+//   4. bw_rowstate (one CTA per chunk): dKd, dQg, dW and dP, the contractions
+//                over the value dimension, by shared-memory tiles;
+//      bw_grads  (one CTA per chunk): every other per-chunk gradient above;
 //   5. bw_norm   (one warp per (token, head)): through the L2 normalisation.
 // Everything lives in the caller's workspace (fp32); each product is a plain
 // loop over its output elements. The factorised exponents need e^-G finite:
@@ -345,6 +347,95 @@ __global__ void __launch_bounds__(kBwThreads, 2) bw_bwd(BwArgs a) {
             a.dS0[(size_t)unit * dk * dv + (size_t)(e / kCols) * dv + c0 + e % kCols] = sG[e];
 }
 
+// 4a. Per chunk, the contractions over the value dimension: dKd = U dS'^T,
+//     dQg = dO S^T, dW = -dU S^T (n x dk) and dP = lower(dO U^T) (C x C). Shared-memory
+//     tiles over 32 value columns at a time: the row operands (U, dO, dU) as they are,
+//     S and dS' transposed; a thread accumulates a 4 x 4 block of each output.
+constexpr int kVb = 32;                 // value columns per tile
+constexpr int kLdA = kVb + 1;           // row-operand tile row length (floats)
+__host__ __device__ inline size_t rs_smem_floats(int dk) { return 3 * (size_t)C * kLdA + 2 * (size_t)kVb * (dk + 4); }
+template <typename T>
+__global__ void __launch_bounds__(kBwThreads) bw_rowstate(BwArgs a) {
+    extern __shared__ float4 smem4[];
+    const int slot = blockIdx.x, unit = slot / a.NC, j = slot % a.NC;
+    const int s = unit / a.H, h = unit % a.H;
+    int64_t t0;
+    int n;
+    chunk_rows(a, s, j, t0, n);
+    if (n == 0) return;
+    const int dk = a.dk, dv = a.dv, tid = threadIdx.x, ldb = dk + 4;
+    const Slot sl{dk, dv};
+    SlotPtr m(a.slots + (size_t)slot * sl.floats(), sl);
+    const T *dout = static_cast<const T *>(a.dout);
+    float *sU = reinterpret_cast<float *>(smem4), *sdO = sU + C * kLdA, *sdU = sdO + C * kLdA;
+    float *sS = sdU + C * kLdA, *sSn = sS + kVb * ldb;  // [value column][state row]
+    const int ngi = dk / 4, rows_per_round = 4 * (kBwThreads / ngi), rounds = C / rows_per_round;
+    for (int round = 0; round < rounds; ++round) {
+        const int r0 = round * rows_per_round + 4 * (tid / ngi), i0 = 4 * (tid % ngi);
+        const int pr0 = 4 * (tid >> 4), pi0 = 4 * (tid & 15);  // the dP block (round 0)
+        float kd[4][4] = {}, qg[4][4] = {}, w[4][4] = {}, dp[4][4] = {};
+        for (int cb = 0; cb < dv; cb += kVb) {
+            __syncthreads();  // the previous tile is consumed
+            for (int e = tid; e < C * kVb; e += kBwThreads) {
+                const int r = e / kVb, c = e % kVb;
+                const bool in = r < n;
+                sU[r * kLdA + c] = in ? m.U[(size_t)r * dv + cb + c] : 0.f;
+                sdU[r * kLdA + c] = in ? m.dU[(size_t)r * dv + cb + c] : 0.f;
+                sdO[r * kLdA + c] = in ? IO<T>::ld(dout + ((size_t)(t0 + r) * a.H + h) * dv + cb + c) : 0.f;
+            }
+            for (int e = tid; e < dk * kVb; e += kBwThreads) {
+                const int i = e / kVb, c = e % kVb;
+                sS[c * ldb + i] = m.S[(size_t)i * dv + cb + c];
+                sSn[c * ldb + i] = m.dSn[(size_t)i * dv + cb + c];
+            }
+            __syncthreads();
+            for (int c = 0; c < kVb; ++c) {
+                const float4 bs = *reinterpret_cast<const float4 *>(sS + c * ldb + i0);
+                const float4 bn = *reinterpret_cast<const float4 *>(sSn + c * ldb + i0);
+                const float vs[4] = {bs.x, bs.y, bs.z, bs.w}, vn[4] = {bn.x, bn.y, bn.z, bn.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float u = sU[(r0 + q) * kLdA + c], o = sdO[(r0 + q) * kLdA + c], du = sdU[(r0 + q) * kLdA + c];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        kd[q][x] += u * vn[x];
+                        qg[q][x] += o * vs[x];
+                        w[q][x] -= du * vs[x];
+                    }
+                }
+                if (round == 0) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float o = sdO[(pr0 + q) * kLdA + c];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) dp[q][x] += o * sU[(pi0 + x) * kLdA + c];
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = r0 + q;
+            if (r < n) {
+                *reinterpret_cast<float4 *>(m.dKd + (size_t)r * dk + i0) = make_float4(kd[q][0], kd[q][1], kd[q][2], kd[q][3]);
+                *reinterpret_cast<float4 *>(m.dQg + (size_t)r * dk + i0) = make_float4(qg[q][0], qg[q][1], qg[q][2], qg[q][3]);
+                *reinterpret_cast<float4 *>(m.dW + (size_t)r * dk + i0) = make_float4(w[q][0], w[q][1], w[q][2], w[q][3]);
+            }
+        }
+        if (round == 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int r = pr0 + q;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int i = pi0 + x;
+                    m.dP[r * C + i] = (r < n && i <= r) ? dp[q][x] : 0.f;
+                }
+            }
+        }
+    }
+}
+
 // 4. Every per-chunk gradient.
 template <typename T>
 __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
@@ -357,31 +448,10 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
     const int dk = a.dk, dv = a.dv, tid = threadIdx.x;
     const Slot sl{dk, dv};
     SlotPtr m(a.slots + (size_t)slot * sl.floats(), sl);
-    const T *dout = static_cast<const T *>(a.dout), *v = static_cast<const T *>(a.v);
-    auto dO = [&](int r, int c) { return IO<T>::ld(dout + ((size_t)(t0 + r) * a.H + h) * dv + c); };
+    const T *v = static_cast<const T *>(a.v);
     auto V = [&](int r, int c) { return IO<T>::ld(v + ((size_t)(t0 + r) * a.H + h) * dv + c); };
     auto beta = [&](int r) { return a.beta[(size_t)(t0 + r) * a.H + h]; };
-    // (1) dKd = U dS'^T, dQg = dO S^T, dW = -dU S^T (n x dk); dP = lower(dO U^T)
-    for (int e = tid; e < n * dk; e += kBwThreads) {
-        const int r = e / dk, i = e % dk;
-        float kd = 0.f, qg = 0.f, w = 0.f;
-        for (int c = 0; c < dv; ++c) {
-            kd += m.U[r * dv + c] * m.dSn[i * dv + c];
-            qg += dO(r, c) * m.S[i * dv + c];
-            w -= m.dU[r * dv + c] * m.S[i * dv + c];
-        }
-        m.dKd[e] = kd;
-        m.dQg[e] = qg;
-        m.dW[e] = w;
-    }
-    for (int e = tid; e < C * C; e += kBwThreads) {
-        const int r = e / C, i = e % C;
-        float acc = 0.f;
-        if (r < n && i <= r)
-            for (int c = 0; c < dv; ++c) acc += dO(r, c) * m.U[i * dv + c];
-        m.dP[e] = acc;
-    }
-    __syncthreads();
+    // (1) dKd, dQg, dW and dP: bw_rowstate
     // (2) dT = lower(dU V^T + dW Kg^T); dV = T^T dU
     for (int e = tid; e < C * C; e += kBwThreads) {
         const int r = e / C, i = e % C;
@@ -504,6 +574,11 @@ cudaError_t run(const BwArgs &a, cudaStream_t st) {
     bw_prep<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
     bw_fwd<<<units * groups, kBwThreads, fwd_smem, st>>>(a);
     bw_bwd<T><<<units * groups, kBwThreads, bwd_smem, st>>>(a);
+    const size_t rs_smem = rs_smem_floats(a.dk) * sizeof(float);
+    if ((e = cudaFuncSetAttribute(bw_rowstate<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs_smem)) !=
+        cudaSuccess)
+        return e;
+    bw_rowstate<T><<<units * a.NC, kBwThreads, rs_smem, st>>>(a);
     bw_grads<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
     const int64_t warps = a.total * a.H;
     if (warps > 0) bw_norm<<<(unsigned)((warps * 32 + kBwThreads - 1) / kBwThreads), kBwThreads, 0, st>>>(a);

@@ -346,8 +346,8 @@ kda_status kda_prefill_conv(const void *q, const void *k, const void *v, const f
  *                (4 dk + 2) * 4 bytes per (token, head): 3.0 GB + 0.5 GB for one sequence of
  *                8192 tokens and 32 heads (3.6 GB). Pass max_seqlen for varlen batches.
  *
- * fp32 CUDA-core arithmetic (a reference-grade implementation; five
- * launches). It factors e^{G_r - G_i} = e^{G_r} e^{-G_i} inside each chunk:
+ * fp32 CUDA-core arithmetic (six launches; the chunk recurrences split by
+ * state column, the value-dimension contractions in shared-memory tiles). It factors e^{G_r - G_i} = e^{G_r} e^{-G_i} inside each chunk:
  * a chunk whose decay range (minus the sum of log_alpha over it) exceeds 60
  * sets device error code 2 (kda_device_error) and its gradients are not valid.
  */
