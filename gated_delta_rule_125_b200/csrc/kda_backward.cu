@@ -27,8 +27,8 @@
 //                chunks' entry states and U, W and Kd staged in shared memory;
 //   3. bw_bwd    (likewise): dU and the state gradient entering each chunk, in
 //                reverse chunk order; dS0;
-//   4. bw_rowstate (one CTA per chunk): dKd, dQg, dW and dP, the contractions
-//                over the value dimension, by shared-memory tiles;
+//   4. bw_rowstate (one CTA per chunk): dKd, dQg, dW, dP and dT, the
+//                contractions over the value (and key) dimension, by shared-memory tiles;
 //      bw_grads  (one CTA per chunk): every other per-chunk gradient above;
 //   5. bw_norm   (one warp per (token, head)): through the L2 normalisation.
 // Everything lives in the caller's workspace (fp32); each product is a plain
@@ -434,6 +434,45 @@ __global__ void __launch_bounds__(kBwThreads) bw_rowstate(BwArgs a) {
             }
         }
     }
+    // dT = lower(dU V^T + dW Kg^T): tiles over the value columns (dU, V), then the key
+    // columns (dW, written above, and Kg); the same 4 x 4 blocks as dP.
+    __syncthreads();  // dW of every row is in the slot
+    {
+        const T *v = static_cast<const T *>(a.v);
+        const int pr0 = 4 * (tid >> 4), pi0 = 4 * (tid & 15);
+        float dt[4][4] = {};
+        float *sR = sU, *sI = sdO;  // [row][32 + 1]: the r rows and the i rows of a tile
+        for (int cb = 0; cb < dv + dk; cb += kVb) {
+            __syncthreads();
+            const bool val = cb < dv;
+            for (int e = tid; e < C * kVb; e += kBwThreads) {
+                const int r = e / kVb, c = e % kVb;
+                const bool in = r < n;
+                sR[r * kLdA + c] = !in ? 0.f : val ? m.dU[(size_t)r * dv + cb + c] : m.dW[(size_t)r * dk + cb - dv + c];
+                sI[r * kLdA + c] = !in ? 0.f
+                                       : val ? IO<T>::ld(v + ((size_t)(t0 + r) * a.H + h) * dv + cb + c)
+                                             : m.Kg[(size_t)r * dk + cb - dv + c];
+            }
+            __syncthreads();
+            for (int c = 0; c < kVb; ++c) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float x0 = sR[(pr0 + q) * kLdA + c];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) dt[q][x] += x0 * sI[(pi0 + x) * kLdA + c];
+                }
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = pr0 + q;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int i = pi0 + x;
+                m.dT[r * C + i] = (r < n && i <= r) ? dt[q][x] : 0.f;
+            }
+        }
+    }
 }
 
 // 4. Every per-chunk gradient.
@@ -448,20 +487,11 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
     const int dk = a.dk, dv = a.dv, tid = threadIdx.x;
     const Slot sl{dk, dv};
     SlotPtr m(a.slots + (size_t)slot * sl.floats(), sl);
-    const T *v = static_cast<const T *>(a.v);
-    auto V = [&](int r, int c) { return IO<T>::ld(v + ((size_t)(t0 + r) * a.H + h) * dv + c); };
+    extern __shared__ float4 smem4[];
+    float *sX = reinterpret_cast<float *>(smem4), *sdT = sX + C * (C + 1), *sY = sdT + C * (C + 1);
     auto beta = [&](int r) { return a.beta[(size_t)(t0 + r) * a.H + h]; };
     // (1) dKd, dQg, dW and dP: bw_rowstate
-    // (2) dT = lower(dU V^T + dW Kg^T); dV = T^T dU
-    for (int e = tid; e < C * C; e += kBwThreads) {
-        const int r = e / C, i = e % C;
-        float acc = 0.f;
-        if (r < n && i <= r) {
-            for (int c = 0; c < dv; ++c) acc += m.dU[r * dv + c] * V(i, c);
-            for (int c = 0; c < dk; ++c) acc += m.dW[r * dk + c] * m.Kg[i * dk + c];
-        }
-        m.dT[e] = acc;
-    }
+    // (2) dT: bw_rowstate; dV = T^T dU
     for (int e = tid; e < n * dv; e += kBwThreads) {
         const int r = e / dv, c = e % dv;
         float acc = 0.f;
@@ -476,12 +506,20 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
         for (int rr = r; rr < n; ++rr) acc += m.T[rr * C + r] * m.dW[rr * dk + c];
         m.dKg[e] = acc;
     }
+    // X, dT and Y in shared memory, rows padded to C + 1 floats (conflict-free by row and by column)
+    constexpr int LD = C + 1;
+    for (int e = tid; e < C * C; e += kBwThreads) {
+        sX[(e / C) * LD + e % C] = m.X[e];
+        sdT[(e / C) * LD + e % C] = m.dT[e];
+    }
+    __syncthreads();
     for (int e = tid; e < C * C; e += kBwThreads) {
         const int r = e / C, i = e % C;
         float acc = 0.f;
         if (r < n && i < n)
-            for (int mm = 0; mm < n; ++mm) acc += m.X[mm * C + r] * m.dT[mm * C + i] * beta(i);
+            for (int mm = 0; mm < n; ++mm) acc += sX[mm * LD + r] * sdT[mm * LD + i] * beta(i);
         m.Y[e] = acc;
+        sY[r * LD + i] = acc;
     }
     __syncthreads();
     // (4) dM = -Y X^T
@@ -489,7 +527,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
         const int r = e / C, i = e % C;
         float acc = 0.f;
         if (r < n && i < n)
-            for (int mm = 0; mm < n; ++mm) acc -= m.Y[r * C + mm] * m.X[i * C + mm];
+            for (int mm = 0; mm < n; ++mm) acc -= sY[r * LD + mm] * sX[i * LD + mm];
         m.dM[e] = acc;
     }
     __syncthreads();
@@ -579,7 +617,11 @@ cudaError_t run(const BwArgs &a, cudaStream_t st) {
         cudaSuccess)
         return e;
     bw_rowstate<T><<<units * a.NC, kBwThreads, rs_smem, st>>>(a);
-    bw_grads<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
+    const size_t gr_smem = 3 * (size_t)C * (C + 1) * sizeof(float);
+    if ((e = cudaFuncSetAttribute(bw_grads<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gr_smem)) !=
+        cudaSuccess)
+        return e;
+    bw_grads<T><<<units * a.NC, kBwThreads, gr_smem, st>>>(a);
     const int64_t warps = a.total * a.H;
     if (warps > 0) bw_norm<<<(unsigned)((warps * 32 + kBwThreads - 1) / kBwThreads), kBwThreads, 0, st>>>(a);
     return cudaGetLastError();
