@@ -42,6 +42,8 @@ namespace {
 constexpr int C = kChunk;  // 64
 constexpr int kBwThreads = 256;
 constexpr float kBwRange = 60.f;
+constexpr int kVb = 32;        // columns per shared-memory tile of the tiled contractions
+constexpr int kLdA = kVb + 1;  // tile row length (floats): rows apart by one bank
 
 // Per-chunk scratch (floats), in this order.
 struct Slot {
@@ -150,36 +152,75 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep(BwArgs a) {
         m.Kd[e] = kv * expf(g - G);
     }
     __syncthreads();
-    // A = strict_lower(Kg Kn^T), P = lower(Qg Kn^T)
-    for (int e = tid; e < C * C; e += kBwThreads) {
-        const int r = e / C, i = e % C;
-        float sa = 0.f, sp = 0.f;
-        if (r < n && i <= r) {
-            for (int c = 0; c < dk; ++c) {
-                sa += m.Kg[r * dk + c] * m.Kn[i * dk + c];
-                sp += m.Qg[r * dk + c] * m.Kn[i * dk + c];
+    // A = strict_lower(Kg Kn^T), P = lower(Qg Kn^T): 32-column tiles of Kg, Qg and Kn
+    // in shared memory, a 4 x 4 block of each per thread
+    extern __shared__ float4 smem4[];
+    float *sm = reinterpret_cast<float *>(smem4);
+    {
+        float *tKg = sm, *tQg = tKg + C * kLdA, *tKn = tQg + C * kLdA;
+        const int r0 = 4 * (tid >> 4), i0 = 4 * (tid & 15);
+        float aa[4][4] = {}, pp[4][4] = {};
+        for (int cb = 0; cb < dk; cb += kVb) {
+            __syncthreads();  // the exponent factors are written; the previous tile is consumed
+            for (int e = tid; e < C * kVb; e += kBwThreads) {
+                const int r = e / kVb, c = e % kVb;
+                const bool in = r < n;
+                tKg[r * kLdA + c] = in ? m.Kg[(size_t)r * dk + cb + c] : 0.f;
+                tQg[r * kLdA + c] = in ? m.Qg[(size_t)r * dk + cb + c] : 0.f;
+                tKn[r * kLdA + c] = in ? m.Kn[(size_t)r * dk + cb + c] : 0.f;
             }
-        }
-        m.A[e] = (r < n && i < r) ? sa : 0.f;
-        m.P[e] = (r < n && i <= r) ? sp : 0.f;
-    }
-    __syncthreads();
-    // X = (I + Diag(beta) A)^-1: column i by forward substitution (rows >= i)
-    const float *bt = a.beta;
-    for (int i = tid; i < C; i += kBwThreads) {
-        for (int r = 0; r < C; ++r) {
-            float x = 0.f;
-            if (r < n && i < n && r >= i) {
-                if (r == i) {
-                    x = 1.f;
-                } else {
-                    float acc = 0.f;
-                    for (int mm = i; mm < r; ++mm) acc += m.A[r * C + mm] * m.X[mm * C + i];
-                    x = -bt[(size_t)(t0 + r) * a.H + h] * acc;
+            __syncthreads();
+            for (int c = 0; c < kVb; ++c) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float kg = tKg[(r0 + q) * kLdA + c], qg = tQg[(r0 + q) * kLdA + c];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const float kn = tKn[(i0 + x) * kLdA + c];
+                        aa[q][x] += kg * kn;
+                        pp[q][x] += qg * kn;
+                    }
                 }
             }
-            m.X[r * C + i] = x;
         }
+        __syncthreads();  // the tiles are consumed: A takes the shared memory (rows of C + 1)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = r0 + q;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const int i = i0 + x;
+                const float av = (r < n && i < r) ? aa[q][x] : 0.f;
+                m.A[r * C + i] = av;
+                sm[r * (C + 1) + i] = av;
+                m.P[r * C + i] = (r < n && i <= r) ? pp[q][x] : 0.f;
+            }
+        }
+    }
+    __syncthreads();
+    // X = (I + Diag(beta) A)^-1: column i by forward substitution (rows >= i), A and X in
+    // shared memory (rows of C + 1 floats)
+    const float *bt = a.beta;
+    {
+        const float *sA = sm;
+        float *sXs = sm + C * (C + 1);
+        for (int i = tid; i < C; i += kBwThreads) {
+            for (int r = 0; r < C; ++r) {
+                float x = 0.f;
+                if (r < n && i < n && r >= i) {
+                    if (r == i) {
+                        x = 1.f;
+                    } else {
+                        float acc = 0.f;
+                        for (int mm = i; mm < r; ++mm) acc += sA[r * (C + 1) + mm] * sXs[mm * (C + 1) + i];
+                        x = -bt[(size_t)(t0 + r) * a.H + h] * acc;
+                    }
+                }
+                sXs[r * (C + 1) + i] = x;
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < C * C; e += kBwThreads) m.X[e] = sXs[(e / C) * (C + 1) + e % C];
     }
     __syncthreads();
     for (int e = tid; e < C * C; e += kBwThreads) {
@@ -351,8 +392,6 @@ __global__ void __launch_bounds__(kBwThreads, 2) bw_bwd(BwArgs a) {
 //     dQg = dO S^T, dW = -dU S^T (n x dk) and dP = lower(dO U^T) (C x C). Shared-memory
 //     tiles over 32 value columns at a time: the row operands (U, dO, dU) as they are,
 //     S and dS' transposed; a thread accumulates a 4 x 4 block of each output.
-constexpr int kVb = 32;                 // value columns per tile
-constexpr int kLdA = kVb + 1;           // row-operand tile row length (floats)
 __host__ __device__ inline size_t rs_smem_floats(int dk) { return 3 * (size_t)C * kLdA + 2 * (size_t)kVb * (dk + 4); }
 template <typename T>
 __global__ void __launch_bounds__(kBwThreads) bw_rowstate(BwArgs a) {
@@ -529,6 +568,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
         if (r < n && i < n)
             for (int mm = 0; mm < n; ++mm) acc -= sY[r * LD + mm] * sX[i * LD + mm];
         m.dM[e] = acc;
+        sdT[r * LD + i] = acc;  // dT is no longer read: dM takes its place
     }
     __syncthreads();
     // (5) dA = strict_lower(Diag(beta) dM); dbeta
@@ -539,7 +579,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
     for (int i = tid; i < n; i += kBwThreads) {
         float acc = 0.f;
         for (int r = 0; r < n; ++r) acc += m.dT[r * C + i] * m.X[r * C + i];
-        for (int mm = 0; mm < i; ++mm) acc += m.dM[i * C + mm] * m.A[i * C + mm];
+        for (int mm = 0; mm < i; ++mm) acc += sdT[i * LD + mm] * m.A[i * C + mm];
         a.dbeta[(size_t)(t0 + i) * a.H + h] = acc;
     }
     __syncthreads();
@@ -557,14 +597,21 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
         m.dQg[e] += qg;
     }
     __syncthreads();
-    // (7)(8) dG, dg, dlog_alpha (reverse cumsum); d q^, d k^ through the exponents
+    // (7)(8) dG, dg, dlog_alpha (reverse cumsum); d q^, d k^ through the exponents.
+    // The row sums of dS' * S first, a warp per state row (coalesced), into shared memory.
+    float *sss = sX;  // X is no longer read
+    for (int c = tid >> 5; c < dk; c += kBwThreads / 32) {
+        float acc = 0.f;
+        for (int cc = tid & 31; cc < dv; cc += 32) acc += m.dSn[c * dv + cc] * m.S[c * dv + cc];
+        for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if ((tid & 31) == 0) sss[c] = acc;
+    }
+    __syncthreads();
     for (int c = tid; c < dk; c += kBwThreads) {
         const float g = m.G[(n - 1) * dk + c];
         float dg = 0.f;
         for (int r = 0; r < n; ++r) dg += m.dKd[r * dk + c] * m.Kd[r * dk + c];
-        float ss = 0.f;
-        for (int cc = 0; cc < dv; ++cc) ss += m.dSn[c * dv + cc] * m.S[c * dv + cc];
-        dg += expf(g) * ss;
+        dg += expf(g) * sss[c];
         float run = 0.f;
         for (int r = n - 1; r >= 0; --r) {
             const int e = r * dk + c;
@@ -609,7 +656,11 @@ cudaError_t run(const BwArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(bw_bwd<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bwd_smem)) !=
         cudaSuccess)
         return e;
-    bw_prep<T><<<units * a.NC, kBwThreads, 0, st>>>(a);
+    const size_t prep_smem = 2 * (size_t)C * (C + 1) * sizeof(float);  // >= the three 64 x 33 tiles
+    if ((e = cudaFuncSetAttribute(bw_prep<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem)) !=
+        cudaSuccess)
+        return e;
+    bw_prep<T><<<units * a.NC, kBwThreads, prep_smem, st>>>(a);
     bw_fwd<<<units * groups, kBwThreads, fwd_smem, st>>>(a);
     bw_bwd<T><<<units * groups, kBwThreads, bwd_smem, st>>>(a);
     const size_t rs_smem = rs_smem_floats(a.dk) * sizeof(float);
