@@ -220,8 +220,9 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------- kda ----
 
-PREFILL_SOURCES = ["gated_delta_rule_125_b200/csrc/kda_prefill_tc.cu", "gated_delta_rule_125_b200/csrc/kda_tc.cuh"]
-DECODE_SOURCES = ["gated_delta_rule_125_b200/csrc/kda_decode.cu"]
+PREFILL_SOURCES = ["gated_delta_rule_125_b200/csrc/kda_prefill_tc.cu", "gated_delta_rule_125_b200/csrc/kda_tc.cuh",
+                   "gated_delta_rule_125_b200/csrc/kda_internal.cuh"]
+DECODE_SOURCES = ["gated_delta_rule_125_b200/csrc/kda_decode.cu", "gated_delta_rule_125_b200/csrc/kda_internal.cuh"]
 
 
 def profiled_traffic(profile, sources):
