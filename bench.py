@@ -46,7 +46,7 @@ METRIC = "KDA prefill tokens/s at H=32,d=128; decode-step HBM GB/s vs B200 peak"
 PREFILL = "prefill_8k"
 T8K, H, D = 8192, 32, 128
 DEC_N = 256
-BACKWARD_LAUNCHES = 6  # bw_prep, bw_fwd, bw_bwd, bw_rowstate, bw_grads, bw_norm
+BACKWARD_LAUNCHES = 7  # bw_offsets, bw_prep, bw_fwd, bw_bwd, bw_rowstate, bw_grads, bw_norm
 # Algorithmic HBM bytes (inputs read once, outputs written once):
 #   prefill per token (all 32 heads): q,k,v bf16 3*32*128*2 + log_alpha 32*128*4 + beta 32*4
 #   + o 32*128*2 = 49,280 B; plus S0 read and S_T written (2 MiB each at H=32).
@@ -607,7 +607,7 @@ def run_kda(args, world, rank, local):
                                   "(bf16) and dL/dS_T (fp32); fp32 CUDA-core kernels",
                       "roofline": {"bound": "hbm", "achieved": bw["gbs"], "peak": hbm, "unit": "GB/s",
                                    "frac": bw["gbs"] / hbm, "traffic": None,
-                                   "kernel": "bw_prep + bw_fwd + bw_bwd + bw_rowstate + bw_grads + bw_norm",
+                                   "kernel": "bw_offsets + bw_prep + bw_fwd + bw_bwd + bw_rowstate + bw_grads + bw_norm",
                                    "algorithmic_bytes": BACKWARD_BYTES, "peak_source": peak_src}}
                      if "ms" in bw else bw),
         "decode_conv": {"value": DECODE_CONV_BYTES / (dconv_us_max * 1e-6) / 1e9, "unit": "GB/s",

@@ -347,7 +347,8 @@ def kda_backward(q, k, v, log_alpha, beta, do, dS_T=None, S0=None, cu_seqlens=No
         max_seqlen = T if cu_seqlens is None else int((cu_seqlens[1:] - cu_seqlens[:-1]).max().item())
     f32 = dict(dtype=torch.float32, device=q.device)
     dq, dkk = torch.empty((T, H, dk), **f32), torch.empty((T, H, dk), **f32)
-    dvv, dla = torch.empty((T, H, dv), **f32), torch.empty((T, H, dk), **f32)
+    dvv = torch.empty((T, H, dv), **f32)
+    dla = torch.empty(tuple(log_alpha.shape), **f32)  # [T,H,dk], or [T,H] with one gate per head
     db = torch.empty((T, H), **f32)
     dS0 = torch.empty((N, H, dk, dv), **f32) if want_dS0 else None
     flags = _flags(l2norm, False, log_alpha.dim() == 2)
@@ -355,7 +356,7 @@ def kda_backward(q, k, v, log_alpha, beta, do, dS_T=None, S0=None, cu_seqlens=No
     if workspace is None:
         nbytes = lib.kda_backward_workspace_size(N, T, max_seqlen, H, dk, dv, code, 64, flags)
         if nbytes == 0:
-            raise KDAError(KDA_ERR_UNSUPPORTED if log_alpha.dim() == 2 else 1, "kda_backward_workspace_size")
+            raise KDAError(KDA_ERR_INVALID_ARG, "kda_backward_workspace_size")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
     rc = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
                           N, T, max_seqlen, H, dk, dv, code, 64, flags, _ptr(do), _ptr(dS_T),

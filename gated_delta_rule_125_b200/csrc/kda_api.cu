@@ -405,18 +405,19 @@ kda_status kda_decode_step_ex(const void *q, const void *k, const void *v, const
 }
 
 namespace {
-int64_t backward_chunks(int64_t total_tokens, int32_t max_seqlen) {
-    const int64_t L = (max_seqlen > 0) ? std::min<int64_t>(max_seqlen, total_tokens) : total_tokens;
-    return std::max<int64_t>(1, (L + kda::kChunk - 1) / kda::kChunk);
+// Chunk slots of the backward: H per chunk of every sequence (bounded by total / 64 + N), kept
+// within one launch grid.
+bool backward_fits(int32_t num_seqs, int64_t total_tokens, int32_t H) {
+    return kda::backward_slots_per_head(num_seqs, total_tokens) * H <= INT32_MAX;
 }
 }  // namespace
 
 size_t kda_backward_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t max_seqlen, int32_t H,
                                    int32_t dk, int32_t dv, kda_dtype dtype, int32_t chunk, uint32_t flags) {
     if (check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags) != KDA_OK) return 0;
-    if (flags & KDA_FLAG_SCALAR_GATE) return 0;
-    return kda::backward_workspace_bytes(num_seqs, H, total_tokens, dk, dv,
-                                         (int)backward_chunks(total_tokens, max_seqlen));
+    (void)max_seqlen;  // the slots follow the sequences' own chunk counts
+    if (!backward_fits(num_seqs, total_tokens, H)) return 0;
+    return kda::backward_workspace_bytes(num_seqs, H, total_tokens, dk, dv);
 }
 
 kda_status kda_backward(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
@@ -427,21 +428,20 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const float
                         size_t workspace_bytes, kda_stream_t stream) {
     kda_status rc = check_prefill_shape(num_seqs, total_tokens, H, dk, dv, dtype, chunk, flags);
     if (rc != KDA_OK) return rc;
-    if (flags & KDA_FLAG_SCALAR_GATE) return KDA_ERR_UNSUPPORTED;
     if (cu_seqlens == nullptr && num_seqs != 1) return KDA_ERR_INVALID_ARG;
     if (total_tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk_out || !dv_out ||
                              !dlog_alpha || !dbeta))
         return KDA_ERR_INVALID_ARG;
-    const int64_t NC = backward_chunks(total_tokens, max_seqlen);
-    if (NC > INT32_MAX) return KDA_ERR_UNSUPPORTED;
-    if (!workspace || workspace_bytes < kda::backward_workspace_bytes(num_seqs, H, total_tokens, dk, dv, (int)NC))
+    if (!backward_fits(num_seqs, total_tokens, H)) return KDA_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < kda::backward_workspace_bytes(num_seqs, H, total_tokens, dk, dv))
         return KDA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 15u)) return KDA_ERR_MISALIGNED;
     kda::BackwardArgs a;
     a.q = q; a.k = k; a.v = v; a.dout = dout;
     a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.dS_T = dS_T; a.cu = cu_seqlens;
-    a.total = total_tokens; a.N = num_seqs; a.H = H; a.dk = dk; a.dv = dv; a.NC = (int)NC;
+    a.total = total_tokens; a.N = num_seqs; a.H = H; a.dk = dk; a.dv = dv;
     a.l2norm = (flags & KDA_FLAG_NO_L2NORM) ? 0 : 1;
+    a.la_scalar = (flags & KDA_FLAG_SCALAR_GATE) ? 1 : 0;
     a.eps = kEps;
     a.dq = dq; a.dk_out = dk_out; a.dv_out = dv_out; a.dlog_alpha = dlog_alpha; a.dbeta = dbeta; a.dS0 = dS0;
     a.ws = workspace;

@@ -19,7 +19,8 @@
 //
 // then through q/max(|q|, eps), k/max(|k|, eps).
 //
-// A CUDA-core implementation in fp32, six launches:
+// A CUDA-core implementation in fp32, seven launches (bw_offsets: the first chunk of each
+// sequence, so that the chunk slots are packed; then):
 //   1. bw_prep   (one CTA per chunk): normalised q, k; G, Qg, Kg, Kn, Kd, A, P,
 //                the unit-lower-triangular inverse X by column forward
 //                substitution, T, W, T V;
@@ -77,14 +78,62 @@ struct BwArgs {
     const float *la, *beta, *S0, *dST;
     const int32_t *cu;
     int64_t total;
-    int N, H, dk, dv, NC;  // NC: chunk slots per (sequence, head)
-    int l2norm;
+    int N, H, dk, dv, NC;  // NC: chunk slots per head, at least the chunks of all sequences
+    int l2norm, la_scalar;
     float eps;
     float *dq, *dkk, *dvv, *dla, *dbeta, *dS0;
-    float *slots;          // N * H * NC slots
+    float *slots;          // NC * H slots: chunk ci of head h in slot ci * H + h
+    int *coff;             // [N + 1]: first chunk of each sequence (prefix sums of ceil(len / 64))
     float *qh, *kh, *dqh, *dkh, *nq, *nk;  // per (token, head)
     int *err;
 };
+
+// Slot of block b of the per-chunk kernels (grid H * NC): chunk ci = b / H of head h = b % H,
+// sequence s the last one whose first chunk is at or before ci, j its chunk; false past the chunks.
+__device__ __forceinline__ bool slot_chunk(const BwArgs &a, int b, int &s, int &h, int &j) {
+    const int ci = b / a.H;
+    h = b % a.H;
+    if (ci >= a.coff[a.N]) return false;
+    int lo = 0, hi = a.N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.coff[mid] <= ci) lo = mid;
+        else hi = mid - 1;
+    }
+    s = lo;
+    j = ci - a.coff[lo];
+    return true;
+}
+__device__ __forceinline__ size_t slot_of(const BwArgs &a, int s, int h, int j) {
+    return (size_t)(a.coff[s] + j) * a.H + h;
+}
+
+// First chunk of each sequence: one CTA, each thread a run of sequences, then a scan of the runs.
+__global__ void __launch_bounds__(1024) bw_offsets(BwArgs a) {
+    __shared__ int part[1024];
+    const int tid = threadIdx.x, per = (a.N + 1023) / 1024, s0 = tid * per, s1 = min(a.N, s0 + per);
+    auto nch = [&](int s) {
+        int64_t bos, eos;
+        seq_bounds(a.cu, s, a.total, bos, eos);
+        return (int)((eos - bos + C - 1) / C);
+    };
+    int sum = 0;
+    for (int s = s0; s < s1; ++s) sum += nch(s);
+    part[tid] = sum;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan of the runs
+        const int v = tid >= off ? part[tid - off] : 0;
+        __syncthreads();
+        part[tid] += v;
+        __syncthreads();
+    }
+    int run = part[tid] - sum;
+    for (int s = s0; s < s1; ++s) {
+        a.coff[s] = run;
+        run += nch(s);
+    }
+    if (tid == 1023) a.coff[a.N] = part[1023];
+}
 
 __device__ __forceinline__ void chunk_rows(const BwArgs &a, int s, int j, int64_t &t0, int &n) {
     int64_t bos, eos;
@@ -97,8 +146,9 @@ __device__ __forceinline__ void chunk_rows(const BwArgs &a, int s, int j, int64_
 // 1. Per chunk: normalised q, k; G, Qg, Kg, Kn, Kd; A, P; X, T; W = T Kg; T V.
 template <typename T>
 __global__ void __launch_bounds__(kBwThreads) bw_prep(BwArgs a) {
-    const int slot = blockIdx.x, unit = slot / a.NC, j = slot % a.NC;
-    const int s = unit / a.H, h = unit % a.H;
+    const int slot = blockIdx.x;
+    int s, h, j;
+    if (!slot_chunk(a, slot, s, h, j)) return;
     int64_t t0;
     int n;
     chunk_rows(a, s, j, t0, n);
@@ -135,7 +185,7 @@ __global__ void __launch_bounds__(kBwThreads) bw_prep(BwArgs a) {
     for (int c = tid; c < dk; c += kBwThreads) {
         float run = 0.f;
         for (int r = 0; r < n; ++r) {
-            run += a.la[(size_t)(t0 + r) * a.H * dk + (size_t)h * dk + c];
+            run += a.la_scalar ? a.la[(size_t)(t0 + r) * a.H + h] : a.la[(size_t)(t0 + r) * a.H * dk + (size_t)h * dk + c];
             m.G[r * dk + c] = run;
         }
         if (-run > kBwRange && a.err) atomicCAS(a.err, 0, 2);
@@ -258,12 +308,13 @@ __global__ void __launch_bounds__(kBwThreads, 2) bw_fwd(BwArgs a) {
     float *sS = reinterpret_cast<float *>(smem4), *sW = sS + dk * kCols, *sKd = sW + C * dk, *sU = sKd + C * dk;
     for (int e = tid; e < dk * kCols; e += kBwThreads)
         sS[e] = a.S0 ? a.S0[(size_t)unit * dk * dv + (size_t)(e / kCols) * dv + c0 + e % kCols] : 0.f;
-    for (int j = 0; j < a.NC; ++j) {
+    const int nchunks = a.coff[s + 1] - a.coff[s];
+    for (int j = 0; j < nchunks; ++j) {
         int64_t t0;
         int n;
         chunk_rows(a, s, j, t0, n);
         if (n == 0) break;
-        SlotPtr m(a.slots + ((size_t)unit * a.NC + j) * sl.floats(), sl);
+        SlotPtr m(a.slots + slot_of(a, s, unit % a.H, j) * sl.floats(), sl);
         for (int e = tid; e < n * dk / 4; e += kBwThreads) {
             reinterpret_cast<float4 *>(sW)[e] = reinterpret_cast<const float4 *>(m.W)[e];
             reinterpret_cast<float4 *>(sKd)[e] = reinterpret_cast<const float4 *>(m.Kd)[e];
@@ -323,12 +374,12 @@ __global__ void __launch_bounds__(kBwThreads, 2) bw_bwd(BwArgs a) {
           *sdO = sP + C * C, *sdU = sdO + C * kCols;
     for (int e = tid; e < dk * kCols; e += kBwThreads)
         sG[e] = a.dST ? a.dST[(size_t)unit * dk * dv + (size_t)(e / kCols) * dv + c0 + e % kCols] : 0.f;
-    for (int j = a.NC - 1; j >= 0; --j) {
+    for (int j = a.coff[s + 1] - a.coff[s] - 1; j >= 0; --j) {
         int64_t t0;
         int n;
         chunk_rows(a, s, j, t0, n);
         if (n == 0) continue;
-        SlotPtr m(a.slots + ((size_t)unit * a.NC + j) * sl.floats(), sl);
+        SlotPtr m(a.slots + slot_of(a, s, h, j) * sl.floats(), sl);
         for (int e = tid; e < n * dk / 4; e += kBwThreads) {
             reinterpret_cast<float4 *>(sA)[e] = reinterpret_cast<const float4 *>(m.Kd)[e];
             reinterpret_cast<float4 *>(sB)[e] = reinterpret_cast<const float4 *>(m.W)[e];
@@ -396,8 +447,9 @@ __host__ __device__ inline size_t rs_smem_floats(int dk) { return 3 * (size_t)C 
 template <typename T>
 __global__ void __launch_bounds__(kBwThreads) bw_rowstate(BwArgs a) {
     extern __shared__ float4 smem4[];
-    const int slot = blockIdx.x, unit = slot / a.NC, j = slot % a.NC;
-    const int s = unit / a.H, h = unit % a.H;
+    const int slot = blockIdx.x;
+    int s, h, j;
+    if (!slot_chunk(a, slot, s, h, j)) return;
     int64_t t0;
     int n;
     chunk_rows(a, s, j, t0, n);
@@ -517,8 +569,9 @@ __global__ void __launch_bounds__(kBwThreads) bw_rowstate(BwArgs a) {
 // 4. Every per-chunk gradient.
 template <typename T>
 __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
-    const int slot = blockIdx.x, unit = slot / a.NC, j = slot % a.NC;
-    const int s = unit / a.H, h = unit % a.H;
+    const int slot = blockIdx.x;
+    int s, h, j;
+    if (!slot_chunk(a, slot, s, h, j)) return;
     int64_t t0;
     int n;
     chunk_rows(a, s, j, t0, n);
@@ -606,6 +659,8 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
         for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if ((tid & 31) == 0) sss[c] = acc;
     }
+    float *srow = sY;  // one gate per (token, head): the per-channel gradients summed per row
+    for (int r = tid; r < C; r += kBwThreads) srow[r] = 0.f;
     __syncthreads();
     for (int c = tid; c < dk; c += kBwThreads) {
         const float g = m.G[(n - 1) * dk + c];
@@ -617,11 +672,16 @@ __global__ void __launch_bounds__(kBwThreads) bw_grads(BwArgs a) {
             const int e = r * dk + c;
             run += m.dQg[e] * m.Qg[e] + m.dKg[e] * m.Kg[e] - m.dKn[e] * m.Kn[e] - m.dKd[e] * m.Kd[e];
             const size_t row = (size_t)(t0 + r) * a.H + h;
-            a.dla[row * dk + c] = run + dg;
+            if (a.la_scalar) atomicAdd(&srow[r], run + dg);
+            else a.dla[row * dk + c] = run + dg;
             const float G = m.G[e];
             a.dqh[row * dk + c] = m.dQg[e] * expf(G);
             a.dkh[row * dk + c] = m.dKg[e] * expf(G) + m.dKn[e] * expf(-G) + m.dKd[e] * expf(g - G);
         }
+    }
+    if (a.la_scalar) {
+        __syncthreads();
+        for (int r = tid; r < n; r += kBwThreads) a.dla[(size_t)(t0 + r) * a.H + h] = srow[r];
     }
 }
 
@@ -660,19 +720,21 @@ cudaError_t run(const BwArgs &a, cudaStream_t st) {
     if ((e = cudaFuncSetAttribute(bw_prep<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)prep_smem)) !=
         cudaSuccess)
         return e;
-    bw_prep<T><<<units * a.NC, kBwThreads, prep_smem, st>>>(a);
+    bw_offsets<<<1, 1024, 0, st>>>(a);
+    const unsigned slots = (unsigned)a.H * (unsigned)a.NC;
+    bw_prep<T><<<slots, kBwThreads, prep_smem, st>>>(a);
     bw_fwd<<<units * groups, kBwThreads, fwd_smem, st>>>(a);
     bw_bwd<T><<<units * groups, kBwThreads, bwd_smem, st>>>(a);
     const size_t rs_smem = rs_smem_floats(a.dk) * sizeof(float);
     if ((e = cudaFuncSetAttribute(bw_rowstate<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rs_smem)) !=
         cudaSuccess)
         return e;
-    bw_rowstate<T><<<units * a.NC, kBwThreads, rs_smem, st>>>(a);
+    bw_rowstate<T><<<slots, kBwThreads, rs_smem, st>>>(a);
     const size_t gr_smem = 3 * (size_t)C * (C + 1) * sizeof(float);
     if ((e = cudaFuncSetAttribute(bw_grads<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gr_smem)) !=
         cudaSuccess)
         return e;
-    bw_grads<T><<<units * a.NC, kBwThreads, gr_smem, st>>>(a);
+    bw_grads<T><<<slots, kBwThreads, gr_smem, st>>>(a);
     const int64_t warps = a.total * a.H;
     if (warps > 0) bw_norm<<<(unsigned)((warps * 32 + kBwThreads - 1) / kBwThreads), kBwThreads, 0, st>>>(a);
     return cudaGetLastError();
@@ -680,29 +742,34 @@ cudaError_t run(const BwArgs &a, cudaStream_t st) {
 
 }  // namespace
 
-size_t backward_workspace_bytes(int N, int H, int64_t total, int dk, int dv, int NC) {
+int64_t backward_slots_per_head(int N, int64_t total) { return total / C + N; }  // >= sum of ceil(len / 64)
+
+size_t backward_workspace_bytes(int N, int H, int64_t total, int dk, int dv) {
     const Slot sl{dk, dv};
-    return ((size_t)N * H * NC * sl.floats() + (size_t)total * H * (4 * (size_t)dk + 2)) * sizeof(float);
+    return ((size_t)backward_slots_per_head(N, total) * H * sl.floats() + (size_t)total * H * (4 * (size_t)dk + 2) +
+            ((size_t)N + 4) / 4 * 4) * sizeof(float);
 }
 
 cudaError_t backward(const BackwardArgs &b, bool bf16, cudaStream_t st) {
     BwArgs a;
     a.q = b.q; a.k = b.k; a.v = b.v; a.dout = b.dout;
     a.la = b.log_alpha; a.beta = b.beta; a.S0 = b.S0; a.dST = b.dS_T; a.cu = b.cu;
-    a.total = b.total; a.N = b.N; a.H = b.H; a.dk = b.dk; a.dv = b.dv; a.NC = b.NC;
-    a.l2norm = b.l2norm; a.eps = b.eps;
+    a.total = b.total; a.N = b.N; a.H = b.H; a.dk = b.dk; a.dv = b.dv;
+    a.NC = (int)backward_slots_per_head(b.N, b.total);
+    a.l2norm = b.l2norm; a.la_scalar = b.la_scalar; a.eps = b.eps;
     a.dq = b.dq; a.dkk = b.dk_out; a.dvv = b.dv_out; a.dla = b.dlog_alpha; a.dbeta = b.dbeta; a.dS0 = b.dS0;
     const Slot sl{b.dk, b.dv};
     float *p = static_cast<float *>(b.ws);
     a.slots = p;
-    p += (size_t)b.N * b.H * b.NC * sl.floats();
+    p += (size_t)a.NC * b.H * sl.floats();
     const size_t th = (size_t)b.total * b.H;
     a.qh = p; p += th * b.dk;
     a.kh = p; p += th * b.dk;
     a.dqh = p; p += th * b.dk;
     a.dkh = p; p += th * b.dk;
     a.nq = p; p += th;
-    a.nk = p;
+    a.nk = p; p += th;
+    a.coff = reinterpret_cast<int *>(p);
     a.err = b.err;
     return bf16 ? run<__nv_bfloat16>(a, st) : run<float>(a, st);
 }

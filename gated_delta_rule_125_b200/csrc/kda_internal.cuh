@@ -145,14 +145,16 @@ struct BackwardArgs {
     const float *log_alpha, *beta, *S0, *dS_T;
     const int32_t *cu;
     int64_t total;
-    int N, H, dk, dv, NC;  // NC: chunks of the longest sequence
+    int N, H, dk, dv;
     int l2norm;
+    int la_scalar;  // log_alpha and dlog_alpha are [T][H]: one gate per (token, head)
     float eps;
     float *dq, *dk_out, *dv_out, *dlog_alpha, *dbeta, *dS0;
     void *ws;
     int *err;
 };
-size_t backward_workspace_bytes(int N, int H, int64_t total, int dk, int dv, int NC);
+int64_t backward_slots_per_head(int N, int64_t total);  // chunk slots per head (>= the chunks)
+size_t backward_workspace_bytes(int N, int H, int64_t total, int dk, int dv);
 cudaError_t backward(const BackwardArgs &b, bool bf16, cudaStream_t st);
 
 // decode step

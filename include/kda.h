@@ -331,23 +331,28 @@ kda_status kda_prefill_conv(const void *q, const void *k, const void *v, const f
  * to q, k, v, log_alpha, beta and S0, given dL/do and dL/dS_T. The pages
  * mention training but give no backward; the chunked reverse-mode algebra
  * implemented here is stated in csrc/kda_backward.cu. The same inputs and
- * rules as kda_prefill (chunk 64; KDA_FLAG_NO_L2NORM honoured; one gate per
- * (token, head) is not supported: KDA_ERR_UNSUPPORTED), plus:
+ * rules as kda_prefill (chunk 64; KDA_FLAG_NO_L2NORM honoured; with
+ * KDA_FLAG_SCALAR_GATE, log_alpha and grad_log_alpha are [T][H]: the gradient
+ * of the one gate per (token, head) is the sum over the key channels of the
+ * broadcast gate's), plus:
  *
  *   dout         [T][H][dv] in the io dtype: dL/do
  *   dS_T         [N][H][dk][dv] fp32: dL/dS_T, or NULL (zero)
  *   grad_q, grad_k        [T][H][dk] fp32 out;  grad_v [T][H][dv] fp32 out
- *   grad_log_alpha        [T][H][dk] fp32 out;  grad_beta [T][H] fp32 out
+ *   grad_log_alpha        [T][H][dk] fp32 out ([T][H] with KDA_FLAG_SCALAR_GATE);  grad_beta [T][H] fp32 out
  *   grad_S0               [N][H][dk][dv] fp32 out, or NULL (not written)
  *   workspace    kda_backward_workspace_size() bytes, 16-byte aligned: fp32 scratch of
  *                about (11 C dk + 9 C^2 + 3 C dv + 2 dk dv) * 4 bytes (C = 64; 737 KB
- *                at dk = dv = 128) for each of N * H * ceil(L / 64) chunk slots,
- *                L = max_seqlen (total_tokens when max_seqlen <= 0), plus about
- *                (4 dk + 2) * 4 bytes per (token, head): 3.0 GB + 0.5 GB for one sequence of
- *                8192 tokens and 32 heads (3.6 GB). Pass max_seqlen for varlen batches.
+ *                at dk = dv = 128) for each of H * (total_tokens / 64 + num_seqs) chunk
+ *                slots (at least one per 64-token chunk of every sequence and head;
+ *                max_seqlen is not needed), plus about (4 dk + 2) * 4 bytes per (token,
+ *                head) and 4 bytes per sequence: 3.0 GB + 0.5 GB for one sequence of 8192
+ *                tokens and 32 heads (3.6 GB).
  *
- * fp32 CUDA-core arithmetic (six launches; the chunk recurrences split by
- * state column, the value-dimension contractions in shared-memory tiles). It factors e^{G_r - G_i} = e^{G_r} e^{-G_i} inside each chunk:
+ * fp32 CUDA-core arithmetic (seven launches: the chunk offsets of the
+ * sequences, then six; the chunk recurrences split by state column, the
+ * value-dimension contractions in shared-memory tiles). It factors
+ * e^{G_r - G_i} = e^{G_r} e^{-G_i} inside each chunk:
  * a chunk whose decay range (minus the sum of log_alpha over it) exceeds 60
  * sets device error code 2 (kda_device_error) and its gradients are not valid.
  */

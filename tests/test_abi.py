@@ -215,7 +215,12 @@ def test_backward_workspace_queries(lib):
     assert a > 0
     assert f(1, 1024, 1024, 32, 128, 128, 1, 64, 0) < a  # per-chunk scratch grows with the chunks
     assert f(2, 8192, 4096, 32, 128, 128, 1, 64, 0) > 0
-    assert f(1, 10, 10, 1, 128, 128, 1, 64, kda.KDA_FLAG_SCALAR_GATE) == 0  # one gate per head: not yet
+    # one gate per head: the same scratch
+    assert f(1, 10, 10, 1, 128, 128, 1, 64, kda.KDA_FLAG_SCALAR_GATE) == f(1, 10, 10, 1, 128, 128, 1, 64, 0) > 0
+    # the chunk slots follow the sequences' own lengths: a varlen batch needs no slots for the
+    # longest sequence's length times the batch (16 sequences of at most 8192 tokens, 62,337 in all)
+    assert f(16, 62337, 8192, 32, 128, 128, 1, 64, 0) < f(1, 62337 + 16 * 64, 62337 + 16 * 64, 32, 128, 128, 1, 64, 0)
+    assert f(16, 62337, 8192, 32, 128, 128, 1, 64, 0) < 16 * f(1, 8192, 8192, 32, 128, 128, 1, 64, 0) / 2
     assert f(1, 10, 10, 1, 96, 128, 1, 64, 0) == 0
     assert f(0, 10, 10, 1, 128, 128, 1, 64, 0) == 0
 
@@ -239,7 +244,6 @@ def backward(lib, **over):
     (dict(N=3), kda.KDA_ERR_INVALID_ARG),
     (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
     (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
-    (dict(flags=kda.KDA_FLAG_SCALAR_GATE), kda.KDA_ERR_UNSUPPORTED),
     (dict(ws=None), kda.KDA_ERR_WORKSPACE),
     (dict(wsb=4096), kda.KDA_ERR_WORKSPACE),
     (dict(ws=A + 4), kda.KDA_ERR_MISALIGNED),

@@ -873,11 +873,18 @@ def test_backward_no_l2norm_no_state_gradient():
     _bw_check(got, inp, do, None, l2norm=False, label="no l2norm")
 
 
-def test_backward_rejects_scalar_gate():
-    inp, do, dST = _bw_inputs([16], 1, 64, torch.float32, seed=53)
-    la = inp["log_alpha"][..., 0].contiguous()
-    with pytest.raises(kda.KDAError):
-        kda.kda_backward(inp["q"], inp["k"], inp["v"], la, inp["beta"], do, dST, inp["S0"], inp["cu_seqlens"])
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 128)])
+def test_backward_scalar_gate(dtype, d):
+    """One gate per (token, head) (the Gated DeltaNet form): log_alpha [T][H], its gradient
+    [T][H], against the oracle's backward with the same per-head gates; varlen with an empty
+    and a one-token sequence."""
+    inp, do, dST = _bw_inputs([90, 0, 1, 140], 2, d, dtype, seed=53)
+    inp["log_alpha"] = inp["log_alpha"][..., 0].contiguous()
+    got = kda.kda_backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], do, dST, inp["S0"],
+                           inp["cu_seqlens"], max_seqlen=140)
+    torch.cuda.synchronize()
+    assert got[3].shape == inp["log_alpha"].shape
+    _bw_check(got, inp, do, dST, label="backward scalar gate %s d=%d" % (dtype, d))
 
 
 def test_backward_flags_strong_decay():
