@@ -197,6 +197,25 @@ def test_short_conv_rejects(lib, over, code):
 
 
 @no_gpu
+@pytest.mark.parametrize("conv,dt,d,code", [
+    (kda.ShortConv(4, A, A, A), 0, 128, kda.KDA_ERR_UNSUPPORTED),      # fp32: the CUDA-core path has no fused form
+    (kda.ShortConv(4, A, A, A), 1, 64, kda.KDA_ERR_UNSUPPORTED),       # d = 64: likewise
+    (kda.ShortConv(5, A, A, A), 1, 128, kda.KDA_ERR_UNSUPPORTED),      # windows up to 4
+    (kda.ShortConv(0, A, A, A), 1, 128, kda.KDA_ERR_UNSUPPORTED),
+    (kda.ShortConv(4, None, A, A), 1, 128, kda.KDA_ERR_INVALID_ARG),
+    (kda.ShortConv(4, A + 2, A, A), 1, 128, kda.KDA_ERR_MISALIGNED),
+    (kda.ShortConv(4, A, A + 8, A), 1, 128, kda.KDA_ERR_MISALIGNED),
+    (kda.ShortConv(4, A, A, A + 4), 1, 128, kda.KDA_ERR_MISALIGNED),
+])
+def test_prefill_conv_rejects(lib, conv, dt, d, code):
+    """kda_prefill_conv validates its convolutions on the host, before any launch."""
+    call = lambda cq, ck, cv: lib.kda_prefill_conv(A, A, A, A, A, None, None, 1, 128, 128, 2, d, d, dt, 64, 0,
+                                                   cq, ck, cv, None, A, A, A, 1 << 30, None)
+    assert call(ctypes.byref(conv), None, None) == code
+    assert call(None, None, ctypes.byref(conv)) == code
+
+
+@no_gpu
 def test_decode_conv_rejects(lib):
     ok = kda.ShortConv(4, A, A, A)
     wide = kda.ShortConv(5, A, A, A)  # the fused decode takes windows up to 4
