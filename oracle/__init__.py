@@ -26,6 +26,13 @@ Functions and the passages they follow (pages cited by title and section):
 * :func:`chunkwise_backward` -- the same gradients through the chunkwise form
   of §5 (a second CPU form: the algebra a chunked GPU backward implements),
   pinned to :func:`backward`.
+* :func:`segment_map` / :func:`segmented` -- the recurrence by segments of a
+  sequence: each token's update is affine in the state (§3), so a segment maps
+  its entry state to its exit state by ``S_out = M S_in + B`` (M the product of
+  the tokens' ``(I - beta k k^T) Diag(alpha)``, B the exit state from zero);
+  the maps of all segments are independent, composed in order, and each
+  segment's outputs then follow from its true entry state (the one-exchange
+  form of splitting a long sequence); pinned to :func:`recurrent`.
 * :func:`short_conv_swish` / :func:`short_conv_step` -- the layer's step before
   the recurrence, §6 and §6.1 (and "Kimi Delta Attention：把遗忘门做到每个通道",
   进状态之前 q/k 还要过一道预处理): a causal short convolution over the token
@@ -177,6 +184,72 @@ def output_gate(o, g, w, eps=1e-6):
     w = np.asarray(w, dtype=np.float64)
     rms = np.sqrt(np.mean(o * o, axis=-1, keepdims=True) + eps)
     return o / rms * w / (1.0 + np.exp(-g))
+
+
+def _unit_rows(x, eps):
+    """x / max(||x||, eps) over the last axis (the L2 normalisation of §6.2)."""
+    n = np.sqrt((x * x).sum(axis=-1, keepdims=True))
+    return x / np.maximum(n, eps)
+
+
+def segment_map(k, v, log_alpha, beta, l2norm=True, eps=1e-6):
+    """Affine map of one (sequence, head) segment of n tokens: ``S_out = M S_in + B``.
+
+    Each token's update ``S <- (I - beta k k^T) Diag(alpha) S + beta k v^T`` (§3) is
+    affine in S, so the segment composes to M = A_n ... A_1 with
+    ``A_t = (I - beta_t k_t k_t^T) Diag(alpha_t)`` and B = the exit state from S_in = 0.
+    k [n, dk], v [n, dv], log_alpha [n, dk] (or [n]: one gate per token), beta [n].
+    Returns ``(M [dk, dk], B [dk, dv])``; fp64, a loop over the tokens.
+    """
+    k, v, la, b = (np.asarray(x, dtype=np.float64) for x in (k, v, log_alpha, beta))
+    n, dk = k.shape
+    if l2norm:
+        k = _unit_rows(k, eps)
+    M, B = np.eye(dk), np.zeros((dk, v.shape[1]))
+    for t in range(n):
+        a = np.exp(la[t]) * np.ones(dk)
+        A = (np.eye(dk) - b[t] * np.outer(k[t], k[t])) * a[None, :]
+        M = A @ M
+        B = A @ B + b[t] * np.outer(k[t], v[t])
+    return M, B
+
+
+def segmented(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, cuts=(), l2norm=True, eps=1e-6):
+    """:func:`recurrent` computed by segments. Every sequence is cut at the offsets
+    ``cuts`` (token positions within the sequence; those outside (0, len) are ignored);
+    each segment's map (:func:`segment_map`) is formed from a zero state, independently
+    of the others; the maps are composed in order from S0 (``S_in`` of a segment is
+    ``M S_in + B`` of the one before); then each segment runs its tokens from its true
+    entry state for the outputs ``o_t = S_t^T q_t``. Returns ``(o [T, H, dv],
+    S_T [N, H, dk, dv])`` like :func:`recurrent`.
+    """
+    q, k, v, la, b = (np.asarray(x, dtype=np.float64) for x in (q, k, v, log_alpha, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.array([0, T]) if cu_seqlens is None else np.asarray(cu_seqlens, dtype=np.int64)
+    N = len(cu) - 1
+    S0 = np.zeros((N, H, dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float64)
+    if l2norm:
+        q, k = _unit_rows(q, eps), _unit_rows(k, eps)
+    o, S_T = np.zeros((T, H, dv)), np.zeros((N, H, dk, dv))
+    for s in range(N):
+        bos, eos = int(cu[s]), int(cu[s + 1])
+        edges = [bos] + sorted(bos + int(c) for c in set(cuts) if 0 < int(c) < eos - bos) + [eos]
+        for h in range(H):
+            gate = la[:, h] if la.ndim == 3 else la[:, h, None] * np.ones((1, dk))
+            maps = [segment_map(k[e0:e1, h], v[e0:e1, h], gate[e0:e1], b[e0:e1, h], l2norm=False)
+                    for e0, e1 in zip(edges[:-1], edges[1:])]
+            S = S0[s, h].copy()
+            for (e0, e1), (M, B) in zip(zip(edges[:-1], edges[1:]), maps):
+                St = S.copy()  # the segment's true entry state
+                for t in range(e0, e1):
+                    a = np.exp(gate[t])
+                    St = (np.eye(dk) - b[t, h] * np.outer(k[t, h], k[t, h])) @ (a[:, None] * St) \
+                        + b[t, h] * np.outer(k[t, h], v[t, h])
+                    o[t, h] = St.T @ q[t, h]
+                S = M @ S + B  # the composed map; equals St
+            S_T[s, h] = S
+    return o, S_T
 
 
 def _silu(x):

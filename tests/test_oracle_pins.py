@@ -723,3 +723,78 @@ def test_chunkwise_backward_equals_token_backward(chunk):
     got = oracle.chunkwise_backward(q, k, v, la, b, do, dST, S0, cu, chunk=chunk)
     for name, g, w in zip(["q", "k", "v", "log_alpha", "beta", "S0"], got, want):
         np.testing.assert_allclose(g, w, rtol=0, atol=1e-12 * max(1.0, np.abs(w).max()), err_msg=name)
+
+
+# ------------------------------------------------ segments of a sequence ----
+# Each token's update is affine in the state ([P1] §3), so a segment of a sequence maps its entry
+# state to its exit state by S_out = M S_in + B; oracle.segmented forms every segment's map from a
+# zero state, composes them in order and replays each segment from its true entry state.
+
+def _seg_case(seed, scalar_gate=False):
+    rng = np.random.default_rng(seed)
+    T, H, dk, dv = 150, 2, 6, 5
+    cu = np.array([0, 70, 70, 150])
+    q, k = rng.normal(size=(T, H, dk)), rng.normal(size=(T, H, dk))
+    v = rng.normal(size=(T, H, dv))
+    la = -np.log1p(np.exp(rng.normal(-3.0, 1.0, size=(T, H) if scalar_gate else (T, H, dk))))
+    b = 1.0 / (1.0 + np.exp(-rng.normal(size=(T, H))))
+    S0 = rng.normal(size=(3, H, dk, dv))
+    return q, k, v, la, b, S0, cu
+
+
+@pytest.mark.parametrize("cuts", [(), (37,), (1, 2, 3), (37, 38, 65, 79), (64,), (500,)])
+@pytest.mark.parametrize("scalar_gate", [False, True])
+def test_segmented_equals_recurrent(cuts, scalar_gate):
+    """Cuts anywhere (on and off 64-token chunk edges, one-token segments, past the end),
+    varlen with an empty sequence, per-channel and per-head gates."""
+    q, k, v, la, b, S0, cu = _seg_case(61 + len(cuts), scalar_gate)
+    la_full = la[..., None] * np.ones(q.shape[2]) if scalar_gate else la  # a per-head gate, broadcast
+    o_ref, S_ref = oracle.recurrent(q, k, v, la_full, b, S0, cu)
+    o, S = oracle.segmented(q, k, v, la, b, S0, cu, cuts=cuts)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12 * max(1.0, np.abs(o_ref).max()))
+    np.testing.assert_allclose(S, S_ref, rtol=0, atol=1e-12 * max(1.0, np.abs(S_ref).max()))
+
+
+def test_segment_map_closed_forms():
+    rng = np.random.default_rng(62)
+    dk, dv = 5, 4
+    k, v = rng.normal(size=(1, dk)), rng.normal(size=(1, dv))
+    la, b = -rng.uniform(0.0, 1.0, size=(1, dk)), np.array([0.7])
+    M, B = oracle.segment_map(k, v, la, b)
+    kh = k[0] / np.linalg.norm(k[0])
+    np.testing.assert_allclose(M, (np.eye(dk) - 0.7 * np.outer(kh, kh)) @ np.diag(np.exp(la[0])), atol=1e-14)
+    np.testing.assert_allclose(B, 0.7 * np.outer(kh, v[0]), atol=1e-14)
+    # beta = 0: a pure decay, M = Diag(exp(sum log_alpha)), B = 0
+    k, v = rng.normal(size=(9, dk)), rng.normal(size=(9, dv))
+    la = -rng.uniform(0.0, 0.5, size=(9, dk))
+    M, B = oracle.segment_map(k, v, la, np.zeros(9))
+    np.testing.assert_allclose(M, np.diag(np.exp(la.sum(0))), atol=1e-14)
+    assert np.abs(B).max() == 0
+
+
+@pytest.mark.parametrize("mistake", ["map order", "drop B", "compose order"])
+def test_segment_pins_catch_planted_mistakes(mistake):
+    """A map multiplied in the wrong order, a dropped B, or segments composed in the wrong
+    order each break the equality with the recurrence."""
+    q, k, v, la, b, S0, cu = _seg_case(63)
+    _, S_ref = oracle.recurrent(q, k, v, la, b, S0, cu)
+    s, h = 0, 1
+    bos, eos = int(cu[s]), int(cu[s + 1])
+    edges = [bos, bos + 23, bos + 51, eos]
+    kh = k[:, h] / np.linalg.norm(k[:, h], axis=-1, keepdims=True)
+    maps = []
+    for e0, e1 in zip(edges[:-1], edges[1:]):
+        if mistake == "map order":  # M = M A instead of A M
+            M, B = np.eye(k.shape[2]), np.zeros((k.shape[2], v.shape[2]))
+            for t in range(e0, e1):
+                A = (np.eye(k.shape[2]) - b[t, h] * np.outer(kh[t], kh[t])) * np.exp(la[t, h])[None, :]
+                M, B = M @ A, A @ B + b[t, h] * np.outer(kh[t], v[t, h])
+            maps.append((M, B))
+        else:
+            maps.append(oracle.segment_map(k[e0:e1, h], v[e0:e1, h], la[e0:e1, h], b[e0:e1, h]))
+    if mistake == "compose order":
+        maps = maps[::-1]
+    S = S0[s, h].copy()
+    for M, B in maps:
+        S = M @ S + (0.0 if mistake == "drop B" else B)
+    assert np.abs(S - S_ref[s, h]).max() > 1e-6
