@@ -798,3 +798,25 @@ def test_segment_pins_catch_planted_mistakes(mistake):
     for M, B in maps:
         S = M @ S + (0.0 if mistake == "drop B" else B)
     assert np.abs(S - S_ref[s, h]).max() > 1e-6
+
+
+def test_chunk_map_from_the_chunkwise_quantities():
+    """The map of one 64-token chunk from the chunkwise quantities a kernel forms
+    (G = cumsum log_alpha, g its last row, Kg = K e^G, Kn = K e^-G, Kd = K e^(g-G),
+    A = strict_lower(Kg Kn^T), T = (I + Diag(beta) A)^-1 Diag(beta), W = T Kg):
+    S' = (Diag(e^g) - Kd^T W) S + Kd^T T V, equal to the token-by-token map."""
+    rng = np.random.default_rng(64)
+    C, dk, dv = 64, 8, 5
+    k, v = rng.normal(size=(C, dk)), rng.normal(size=(C, dv))
+    la = -np.log1p(np.exp(rng.normal(-3.0, 1.0, size=(C, dk))))
+    b = 1.0 / (1.0 + np.exp(-rng.normal(size=C)))
+    M_ref, B_ref = oracle.segment_map(k, v, la, b)
+    kh = k / np.linalg.norm(k, axis=1, keepdims=True)
+    G = np.cumsum(la, axis=0)
+    g = G[-1]
+    Kg, Kn, Kd = kh * np.exp(G), kh * np.exp(-G), kh * np.exp(g - G)
+    A = np.tril(Kg @ Kn.T, -1)
+    T = np.linalg.solve(np.eye(C) + b[:, None] * A, np.diag(b))
+    W = T @ Kg
+    np.testing.assert_allclose(np.diag(np.exp(g)) - Kd.T @ W, M_ref, atol=1e-12)
+    np.testing.assert_allclose(Kd.T @ (T @ v), B_ref, atol=1e-12)
