@@ -269,3 +269,27 @@ def backward(lib, **over):
 ])
 def test_backward_rejects(lib, over, code):
     assert backward(lib, **over) == code
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/kda.h is a C header (C99, no C++ or torch types) and a C program links against
+    libkda.so and calls it (version and status strings need no GPU)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "use_kda.c"
+    src.write_text('#include "kda.h"\n#include <stdio.h>\n#include <string.h>\n'
+                   'int main(void) {\n'
+                   '    if (kda_version() <= 0) return 1;\n'
+                   '    if (strlen(kda_status_string(KDA_ERR_WORKSPACE)) == 0) return 2;\n'
+                   '    printf("%d\\n", (int)kda_version());\n'
+                   '    return 0;\n}\n')
+    libdir = os.path.dirname(kda.library_path())
+    exe = tmp_path / "use_kda"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(root, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lkda", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    assert int(out) == lib.kda_version()
